@@ -1,0 +1,640 @@
+#!/usr/bin/env python
+"""Throughput of the fused RHT16 + FP4 quantizer on B200: GB/s of algorithmic bytes.
+
+Default workload (one step = one pass of the hot path over one batch): the dense-1.5B-like
+linear-layer operands X [8192, 2048] (Student-t, nu=4) and W [8192, 2048] (N(0, 0.02)) quantized
+on the UFP4 fwd_y path -- RHT16 + E1M2 round-to-nearest-even, FP32 1x16 scales, along K=2048 --
+as one launch over the stacked [16384, 2048] operands. Algorithmic bytes: 2 (bf16 in) + 0.5
+(codes) + 0.25 (FP32 scale) per element.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload c2|...]
+
+Timing: inputs resident in HBM, rotating through enough buffer sets that every launch reads
+data evicted from L2; steps replayed from a CUDA graph; CUDA events on the launching stream,
+barrier + synchronize around the timed region, max over ranks. Prints one JSON line (rank 0).
+"""
+import argparse
+import concurrent.futures as cf
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused RHT+FP4-quantize GB/s (BF16 in) and fraction of B200 HBM peak"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=40000)
+    p.add_argument("--warmup", type=int, default=400)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="c2",
+                   choices=["c2", "c2-quant-only", "c2-unfused", "c3", "c4-nvfp4", "c4-nvfp4-given",
+                            "c4-nvint4", "c4-mxfp4", "c4-if4", "c5-moe-ufp4", "c5-moe-e2m1",
+                            "c5-dense-ufp4", "c5-dense-e2m1"])
+    p.add_argument("--no-extras", action="store_true", help="skip e2e, ratios and CPU baseline")
+    a = p.parse_args()
+    if a.warmup < 3:
+        p.error("--warmup must be >= 3")
+    return a
+
+
+# ---------------------------------------------------------------------------- peaks / clocks
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (earlier measurement on this pool)"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid):
+        self.uuid = gpu_uuid
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in out.splitlines():
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_scaled_bit_rht16_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current sources."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get(kernel_key)
+        if rec and rec.get("source_sha") == kernel_source_sha():
+            return rec["bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------------------- workloads
+
+class Workload:
+    """One step of a workload over R rotating buffer sets. Subclasses fill in the sizes, the
+    device buffers and enqueue()."""
+    name = ""
+    desc = ""
+    kernel_key = ""
+    launches_per_step = 1
+
+    def elements(self):
+        raise NotImplementedError
+
+    def bytes_per_step(self):
+        raise NotImplementedError
+
+    def set_bytes(self):
+        raise NotImplementedError
+
+
+def _dev_bf16(bits, device):
+    import numpy as np
+    import torch
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(device)
+
+
+class RowWorkload(Workload):
+    """fp4q_rht_quantize over one [rows, cols] bf16 tensor per step."""
+
+    def __init__(self, name, desc, make_input, cfg, kernel_key, unfused=False):
+        self.name, self.desc, self.cfg, self.kernel_key = name, desc, cfg, kernel_key
+        self.make_input = make_input
+        self.unfused = unfused
+        self.launches_per_step = 2 if unfused else 1
+        self.given = name.endswith("given")
+
+    def setup(self, device, l2_bytes):
+        import torch
+        import block_scaled_bit_rht16_b200 as fq
+        self.fq = fq
+        bits = self.make_input()
+        self.rows, self.cols = bits.shape
+        self.host_bits = bits
+        x0 = _dev_bf16(bits, device)
+        self.R = max(2, math.ceil(2 * l2_bytes / self.set_bytes()) + 1)
+        self.sets = []
+        for r in range(self.R):
+            x = x0 if r == 0 else x0.clone()
+            out = fq.Quantized(*fq._alloc_outputs(self.cfg, self.rows, self.cols, device), None, None,
+                               fq.alloc_workspace(self.cfg, self.rows, self.cols, device))
+            if self.cfg.scale == fq.FP4Q_SCALE_E4M3_1x16_TENSOR:
+                out.tensor_scale = torch.full((1,), 0.01, dtype=torch.float32, device=device)
+            y = torch.empty_like(x) if self.unfused else None
+            self.sets.append((x, out, y))
+        if self.cfg.scale == fq.FP4Q_SCALE_E4M3_1x16_TENSOR and not self.given:
+            self.launches_per_step = 2   # amax pass + quantize pass
+
+    def elements(self):
+        return self.rows * self.cols
+
+    def bytes_per_step(self):
+        import block_scaled_bit_rht16_b200 as fq
+        per = 2.0 + 0.5   # bf16 in, codes out
+        scale = self.cfg.scale
+        if scale == fq.FP4Q_SCALE_FP32_1x16:
+            per += 0.25
+        elif scale == fq.FP4Q_SCALE_E4M3_1x16_TENSOR:
+            per += 1.0 / 16
+            if not self.given:
+                per += 2.0   # the amax pass reads the input once more
+        else:
+            per += 1.0 / 32
+        return per * self.elements()
+
+    def set_bytes(self):
+        return self.bytes_per_step() + (4.0 * self.elements() if self.unfused else 0.0)
+
+    def enqueue(self, i, stream):
+        x, out, y = self.sets[i % self.R]
+        if self.unfused:
+            self.fq.rht16(x, self.cfg.sign_mask, out=y, stream=stream)
+            self.fq.rht_quantize(self.quant_only_cfg(), y, out=out, stream=stream)
+        else:
+            self.fq.rht_quantize(self.cfg, x, out=out, tensor_scale=out.tensor_scale,
+                                 tensor_scale_given=self.given, stream=stream)
+
+    def quant_only_cfg(self):
+        from dataclasses import replace
+        return replace(self.cfg, rht=0, sign_mask=0)
+
+    # e2e through the public API with host buffers
+    def e2e_setup(self, device):
+        import torch
+        self.h_in = torch.from_numpy(self.host_bits.view("int16")).view(torch.bfloat16).pin_memory()
+        x, out, _ = self.sets[0]
+        self.h_codes = torch.empty(out.codes.shape, dtype=out.codes.dtype).pin_memory()
+        self.h_scales = torch.empty(out.scales.shape, dtype=out.scales.dtype).pin_memory()
+        return self.h_in.numel() * 2, self.h_codes.numel() + self.h_scales.numel() * self.h_scales.element_size()
+
+    def e2e_step(self, stream):
+        import torch
+        x, out, _ = self.sets[0]
+        with torch.cuda.stream(stream):
+            x.copy_(self.h_in, non_blocking=True)
+            self.fq.rht_quantize(self.cfg, x, out=out, tensor_scale=out.tensor_scale,
+                                 tensor_scale_given=self.given, stream=stream)
+            self.h_codes.copy_(out.codes, non_blocking=True)
+            self.h_scales.copy_(out.scales, non_blocking=True)
+
+
+class DualWorkload(Workload):
+    def __init__(self, name, desc, make_input, rc, cc, kernel_key):
+        self.name, self.desc, self.rc, self.cc, self.kernel_key = name, desc, rc, cc, kernel_key
+        self.make_input = make_input
+
+    def setup(self, device, l2_bytes):
+        import torch
+        import block_scaled_bit_rht16_b200 as fq
+        self.fq = fq
+        bits = self.make_input()
+        self.rows, self.cols = bits.shape
+        self.host_bits = bits
+        x0 = _dev_bf16(bits, device)
+        self.R = max(2, math.ceil(2 * l2_bytes / self.set_bytes()) + 1)
+        self.sets = []
+        M, N = self.rows, self.cols
+        for r in range(self.R):
+            x = x0 if r == 0 else x0.clone()
+            out = fq.Dual(torch.empty((M, N // 2), dtype=torch.uint8, device=device),
+                          torch.empty((M, N // 16), dtype=torch.float32, device=device),
+                          torch.empty((N, M // 2), dtype=torch.uint8, device=device),
+                          torch.empty((N, M // 16), dtype=torch.float32, device=device))
+            self.sets.append((x, out))
+
+    def elements(self):
+        return self.rows * self.cols
+
+    def bytes_per_step(self):
+        return 3.5 * self.elements()
+
+    def set_bytes(self):
+        return self.bytes_per_step()
+
+    def enqueue(self, i, stream):
+        x, out = self.sets[i % self.R]
+        self.fq.quantize_dual(self.rc, self.cc, x, out=out, stream=stream)
+
+    def e2e_setup(self, device):
+        import torch
+        self.h_in = torch.from_numpy(self.host_bits.view("int16")).view(torch.bfloat16).pin_memory()
+        x, out = self.sets[0]
+        self.h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory()
+                      for t in (out.codes_row, out.scales_row, out.codes_col, out.scales_col)]
+        return self.h_in.numel() * 2, sum(t.numel() * t.element_size() for t in self.h_out)
+
+    def e2e_step(self, stream):
+        import torch
+        x, out = self.sets[0]
+        with torch.cuda.stream(stream):
+            x.copy_(self.h_in, non_blocking=True)
+            self.fq.quantize_dual(self.rc, self.cc, x, out=out, stream=stream)
+            for h, d in zip(self.h_out, (out.codes_row, out.scales_row, out.codes_col, out.scales_col)):
+                h.copy_(d, non_blocking=True)
+
+
+def make_workload(name):
+    import numpy as np
+    import block_scaled_bit_rht16_b200 as fq
+    from block_scaled_bit_rht16_b200 import synth
+
+    def c2_input():
+        x, w = synth.workload2()
+        return np.concatenate([x, w], axis=0)
+
+    if name.startswith("c2"):
+        mask = fq.sign_mask_from_seed(synth.sign_seed(2))
+        cfg = fq.recipe("ufp4", "fwd_y", "x", sign_mask=mask)
+        desc = ("dense-1.5B-like operands X[8192,2048] Student-t(4) + W[8192,2048] N(0,0.02), "
+                "UFP4 fwd_y: RHT16 + E1M2 RTNE, FP32 1x16 scales along K=2048, one launch over "
+                "the stacked [16384,2048]")
+        if name == "c2-quant-only":
+            from dataclasses import replace
+            return RowWorkload(name, desc + " -- rotation off (quantize only)", c2_input,
+                               replace(cfg, rht=0, sign_mask=0), "quantize_kernel<E1M2,FP32,RTNE>")
+        if name == "c2-unfused":
+            return RowWorkload(name, desc + " -- unfused: rotation pass to bf16, then quantize",
+                               c2_input, cfg, "rht16_kernel+quantize_kernel", unfused=True)
+        return RowWorkload(name, desc, c2_input, cfg, "quantize_kernel<E1M2,FP32,RTNE>")
+    if name == "c3":
+        mask = fq.sign_mask_from_seed(synth.sign_seed(3))
+        rc = fq.recipe("ufp4", "bwd_dx", "dy", sign_mask=mask, sr_seed=synth.SR_SEED)
+        cc = fq.recipe("ufp4", "bwd_dw", "dy", sign_mask=mask, sr_seed=synth.SR_SEED)
+        return DualWorkload(name, "backward dY[8192,8192] N(0,1e-3) with 0.01% x100, RHT16 + E1M2 "
+                            "SR in row and column orientation from one read", synth.workload3, rc, cc,
+                            "dual_kernel<E1M2,SR,SR>")
+    if name.startswith("c4"):
+        mask = fq.sign_mask_from_seed(synth.sign_seed(4))
+        kind = name.split("-", 1)[1]
+        grid = {"nvfp4": fq.FP4Q_GRID_E2M1, "nvfp4-given": fq.FP4Q_GRID_E2M1, "nvint4": fq.FP4Q_GRID_INT4,
+                "mxfp4": fq.FP4Q_GRID_E2M1, "if4": fq.FP4Q_GRID_IF4}[kind]
+        scale = fq.FP4Q_SCALE_UE8M0_1x32 if kind == "mxfp4" else fq.FP4Q_SCALE_E4M3_1x16_TENSOR
+        cfg = fq.Config(grid=grid, scale=scale, rht=1, sign_mask=mask)
+        return RowWorkload(name, "[16384,5120] Laplace(0,1), RHT16, %s" % kind, synth.workload4, cfg,
+                           "quantize_kernel<%s>" % kind)
+    if name.startswith("c5"):
+        mask = fq.sign_mask_from_seed(synth.sign_seed(5))
+        ufp4 = name.endswith("ufp4")
+        cfg = fq.recipe("ufp4" if ufp4 else "e2m1", "fwd_y", "x", sign_mask=mask)
+        if "moe" in name:
+            def inp():
+                return np.concatenate([synth.workload5_expert(e) for e in range(64)], axis=0)
+            desc = "MoE experts [64,2048,7168] as [131072,7168], sigma_e log-uniform [0.1,10]"
+        else:
+            def inp():
+                return synth.workload5_dense_rows(0, 32768)
+            desc = "dense [32768,8192] N(0,1)"
+        desc += ", %s fwd_y" % ("UFP4 RHT16+E1M2" if ufp4 else "E2M1 baseline (no rotation)")
+        return RowWorkload(name, desc, inp, cfg, "quantize_kernel")
+    raise ValueError(name)
+
+
+# ---------------------------------------------------------------------------- timing (ours)
+
+def time_graph(wl, steps, warmup, stream, per_launch_events=True):
+    """Warm up, capture a graph of G steps (with per-step event pairs), replay it to run exactly
+    `steps` steps. Returns (total_ms, per_step_kernel_ms or None)."""
+    import torch
+    for i in range(warmup):
+        wl.enqueue(i, stream)
+    torch.cuda.synchronize()
+    G = wl.R * max(1, min(steps, 64 * wl.R) // wl.R) if steps >= wl.R else steps
+    full, rem = divmod(steps, G)
+    def ev():
+        try:   # an event recorded as a node of the captured graph
+            return torch.cuda.Event(enable_timing=True, external=True)
+        except TypeError:
+            return torch.cuda.Event(enable_timing=True)
+    evs = [(ev(), ev()) for _ in range(G)]
+
+    def capture(n, with_events):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                if with_events:
+                    evs[i][0].record(stream)
+                wl.enqueue(i, stream)
+                if with_events:
+                    evs[i][1].record(stream)
+        return g
+
+    try:
+        g_main = capture(G, per_launch_events)
+    except Exception:
+        per_launch_events = False
+        g_main = capture(G, False)
+    g_rem = capture(rem, False) if rem else None
+    g_main.replay()
+    torch.cuda.synchronize()
+    return g_main, g_rem, full, evs if per_launch_events else None
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 2**20)
+    import block_scaled_bit_rht16_b200 as fq
+    fq._lib.load()
+
+    wl = make_workload(args.workload)
+    wl.setup(dev, l2)
+    stream = torch.cuda.Stream(device=dev)
+    g_main, g_rem, full, evs = time_graph(wl, args.steps, args.warmup, stream)
+
+    sampler = ClockSampler("GPU-" + str(props.uuid)) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(full):
+        g_main.replay()
+    if g_rem is not None:
+        g_rem.replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    bytes_step = wl.bytes_per_step()
+    value = world * bytes_step / (ms_per_step * 1e-3) / 1e9
+
+    kernel_ms = None
+    if evs is not None:
+        try:
+            kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+        except Exception:
+            kernel_ms = None
+    peak, peak_src = hbm_peak()
+    achieved = bytes_step / wl.launches_per_step / ((kernel_ms if kernel_ms else ms_per_step) * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": profiled_traffic(wl.kernel_key),
+                "kernel": wl.kernel_key, "peak_source": peak_src,
+                "kernel_us": round((kernel_ms or ms_per_step) * 1e3, 3),
+                "algorithmic_bytes_per_launch": bytes_step / wl.launches_per_step}
+
+    extras = {}
+    if not args.no_extras:
+        extras["e2e"] = measure_e2e(wl, stream, world)
+        if args.workload == "c2":
+            extras["ratios"] = measure_ratios(args, stream, dev, l2, kernel_ms or ms_per_step)
+    del g_main, g_rem
+    if world > 1:
+        dist.barrier()
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": wl.desc, "elements_per_step": wl.elements(),
+                   "algorithmic_bytes_per_step": bytes_step,
+                   "l2": "rotating %d input/output sets (%.0f MiB total > 2x L2 of %.0f MiB)"
+                         % (wl.R, wl.R * wl.set_bytes() / 2**20, l2 / 2**20),
+                   "launch": "CUDA graph replay, %d launch(es) per step" % wl.launches_per_step,
+                   "parallelism": "dp%d (independent rows per rank, no collective)" % world},
+        "hbm_frac": round(value / world / peak, 4),
+        "roofline": roofline,
+        "gpu_launches": args.steps * wl.launches_per_step,
+        "clocks": clocks,
+    }
+    line.update({k: v for k, v in extras.items() if k != "ratios"})
+    if "ratios" in extras:
+        line["ratios"] = extras["ratios"]
+    if rank == 0 and world == 1 and not args.no_extras:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def measure_e2e(wl, stream, world, steps=30):
+    """Same metric through the public API with pinned host buffers: H2D copy of the step's
+    inputs, the quantize call, D2H copy of codes and scales, all inside the timed region."""
+    import torch
+    h2d, d2h = wl.e2e_setup(stream.device)
+    for _ in range(3):
+        wl.e2e_step(stream)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        wl.e2e_step(stream)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    return {"value": round(world * wl.bytes_per_step() / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": round(ms, 4)}
+
+
+def measure_ratios(args, stream, dev, l2, fused_kernel_ms):
+    """Time relative to quantize-only (rotation off), as the UFP4 pages report it: fused and
+    unfused (rotation pass to bf16, then quantize-only), kernel time per step."""
+    out = {}
+    per = {}
+    for name in ("c2-quant-only", "c2-unfused"):
+        wl = make_workload(name)
+        wl.setup(dev, l2)
+        steps = 64 * wl.R
+        g, _, _, evs = time_graph(wl, steps, 20, stream)
+        g.replay()
+        import torch
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(20):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        per[name] = a.elapsed_time(b) / (20 * steps)
+        del g, wl
+        torch.cuda.empty_cache()
+    qo = per["c2-quant-only"]
+    out["quant_only_us_per_step"] = round(qo * 1e3, 3)
+    out["fused_over_quant_only"] = round(fused_kernel_ms / qo, 4)
+    out["unfused_over_quant_only"] = round(per["c2-unfused"] / qo, 4)
+    out["pages_sm100"] = {"fused": 1.07, "unfused": 1.41}
+    return out
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+
+def _oracle_cfg(cfg):
+    import oracle as O
+    import block_scaled_bit_rht16_b200 as fq
+    g = {fq.FP4Q_GRID_E2M1: O.GRID_E2M1, fq.FP4Q_GRID_E1M2: O.GRID_E1M2, fq.FP4Q_GRID_INT4: O.GRID_INT4,
+         fq.FP4Q_GRID_IF4: O.GRID_IF4}[cfg.grid]
+    s = {fq.FP4Q_SCALE_FP32_1x16: O.SCALE_FP32_1x16, fq.FP4Q_SCALE_E4M3_1x16_TENSOR: O.SCALE_E4M3_1x16,
+         fq.FP4Q_SCALE_UE8M0_1x32: O.SCALE_UE8M0_1x32}[cfg.scale]
+    return O.OracleConfig(grid=g, scale=s, round=O.ROUND_SR if cfg.round else O.ROUND_RTNE, rht=cfg.rht,
+                          sign_mask=cfg.sign_mask, sr_stream=cfg.sr_stream, sr_seed=cfg.sr_seed)
+
+
+def oracle_pass(cfg, bits, rows_total, threads):
+    """The oracle over `rows_total` rows of `bits` (cycled), chunked over a thread pool (the
+    ctypes call releases the GIL). Returns seconds."""
+    import oracle as O
+    oc = _oracle_cfg(cfg)
+    chunk = 64
+    starts = [(r % bits.shape[0]) for r in range(0, rows_total, chunk)]
+
+    def one(r0):
+        r1 = min(r0 + chunk, bits.shape[0])
+        O.quantize(oc, bits[r0:r1], row0=r0,
+                   tensor_scale=0.01 if oc.scale == O.SCALE_E4M3_1x16 else None)
+
+    t = time.perf_counter()
+    if threads > 1:
+        with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(one, starts))
+    else:
+        for r0 in starts:
+            one(r0)
+    return time.perf_counter() - t
+
+
+def cpu_baseline(wl, budget_s=12.0):
+    cores = len(os.sched_getaffinity(0))
+    cfg = getattr(wl, "cfg", None) or wl.rc
+    bits = wl.host_bits
+    probe_rows = 256
+    t = oracle_pass(cfg, bits, probe_rows, cores)
+    rows = int(min(bits.shape[0], max(probe_rows, probe_rows * budget_s / max(t, 1e-6) / 4)))
+    t = oracle_pass(cfg, bits, rows, cores)
+    per_elem = wl.bytes_per_step() / wl.elements()
+    gbs = rows * bits.shape[1] * per_elem / t / 1e9
+    return {"value": round(gbs, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": "%d of %d rows of the step's tensor (%.1f s wall on %d threads)"
+                      % (rows, bits.shape[0], t, cores)}
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle as it stands, timed on the host cores on a bounded
+    sample of the same workload per step (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from block_scaled_bit_rht16_b200 import synth
+    import numpy as np
+    import block_scaled_bit_rht16_b200 as fq
+    mask = fq.sign_mask_from_seed(synth.sign_seed(2))
+    cfg = fq.recipe("ufp4", "fwd_y", "x", sign_mask=mask)
+    x, w = synth.workload2()
+    bits = np.concatenate([x, w], axis=0)
+    cores = len(os.sched_getaffinity(0))
+    t1 = oracle_pass(cfg, bits, 64, 1)   # rows per second on one core
+    rate = 64 / max(t1, 1e-6) * max(1, cores) * 0.7
+    budget = 120.0
+    rows = max(1, min(bits.shape[0], int(rate * budget / (args.steps + args.warmup))))
+    threads = cores if rows >= 64 * cores else 1
+    for i in range(args.warmup):
+        oracle_pass(cfg, bits, rows, threads)
+    t = 0.0
+    for i in range(args.steps):
+        t += oracle_pass(cfg, bits, rows, threads)
+    bytes_per_elem = 2.75
+    value = args.steps * rows * bits.shape[1] * bytes_per_elem / t / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(t / args.steps * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "dense-1.5B-like operands X[8192,2048] + W[8192,2048], UFP4 fwd_y "
+                                   "(RHT16 + E1M2 RTNE, FP32 1x16), CPU oracle on %d rows per step" % rows},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": "%d rows x 2048 per step, cycled through the stacked X,W" % rows},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

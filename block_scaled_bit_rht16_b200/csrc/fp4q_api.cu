@@ -1,0 +1,301 @@
+// fp4q_api.cu -- the C ABI declared in include/fp4q.h: host-side validation, workspace layout
+// and kernel dispatch. Every argument is checked before anything is enqueued; a rejected call
+// launches nothing.
+#include <cmath>
+#include <cstring>
+
+#include "../../include/fp4q.h"
+#include "fp4q_kernels.cuh"
+
+using namespace fp4q;
+
+namespace {
+
+bool aligned(const void* p, size_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+
+uint64_t host_splitmix64(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Per bf16 pair k: bit 15 flips element 2k, bit 31 flips element 2k+1.
+void sign_words(uint32_t mask, bool rht, uint32_t* sw) {
+  for (int k = 0; k < 8; ++k) {
+    sw[k] = 0u;
+    if (!rht) continue;
+    if ((mask >> (2 * k)) & 1u) sw[k] |= 0x00008000u;
+    if ((mask >> (2 * k + 1)) & 1u) sw[k] |= 0x80000000u;
+  }
+}
+
+fp4q_status check_cfg(const fp4q_config* cfg) {
+  if (cfg == nullptr) return FP4Q_ERR_INVALID_ARG;
+  if (cfg->grid < FP4Q_GRID_E2M1 || cfg->grid > FP4Q_GRID_IF4) return FP4Q_ERR_INVALID_ARG;
+  if (cfg->scale < FP4Q_SCALE_FP32_1x16 || cfg->scale > FP4Q_SCALE_UE8M0_1x32) return FP4Q_ERR_INVALID_ARG;
+  if (cfg->round != FP4Q_ROUND_RTNE && cfg->round != FP4Q_ROUND_SR) return FP4Q_ERR_INVALID_ARG;
+  if (cfg->rht != 0 && cfg->rht != 1) return FP4Q_ERR_INVALID_ARG;
+  if (cfg->sign_mask > 0xFFFFu) return FP4Q_ERR_INVALID_ARG;
+  if (cfg->outputs & ~(uint32_t)(FP4Q_OUT_CODES | FP4Q_OUT_DEQUANT | FP4Q_OUT_STATS)) return FP4Q_ERR_INVALID_ARG;
+  if (cfg->reserved != 0u) return FP4Q_ERR_INVALID_ARG;
+  if (cfg->grid == FP4Q_GRID_IF4 &&
+      (cfg->scale != FP4Q_SCALE_E4M3_1x16_TENSOR || cfg->round != FP4Q_ROUND_RTNE))
+    return FP4Q_ERR_UNSUPPORTED;
+  if (cfg->scale == FP4Q_SCALE_UE8M0_1x32 && cfg->grid != FP4Q_GRID_E2M1) return FP4Q_ERR_UNSUPPORTED;
+  return FP4Q_OK;
+}
+
+int block_elems(const fp4q_config* cfg) { return cfg->scale == FP4Q_SCALE_UE8M0_1x32 ? 32 : 16; }
+
+size_t stats_bytes() { return (size_t)kStatsCtas * ST_LEN * sizeof(double); }
+
+fp4q_status check_shape(int64_t rows, int64_t cols, int64_t ld, int unit) {
+  if (rows < 0 || cols < 0) return FP4Q_ERR_SHAPE;
+  if (cols % unit != 0) return FP4Q_ERR_SHAPE;
+  if (ld < cols) return FP4Q_ERR_SHAPE;
+  if (rows > 1 && ld % 8 != 0) return FP4Q_ERR_ALIGN;   // every row starts 16-byte aligned
+  return FP4Q_OK;
+}
+
+fp4q_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP4Q_OK : FP4Q_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* fp4q_status_string(fp4q_status s) {
+  switch (s) {
+    case FP4Q_OK: return "ok";
+    case FP4Q_ERR_INVALID_ARG: return "invalid argument";
+    case FP4Q_ERR_SHAPE: return "invalid shape";
+    case FP4Q_ERR_ALIGN: return "misaligned pointer or row pitch";
+    case FP4Q_ERR_UNSUPPORTED: return "unsupported configuration";
+    case FP4Q_ERR_WORKSPACE: return "workspace missing or too small";
+    case FP4Q_ERR_CUDA: return "CUDA error";
+    case FP4Q_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+uint32_t fp4q_sign_mask_from_seed(uint64_t seed) { return (uint32_t)(host_splitmix64(seed) & 0xFFFFu); }
+
+size_t fp4q_workspace_size(const fp4q_config* cfg, int64_t rows, int64_t cols) {
+  if (check_cfg(cfg) != FP4Q_OK || rows < 0 || cols < 0) return 0;
+  const bool stats = (cfg->outputs & FP4Q_OUT_STATS) != 0;
+  const bool nv = cfg->scale == FP4Q_SCALE_E4M3_1x16_TENSOR;
+  if (!stats && !nv) return 0;
+  return sizeof(WsHeader) + (stats ? stats_bytes() : 0);
+}
+
+fp4q_status fp4q_rht_quantize(const fp4q_config* cfg, const void* x, int64_t rows, int64_t cols,
+                              int64_t ld, uint8_t* codes, void* scales, float* tensor_scale,
+                              int32_t tensor_scale_given, void* dequant, void* workspace,
+                              size_t workspace_bytes, fp4q_stream_t stream) {
+  fp4q_status st = check_cfg(cfg);
+  if (st != FP4Q_OK) return st;
+  const int unit = block_elems(cfg);
+  st = check_shape(rows, cols, ld, unit);
+  if (st != FP4Q_OK) return st;
+  const bool want_deq = (cfg->outputs & FP4Q_OUT_DEQUANT) != 0;
+  const bool want_stats = (cfg->outputs & FP4Q_OUT_STATS) != 0;
+  const bool nv = cfg->scale == FP4Q_SCALE_E4M3_1x16_TENSOR;
+  const bool compute_alpha = nv && !tensor_scale_given;
+  const bool empty = rows == 0 || cols == 0;
+  if (!empty && (x == nullptr || codes == nullptr || scales == nullptr)) return FP4Q_ERR_INVALID_ARG;
+  if (want_deq && !empty && dequant == nullptr) return FP4Q_ERR_INVALID_ARG;
+  if (nv && tensor_scale == nullptr) return FP4Q_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(codes, unit == 32 ? 16 : 8) || !aligned(scales, 4) ||
+      !aligned(dequant, 16) || !aligned(tensor_scale, 4) || !aligned(workspace, 256))
+    return FP4Q_ERR_ALIGN;
+  const size_t need = fp4q_workspace_size(cfg, rows, cols);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return FP4Q_ERR_WORKSPACE;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  WsHeader* ws = reinterpret_cast<WsHeader*>(workspace);
+  if (need > 0) {
+    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), s) != cudaSuccess) return FP4Q_ERR_CUDA;
+  }
+  if (empty) {
+    if (compute_alpha && cudaMemsetAsync(tensor_scale, 0, sizeof(float), s) != cudaSuccess)
+      return FP4Q_ERR_CUDA;
+    return FP4Q_OK;
+  }
+
+  QuantArgs a{};
+  a.x = static_cast<const uint16_t*>(x);
+  a.rows = rows;
+  a.cols = cols;
+  a.ld = ld;
+  a.units_per_row = cols / unit;
+  a.nunits = rows * a.units_per_row;
+  a.codes = codes;
+  a.scales = scales;
+  a.deq = want_deq ? static_cast<uint16_t*>(dequant) : nullptr;
+  a.ts_in = (nv && tensor_scale_given) ? tensor_scale : nullptr;
+  a.ts_out = compute_alpha ? tensor_scale : nullptr;
+  a.ws = need > 0 ? ws : nullptr;
+  a.partials = want_stats ? reinterpret_cast<double*>(static_cast<char*>(workspace) + sizeof(WsHeader)) : nullptr;
+  sign_words(cfg->sign_mask, cfg->rht != 0, a.sw);
+  a.c = cfg->rht ? 4.0f : 1.0f;
+  a.cinv = cfg->rht ? 0.25f : 1.0f;
+  a.seedx = cfg->sr_seed ^ ((uint64_t)(cfg->sr_stream & 1u) << 63);
+  a.contiguous = (ld == cols) ? 1 : 0;
+
+  if (compute_alpha) {
+    QuantArgs am = a;
+    if (cfg->scale == FP4Q_SCALE_E4M3_1x16_TENSOR) {
+      am.units_per_row = cols / 16;
+      am.nunits = rows * am.units_per_row;
+    }
+    if (launch_amax(am, s) != cudaSuccess) return FP4Q_ERR_CUDA;
+  }
+  return cuda_status(launch_quantize(cfg->grid, cfg->scale, cfg->round, want_stats, a, s));
+}
+
+fp4q_status fp4q_if4_select(const fp4q_config* cfg, const void* x, int64_t rows, int64_t cols,
+                            int64_t ld, uint8_t* codes, uint8_t* scales_flagged,
+                            float* tensor_scale, int32_t tensor_scale_given, void* dequant,
+                            void* workspace, size_t workspace_bytes, fp4q_stream_t stream) {
+  if (cfg == nullptr) return FP4Q_ERR_INVALID_ARG;
+  fp4q_config c = *cfg;
+  c.grid = FP4Q_GRID_IF4;
+  c.scale = FP4Q_SCALE_E4M3_1x16_TENSOR;
+  return fp4q_rht_quantize(&c, x, rows, cols, ld, codes, scales_flagged, tensor_scale,
+                           tensor_scale_given, dequant, workspace, workspace_bytes, stream);
+}
+
+fp4q_status fp4q_quantize_dual(const fp4q_config* row_cfg, const fp4q_config* col_cfg,
+                               const void* dy, int64_t M, int64_t N, int64_t ld,
+                               uint8_t* codes_row, void* scales_row, uint8_t* codes_col,
+                               void* scales_col, void* workspace, size_t workspace_bytes,
+                               fp4q_stream_t stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  fp4q_status st = check_cfg(row_cfg);
+  if (st != FP4Q_OK) return st;
+  st = check_cfg(col_cfg);
+  if (st != FP4Q_OK) return st;
+  for (const fp4q_config* c : {row_cfg, col_cfg}) {
+    if (c->scale != FP4Q_SCALE_FP32_1x16 || c->grid == FP4Q_GRID_IF4) return FP4Q_ERR_UNSUPPORTED;
+    if (c->outputs & (FP4Q_OUT_DEQUANT | FP4Q_OUT_STATS)) return FP4Q_ERR_UNSUPPORTED;
+  }
+  if (row_cfg->grid != col_cfg->grid) return FP4Q_ERR_UNSUPPORTED;
+  if (M < 0 || N < 0 || M % 16 != 0 || N % 16 != 0 || ld < N) return FP4Q_ERR_SHAPE;
+  if (M > 1 && ld % 8 != 0) return FP4Q_ERR_ALIGN;
+  const bool empty = M == 0 || N == 0;
+  if (!empty && (dy == nullptr || codes_row == nullptr || scales_row == nullptr ||
+                 codes_col == nullptr || scales_col == nullptr))
+    return FP4Q_ERR_INVALID_ARG;
+  if (!aligned(dy, 16) || !aligned(codes_row, 8) || !aligned(codes_col, 8) ||
+      !aligned(scales_row, 4) || !aligned(scales_col, 4))
+    return FP4Q_ERR_ALIGN;
+  if (empty) return FP4Q_OK;
+  DualArgs a{};
+  a.dy = static_cast<const uint16_t*>(dy);
+  a.M = M;
+  a.N = N;
+  a.ld = ld;
+  a.codes_row = codes_row;
+  a.scales_row = static_cast<float*>(scales_row);
+  a.codes_col = codes_col;
+  a.scales_col = static_cast<float*>(scales_col);
+  sign_words(row_cfg->sign_mask, row_cfg->rht != 0, a.sw_row);
+  sign_words(col_cfg->sign_mask, col_cfg->rht != 0, a.sw_col);
+  a.c_row = row_cfg->rht ? 4.0f : 1.0f;
+  a.cinv_row = row_cfg->rht ? 0.25f : 1.0f;
+  a.c_col = col_cfg->rht ? 4.0f : 1.0f;
+  a.cinv_col = col_cfg->rht ? 0.25f : 1.0f;
+  a.seedx_row = row_cfg->sr_seed ^ ((uint64_t)(row_cfg->sr_stream & 1u) << 63);
+  a.seedx_col = col_cfg->sr_seed ^ ((uint64_t)(col_cfg->sr_stream & 1u) << 63);
+  a.round_row = row_cfg->round;
+  a.round_col = col_cfg->round;
+  a.grid_row = row_cfg->grid;
+  a.grid_col = col_cfg->grid;
+  return cuda_status(launch_dual(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fp4q_status fp4q_dequantize(const fp4q_config* cfg, const uint8_t* codes, const void* scales,
+                            const float* tensor_scale, int64_t rows, int64_t cols,
+                            int32_t inverse_rht, void* out, fp4q_stream_t stream) {
+  fp4q_status st = check_cfg(cfg);
+  if (st != FP4Q_OK) return st;
+  if (inverse_rht != 0 && inverse_rht != 1) return FP4Q_ERR_INVALID_ARG;
+  st = check_shape(rows, cols, cols, block_elems(cfg));
+  if (st != FP4Q_OK) return st;
+  const bool empty = rows == 0 || cols == 0;
+  const bool nv = cfg->scale == FP4Q_SCALE_E4M3_1x16_TENSOR;
+  if (!empty && (codes == nullptr || scales == nullptr || out == nullptr)) return FP4Q_ERR_INVALID_ARG;
+  if (!empty && nv && tensor_scale == nullptr) return FP4Q_ERR_INVALID_ARG;
+  if (!aligned(codes, 8) || !aligned(out, 16) || !aligned(scales, 4) || !aligned(tensor_scale, 4))
+    return FP4Q_ERR_ALIGN;
+  if (empty) return FP4Q_OK;
+  uint32_t sw[8];
+  sign_words(cfg->sign_mask, true, sw);
+  return cuda_status(launch_dequant(cfg->grid, cfg->scale, codes, scales, tensor_scale, rows, cols,
+                                    sw, inverse_rht != 0, static_cast<uint16_t*>(out),
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fp4q_status fp4q_rht16(const void* x, int64_t rows, int64_t cols, int64_t ld, uint32_t sign_mask,
+                       void* out, int32_t out_fp32, fp4q_stream_t stream) {
+  if (sign_mask > 0xFFFFu || (out_fp32 != 0 && out_fp32 != 1)) return FP4Q_ERR_INVALID_ARG;
+  fp4q_status st = check_shape(rows, cols, ld, 16);
+  if (st != FP4Q_OK) return st;
+  const bool empty = rows == 0 || cols == 0;
+  if (!empty && (x == nullptr || out == nullptr)) return FP4Q_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(out, 16)) return FP4Q_ERR_ALIGN;
+  if (empty) return FP4Q_OK;
+  uint32_t sw[8];
+  sign_words(sign_mask, true, sw);
+  return cuda_status(launch_rht16(static_cast<const uint16_t*>(x), rows, cols, ld, sw, out,
+                                  out_fp32 != 0, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fp4q_status fp4q_stats(const void* workspace, size_t workspace_bytes, fp4q_stats_t* host_out,
+                       fp4q_stream_t stream) {
+  if (workspace == nullptr || host_out == nullptr) return FP4Q_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return FP4Q_ERR_ALIGN;
+  if (workspace_bytes < sizeof(WsHeader) + stats_bytes()) return FP4Q_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  WsHeader* ws = reinterpret_cast<WsHeader*>(const_cast<void*>(workspace));
+  const double* partials = reinterpret_cast<const double*>(static_cast<const char*>(workspace) + sizeof(WsHeader));
+  if (launch_stats_reduce(ws, partials, s) != cudaSuccess) return FP4Q_ERR_CUDA;
+  WsHeader h;
+  if (cudaMemcpyAsync(&h, ws, sizeof h, cudaMemcpyDeviceToHost, s) != cudaSuccess) return FP4Q_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FP4Q_ERR_CUDA;
+
+  std::memset(host_out, 0, sizeof *host_out);
+  const double* r = h.reduced;
+  host_out->sum_y2 = r[ST_SUM_Y2];
+  host_out->sum_err2 = r[ST_SUM_ERR2];
+  host_out->sum_y_xhat = r[ST_SUM_YXHAT];
+  host_out->n = r[ST_N];
+  for (int c = 0; c < 8; ++c) {
+    host_out->cell_count[c] = r[ST_CELL_N + c];
+    host_out->cell_err[c] = r[ST_CELL_ERR + c];
+    host_out->cell_mean_err[c] = r[ST_CELL_N + c] > 0 ? r[ST_CELL_ERR + c] / r[ST_CELL_N + c] : NAN;
+  }
+  host_out->if4_fp4_blocks = r[ST_IF4_FP4];
+  host_out->blocks = r[ST_BLOCKS];
+  const double y2 = host_out->sum_y2, e2 = host_out->sum_err2;
+  host_out->sqnr_db = e2 == 0.0 ? INFINITY : (y2 > 0.0 ? 10.0 * std::log10(y2 / e2) : -INFINITY);
+  host_out->alpha = y2 > 0.0 ? host_out->sum_y_xhat / y2 : 1.0;
+  host_out->mse = host_out->n > 0 ? e2 / host_out->n : 0.0;
+  host_out->nmse = y2 > 0.0 ? e2 / y2 : 0.0;
+  host_out->if4_fp4_fraction = host_out->blocks > 0 ? host_out->if4_fp4_blocks / host_out->blocks : 0.0;
+  host_out->status = h.status == 0 ? FP4Q_OK : FP4Q_ERR_TIMEOUT;
+  return host_out->status == FP4Q_OK ? FP4Q_OK : FP4Q_ERR_TIMEOUT;
+}
+
+fp4q_status fp4q_check_division(uint64_t seed, uint64_t n, unsigned long long* mismatches,
+                                fp4q_stream_t stream) {
+  if (mismatches == nullptr) return FP4Q_ERR_INVALID_ARG;
+  if (!aligned(mismatches, 8)) return FP4Q_ERR_ALIGN;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(mismatches, 0, sizeof(unsigned long long), s) != cudaSuccess) return FP4Q_ERR_CUDA;
+  if (n == 0) return FP4Q_OK;
+  return cuda_status(launch_division_check(seed, n, mismatches, s));
+}
+
+}  // extern "C"

@@ -1,0 +1,184 @@
+// fp4q_device.cuh -- device building blocks of the fused RHT16 + 4-bit quantizer (sm_100a).
+//
+// Layout of a 16-element block in registers: eight float2 P[i] = (v_i, v_{i+8}), i = 0..7.
+// Butterfly stages h = 1, 2, 4 pair P[i] with P[i+h] and run as packed f32x2 adds (one
+// instruction per two elements); stage h = 8 pairs the two lanes of each P[i] and runs scalar.
+// Every operation is the same IEEE binary32 operation, in the same stage order, as the
+// definition (butterfly stages 1, 2, 4, 8, each (a+b, a-b)), so the result is bit-identical.
+//
+// Sources: "蚂蚁集团揭秘：为什么给AI"降精度省电"会悄悄让它越来越笨？" (techwalker.com), section
+// 六 Q5 (16-point rotation fused with the 16-element quantization block); "当你的 GPU 学不会算账"
+// (zhichai.net/topic/178208020), sections "E2M1" and "UFP4" (grids, recipe table).
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fp4q {
+
+enum Grid { kE2M1 = 0, kE1M2 = 1, kINT4 = 2, kIF4 = 3 };
+enum Scale { kFP32 = 0, kE4M3 = 1, kUE8M0 = 2 };
+enum Round { kRTNE = 0, kSR = 1 };
+
+// ------------------------------------------------------------------ bf16 / packed helpers
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+// a - b as fma(b, -1, a): one rounding of the exact difference, like a plain subtraction.
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
+}
+
+// Load-side: eight 32-bit words (bf16 pairs) -> P[8], with the sign diagonal applied by
+// flipping the bf16 sign bits (exact). sw[k] holds the flips of elements 2k (bit 15) and
+// 2k+1 (bit 31).
+__device__ __forceinline__ void unpack16(const uint4& lo, const uint4& hi, const uint32_t* sw,
+                                         float2* P) {
+  const uint32_t w[8] = {lo.x ^ sw[0], lo.y ^ sw[1], lo.z ^ sw[2], lo.w ^ sw[3],
+                         hi.x ^ sw[4], hi.y ^ sw[5], hi.z ^ sw[6], hi.w ^ sw[7]};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    P[2 * k] = make_float2(bf_lo(w[k]), bf_lo(w[k + 4]));
+    P[2 * k + 1] = make_float2(bf_hi(w[k]), bf_hi(w[k + 4]));
+  }
+}
+
+// v <- H16 v in natural (Sylvester) order, stages h = 1, 2, 4, 8. No 1/4 here: callers fold the
+// exact power-of-two normalisation into the scale.
+__device__ __forceinline__ void fwht16(float2* P) {
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if ((i & h) == 0) {
+        const float2 a = P[i], b = P[i + h];
+        P[i] = add2(a, b);
+        P[i + h] = sub2(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float a = P[i].x, b = P[i].y;
+    P[i] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+  }
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// max_i |v_i| over the 16 elements (exact, order-free).
+__device__ __forceinline__ float absmax16(const float2* P) {
+  float m0 = max3(fabsf(P[0].x), fabsf(P[0].y), fabsf(P[1].x));
+  float m1 = max3(fabsf(P[1].y), fabsf(P[2].x), fabsf(P[2].y));
+  float m2 = max3(fabsf(P[3].x), fabsf(P[3].y), fabsf(P[4].x));
+  float m3 = max3(fabsf(P[4].y), fabsf(P[5].x), fabsf(P[5].y));
+  float m4 = max3(fabsf(P[6].x), fabsf(P[6].y), fabsf(P[7].x));
+  float m5 = max3(m0, m1, fabsf(P[7].y));
+  return max3(m2, m3, max3(m4, m5, 0.0f));
+}
+
+// ------------------------------------------------------------------ exact division
+//
+// v = RN(y / s) for a whole block, with y = c^-1 * vraw (c = 4 with rotation, 1 without; an
+// exact power of two). The quotient is Markstein's correction step (P. Markstein, "Computation
+// of elementary functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990):
+// with R = RN(1/S) and q0 = RN(a R), the remainder r = a - q0 S is exact under an FMA and
+// q1 = RN(q0 + r R) is the correctly rounded a/S. Here S = c*s and a = vraw, so a/S = y/s.
+// The step is valid while S and 1/S are normal with headroom and |a| >= 2^-100 * max(1, S);
+// Smaller |a| give quotients below 2^-99, which every rounding rule here maps to a zero code
+// (stochastic rounding recomputes them with the IEEE division, see div_tiny_fix).
+struct Divider {
+  float2 R2, nS2;   // (R, R), (-S, -S)
+  float S, R;
+  bool fast;        // the block's S is in the range where the correction step is exact
+};
+
+__device__ __forceinline__ Divider make_divider(float s, float c) {
+  Divider d;
+  d.S = __fmul_rn(s, c);
+  d.fast = (d.S >= 0x1p-90f) && (d.S <= 0x1p+90f);
+  d.R = d.fast ? __frcp_rn(d.S) : 0.0f;
+  d.R2 = make_float2(d.R, d.R);
+  d.nS2 = make_float2(-d.S, -d.S);
+  return d;
+}
+
+// Quotients of a packed pair (signed; -0 inputs give +0, callers take signs from vraw).
+__device__ __forceinline__ float2 div2(const Divider& d, float2 a) {
+  const float2 q0 = __fmul2_rn(a, d.R2);
+  const float2 r = __ffma2_rn(q0, d.nS2, a);
+  return __ffma2_rn(r, d.R2, q0);
+}
+
+// ------------------------------------------------------------------ grids
+
+template <int G> struct GridInfo;
+template <> struct GridInfo<kE2M1> { static constexpr float qmax = 6.0f; };
+template <> struct GridInfo<kE1M2> { static constexpr float qmax = 3.5f; };
+template <> struct GridInfo<kINT4> { static constexpr float qmax = 7.0f; };
+template <> struct GridInfo<kIF4> { static constexpr float qmax = 6.0f; };
+
+// E2M1 codes of two values, hardware round-to-nearest-even with saturation to +-6; the sign of
+// each input (including -0) is kept. Result: a in bits 4..7, b in bits 0..3.
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float a, float b) {
+  uint32_t r;
+  asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u32.u8 %0, t; }"
+      : "=r"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// Signed value of two E2M1 codes packed in a byte (exact decode): low nibble -> .x.
+__device__ __forceinline__ float2 e2m1x2_to_f32(uint32_t byte) {
+  uint32_t h2;
+  asm("{ .reg .b8 t; cvt.u8.u32 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }" : "=r"(h2) : "r"(byte));
+  __half2 h = *reinterpret_cast<__half2*>(&h2);
+  return __half22float2(h);
+}
+
+// E4M3 (satfinite, round to nearest even) of a non-negative float -> byte.
+__device__ __forceinline__ uint32_t cvt_e4m3(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+  return r & 0xFFu;
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
+  uint32_t h2;
+  const uint16_t b = static_cast<uint16_t>(byte & 0x7Fu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(b));
+  __half2 h = *reinterpret_cast<__half2*>(&h2);
+  return __low2float(h);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// ------------------------------------------------------------------ stochastic rounding source
+
+__device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// 64 random bits for the element pair (2p, 2p+1); seedx = seed ^ (stream << 63).
+__device__ __forceinline__ uint64_t sr_pair_bits(uint64_t seedx, uint64_t pair) {
+  return splitmix64(seedx ^ (pair * 0x9E3779B97F4A7C15ull));
+}
+
+// Round-up decision r < frac with r = (u >> 8) * 2^-24, taken exactly as
+// (u >> 8) < frac * 2^24 (both sides exact in FP32).
+__device__ __forceinline__ bool sr_up(uint32_t u, float frac) {
+  return __uint2float_rn(u >> 8) < __fmul_rn(frac, 16777216.0f);
+}
+
+}  // namespace fp4q

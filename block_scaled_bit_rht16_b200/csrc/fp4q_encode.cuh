@@ -1,0 +1,277 @@
+// fp4q_encode.cuh -- per-block encoder shared by the row and dual-orientation kernels.
+//
+// Input: one 16-element block as P[8] = (v_i, v_{i+8}) after the butterfly (not yet times 1/4),
+// the block's dequant multiplier s (0 marks an all-zero block) and its Divider. Output: the
+// 8-byte code word pair, optional bf16 dequant, optional statistics.
+//
+// Rounding follows "蚂蚁集团揭秘…" (techwalker.com) section 二 (round to nearest, ties to even
+// code) and "低精度量化技术：IF4…" (bxzpzcl.cn/news/2320061) section 6.1 (stochastic rounding
+// floor(x) + (random() < frac), applied between adjacent grid points) and sections 3.1-3.2
+// (IF4: FP4 candidate vs INT4 * 7/6 candidate, smaller squared error wins).
+#pragma once
+#include <cuda_fp16.h>
+
+#include "fp4q_device.cuh"
+#include "fp4q_kernels.cuh"
+
+namespace fp4q {
+
+struct EncCtx {
+  float cinv;       // y = cinv * vraw
+  uint64_t seedx;   // SR: seed ^ (stream << 63)
+};
+
+__device__ __forceinline__ uint32_t sign_bit(float x) { return __float_as_uint(x) >> 31; }
+
+// Small exact integer m (0..15) as a float.
+__device__ __forceinline__ float small_int_f32(uint32_t m) {
+  return __fadd_rn(__uint_as_float(0x4B000000u | m), -8388608.0f);
+}
+
+// Uniform grids (E1M2: step 1/2, qmax 3.5; INT4: step 1, qmax 7). Returns the nibble; val is
+// the code's signed value in scaled units, mag the magnitude code.
+template <int G, int R>
+__device__ __forceinline__ uint32_t round_uniform(float q, float vraw, uint32_t rnd, float& val,
+                                                  uint32_t& mag) {
+  constexpr float qmax = GridInfo<G>::qmax;
+  constexpr float inv_step = (G == kE1M2) ? 2.0f : 1.0f;
+  const float t = __fmul_rn(fminf(fabsf(q), qmax), inv_step);   // |v| in steps, exact
+  uint32_t m;
+  if constexpr (R == kRTNE) {
+    m = __float_as_uint(__fadd_rn(t, 8388608.0f)) & 0xFu;        // round half to even
+  } else {
+    const float fl = floorf(t);
+    const float frac = __fsub_rn(t, fl);                          // exact
+    m = (__float_as_uint(__fadd_rn(fl, 8388608.0f)) & 0xFu) + (sr_up(rnd, frac) ? 1u : 0u);
+  }
+  const uint32_t neg = sign_bit(vraw);
+  mag = m;
+  if constexpr (G == kE1M2) {
+    const float g = __fmul_rn(small_int_f32(m), 0.5f);
+    val = __uint_as_float(__float_as_uint(g) | (neg << 31));      // -0 stays -0 (code 0x8)
+    return m | (neg << 3);
+  } else {
+    const float g = small_int_f32(m);
+    val = (neg && m) ? -g : g;                                    // two's complement has no -0
+    return (neg ? (0u - m) : m) & 0xFu;
+  }
+}
+
+// E2M1 stochastic rounding of one value: the chosen grid point, signed like vraw.
+__device__ __forceinline__ float e2m1_sr_value(float q, float vraw, uint32_t rnd) {
+  const float a = fminf(fabsf(q), 6.0f);
+  const bool lo = a < 2.0f, mid = a < 4.0f;
+  const float inv_step = lo ? 2.0f : (mid ? 1.0f : 0.5f);
+  const float step = lo ? 0.5f : (mid ? 1.0f : 2.0f);
+  const float t = __fmul_rn(a, inv_step);   // exact
+  const float fl = floorf(t);
+  const float frac = __fsub_rn(t, fl);      // exact
+  const float k = sr_up(rnd, frac) ? __fadd_rn(fl, 1.0f) : fl;
+  const float g = __fmul_rn(k, step);       // exact: a grid point
+  return __uint_as_float(__float_as_uint(g) | (__float_as_uint(vraw) & 0x80000000u));
+}
+
+__device__ __forceinline__ float with_sign_of(float q, float vraw) {
+  return __uint_as_float((__float_as_uint(q) & 0x7FFFFFFFu) | (__float_as_uint(vraw) & 0x80000000u));
+}
+
+// ------------------------------------------------------------------ statistics accumulator
+
+struct StatsAcc {
+  double y2, err2, yx, blocks, if4_fp4;
+  double* cell_err;    // shared [8][kThreads]
+  uint32_t* cell_n;    // shared [8][kThreads]
+
+  // cell error |val| - |q| is formed in FP64 (exact for two floats)
+  __device__ __forceinline__ void element(float y, float xhat, uint32_t mag, float val, float q) {
+    y2 += (double)y * (double)y;
+    const double d = (double)y - (double)xhat;
+    err2 += d * d;
+    yx += (double)y * (double)xhat;
+    cell_err[mag * kThreads + threadIdx.x] += fabs((double)val) - fabs((double)q);
+    cell_n[mag * kThreads + threadIdx.x] += 1u;
+  }
+};
+
+__device__ __forceinline__ float elem_x(const float2* A, int e) { return e < 8 ? A[e].x : A[e - 8].y; }
+
+// Encodes one block. pair0 = (logical index of element 0) / 2 for the SR counter.
+// Returns the IF4 flag (0x80 for an INT4 block, else 0).
+template <int G, int R, bool STATS>
+__device__ __forceinline__ uint32_t encode16(const EncCtx& ctx, const float2* P, uint64_t pair0,
+                                             uint8_t* codes, uint16_t* deq, float s,
+                                             const Divider& dv, StatsAcc* acc) {
+  const bool zero = (s == 0.0f);
+  constexpr bool kExactSmall = (R == kSR) || (G == kIF4);
+  float2 Q[8];
+  if (zero) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) Q[i] = make_float2(0.0f, 0.0f);
+  } else if (dv.fast) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) Q[i] = div2(dv, P[i]);
+    if constexpr (kExactSmall) {
+      // the correction step is exact for quotients >= 2^-20; smaller nonzero ones (rare) are
+      // recomputed with the IEEE division so stochastic rounding and IF4 errors stay exact
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (fabsf(Q[i].x) < 0x1p-19f && P[i].x != 0.0f) Q[i].x = __fdiv_rn(__fmul_rn(P[i].x, ctx.cinv), s);
+        if (fabsf(Q[i].y) < 0x1p-19f && P[i].y != 0.0f) Q[i].y = __fdiv_rn(__fmul_rn(P[i].y, ctx.cinv), s);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      Q[i] = make_float2(__fdiv_rn(__fmul_rn(P[i].x, ctx.cinv), s),
+                         __fdiv_rn(__fmul_rn(P[i].y, ctx.cinv), s));
+  }
+
+  // 32 random bits per element: pair j covers elements 2j (low half) and 2j+1 (high half)
+  uint32_t rnd[16];
+  if constexpr (R == kSR) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint64_t h = sr_pair_bits(ctx.seedx, pair0 + (uint64_t)j);
+      rnd[2 * j] = (uint32_t)h;
+      rnd[2 * j + 1] = (uint32_t)(h >> 32);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) rnd[j] = 0u;
+  }
+
+  const bool need_val = STATS || (deq != nullptr) || (G == kIF4);
+  float val[16];
+  uint32_t mag[16];
+  uint32_t w0 = 0u, w1 = 0u, flag = 0u;
+
+  if constexpr (G == kE1M2 || G == kINT4) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      w0 |= round_uniform<G, R>(Q[i].x, P[i].x, rnd[i], val[i], mag[i]) << (4 * i);
+      w1 |= round_uniform<G, R>(Q[i].y, P[i].y, rnd[i + 8], val[i + 8], mag[i + 8]) << (4 * i);
+    }
+  } else {  // E2M1 (and the FP4 candidate of IF4): hardware RNE conversion of signed values
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float e0, e1, f0, f1;   // elements 2j, 2j+1 (word 0) and 8+2j, 9+2j (word 1)
+      if constexpr (R == kSR) {
+        e0 = e2m1_sr_value(Q[2 * j].x, P[2 * j].x, rnd[2 * j]);
+        e1 = e2m1_sr_value(Q[2 * j + 1].x, P[2 * j + 1].x, rnd[2 * j + 1]);
+        f0 = e2m1_sr_value(Q[2 * j].y, P[2 * j].y, rnd[2 * j + 8]);
+        f1 = e2m1_sr_value(Q[2 * j + 1].y, P[2 * j + 1].y, rnd[2 * j + 9]);
+      } else {
+        e0 = with_sign_of(Q[2 * j].x, P[2 * j].x);
+        e1 = with_sign_of(Q[2 * j + 1].x, P[2 * j + 1].x);
+        f0 = with_sign_of(Q[2 * j].y, P[2 * j].y);
+        f1 = with_sign_of(Q[2 * j + 1].y, P[2 * j + 1].y);
+      }
+      w0 |= cvt_e2m1x2(e1, e0) << (8 * j);
+      w1 |= cvt_e2m1x2(f1, f0) << (8 * j);
+    }
+    if (need_val) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 d0 = e2m1x2_to_f32((w0 >> (8 * j)) & 0xFFu);
+        const float2 d1 = e2m1x2_to_f32((w1 >> (8 * j)) & 0xFFu);
+        val[2 * j] = d0.x;
+        val[2 * j + 1] = d0.y;
+        val[8 + 2 * j] = d1.x;
+        val[9 + 2 * j] = d1.y;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        mag[e] = (w0 >> (4 * e)) & 7u;
+        mag[e + 8] = (w1 >> (4 * e)) & 7u;
+      }
+    }
+    if constexpr (G == kIF4) {
+      const float r76 = __fdiv_rn(7.0f, 6.0f), r67 = __fdiv_rn(6.0f, 7.0f);
+      float vint[16];
+      uint32_t mint[16];
+      uint32_t i0 = 0u, i1 = 0u;
+      float2 Efp[8], Eint[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float d_fp[2], d_int[2];
+#pragma unroll
+        for (int l = 0; l < 2; ++l) {
+          const int e = i + 8 * l;
+          const float q = l ? Q[i].y : Q[i].x;
+          const float w = __fmul_rn(q, r76);
+          const uint32_t m = __float_as_uint(__fadd_rn(fminf(fabsf(w), 7.0f), 8388608.0f)) & 0xFu;
+          const bool n = sign_bit(w) && m;
+          const float k = small_int_f32(m);
+          vint[e] = __fmul_rn(n ? -k : k, r67);
+          mint[e] = m;
+          const uint32_t nib = (n ? (0u - m) : m) & 0xFu;
+          if (l) i1 |= nib << (4 * i); else i0 |= nib << (4 * i);
+          d_fp[l] = __fsub_rn(val[e], q);
+          d_int[l] = __fsub_rn(vint[e], q);
+        }
+        Efp[i] = make_float2(__fmul_rn(d_fp[0], d_fp[0]), __fmul_rn(d_fp[1], d_fp[1]));
+        Eint[i] = make_float2(__fmul_rn(d_int[0], d_int[0]), __fmul_rn(d_int[1], d_int[1]));
+      }
+      // balanced pairwise sums over elements 0..15 ((e0+e1)+(e2+e3))..., both halves at once
+#pragma unroll
+      for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 8; i += 2 * h) {
+          Efp[i] = add2(Efp[i], Efp[i + h]);
+          Eint[i] = add2(Eint[i], Eint[i + h]);
+        }
+      }
+      const float sse_fp = __fadd_rn(Efp[0].x, Efp[0].y);
+      const float sse_int = __fadd_rn(Eint[0].x, Eint[0].y);
+      if (!zero && sse_int < sse_fp) {
+        flag = 0x80u;
+        w0 = i0;
+        w1 = i1;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          val[e] = vint[e];
+          mag[e] = mint[e];
+        }
+      }
+    }
+  }
+  if (zero) {
+    w0 = 0u;
+    w1 = 0u;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      val[e] = 0.0f;
+      mag[e] = 0u;
+    }
+  }
+
+  __stcs(reinterpret_cast<uint2*>(codes), make_uint2(w0, w1));
+
+  if (deq != nullptr || STATS) {
+    float xh[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) xh[e] = __fmul_rn(val[e], s);
+    if (deq != nullptr) {
+      uint4 o0, o1;
+      o0.x = pack_bf16x2(xh[0], xh[1]);   o0.y = pack_bf16x2(xh[2], xh[3]);
+      o0.z = pack_bf16x2(xh[4], xh[5]);   o0.w = pack_bf16x2(xh[6], xh[7]);
+      o1.x = pack_bf16x2(xh[8], xh[9]);   o1.y = pack_bf16x2(xh[10], xh[11]);
+      o1.z = pack_bf16x2(xh[12], xh[13]); o1.w = pack_bf16x2(xh[14], xh[15]);
+      uint4* d = reinterpret_cast<uint4*>(deq);
+      __stcs(d, o0);
+      __stcs(d + 1, o1);
+    }
+    if constexpr (STATS) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float y = __fmul_rn(elem_x(P, e), ctx.cinv);
+        acc->element(y, xh[e], mag[e], val[e], zero ? 0.0f : elem_x(Q, e));
+      }
+      acc->blocks += 1.0;
+      if (G == kIF4 && flag == 0u) acc->if4_fp4 += 1.0;
+    }
+  }
+  return flag;
+}
+
+}  // namespace fp4q

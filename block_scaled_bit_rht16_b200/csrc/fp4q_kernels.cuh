@@ -1,0 +1,73 @@
+// fp4q_kernels.cuh -- kernel argument blocks and launch entry points shared by the host layer.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fp4q {
+
+// Raw statistics record (doubles), one per CTA in the workspace and once reduced.
+enum {
+  ST_SUM_Y2 = 0, ST_SUM_ERR2 = 1, ST_SUM_YXHAT = 2, ST_N = 3, ST_CELL_N = 4, ST_CELL_ERR = 12,
+  ST_IF4_FP4 = 20, ST_BLOCKS = 21, ST_LEN = 24
+};
+
+// Workspace layout: a 256-byte header, then (with statistics) kStatsCtas raw records.
+struct WsHeader {
+  uint32_t magic;       // kWsMagic once a statistics-producing call has been enqueued
+  uint32_t n_partials;  // raw records that follow
+  uint32_t amax_bits;   // rotated-tensor amax (bit pattern of a non-negative float)
+  int32_t status;       // device status word (0 ok)
+  double reduced[ST_LEN];  // fp4q_stats writes the fixed-order reduction here
+  uint8_t pad[256 - 16 - 8 * ST_LEN];
+};
+static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
+constexpr uint32_t kWsMagic = 0x51345046u;   // "FP4Q"
+constexpr int kStatsCtas = 512;               // fixed grid of statistics-producing launches
+constexpr int kThreads = 256;
+
+struct QuantArgs {
+  const uint16_t* x;
+  int64_t rows, cols, ld;
+  int64_t nunits;          // blocks of 16 (32 for UE8M0) in the tensor
+  int64_t units_per_row;
+  uint8_t* codes;
+  void* scales;
+  uint16_t* deq;           // optional
+  const float* ts_in;      // E4M3: alpha supplied by the caller
+  float* ts_out;           // E4M3: where the computed alpha goes
+  WsHeader* ws;            // header (amax, status) or null
+  double* partials;        // statistics records or null
+  uint32_t sw[8];          // sign flips per bf16 pair (all 0 without rotation)
+  float c, cinv;           // 4, 1/4 with rotation; 1, 1 without
+  uint64_t seedx;          // SR: seed ^ (stream << 63)
+  int contiguous;          // ld == cols
+};
+
+struct DualArgs {
+  const uint16_t* dy;
+  int64_t M, N, ld;
+  uint8_t* codes_row; float* scales_row;
+  uint8_t* codes_col; float* scales_col;
+  uint32_t sw_row[8], sw_col[8];
+  float c_row, cinv_row, c_col, cinv_col;
+  uint64_t seedx_row, seedx_col;
+  int round_row, round_col;   // per orientation
+  int grid_row, grid_col;
+};
+
+// Host-side launchers (fp4q_row.cu / fp4q_dual.cu). Return the CUDA error of the launch.
+cudaError_t launch_quantize(int grid, int scale, int round, bool stats, const QuantArgs& a,
+                            cudaStream_t st);
+cudaError_t launch_amax(const QuantArgs& a, cudaStream_t st);
+cudaError_t launch_rht16(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                         const uint32_t* sw, void* out, bool out_fp32, cudaStream_t st);
+cudaError_t launch_dequant(int grid, int scale, const uint8_t* codes, const void* scales,
+                           const float* ts, int64_t rows, int64_t cols, const uint32_t* sw,
+                           bool inverse, uint16_t* out, cudaStream_t st);
+cudaError_t launch_stats_reduce(WsHeader* ws, const double* partials, cudaStream_t st);
+cudaError_t launch_dual(const DualArgs& a, cudaStream_t st);
+cudaError_t launch_division_check(uint64_t seed, uint64_t n, unsigned long long* bad,
+                                  cudaStream_t st);
+
+}  // namespace fp4q

@@ -1,0 +1,564 @@
+// fp4q_row.cu -- row-orientation kernels of the fused RHT16 + block-scaled 4-bit quantizer.
+//
+// One thread owns one scale block (16 elements; 32 for UE8M0) end to end: two (four) 128-bit
+// coalesced loads, sign flips on the bf16 bits, the 16-point butterfly in registers (packed
+// f32x2), block absmax, the scale, exact quotients, rounding, nibble packing, one 8-byte
+// (16-byte) code store and the scale store. Consecutive threads own consecutive blocks, so a
+// warp reads 1 KiB and writes 256 B of codes contiguously. The grid is persistent (SM count x
+// resident CTAs) and each thread keeps two blocks in flight.
+//
+// Sources: "蚂蚁集团揭秘…" (techwalker.com), section 六 Q5 (16-point rotation fused with the
+// 16-element quantization block); "当你的 GPU 学不会算账" (zhichai.net/topic/178208020),
+// section "UFP4：换一把尺子" (recipe table: 1x16 blocks, FP32 scale, SR on dY);
+// "低精度量化技术：IF4…" (bxzpzcl.cn/news/2320061), section 3.2 (E4M3 block scale + FP32
+// tensor scale); "AMD全新研究揭示…" (cannews.ca/article/21387), MXFP4 section (32-element
+// blocks, shared E8M0 exponent).
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "fp4q_device.cuh"
+#include "fp4q_encode.cuh"
+#include "fp4q_kernels.cuh"
+
+namespace fp4q {
+namespace {
+
+__device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
+  return __ldcs(reinterpret_cast<const uint4*>(p));
+}
+
+__device__ __forceinline__ int64_t unit_offset(const QuantArgs& a, int64_t u, int unit) {
+  if (a.contiguous) return u * unit;
+  const int64_t r = u / a.units_per_row;
+  return r * a.ld + (u - r * a.units_per_row) * unit;
+}
+
+__device__ __forceinline__ void rotate_if(const QuantArgs& a, float2* P) {
+  if (a.c != 1.0f) fwht16(P);
+}
+
+// Fixed-order reduction of the per-thread statistics into this CTA's raw record.
+__device__ void stats_finish(const StatsAcc& acc, double* partials) {
+  __shared__ double red[5][kThreads];
+  red[0][threadIdx.x] = acc.y2;
+  red[1][threadIdx.x] = acc.err2;
+  red[2][threadIdx.x] = acc.yx;
+  red[3][threadIdx.x] = acc.blocks;
+  red[4][threadIdx.x] = acc.if4_fp4;
+  __syncthreads();
+  double* out = partials + (size_t)blockIdx.x * ST_LEN;
+  const int t = threadIdx.x;
+  if (t < 5) {
+    const int dst[5] = {ST_SUM_Y2, ST_SUM_ERR2, ST_SUM_YXHAT, ST_BLOCKS, ST_IF4_FP4};
+    double s = 0.0;
+    for (int i = 0; i < kThreads; ++i) s += red[t][i];
+    out[dst[t]] = s;
+  } else if (t >= 32 && t < 40) {
+    const int c = t - 32;
+    double s = 0.0, n = 0.0;
+    for (int i = 0; i < kThreads; ++i) {
+      s += acc.cell_err[c * kThreads + i];
+      n += (double)acc.cell_n[c * kThreads + i];
+    }
+    out[ST_CELL_ERR + c] = s;
+    out[ST_CELL_N + c] = n;
+  } else if (t == 64) {
+    double n = 0.0;
+    for (int i = 0; i < 8 * kThreads; ++i) n += (double)acc.cell_n[i];
+    out[ST_N] = n;
+    out[22] = 0.0;
+    out[23] = 0.0;
+  }
+}
+
+// MXFP4 block: 32 elements (two rotated 16-blocks P, Q) scaled by 2^-e (exact multiply by
+// `mult` = 2^-e * cinv), E2M1 with saturation.
+template <int R, bool STATS>
+__device__ __forceinline__ void encode_mx(const EncCtx& ctx, const float2* P, const float2* Q,
+                                          uint64_t pair0, uint8_t* codes, uint16_t* deq, float s,
+                                          float mult, bool zero, StatsAcc* acc) {
+  const float2 m2 = make_float2(mult, mult);
+  uint32_t w[4];
+  float val[32], vq[32];
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const float2* H = half ? Q : P;
+    float2 V[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) V[i] = __fmul2_rn(H[i], m2);   // exact scaling, sign kept
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      vq[16 * half + i] = V[i].x;
+      vq[16 * half + 8 + i] = V[i].y;
+    }
+    uint32_t rnd[16];
+    if constexpr (R == kSR) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint64_t h = sr_pair_bits(ctx.seedx, pair0 + 8u * half + (uint64_t)j);
+        rnd[2 * j] = (uint32_t)h;
+        rnd[2 * j + 1] = (uint32_t)(h >> 32);
+      }
+    }
+    uint32_t wa = 0u, wb = 0u;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float e0 = V[2 * j].x, e1 = V[2 * j + 1].x, f0 = V[2 * j].y, f1 = V[2 * j + 1].y;
+      if constexpr (R == kSR) {
+        e0 = e2m1_sr_value(e0, e0, rnd[2 * j]);
+        e1 = e2m1_sr_value(e1, e1, rnd[2 * j + 1]);
+        f0 = e2m1_sr_value(f0, f0, rnd[2 * j + 8]);
+        f1 = e2m1_sr_value(f1, f1, rnd[2 * j + 9]);
+      }
+      wa |= cvt_e2m1x2(e1, e0) << (8 * j);
+      wb |= cvt_e2m1x2(f1, f0) << (8 * j);
+    }
+    if (zero) {
+      wa = 0u;
+      wb = 0u;
+    }
+    w[2 * half] = wa;
+    w[2 * half + 1] = wb;
+  }
+  __stcs(reinterpret_cast<uint4*>(codes), make_uint4(w[0], w[1], w[2], w[3]));
+  if (deq != nullptr || STATS) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 d = e2m1x2_to_f32((w[k] >> (8 * j)) & 0xFFu);
+        val[8 * k + 2 * j] = d.x;
+        val[8 * k + 2 * j + 1] = d.y;
+      }
+    float xh[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) xh[e] = __fmul_rn(val[e], s);
+    if (deq != nullptr) {
+      uint4* d = reinterpret_cast<uint4*>(deq);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint4 o;
+        o.x = pack_bf16x2(xh[8 * k + 0], xh[8 * k + 1]);
+        o.y = pack_bf16x2(xh[8 * k + 2], xh[8 * k + 3]);
+        o.z = pack_bf16x2(xh[8 * k + 4], xh[8 * k + 5]);
+        o.w = pack_bf16x2(xh[8 * k + 6], xh[8 * k + 7]);
+        __stcs(d + k, o);
+      }
+    }
+    if constexpr (STATS) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float2* H = (e < 16) ? P : Q;
+        const float y = __fmul_rn(elem_x(H, e & 15), ctx.cinv);
+        const uint32_t mag = (w[e >> 3] >> (4 * (e & 7))) & 7u;
+        acc->element(y, xh[e], mag, val[e], zero ? 0.0f : vq[e]);
+      }
+      acc->blocks += 1.0;
+    }
+  }
+}
+
+template <int G, int S, int R, bool STATS>
+__global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantArgs a) {
+  constexpr float qmax = GridInfo<G>::qmax;
+  constexpr int kUnit = (S == kUE8M0) ? 32 : 16;
+  constexpr int kVec = kUnit / 8;   // 16-byte loads per unit
+
+  float alpha = 0.0f, denom = 0.0f;
+  if constexpr (S == kE4M3) {
+    if (a.ts_in != nullptr) {
+      alpha = *a.ts_in;
+    } else {
+      const float A = __uint_as_float(a.ws->amax_bits);
+      alpha = __fdiv_rn(A, __fmul_rn(qmax, 448.0f));
+      if (a.ts_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *a.ts_out = alpha;
+    }
+    denom = __fmul_rn(alpha, qmax);
+  }
+
+  StatsAcc acc;
+  if constexpr (STATS) {
+    __shared__ double s_cell_err[8 * kThreads];
+    __shared__ uint32_t s_cell_n[8 * kThreads];
+    acc.y2 = acc.err2 = acc.yx = acc.blocks = acc.if4_fp4 = 0.0;
+    acc.cell_err = s_cell_err;
+    acc.cell_n = s_cell_n;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      s_cell_err[c * kThreads + threadIdx.x] = 0.0;
+      s_cell_n[c * kThreads + threadIdx.x] = 0u;
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      a.ws->magic = kWsMagic;
+      a.ws->n_partials = gridDim.x;
+    }
+  }
+  const EncCtx ctx{a.cinv, a.seedx};
+
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < a.nunits; u += 2 * stride) {
+    uint4 buf[2][kVec];
+    const int64_t uu[2] = {u, u + stride};
+    const bool has2 = uu[1] < a.nunits;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      if (k == 1 && !has2) break;
+      const uint16_t* src = a.x + unit_offset(a, uu[k], kUnit);
+#pragma unroll
+      for (int v = 0; v < kVec; ++v) buf[k][v] = ld_stream(src + 8 * v);
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      if (k == 1 && !has2) break;
+      const int64_t un = uu[k];
+      uint16_t* deq = a.deq ? a.deq + un * kUnit : nullptr;
+      if constexpr (S != kUE8M0) {
+        float2 P[8];
+        unpack16(buf[k][0], buf[k][1], a.sw, P);
+        rotate_if(a, P);
+        const float amax_y = __fmul_rn(absmax16(P), a.cinv);
+        float s;
+        uint32_t sbyte = 0u;
+        if constexpr (S == kFP32) {
+          s = __fdiv_rn(amax_y, qmax);
+        } else {
+          const float delta = denom > 0.0f ? __fdiv_rn(amax_y, denom) : 0.0f;
+          sbyte = cvt_e4m3(delta);
+          s = __fmul_rn(e4m3_to_f32(sbyte), alpha);
+        }
+        const Divider dv = make_divider(s, a.c);
+        const uint32_t flag = encode16<G, R, STATS>(ctx, P, (uint64_t)un * 8u, a.codes + un * 8,
+                                                    deq, s, dv, STATS ? &acc : nullptr);
+        if constexpr (S == kFP32) {
+          __stcs(reinterpret_cast<float*>(a.scales) + un, s);
+        } else {
+          reinterpret_cast<uint8_t*>(a.scales)[un] = (uint8_t)(sbyte | flag);
+        }
+      } else {
+        float2 P[8], Q[8];
+        unpack16(buf[k][0], buf[k][1], a.sw, P);
+        unpack16(buf[k][2], buf[k][3], a.sw, Q);
+        rotate_if(a, P);
+        rotate_if(a, Q);
+        const float amax_y = __fmul_rn(fmaxf(absmax16(P), absmax16(Q)), a.cinv);
+        int e = -127;
+        if (amax_y != 0.0f) {
+          const int E = (int)(__float_as_uint(amax_y) >> 23);   // biased exponent
+          e = (E == 0) ? -127 : max(-127, min(127, E - 127 - 2));
+        }
+        const float s = (e >= -126) ? __uint_as_float((uint32_t)(127 + e) << 23) : 0x1p-127f;
+        const float mult = __fmul_rn(__uint_as_float((uint32_t)(127 - e) << 23), a.cinv);
+        encode_mx<R, STATS>(ctx, P, Q, (uint64_t)un * 16u, a.codes + un * 16, deq, s, mult,
+                            amax_y == 0.0f, STATS ? &acc : nullptr);
+        reinterpret_cast<uint8_t*>(a.scales)[un] = (uint8_t)(e + 127);
+      }
+    }
+  }
+  if constexpr (STATS) stats_finish(acc, a.partials);
+}
+
+// Amax of the rotated tensor: per-warp maximum of the bit patterns (non-negative floats order
+// like unsigned integers), one atomicMax per warp into the workspace header.
+__global__ void __launch_bounds__(kThreads) amax_kernel(const QuantArgs a) {
+  uint32_t m = 0u;
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < a.nunits; u += stride) {
+    const uint16_t* src = a.x + unit_offset(a, u, 16);
+    float2 P[8];
+    unpack16(ld_stream(src), ld_stream(src + 8), a.sw, P);
+    rotate_if(a, P);
+    m = max(m, __float_as_uint(__fmul_rn(absmax16(P), a.cinv)));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0 && m != 0u) atomicMax(&a.ws->amax_bits, m);
+}
+
+// The rotation alone: y = 1/4 H16 D x, stored bf16 (RNE) or FP32.
+__global__ void __launch_bounds__(kThreads) rht16_kernel(const QuantArgs a, int out_fp32, void* out) {
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < a.nunits; u += stride) {
+    const uint16_t* src = a.x + unit_offset(a, u, 16);
+    float2 P[8];
+    unpack16(ld_stream(src), ld_stream(src + 8), a.sw, P);
+    fwht16(P);
+    float y[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) y[e] = __fmul_rn(elem_x(P, e), 0.25f);
+    if (out_fp32) {
+      float4* d = reinterpret_cast<float4*>(out) + u * 4;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) __stcs(d + k, make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]));
+    } else {
+      uint4 o0, o1;
+      o0.x = pack_bf16x2(y[0], y[1]);   o0.y = pack_bf16x2(y[2], y[3]);
+      o0.z = pack_bf16x2(y[4], y[5]);   o0.w = pack_bf16x2(y[6], y[7]);
+      o1.x = pack_bf16x2(y[8], y[9]);   o1.y = pack_bf16x2(y[10], y[11]);
+      o1.z = pack_bf16x2(y[12], y[13]); o1.w = pack_bf16x2(y[14], y[15]);
+      uint4* d = reinterpret_cast<uint4*>(out) + u * 2;
+      __stcs(d, o0);
+      __stcs(d + 1, o1);
+    }
+  }
+}
+
+// Codes back to bf16 (optionally through the inverse rotation x = D 1/4 H16 xhat).
+struct DeqArgs {
+  const uint8_t* codes;
+  const void* scales;
+  const float* ts;
+  uint16_t* out;
+  int64_t nunits;    // 16-element blocks
+  uint32_t sw[8];
+  int inverse;
+};
+
+template <int G, int S>
+__global__ void __launch_bounds__(kThreads) dequant_kernel(const DeqArgs a) {
+  const float alpha = (S == kE4M3) ? *a.ts : 0.0f;
+  const float r67 = __fdiv_rn(6.0f, 7.0f);
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < a.nunits; u += stride) {
+    const uint2 cw = __ldcs(reinterpret_cast<const uint2*>(a.codes) + u);
+    float s;
+    bool int_block = false;
+    if constexpr (S == kFP32) {
+      s = reinterpret_cast<const float*>(a.scales)[u];
+    } else if constexpr (S == kE4M3) {
+      const uint32_t b = reinterpret_cast<const uint8_t*>(a.scales)[u];
+      int_block = (G == kIF4) && (b & 0x80u);
+      s = __fmul_rn(e4m3_to_f32(b & 0x7Fu), alpha);
+    } else {
+      const int e = (int)reinterpret_cast<const uint8_t*>(a.scales)[u >> 1] - 127;
+      s = (e >= -126) ? __uint_as_float((uint32_t)(127 + e) << 23) : 0x1p-127f;
+    }
+    float v[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint32_t nib = ((e < 8 ? cw.x : cw.y) >> (4 * (e & 7))) & 0xFu;
+      float q;
+      if (G == kINT4 || int_block) {
+        const uint32_t m = (nib & 8u) ? 16u - nib : nib;
+        const float k = small_int_f32(m);
+        q = (nib & 8u) ? -k : k;
+        if (int_block) q = __fmul_rn(q, r67);
+      } else if (G == kE1M2) {
+        const float g = __fmul_rn(small_int_f32(nib & 7u), 0.5f);
+        q = __uint_as_float(__float_as_uint(g) | ((nib & 8u) << 28));
+      } else {
+        const float2 d = e2m1x2_to_f32(nib);
+        q = d.x;
+      }
+      v[e] = __fmul_rn(q, s);
+    }
+    if (a.inverse) {
+      float2 P[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) P[i] = make_float2(v[i], v[i + 8]);
+      fwht16(P);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float t = __fmul_rn(elem_x(P, e), 0.25f);
+        // element e's sign flip: word e >> 1 of sw, bit 15 (even e) or bit 31 (odd e)
+        const uint32_t flip = (a.sw[e >> 1] >> ((e & 1) ? 31 : 15)) & 1u;
+        v[e] = __uint_as_float(__float_as_uint(t) ^ (flip << 31));
+      }
+    }
+    uint4 o0, o1;
+    o0.x = pack_bf16x2(v[0], v[1]);   o0.y = pack_bf16x2(v[2], v[3]);
+    o0.z = pack_bf16x2(v[4], v[5]);   o0.w = pack_bf16x2(v[6], v[7]);
+    o1.x = pack_bf16x2(v[8], v[9]);   o1.y = pack_bf16x2(v[10], v[11]);
+    o1.z = pack_bf16x2(v[12], v[13]); o1.w = pack_bf16x2(v[14], v[15]);
+    uint4* d = reinterpret_cast<uint4*>(a.out) + u * 2;
+    __stcs(d, o0);
+    __stcs(d + 1, o1);
+  }
+}
+
+// Fixed-order FP64 reduction of the per-CTA records into the header (one thread per field).
+__global__ void stats_reduce_kernel(WsHeader* ws, const double* partials) {
+  const int f = threadIdx.x;
+  if (f >= ST_LEN) return;
+  double s = 0.0;
+  const uint32_t n = (ws->magic == kWsMagic) ? min(ws->n_partials, (uint32_t)kStatsCtas) : 0u;
+  for (uint32_t i = 0; i < n; ++i) s += partials[(size_t)i * ST_LEN + f];
+  ws->reduced[f] = s;
+}
+
+// Self-check of the exact-quotient step: pseudo-random pairs (s, y) with s in [2^-60, 2^90)
+// and y / s in [2^-20, 8), with and without the folded 1/4, compared with IEEE division.
+__global__ void __launch_bounds__(kThreads) division_check_kernel(uint64_t seed, uint64_t n,
+                                                                  unsigned long long* bad) {
+  unsigned long long local = 0;
+  const uint64_t stride = (uint64_t)gridDim.x * kThreads;
+  for (uint64_t i = (uint64_t)blockIdx.x * kThreads + threadIdx.x; i < n; i += stride) {
+    const uint64_t h = splitmix64(seed ^ (i * 0x9E3779B97F4A7C15ull));
+    const uint64_t g = splitmix64(h);
+    const int es = (int)(h % 151u) - 60;                        // 2^-60 .. 2^90
+    const float s = __uint_as_float(((uint32_t)(127 + es) << 23) | (uint32_t)(h >> 41));
+    const int et = (int)((h >> 8) % 24u) - 21;                  // 2^-21 .. 2^2 (times [1,2))
+    const float t = __uint_as_float(((uint32_t)(127 + et) << 23) | (uint32_t)(g & 0x7FFFFFu));
+    float y = __fmul_rn(s, t);
+    if (g >> 63) y = -y;
+    for (int rot = 0; rot < 2; ++rot) {
+      const float c = rot ? 4.0f : 1.0f;
+      const Divider dv = make_divider(s, c);
+      if (!dv.fast) continue;
+      const float vraw = __fmul_rn(y, c);
+      const float2 q = div2(dv, make_float2(vraw, -vraw));
+      const float want = __fdiv_rn(y, s);
+      if (fabsf(want) < 0x1p-20f) continue;
+      if (__float_as_uint(fabsf(q.x)) != __float_as_uint(fabsf(want)) ||
+          __float_as_uint(fabsf(q.y)) != __float_as_uint(fabsf(want)))
+        ++local;
+    }
+  }
+  if (local) atomicAdd(bad, local);
+}
+
+// ------------------------------------------------------------------ launch helpers
+
+// Resident CTAs of `kernel` on the current device (SM count x occupancy), queried once per
+// (kernel, device) and cached, so that launches inside a stream capture do no queries.
+template <class K>
+int resident_ctas(K kernel) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  int sms = 148, per_sm = 1;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0);
+  const int n = sms * std::max(per_sm, 1);
+  cache.emplace(key, n);
+  return n;
+}
+
+template <class K>
+int persistent_grid(K kernel, int64_t work_threads) {
+  const int64_t need = (work_threads + kThreads - 1) / kThreads;
+  return (int)std::max<int64_t>(1, std::min<int64_t>(need, resident_ctas(kernel)));
+}
+
+template <int G, int S, int R, bool STATS>
+cudaError_t launch_q(const QuantArgs& a, cudaStream_t st) {
+  auto k = quantize_kernel<G, S, R, STATS>;
+  int grid;
+  if (STATS) {
+    grid = kStatsCtas;
+  } else {
+    // two units per thread per iteration
+    grid = persistent_grid(k, (a.nunits + 1) / 2);
+  }
+  k<<<grid, kThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int G, int S, int R>
+cudaError_t launch_q_stats(bool stats, const QuantArgs& a, cudaStream_t st) {
+  return stats ? launch_q<G, S, R, true>(a, st) : launch_q<G, S, R, false>(a, st);
+}
+
+template <int G, int S>
+cudaError_t launch_q_round(int round, bool stats, const QuantArgs& a, cudaStream_t st) {
+  return round == kSR ? launch_q_stats<G, S, kSR>(stats, a, st)
+                      : launch_q_stats<G, S, kRTNE>(stats, a, st);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(int grid, int scale, int round, bool stats, const QuantArgs& a,
+                            cudaStream_t st) {
+  if (scale == kFP32) {
+    if (grid == kE2M1) return launch_q_round<kE2M1, kFP32>(round, stats, a, st);
+    if (grid == kE1M2) return launch_q_round<kE1M2, kFP32>(round, stats, a, st);
+    if (grid == kINT4) return launch_q_round<kINT4, kFP32>(round, stats, a, st);
+  } else if (scale == kE4M3) {
+    if (grid == kE2M1) return launch_q_round<kE2M1, kE4M3>(round, stats, a, st);
+    if (grid == kE1M2) return launch_q_round<kE1M2, kE4M3>(round, stats, a, st);
+    if (grid == kINT4) return launch_q_round<kINT4, kE4M3>(round, stats, a, st);
+    if (grid == kIF4) return launch_q_stats<kIF4, kE4M3, kRTNE>(stats, a, st);
+  } else if (scale == kUE8M0) {
+    if (grid == kE2M1) return launch_q_round<kE2M1, kUE8M0>(round, stats, a, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_amax(const QuantArgs& a, cudaStream_t st) {
+  amax_kernel<<<persistent_grid(amax_kernel, a.nunits), kThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rht16(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                         const uint32_t* sw, void* out, bool out_fp32, cudaStream_t st) {
+  QuantArgs a{};
+  a.x = x;
+  a.rows = rows;
+  a.cols = cols;
+  a.ld = ld;
+  a.units_per_row = cols / 16;
+  a.nunits = rows * a.units_per_row;
+  a.contiguous = (ld == cols);
+  for (int k = 0; k < 8; ++k) a.sw[k] = sw[k];
+  a.c = 4.0f;
+  a.cinv = 0.25f;
+  if (a.nunits == 0) return cudaSuccess;
+  rht16_kernel<<<persistent_grid(rht16_kernel, a.nunits), kThreads, 0, st>>>(a, out_fp32 ? 1 : 0, out);
+  return cudaGetLastError();
+}
+
+template <int G, int S>
+cudaError_t launch_dq(const DeqArgs& a, cudaStream_t st) {
+  auto k = dequant_kernel<G, S>;
+  k<<<persistent_grid(k, a.nunits), kThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequant(int grid, int scale, const uint8_t* codes, const void* scales,
+                           const float* ts, int64_t rows, int64_t cols, const uint32_t* sw,
+                           bool inverse, uint16_t* out, cudaStream_t st) {
+  DeqArgs a{};
+  a.codes = codes;
+  a.scales = scales;
+  a.ts = ts;
+  a.out = out;
+  a.nunits = rows * (cols / 16);
+  for (int k = 0; k < 8; ++k) a.sw[k] = sw[k];
+  a.inverse = inverse ? 1 : 0;
+  if (a.nunits == 0) return cudaSuccess;
+  if (scale == kFP32) {
+    if (grid == kE2M1) return launch_dq<kE2M1, kFP32>(a, st);
+    if (grid == kE1M2) return launch_dq<kE1M2, kFP32>(a, st);
+    if (grid == kINT4) return launch_dq<kINT4, kFP32>(a, st);
+  } else if (scale == kE4M3) {
+    if (grid == kE2M1) return launch_dq<kE2M1, kE4M3>(a, st);
+    if (grid == kE1M2) return launch_dq<kE1M2, kE4M3>(a, st);
+    if (grid == kINT4) return launch_dq<kINT4, kE4M3>(a, st);
+    if (grid == kIF4) return launch_dq<kIF4, kE4M3>(a, st);
+  } else if (scale == kUE8M0) {
+    if (grid == kE2M1) return launch_dq<kE2M1, kUE8M0>(a, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_division_check(uint64_t seed, uint64_t n, unsigned long long* bad,
+                                  cudaStream_t st) {
+  division_check_kernel<<<persistent_grid(division_check_kernel, (int64_t)std::min<uint64_t>(n, 1ull << 40)),
+                          kThreads, 0, st>>>(seed, n, bad);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stats_reduce(WsHeader* ws, const double* partials, cudaStream_t st) {
+  stats_reduce_kernel<<<1, 32, 0, st>>>(ws, partials);
+  return cudaGetLastError();
+}
+
+}  // namespace fp4q

@@ -1,0 +1,159 @@
+"""Host-side checks of the C-ABI library (no GPU): it loads, exports every symbol the header
+declares, its structs match the ctypes mirror byte for byte, and invalid arguments are rejected
+with the documented status before anything is launched."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle as O
+import block_scaled_bit_rht16_b200 as fq
+from block_scaled_bit_rht16_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp4q.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp4q_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    names = _declared()
+    assert names == sorted(_lib.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True).stdout
+    for n in names:
+        assert re.search(r"\bT %s$" % n, out, flags=re.M), n
+
+
+def test_struct_layout_matches_header(tmp_path):
+    prog = tmp_path / "layout.c"
+    prog.write_text('''#include <stdio.h>
+#include <stddef.h>
+#include "fp4q.h"
+int main(void) {
+  printf("%zu %zu %zu %zu %zu\\n", sizeof(fp4q_config), offsetof(fp4q_config, sr_seed),
+         offsetof(fp4q_config, outputs), sizeof(fp4q_stats_t), offsetof(fp4q_stats_t, status));
+  return 0;
+}''')
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(prog), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True).stdout.split()]
+    want = [ctypes.sizeof(_lib.fp4q_config), _lib.fp4q_config.sr_seed.offset,
+            _lib.fp4q_config.outputs.offset, ctypes.sizeof(_lib.fp4q_stats_t),
+            _lib.fp4q_stats_t.status.offset]
+    assert got == want
+
+
+def test_status_strings():
+    lib = _lib.load()
+    for s in range(8):
+        assert lib.fp4q_status_string(s)
+    assert lib.fp4q_status_string(0) == b"ok"
+    assert lib.fp4q_status_string(99) == b"unknown status"
+
+
+def test_sign_mask_from_seed_matches_oracle():
+    for seed in (0, 1, 0x5EED0001, 0x5EED0005, 2**63 + 17):
+        assert fq.sign_mask_from_seed(seed) == O.sign_mask_from_seed(seed)
+
+
+def test_workspace_sizes():
+    assert fq.workspace_size(fq.Config(), 128, 256) == 0
+    base = fq.workspace_size(fq.Config(scale=fq.FP4Q_SCALE_E4M3_1x16_TENSOR, grid=fq.FP4Q_GRID_E2M1), 128, 256)
+    assert base == 256
+    st = fq.workspace_size(fq.Config(stats=True), 128, 256)
+    assert st > 256 and st % 8 == 0
+    assert fq.workspace_size(fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=fq.FP4Q_SCALE_UE8M0_1x32), 1, 32) == 0
+
+
+FAKE = 1 << 20   # a 256-byte-aligned non-null address; never dereferenced: validation fails first
+
+
+def _q(cfg=None, x=FAKE, rows=4, cols=32, ld=32, codes=FAKE, scales=FAKE, ts=None, given=0,
+       deq=None, ws=None, ws_bytes=0):
+    lib = _lib.load()
+    c = (cfg or fq.Config()).c()
+    return lib.fp4q_rht_quantize(ctypes.byref(c), x, rows, cols, ld, codes, scales, ts, given, deq,
+                                 ws, ws_bytes, None)
+
+
+def test_rejects_bad_arguments_before_launch():
+    assert _q(x=None) == _lib.FP4Q_ERR_INVALID_ARG
+    assert _q(codes=None) == _lib.FP4Q_ERR_INVALID_ARG
+    assert _q(cols=24, ld=24) == _lib.FP4Q_ERR_SHAPE
+    assert _q(rows=-1) == _lib.FP4Q_ERR_SHAPE
+    assert _q(ld=16) == _lib.FP4Q_ERR_SHAPE
+    assert _q(ld=36) == _lib.FP4Q_ERR_ALIGN
+    assert _q(x=FAKE + 8) == _lib.FP4Q_ERR_ALIGN
+    assert _q(codes=FAKE + 4) == _lib.FP4Q_ERR_ALIGN
+    assert _q(fq.Config(dequant=True)) == _lib.FP4Q_ERR_INVALID_ARG          # dequant requested, NULL
+    assert _q(fq.Config(stats=True)) == _lib.FP4Q_ERR_WORKSPACE              # stats need a workspace
+    assert _q(fq.Config(stats=True), ws=FAKE, ws_bytes=100) == _lib.FP4Q_ERR_WORKSPACE
+    assert _q(fq.Config(stats=True), ws=FAKE + 64, ws_bytes=1 << 20) == _lib.FP4Q_ERR_ALIGN
+    e4 = fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=fq.FP4Q_SCALE_E4M3_1x16_TENSOR)
+    assert _q(e4) == _lib.FP4Q_ERR_INVALID_ARG                               # tensor scale missing
+    assert _q(e4, ts=FAKE) == _lib.FP4Q_ERR_WORKSPACE                        # amax pass needs one
+    assert _q(fq.Config(grid=7)) == _lib.FP4Q_ERR_INVALID_ARG
+    assert _q(fq.Config(scale=9)) == _lib.FP4Q_ERR_INVALID_ARG
+    assert _q(fq.Config(round=2)) == _lib.FP4Q_ERR_INVALID_ARG
+    assert _q(fq.Config(rht=2)) == _lib.FP4Q_ERR_INVALID_ARG
+    assert _q(fq.Config(sign_mask=1 << 16)) == _lib.FP4Q_ERR_INVALID_ARG
+    assert _q(fq.Config(grid=fq.FP4Q_GRID_IF4)) == _lib.FP4Q_ERR_UNSUPPORTED  # IF4 needs E4M3
+    assert _q(fq.Config(grid=fq.FP4Q_GRID_E1M2, scale=fq.FP4Q_SCALE_UE8M0_1x32)) == _lib.FP4Q_ERR_UNSUPPORTED
+    mx = fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=fq.FP4Q_SCALE_UE8M0_1x32)
+    assert _q(mx, cols=48, ld=48) == _lib.FP4Q_ERR_SHAPE
+    assert _q(mx, codes=FAKE + 8) == _lib.FP4Q_ERR_ALIGN
+    c = fq.Config().c()
+    c.reserved = 1
+    assert _lib.load().fp4q_rht_quantize(ctypes.byref(c), FAKE, 4, 32, 32, FAKE, FAKE, None, 0, None,
+                                         None, 0, None) == _lib.FP4Q_ERR_INVALID_ARG
+    assert _lib.load().fp4q_rht_quantize(None, FAKE, 4, 32, 32, FAKE, FAKE, None, 0, None, None, 0,
+                                         None) == _lib.FP4Q_ERR_INVALID_ARG
+
+
+def test_dual_dequant_rht_stats_validation():
+    lib = _lib.load()
+    r, c = fq.Config(round=fq.FP4Q_ROUND_SR).c(), fq.Config(round=fq.FP4Q_ROUND_SR, sr_stream=1).c()
+    dual = lambda rc=r, cc=c, M=32, N=32, ld=32, dy=FAKE, cr=FAKE: lib.fp4q_quantize_dual(
+        ctypes.byref(rc), ctypes.byref(cc), dy, M, N, ld, cr, FAKE, FAKE, FAKE, None, 0, None)
+    assert dual(M=24) == _lib.FP4Q_ERR_SHAPE
+    assert dual(N=40, ld=40) == _lib.FP4Q_ERR_SHAPE
+    assert dual(dy=None) == _lib.FP4Q_ERR_INVALID_ARG
+    assert dual(cr=FAKE + 4) == _lib.FP4Q_ERR_ALIGN
+    e2 = fq.Config(grid=fq.FP4Q_GRID_E2M1).c()
+    assert dual(cc=e2) == _lib.FP4Q_ERR_UNSUPPORTED
+    nv = fq.Config(scale=fq.FP4Q_SCALE_E4M3_1x16_TENSOR).c()
+    assert dual(rc=nv) == _lib.FP4Q_ERR_UNSUPPORTED
+    assert dual(rc=fq.Config(dequant=True).c()) == _lib.FP4Q_ERR_UNSUPPORTED
+    d = fq.Config().c()
+    assert lib.fp4q_dequantize(ctypes.byref(d), None, FAKE, None, 4, 32, 0, FAKE, None) == _lib.FP4Q_ERR_INVALID_ARG
+    assert lib.fp4q_dequantize(ctypes.byref(d), FAKE, FAKE, None, 4, 24, 0, FAKE, None) == _lib.FP4Q_ERR_SHAPE
+    assert lib.fp4q_dequantize(ctypes.byref(d), FAKE, FAKE, None, 4, 32, 2, FAKE, None) == _lib.FP4Q_ERR_INVALID_ARG
+    assert lib.fp4q_dequantize(ctypes.byref(nv), FAKE, FAKE, None, 4, 32, 0, FAKE, None) == _lib.FP4Q_ERR_INVALID_ARG
+    assert lib.fp4q_rht16(FAKE, 4, 24, 24, 0, FAKE, 0, None) == _lib.FP4Q_ERR_SHAPE
+    assert lib.fp4q_rht16(FAKE, 4, 32, 32, 1 << 17, FAKE, 0, None) == _lib.FP4Q_ERR_INVALID_ARG
+    assert lib.fp4q_rht16(FAKE + 2, 4, 32, 32, 0, FAKE, 0, None) == _lib.FP4Q_ERR_ALIGN
+    st = _lib.fp4q_stats_t()
+    assert lib.fp4q_stats(None, 0, ctypes.byref(st), None) == _lib.FP4Q_ERR_INVALID_ARG
+    assert lib.fp4q_stats(FAKE, 256, ctypes.byref(st), None) == _lib.FP4Q_ERR_WORKSPACE
+
+
+def test_recipe_presets():
+    # UFP4 recipe table: rotation on every path, SR on dY only; E2M1 baseline: rotation on bwd_dw
+    for path in ("fwd_y", "bwd_dx", "bwd_dw"):
+        u = fq.recipe("ufp4", path, "x", sign_mask=0x1234)
+        assert u.grid == fq.FP4Q_GRID_E1M2 and u.rht == 1 and u.round == fq.FP4Q_ROUND_RTNE
+        e = fq.recipe("e2m1", path, "x", sign_mask=0x1234)
+        assert e.grid == fq.FP4Q_GRID_E2M1 and e.rht == (1 if path == "bwd_dw" else 0)
+    dy = fq.recipe("ufp4", "bwd_dw", "dy", sr_seed=5)
+    assert dy.round == fq.FP4Q_ROUND_SR and dy.sr_stream == 1
+    assert fq.recipe("ufp4", "bwd_dx", "dy").sr_stream == 0

@@ -1,0 +1,279 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle, element by element.
+
+Codes, scale bytes/floats, tensor scales and bf16 dequant outputs must be bit-identical;
+statistics must agree to 1e-5 relative (the oracle sums in FP64 in another order).
+Shapes span several persistent-grid iterations and ragged tails; edge blocks cover zeros,
+negative zeros, ties, single nonzeros, bf16 subnormals, huge values and extreme dynamic range.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import block_scaled_bit_rht16_b200 as fq
+from block_scaled_bit_rht16_b200 import synth, _lib
+from helpers import bf16_bits, host, ocfg, to_dev
+
+pytestmark = pytest.mark.gpu
+
+MASK = 0xB5E1
+E2M1, E1M2, INT4, IF4 = fq.FP4Q_GRID_E2M1, fq.FP4Q_GRID_E1M2, fq.FP4Q_GRID_INT4, fq.FP4Q_GRID_IF4
+FP32, E4M3, UE8M0 = fq.FP4Q_SCALE_FP32_1x16, fq.FP4Q_SCALE_E4M3_1x16_TENSOR, fq.FP4Q_SCALE_UE8M0_1x32
+RTNE, SR = fq.FP4Q_ROUND_RTNE, fq.FP4Q_ROUND_SR
+
+COMBOS = [(E2M1, FP32, RTNE), (E1M2, FP32, RTNE), (INT4, FP32, RTNE),
+          (E2M1, FP32, SR), (E1M2, FP32, SR), (INT4, FP32, SR),
+          (E2M1, E4M3, RTNE), (INT4, E4M3, RTNE), (E1M2, E4M3, RTNE), (E2M1, E4M3, SR),
+          (IF4, E4M3, RTNE), (E2M1, UE8M0, RTNE), (E2M1, UE8M0, SR)]
+STAT_KEYS = ["sum_y2", "sum_err2", "sum_y_xhat"]
+
+
+def _cid(c):
+    return "%s-%s-%s" % ({0: "e2m1", 1: "e1m2", 2: "int4", 3: "if4"}[c[0]],
+                         {0: "fp32", 1: "e4m3", 2: "ue8m0"}[c[1]], {0: "rtne", 1: "sr"}[c[2]])
+
+
+def gpu_quantize(cfg, x_bits, ld=None, tensor_scale=None):
+    x = to_dev(x_bits, ld)
+    ts = None
+    if tensor_scale is not None:
+        ts = torch.tensor([tensor_scale], dtype=torch.float32, device="cuda")
+    out = fq.rht_quantize(cfg, x, tensor_scale=ts, tensor_scale_given=tensor_scale is not None)
+    torch.cuda.synchronize()
+    return out
+
+
+def compare_quant(cfg, x_bits, out, row0=0, tensor_scale=None, check_stats=True):
+    ref = O.quantize(ocfg(cfg), x_bits, row0=row0, tensor_scale=tensor_scale,
+                     dequant=cfg.dequant, stats=cfg.stats and check_stats)
+    np.testing.assert_array_equal(host(out.codes), ref["codes"])
+    np.testing.assert_array_equal(host(out.scales), ref["scales"])
+    if cfg.scale == E4M3:
+        assert host(out.tensor_scale)[0] == np.float32(ref["tensor_scale"])
+    if cfg.dequant:
+        np.testing.assert_array_equal(bf16_bits(out.dequant), ref["dequant"])
+    if cfg.stats and check_stats:
+        compare_stats(fq.stats(out.workspace), O.finalize_stats(ref["stats_raw"]), ref["stats_raw"])
+    return ref
+
+
+def compare_stats(g, o, raw):
+    for k, i in zip(STAT_KEYS, (O.ST_SUM_Y2, O.ST_SUM_ERR2, O.ST_SUM_YXHAT)):
+        assert g[k] == pytest.approx(raw[i], rel=1e-5, abs=1e-30), k
+    assert g["n"] == raw[O.ST_N]
+    assert g["blocks"] == raw[O.ST_BLOCKS]
+    assert g["if4_fp4_blocks"] == raw[O.ST_IF4_FP4]
+    np.testing.assert_array_equal(g["cell_count"], raw[O.ST_CELL_N:O.ST_CELL_N + 8])
+    np.testing.assert_allclose(g["cell_err"], raw[O.ST_CELL_ERR:O.ST_CELL_ERR + 8], rtol=1e-5, atol=1e-9)
+    if math.isfinite(o["sqnr_db"]):
+        assert g["sqnr_db"] == pytest.approx(o["sqnr_db"], rel=1e-5)
+    else:
+        assert g["sqnr_db"] == o["sqnr_db"]
+    assert g["alpha"] == pytest.approx(o["alpha"], rel=1e-5)
+    cm, om = np.array(g["cell_mean_err"]), o["cell_mean_err"]
+    np.testing.assert_array_equal(np.isnan(cm), np.isnan(om))
+    ok = ~np.isnan(om)
+    np.testing.assert_allclose(cm[ok], om[ok], rtol=1e-5, atol=1e-9)
+    assert g["status"] == 0
+
+
+# ------------------------------------------------------------------ all configurations
+
+@pytest.mark.parametrize("combo", COMBOS, ids=_cid)
+@pytest.mark.parametrize("rht", [0, 1])
+def test_small_ragged_all_outputs(combo, rht):
+    grid, scale, rnd = combo
+    cfg = fq.Config(grid=grid, scale=scale, round=rnd, rht=rht, sign_mask=MASK, sr_seed=0x1234ABCD,
+                    dequant=True, stats=True)
+    for rows, cols, kind in [(1, 32, "normal"), (37, 96, "t4"), (130, 1056, "laplace")]:
+        x = synth.small(rows * 7 + cols, rows, cols, kind)
+        compare_quant(cfg, x, gpu_quantize(cfg, x))
+
+
+@pytest.mark.parametrize("combo", COMBOS, ids=_cid)
+def test_many_grid_iterations(combo):
+    # 4M elements: each thread of the persistent grid runs several iterations (and a ragged
+    # last one); statistics off to keep the oracle quick
+    grid, scale, rnd = combo
+    cfg = fq.Config(grid=grid, scale=scale, round=rnd, rht=1, sign_mask=0x0F0F, sr_seed=77)
+    x = synth.small(5, 1031, 4096, "t4")
+    compare_quant(cfg, x, gpu_quantize(cfg, x))
+
+
+@pytest.mark.parametrize("combo", [(E1M2, FP32, RTNE), (E2M1, E4M3, RTNE), (IF4, E4M3, RTNE),
+                                   (E2M1, UE8M0, SR), (INT4, FP32, SR)], ids=_cid)
+def test_strided_input_and_given_tensor_scale(combo):
+    grid, scale, rnd = combo
+    cfg = fq.Config(grid=grid, scale=scale, round=rnd, sign_mask=0x8001, sr_seed=5, dequant=True)
+    x = synth.small(9, 67, 320, "normal", 3.0)
+    ts = np.float32(0.0123) if scale == E4M3 else None
+    out = gpu_quantize(cfg, x, ld=320 + 24, tensor_scale=ts)
+    compare_quant(cfg, x, out, tensor_scale=ts)
+
+
+def test_empty_inputs():
+    for cfg in [fq.Config(), fq.Config(grid=E2M1, scale=E4M3, stats=True, dequant=True)]:
+        for rows, cols in [(0, 64), (8, 0)]:
+            x = torch.empty((rows, cols), dtype=torch.bfloat16, device="cuda")
+            out = fq.rht_quantize(cfg, x)
+            torch.cuda.synchronize()
+            assert out.codes.numel() == 0
+            if cfg.scale == E4M3:
+                assert host(out.tensor_scale)[0] == 0.0
+            if cfg.stats:
+                s = fq.stats(out.workspace)
+                assert s["n"] == 0 and s["blocks"] == 0
+
+
+# ------------------------------------------------------------------ edge blocks
+
+def _edge_matrix(scale_unit=1.0):
+    """Rows of 32 crafted values (two 16-blocks each), all finite with |x| < 2^123 after the
+    scaling by `unit` (so that sums of 16 stay finite)."""
+    f = np.float32
+    rows = []
+    z = np.zeros(32, f)
+    rows.append(z)                                             # all zero
+    rows.append(np.full(32, -0.0, f))                          # negative zeros
+    r = z.copy(); r[5] = -3.0; rows.append(r)                  # single nonzero
+    rows.append(np.full(32, 1.7, f))                           # all equal
+    rows.append(np.full(32, -2.5, f))
+    ties = np.array([6, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25, -0.75, -1.25, -1.75, -2.5,
+                     -3.5, -5.0, 0.0], f)
+    rows.append(np.concatenate([ties, ties[::-1]]))            # E2M1 midpoints with s = 1
+    ties2 = np.array([3.5, 0.25, 0.75, 1.25, 1.75, 2.25, 2.75, 3.25, -0.25, -0.75, -1.25, -1.75,
+                      -2.25, -2.75, -3.25, -0.0], f)
+    rows.append(np.concatenate([ties2, -ties2]))               # E1M2 midpoints with s = 1
+    ties3 = np.array([7, 0.5, 1.5, 2.5, 3.5, 4.5, 5.5, 6.5, -0.5, -1.5, -2.5, -3.5, -4.5, -5.5, -6.5, 0], f)
+    rows.append(np.concatenate([ties3, ties3]))                # INT4 midpoints with s = 1
+    sub = np.float32(2.0 ** -130)
+    rows.append(np.array([sub * (k % 5 - 2) for k in range(32)], f))   # bf16 subnormals
+    rows.append(np.array([1e24 * ((-1) ** k) * (1 + k / 64) for k in range(32)], f))   # huge
+    dyn = np.full(32, 1e-35, f); dyn[0] = 1e20; dyn[17] = -1e20; dyn[3] = -3e-38
+    rows.append(dyn)                                           # dynamic range beyond 2^180
+    mix = np.array([(1e-6 if k % 3 else 1.0) * ((-1) ** k) for k in range(32)], f)
+    rows.append(mix)                                           # small quotients next to large
+    r = z.copy(); r[::4] = -0.0; r[1] = 2.0 ** -133; rows.append(r)   # smallest bf16 subnormal
+    return synth.to_bf16_bits(np.stack(rows) * np.float32(scale_unit))
+
+
+@pytest.mark.parametrize("combo", COMBOS, ids=_cid)
+@pytest.mark.parametrize("rht", [0, 1])
+@pytest.mark.parametrize("unit", [1.0, 2.0 ** -100, 2.0 ** 40])
+def test_edge_blocks(combo, rht, unit):
+    grid, scale, rnd = combo
+    x = _edge_matrix(unit)
+    cfg = fq.Config(grid=grid, scale=scale, round=rnd, rht=rht, sign_mask=0x5A5A, sr_seed=3,
+                    dequant=True, stats=True)
+    compare_quant(cfg, x, gpu_quantize(cfg, x))
+    if scale == E4M3:   # the same blocks under a given (stale, too small) tensor scale
+        ts = np.float32(1e-4)
+        compare_quant(cfg, x, gpu_quantize(cfg, x, tensor_scale=ts), tensor_scale=ts)
+
+
+def test_edge_blocks_inside_random_data():
+    # edge rows scattered through a larger random tensor, so they share warps with normal blocks
+    base = synth.small(31, 512, 512, "normal")
+    edge = _edge_matrix()
+    idx = np.random.default_rng(0).choice(512, size=edge.shape[0], replace=False)
+    for j, i in enumerate(idx):
+        base[i, 64:96] = edge[j]
+    for combo in COMBOS:
+        cfg = fq.Config(grid=combo[0], scale=combo[1], round=combo[2], sign_mask=0x1357, sr_seed=11,
+                        dequant=True)
+        compare_quant(cfg, base, gpu_quantize(cfg, base))
+
+
+# ------------------------------------------------------------------ exact quotient step
+
+def test_division_step_matches_ieee_division():
+    lib = _lib.load()
+    bad = torch.zeros(1, dtype=torch.int64, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    import ctypes
+    for seed in (1, 2, 3):
+        assert lib.fp4q_check_division(seed, 1 << 28, ctypes.c_void_p(bad.data_ptr()),
+                                       ctypes.c_void_p(s)) == 0
+        torch.cuda.synchronize()
+        assert int(bad.item()) == 0
+
+
+# ------------------------------------------------------------------ dual orientation
+
+@pytest.mark.parametrize("grid", [E1M2, E2M1, INT4])
+@pytest.mark.parametrize("rounds", [(SR, SR), (RTNE, RTNE), (RTNE, SR)])
+@pytest.mark.parametrize("rhts", [(1, 1), (0, 1)])
+def test_dual_matches_row_and_transposed_oracle(grid, rounds, rhts):
+    for M, N, ld in [(16, 16, 16), (144, 80, 80), (400, 272, 288)]:
+        dy = synth.small(M + N, M, N, "normal", 1e-3)
+        rc = fq.Config(grid=grid, round=rounds[0], rht=rhts[0], sign_mask=0x3C5A, sr_seed=0x5A5A0003)
+        cc = fq.Config(grid=grid, round=rounds[1], rht=rhts[1], sign_mask=0xA5C3, sr_seed=0x5A5A0003,
+                       sr_stream=1)
+        out = fq.quantize_dual(rc, cc, to_dev(dy, ld))
+        torch.cuda.synchronize()
+        r = O.quantize(ocfg(rc), dy)
+        c = O.quantize(ocfg(cc), np.ascontiguousarray(dy.T))
+        np.testing.assert_array_equal(host(out.codes_row), r["codes"])
+        np.testing.assert_array_equal(host(out.scales_row), r["scales"])
+        np.testing.assert_array_equal(host(out.codes_col), c["codes"])
+        np.testing.assert_array_equal(host(out.scales_col), c["scales"])
+
+
+def test_dual_edge_blocks():
+    e = _edge_matrix()                        # [13, 32]
+    dy = np.zeros((208, 64), np.uint16)
+    dy[:13, :32] = e
+    dy[13:26, 32:] = e
+    dy[40:72, :13] = e.T
+    rc = fq.Config(round=SR, sign_mask=0x0FF0, sr_seed=9)
+    cc = fq.Config(round=SR, sign_mask=0x0FF0, sr_seed=9, sr_stream=1)
+    out = fq.quantize_dual(rc, cc, to_dev(dy))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host(out.codes_row), O.quantize(ocfg(rc), dy)["codes"])
+    np.testing.assert_array_equal(host(out.codes_col), O.quantize(ocfg(cc), np.ascontiguousarray(dy.T))["codes"])
+
+
+# ------------------------------------------------------------------ dequantize / rotation alone
+
+@pytest.mark.parametrize("combo", [(E2M1, FP32, RTNE), (E1M2, FP32, RTNE), (INT4, FP32, SR),
+                                   (E2M1, E4M3, RTNE), (INT4, E4M3, RTNE), (IF4, E4M3, RTNE),
+                                   (E2M1, UE8M0, RTNE)], ids=_cid)
+@pytest.mark.parametrize("inverse", [False, True])
+def test_dequantize(combo, inverse):
+    grid, scale, rnd = combo
+    cfg = fq.Config(grid=grid, scale=scale, round=rnd, sign_mask=0x2468, sr_seed=1)
+    x = synth.small(17, 75, 320, "laplace")
+    q = gpu_quantize(cfg, x)
+    d = fq.dequantize(cfg, q.codes, q.scales, q.tensor_scale, inverse_rht=inverse)
+    torch.cuda.synchronize()
+    ts = float(host(q.tensor_scale)[0]) if scale == E4M3 else 0.0
+    ref = O.dequantize(ocfg(cfg), host(q.codes), host(q.scales), ts, 75, 320, inverse_rht=inverse)
+    np.testing.assert_array_equal(bf16_bits(d), ref)
+
+
+def test_rotation_alone():
+    x = synth.small(3, 129, 2048, "t4")
+    for fp32 in (True, False):
+        y = fq.rht16(to_dev(x, 2048 + 64), 0x7E57, out_fp32=fp32)
+        torch.cuda.synchronize()
+        yf, yb = O.rht16_rows(x, 0x7E57)
+        if fp32:
+            np.testing.assert_array_equal(host(y).view(np.uint32), yf.view(np.uint32))
+        else:
+            np.testing.assert_array_equal(bf16_bits(y), yb)
+
+
+def test_unfused_pipeline_equals_fused_on_fp32_intermediate():
+    # quantize-only on the FP32 rotation is not expressible (inputs are bf16), but the
+    # rotation-alone output in bf16 fed to quantize-only must match the oracle doing the same
+    x = synth.small(8, 64, 512, "normal")
+    mask = 0x1111
+    yb = fq.rht16(to_dev(x), mask)
+    cfg = fq.Config(rht=0)
+    q = fq.rht_quantize(cfg, yb)
+    torch.cuda.synchronize()
+    _, yref = O.rht16_rows(x, mask)
+    ref = O.quantize(ocfg(cfg), yref)
+    np.testing.assert_array_equal(host(q.codes), ref["codes"])
