@@ -145,11 +145,13 @@ double orc_decode_nibble(int grid, uint8_t nib) {
 /* ------------------------------------------------------------------------------------ */
 /* Rounding.
  *
- * RTNE [UFP4-B section 二]: the nearest grid point; on a tie the even code (R5). Values
- * beyond the largest magnitude map to it (saturation), which nearest-point search does by
- * itself. Distances are exact in double (a float minus a grid point of few bits). */
+ * RTNE [UFP4-B section 二]: the nearest grid point; on a tie the even code (R5). Values at or
+ * beyond the largest magnitude map to it (saturation). Below it, distances are exact in double
+ * (a float under 8 minus a grid point of few bits); far above it they would not be, which is
+ * why saturation is decided first. */
 
 static int nearest_magnitude_code(const double* g, double a) {
+  if (a >= g[7]) return 7;
   int best = 0;
   double bd = fabs(a - g[0]);
   for (int c = 1; c < 8; ++c) {

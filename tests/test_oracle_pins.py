@@ -87,6 +87,15 @@ def test_rtne_against_independent_formula(grid):
     np.testing.assert_array_equal(np.sign(got[nz]), np.sign(want[nz]))
 
 
+@pytest.mark.parametrize("grid", [O.GRID_E2M1, O.GRID_E1M2, O.GRID_INT4])
+def test_rtne_saturates_far_above_qmax(grid):
+    # the nearest point to anything above the largest magnitude is that magnitude
+    g = O.grid_magnitudes(grid)
+    v = np.float32([g[7] * 1.01, 1e10, 2.0 ** 60, 3e38, -1e30, -(2.0 ** 100)])
+    got = _value_of(grid, O.round_rtne(grid, v))
+    np.testing.assert_array_equal(got, np.copysign(g[7], v))
+
+
 def test_rtne_tie_table_reading():
     # reading R5: ties go to the even code
     v = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
