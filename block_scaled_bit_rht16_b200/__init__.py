@@ -85,7 +85,8 @@ def _check_input(x, name="x"):
         raise TypeError("%s must be a 2-D bfloat16 CUDA tensor" % name)
     if x.stride(1) != 1 and x.numel() > 0:
         raise ValueError("%s must have unit column stride" % name)
-    return x.shape[0], x.shape[1], (x.stride(0) if x.shape[0] > 1 else x.shape[1])
+    ld = x.stride(0) if (x.shape[0] > 1 and x.numel() > 0) else x.shape[1]
+    return x.shape[0], x.shape[1], ld
 
 
 def sign_mask_from_seed(seed: int) -> int:

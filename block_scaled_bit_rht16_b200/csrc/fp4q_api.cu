@@ -53,6 +53,7 @@ size_t stats_bytes() { return (size_t)kStatsCtas * ST_LEN * sizeof(double); }
 fp4q_status check_shape(int64_t rows, int64_t cols, int64_t ld, int unit) {
   if (rows < 0 || cols < 0) return FP4Q_ERR_SHAPE;
   if (cols % unit != 0) return FP4Q_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return FP4Q_OK;            // empty: nothing is read
   if (ld < cols) return FP4Q_ERR_SHAPE;
   if (rows > 1 && ld % 8 != 0) return FP4Q_ERR_ALIGN;   // every row starts 16-byte aligned
   return FP4Q_OK;
@@ -181,8 +182,9 @@ fp4q_status fp4q_quantize_dual(const fp4q_config* row_cfg, const fp4q_config* co
     if (c->outputs & (FP4Q_OUT_DEQUANT | FP4Q_OUT_STATS)) return FP4Q_ERR_UNSUPPORTED;
   }
   if (row_cfg->grid != col_cfg->grid) return FP4Q_ERR_UNSUPPORTED;
-  if (M < 0 || N < 0 || M % 16 != 0 || N % 16 != 0 || ld < N) return FP4Q_ERR_SHAPE;
-  if (M > 1 && ld % 8 != 0) return FP4Q_ERR_ALIGN;
+  if (M < 0 || N < 0 || M % 16 != 0 || N % 16 != 0) return FP4Q_ERR_SHAPE;
+  if (M > 0 && N > 0 && ld < N) return FP4Q_ERR_SHAPE;
+  if (M > 1 && N > 0 && ld % 8 != 0) return FP4Q_ERR_ALIGN;
   const bool empty = M == 0 || N == 0;
   if (!empty && (dy == nullptr || codes_row == nullptr || scales_row == nullptr ||
                  codes_col == nullptr || scales_col == nullptr))
