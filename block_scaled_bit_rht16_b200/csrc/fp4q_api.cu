@@ -142,6 +142,7 @@ fp4q_status fp4q_rht_quantize(const fp4q_config* cfg, const void* x, int64_t row
   a.cinv = cfg->rht ? 0.25f : 1.0f;
   a.seedx = cfg->sr_seed ^ ((uint64_t)(cfg->sr_stream & 1u) << 63);
   a.contiguous = (ld == cols) ? 1 : 0;
+  a.vec32 = (reinterpret_cast<uintptr_t>(x) % 32 == 0 && (rows == 1 || ld % 16 == 0)) ? 1 : 0;
 
   if (compute_alpha) {
     QuantArgs am = a;
@@ -296,7 +297,6 @@ fp4q_status fp4q_check_division(uint64_t seed, uint64_t n, unsigned long long* m
   if (!aligned(mismatches, 8)) return FP4Q_ERR_ALIGN;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(mismatches, 0, sizeof(unsigned long long), s) != cudaSuccess) return FP4Q_ERR_CUDA;
-  if (n == 0) return FP4Q_OK;
   return cuda_status(launch_division_check(seed, n, mismatches, s));
 }
 

@@ -42,7 +42,6 @@ __global__ void __launch_bounds__(kThreads) dual_kernel(const DualArgs a) {
   }
   __syncthreads();
 
-  constexpr float qmax = GridInfo<G>::qmax;
   const EncCtx ctx_row{a.cinv_row, a.seedx_row};
   const EncCtx ctx_col{a.cinv_col, a.seedx_col};
 
@@ -56,7 +55,7 @@ __global__ void __launch_bounds__(kThreads) dual_kernel(const DualArgs a) {
     float2 P[8];
     unpack16(src[0], src[1], a.sw_row, P);
     if (a.c_row != 1.0f) fwht16(P);
-    const float s = __fdiv_rn(__fmul_rn(absmax16(P), a.cinv_row), qmax);
+    const float s = div_qmax<G>(__fmul_rn(absmax16(P), a.cinv_row));
     const Divider dv = make_divider(s, a.c_row);
     const int64_t u = (m * a.N + n) >> 4;   // 16-block index in [M, N/16]
     encode16<G, RR, false>(ctx_row, P, (uint64_t)u * 8u, a.codes_row + u * 8, nullptr, s, dv,
@@ -83,7 +82,7 @@ __global__ void __launch_bounds__(kThreads) dual_kernel(const DualArgs a) {
     unpack16(make_uint4(wd[0], wd[1], wd[2], wd[3]), make_uint4(wd[4], wd[5], wd[6], wd[7]),
              a.sw_col, P);
     if (a.c_col != 1.0f) fwht16(P);
-    const float s = __fdiv_rn(__fmul_rn(absmax16(P), a.cinv_col), qmax);
+    const float s = div_qmax<G>(__fmul_rn(absmax16(P), a.cinv_col));
     const Divider dv = make_divider(s, a.c_col);
     const int64_t u = (n * a.M + m) >> 4;   // 16-block index in [N, M/16]
     encode16<G, RC, false>(ctx_col, P, (uint64_t)u * 8u, a.codes_col + u * 8, nullptr, s, dv,

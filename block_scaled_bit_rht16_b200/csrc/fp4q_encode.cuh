@@ -75,6 +75,115 @@ __device__ __forceinline__ float with_sign_of(float q, float vraw) {
   return __uint_as_float((__float_as_uint(q) & 0x7FFFFFFFu) | (__float_as_uint(vraw) & 0x80000000u));
 }
 
+// ------------------------------------------------------------------ lean encoder (hot path)
+//
+// FP32 1x16 scale, round to nearest even, codes only. Per element pair one packed FMA forms
+// t = 1.5 * 2^23 + v / step, whose float rounding is exactly round-half-even of v / step and
+// whose low four bits are that integer in two's complement. Funnel shifts pack the low nibbles
+// of eight such words (discarding the rest); E1M2 then turns the two's complement nibbles into
+// sign-magnitude with word-wide integer operations and takes each sign bit from the rotated
+// value itself (so a negative value that rounds to zero keeps its sign).
+
+// Exact RN(a / qmax) for the grid's compile-time qmax: one multiply and two FMAs (the same
+// correction step as the element quotients, with the divisor's correctly rounded reciprocal
+// folded at compile time), or the IEEE division outside the range where that step is exact.
+template <int G>
+__device__ __forceinline__ float div_qmax(float a) {
+  constexpr float qmax = GridInfo<G>::qmax;
+  constexpr float r = 1.0f / qmax;
+  if (a >= 0x1p-100f && a <= 0x1p+100f) {
+    const float s0 = __fmul_rn(a, r);
+    const float e = __fmaf_rn(-s0, qmax, a);
+    return __fmaf_rn(e, r, s0);
+  }
+  return __fdiv_rn(a, qmax);
+}
+
+// Low nibbles of t[0..7] packed into one word, t[0] in bits 0..3 (bits above each nibble of
+// t are ignored).
+__device__ __forceinline__ uint32_t pack_low_nibbles(const uint32_t* t) {
+  uint32_t w = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w = __funnelshift_r(w, t[i], 4);
+  return w;
+}
+
+// Sign bits of f[0..7] at bit 4i+3.
+__device__ __forceinline__ uint32_t pack_signs(const float* f) {
+  uint32_t w = 0u;
+#pragma unroll
+  for (int i = 7; i >= 0; --i) w = __funnelshift_l(__float_as_uint(f[i]), w, 4);
+  return w & 0x88888888u;
+}
+
+// Two's complement nibbles (-7..7) -> magnitudes 0..7 in the same nibbles.
+__device__ __forceinline__ uint32_t nibble_magnitudes(uint32_t w) {
+  const uint32_t neg = (w >> 3) & 0x11111111u;
+  return (w ^ (neg * 15u)) + neg;
+}
+
+// Codes of one block on E1M2 / INT4 / E2M1 from the rotated raw values P (y = cinv * P) with
+// block scale s (already known nonzero or zero). Returns the two code words.
+template <int G>
+__device__ __forceinline__ uint2 encode_lean(const float2* P, float s, const Divider& dv,
+                                             float cinv) {
+  if (s == 0.0f) return make_uint2(0u, 0u);
+  constexpr float qmax = GridInfo<G>::qmax;
+  float2 Q[8];
+  if (dv.fast) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) Q[i] = div2(dv, P[i]);
+  } else {
+    // block scale outside the exact range of the correction step (tiny or huge data):
+    // IEEE division, then the saturation the fast range never needs
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float qx = __fdiv_rn(__fmul_rn(P[i].x, cinv), s);
+      const float qy = __fdiv_rn(__fmul_rn(P[i].y, cinv), s);
+      Q[i] = make_float2(fminf(fmaxf(qx, -qmax), qmax), fminf(fmaxf(qy, -qmax), qmax));
+    }
+  }
+  if constexpr (G == kE2M1) {
+    uint32_t w[2];
+#pragma unroll
+    for (int l = 0; l < 2; ++l) {
+      uint32_t b[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float lo = l ? with_sign_of(Q[2 * j].y, P[2 * j].y) : with_sign_of(Q[2 * j].x, P[2 * j].x);
+        const float hi = l ? with_sign_of(Q[2 * j + 1].y, P[2 * j + 1].y)
+                           : with_sign_of(Q[2 * j + 1].x, P[2 * j + 1].x);
+        b[j] = cvt_e2m1x2(hi, lo);
+      }
+      w[l] = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+    }
+    return make_uint2(w[0], w[1]);
+  } else {
+    constexpr float inv_step = (G == kE1M2) ? 2.0f : 1.0f;
+    const float2 m2 = make_float2(inv_step, inv_step);
+    const float2 c2 = make_float2(12582912.0f, 12582912.0f);   // 1.5 * 2^23
+    uint32_t t0[8], t1[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 t = __ffma2_rn(Q[i], m2, c2);
+      t0[i] = __float_as_uint(t.x);
+      t1[i] = __float_as_uint(t.y);
+    }
+    uint32_t w0 = pack_low_nibbles(t0), w1 = pack_low_nibbles(t1);
+    if constexpr (G == kE1M2) {
+      float v0[8], v1[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v0[i] = P[i].x;
+        v1[i] = P[i].y;
+      }
+      w0 = nibble_magnitudes(w0) | pack_signs(v0);
+      w1 = nibble_magnitudes(w1) | pack_signs(v1);
+    }
+    return make_uint2(w0, w1);
+  }
+}
+
 // ------------------------------------------------------------------ statistics accumulator
 
 struct StatsAcc {

@@ -42,6 +42,7 @@ struct QuantArgs {
   float c, cinv;           // 4, 1/4 with rotation; 1, 1 without
   uint64_t seedx;          // SR: seed ^ (stream << 63)
   int contiguous;          // ld == cols
+  int vec32;               // every unit starts 32-byte aligned: one 256-bit load per 16 elements
 };
 
 struct DualArgs {

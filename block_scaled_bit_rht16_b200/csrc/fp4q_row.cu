@@ -31,6 +31,20 @@ __device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
   return __ldcs(reinterpret_cast<const uint4*>(p));
 }
 
+// 16 bf16 (32 bytes): one 256-bit load when the address is 32-byte aligned (the host sets
+// vec32 only when every unit start is), else two 128-bit loads. Read-only, streamed past L1.
+__device__ __forceinline__ void load16(const uint16_t* p, bool vec32, uint4& lo, uint4& hi) {
+  if (vec32) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w),
+                   "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+                 : "l"(p));
+  } else {
+    lo = ld_stream(p);
+    hi = ld_stream(p + 8);
+  }
+}
+
 __device__ __forceinline__ int64_t unit_offset(const QuantArgs& a, int64_t u, int unit) {
   if (a.contiguous) return u * unit;
   const int64_t r = u / a.units_per_row;
@@ -209,7 +223,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantArgs a) {
       if (k == 1 && !has2) break;
       const uint16_t* src = a.x + unit_offset(a, uu[k], kUnit);
 #pragma unroll
-      for (int v = 0; v < kVec; ++v) buf[k][v] = ld_stream(src + 8 * v);
+      for (int v = 0; v < kVec; v += 2) load16(src + 8 * v, a.vec32 != 0, buf[k][v], buf[k][v + 1]);
     }
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
@@ -224,7 +238,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantArgs a) {
         float s;
         uint32_t sbyte = 0u;
         if constexpr (S == kFP32) {
-          s = __fdiv_rn(amax_y, qmax);
+          s = div_qmax<G>(amax_y);
         } else {
           const float delta = denom > 0.0f ? __fdiv_rn(amax_y, denom) : 0.0f;
           sbyte = cvt_e4m3(delta);
@@ -261,15 +275,43 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantArgs a) {
   if constexpr (STATS) stats_finish(acc, a.partials);
 }
 
+// The hot path: FP32 1x16 scale, round to nearest even, codes and scales only.
+template <int G>
+__global__ void __launch_bounds__(kThreads) lean_kernel(const QuantArgs a) {
+  const bool vec32 = a.vec32 != 0;
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < a.nunits; u += 2 * stride) {
+    uint4 lo[2], hi[2];
+    const int64_t uu[2] = {u, u + stride};
+    const bool has2 = uu[1] < a.nunits;
+    load16(a.x + unit_offset(a, uu[0], 16), vec32, lo[0], hi[0]);
+    if (has2) load16(a.x + unit_offset(a, uu[1], 16), vec32, lo[1], hi[1]);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      if (k == 1 && !has2) break;
+      const int64_t un = uu[k];
+      float2 P[8];
+      unpack16(lo[k], hi[k], a.sw, P);
+      rotate_if(a, P);
+      const float s = div_qmax<G>(__fmul_rn(absmax16(P), a.cinv));
+      const Divider dv = make_divider(s, a.c);
+      const uint2 w = encode_lean<G>(P, s, dv, a.cinv);
+      __stcs(reinterpret_cast<uint2*>(a.codes) + un, w);
+      __stcs(reinterpret_cast<float*>(a.scales) + un, s);
+    }
+  }
+}
+
 // Amax of the rotated tensor: per-warp maximum of the bit patterns (non-negative floats order
 // like unsigned integers), one atomicMax per warp into the workspace header.
 __global__ void __launch_bounds__(kThreads) amax_kernel(const QuantArgs a) {
   uint32_t m = 0u;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < a.nunits; u += stride) {
-    const uint16_t* src = a.x + unit_offset(a, u, 16);
+    uint4 lo, hi;
+    load16(a.x + unit_offset(a, u, 16), a.vec32 != 0, lo, hi);
     float2 P[8];
-    unpack16(ld_stream(src), ld_stream(src + 8), a.sw, P);
+    unpack16(lo, hi, a.sw, P);
     rotate_if(a, P);
     m = max(m, __float_as_uint(__fmul_rn(absmax16(P), a.cinv)));
   }
@@ -282,9 +324,10 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const QuantArgs a) {
 __global__ void __launch_bounds__(kThreads) rht16_kernel(const QuantArgs a, int out_fp32, void* out) {
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < a.nunits; u += stride) {
-    const uint16_t* src = a.x + unit_offset(a, u, 16);
+    uint4 lo, hi;
+    load16(a.x + unit_offset(a, u, 16), a.vec32 != 0, lo, hi);
     float2 P[8];
-    unpack16(ld_stream(src), ld_stream(src + 8), a.sw, P);
+    unpack16(lo, hi, a.sw, P);
     fwht16(P);
     float y[16];
 #pragma unroll
@@ -395,6 +438,18 @@ __global__ void __launch_bounds__(kThreads) division_check_kernel(uint64_t seed,
                                                                   unsigned long long* bad) {
   unsigned long long local = 0;
   const uint64_t stride = (uint64_t)gridDim.x * kThreads;
+  // every mantissa of a in [1, 4) for the three compile-time divisors (the scale quotient
+  // a / qmax); by scale invariance this covers all a in [2^-100, 2^100]
+  for (uint64_t i = (uint64_t)blockIdx.x * kThreads + threadIdx.x; i < (3ull << 24); i += stride) {
+    const uint32_t m = (uint32_t)(i & 0xFFFFFFu);
+    const float a = __uint_as_float(((127u + (m >> 23)) << 23) | (m & 0x7FFFFFu));
+    const int g = (int)(i >> 24);
+    float got, want;
+    if (g == 0) { got = div_qmax<kE2M1>(a); want = __fdiv_rn(a, 6.0f); }
+    else if (g == 1) { got = div_qmax<kE1M2>(a); want = __fdiv_rn(a, 3.5f); }
+    else { got = div_qmax<kINT4>(a); want = __fdiv_rn(a, 7.0f); }
+    if (__float_as_uint(got) != __float_as_uint(want)) ++local;
+  }
   for (uint64_t i = (uint64_t)blockIdx.x * kThreads + threadIdx.x; i < n; i += stride) {
     const uint64_t h = splitmix64(seed ^ (i * 0x9E3779B97F4A7C15ull));
     const uint64_t g = splitmix64(h);
@@ -475,8 +530,20 @@ cudaError_t launch_q_round(int round, bool stats, const QuantArgs& a, cudaStream
 
 }  // namespace
 
+template <int G>
+cudaError_t launch_lean(const QuantArgs& a, cudaStream_t st) {
+  auto k = lean_kernel<G>;
+  k<<<persistent_grid(k, (a.nunits + 1) / 2), kThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quantize(int grid, int scale, int round, bool stats, const QuantArgs& a,
                             cudaStream_t st) {
+  if (scale == kFP32 && round == kRTNE && !stats && a.deq == nullptr) {
+    if (grid == kE2M1) return launch_lean<kE2M1>(a, st);
+    if (grid == kE1M2) return launch_lean<kE1M2>(a, st);
+    if (grid == kINT4) return launch_lean<kINT4>(a, st);
+  }
   if (scale == kFP32) {
     if (grid == kE2M1) return launch_q_round<kE2M1, kFP32>(round, stats, a, st);
     if (grid == kE1M2) return launch_q_round<kE1M2, kFP32>(round, stats, a, st);
@@ -510,6 +577,7 @@ cudaError_t launch_rht16(const uint16_t* x, int64_t rows, int64_t cols, int64_t 
   for (int k = 0; k < 8; ++k) a.sw[k] = sw[k];
   a.c = 4.0f;
   a.cinv = 0.25f;
+  a.vec32 = (reinterpret_cast<uintptr_t>(x) % 32 == 0) && (rows == 1 || ld % 16 == 0);
   if (a.nunits == 0) return cudaSuccess;
   rht16_kernel<<<persistent_grid(rht16_kernel, a.nunits), kThreads, 0, st>>>(a, out_fp32 ? 1 : 0, out);
   return cudaGetLastError();

@@ -83,10 +83,13 @@ def compare_stats(g, o, raw):
 
 @pytest.mark.parametrize("combo", COMBOS, ids=_cid)
 @pytest.mark.parametrize("rht", [0, 1])
-def test_small_ragged_all_outputs(combo, rht):
+@pytest.mark.parametrize("outs", ["all", "codes"])
+def test_small_ragged(combo, rht, outs):
+    # "codes" without dequant/statistics takes the lean kernel for FP32 + RTNE
     grid, scale, rnd = combo
+    full = outs == "all"
     cfg = fq.Config(grid=grid, scale=scale, round=rnd, rht=rht, sign_mask=MASK, sr_seed=0x1234ABCD,
-                    dequant=True, stats=True)
+                    dequant=full, stats=full)
     for rows, cols, kind in [(1, 32, "normal"), (37, 96, "t4"), (130, 1056, "laplace")]:
         x = synth.small(rows * 7 + cols, rows, cols, kind)
         compare_quant(cfg, x, gpu_quantize(cfg, x))
@@ -102,15 +105,32 @@ def test_many_grid_iterations(combo):
     compare_quant(cfg, x, gpu_quantize(cfg, x))
 
 
-@pytest.mark.parametrize("combo", [(E1M2, FP32, RTNE), (E2M1, E4M3, RTNE), (IF4, E4M3, RTNE),
-                                   (E2M1, UE8M0, SR), (INT4, FP32, SR)], ids=_cid)
-def test_strided_input_and_given_tensor_scale(combo):
+@pytest.mark.parametrize("combo", [(E1M2, FP32, RTNE), (E2M1, FP32, RTNE), (INT4, FP32, RTNE),
+                                   (E2M1, E4M3, RTNE), (IF4, E4M3, RTNE), (E2M1, UE8M0, SR),
+                                   (INT4, FP32, SR)], ids=_cid)
+@pytest.mark.parametrize("ld", [320 + 24, 320 + 32])   # 16-byte and 32-byte aligned rows
+@pytest.mark.parametrize("deq", [False, True])
+def test_strided_input_and_given_tensor_scale(combo, ld, deq):
     grid, scale, rnd = combo
-    cfg = fq.Config(grid=grid, scale=scale, round=rnd, sign_mask=0x8001, sr_seed=5, dequant=True)
+    cfg = fq.Config(grid=grid, scale=scale, round=rnd, sign_mask=0x8001, sr_seed=5, dequant=deq)
     x = synth.small(9, 67, 320, "normal", 3.0)
     ts = np.float32(0.0123) if scale == E4M3 else None
-    out = gpu_quantize(cfg, x, ld=320 + 24, tensor_scale=ts)
+    out = gpu_quantize(cfg, x, ld=ld, tensor_scale=ts)
     compare_quant(cfg, x, out, tensor_scale=ts)
+
+
+@pytest.mark.parametrize("grid", [E1M2, E2M1, INT4])
+def test_input_only_16_byte_aligned(grid):
+    # a view starting 8 elements into its storage: 16-byte but not 32-byte aligned
+    x = synth.small(10, 33, 256, "t4")
+    big = np.zeros((33, 264), np.uint16)
+    big[:, 8:] = x
+    t = to_dev(big)[:, 8:]
+    assert t.data_ptr() % 32 == 16
+    cfg = fq.Config(grid=grid, sign_mask=0x0F0F)
+    out = fq.rht_quantize(cfg, t)
+    torch.cuda.synchronize()
+    compare_quant(cfg, x, out)
 
 
 def test_empty_inputs():
@@ -162,11 +182,13 @@ def _edge_matrix(scale_unit=1.0):
 @pytest.mark.parametrize("combo", COMBOS, ids=_cid)
 @pytest.mark.parametrize("rht", [0, 1])
 @pytest.mark.parametrize("unit", [1.0, 2.0 ** -100, 2.0 ** 40])
-def test_edge_blocks(combo, rht, unit):
+@pytest.mark.parametrize("outs", ["all", "codes"])
+def test_edge_blocks(combo, rht, unit, outs):
     grid, scale, rnd = combo
     x = _edge_matrix(unit)
+    full = outs == "all"
     cfg = fq.Config(grid=grid, scale=scale, round=rnd, rht=rht, sign_mask=0x5A5A, sr_seed=3,
-                    dequant=True, stats=True)
+                    dequant=full, stats=full)
     compare_quant(cfg, x, gpu_quantize(cfg, x))
     if scale == E4M3:   # the same blocks under a given (stale, too small) tensor scale
         ts = np.float32(1e-4)
@@ -181,9 +203,10 @@ def test_edge_blocks_inside_random_data():
     for j, i in enumerate(idx):
         base[i, 64:96] = edge[j]
     for combo in COMBOS:
-        cfg = fq.Config(grid=combo[0], scale=combo[1], round=combo[2], sign_mask=0x1357, sr_seed=11,
-                        dequant=True)
-        compare_quant(cfg, base, gpu_quantize(cfg, base))
+        for deq in (False, True):
+            cfg = fq.Config(grid=combo[0], scale=combo[1], round=combo[2], sign_mask=0x1357,
+                            sr_seed=11, dequant=deq)
+            compare_quant(cfg, base, gpu_quantize(cfg, base))
 
 
 # ------------------------------------------------------------------ exact quotient step
