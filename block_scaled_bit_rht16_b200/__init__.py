@@ -210,6 +210,14 @@ def rht16(x, sign_mask: int, *, out_fp32: bool = False, out=None, stream=None):
     return out
 
 
+def device_status(clear: bool = False, stream=None) -> int:
+    """fp4q_device_status: the library's sticky device status bits (0 when all is well)."""
+    v = ctypes.c_int32(0)
+    _lib.check(_lib.load().fp4q_device_status(ctypes.byref(v), int(bool(clear)), _stream_ptr(stream)),
+               "fp4q_device_status")
+    return int(v.value)
+
+
 def stats(workspace, stream=None) -> dict:
     """fp4q_stats: reduce and fetch the statistics a stats-enabled call left in `workspace`."""
     res = _lib.fp4q_stats_t()

@@ -300,4 +300,14 @@ fp4q_status fp4q_check_division(uint64_t seed, uint64_t n, unsigned long long* m
   return cuda_status(launch_division_check(seed, n, mismatches, s));
 }
 
+fp4q_status fp4q_device_status(int32_t* status_bits, int32_t clear, fp4q_stream_t stream) {
+  if (status_bits == nullptr || (clear != 0 && clear != 1)) return FP4Q_ERR_INVALID_ARG;
+  return cuda_status(read_device_status(status_bits, clear != 0, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fp4q_status fp4q_check_wait_timeout(uint64_t limit_ns, fp4q_stream_t stream) {
+  if (limit_ns == 0 || limit_ns > 1000000000ull) return FP4Q_ERR_INVALID_ARG;
+  return cuda_status(launch_wait_timeout_check(limit_ns, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -89,9 +89,10 @@ __device__ __forceinline__ float absmax16(const float2* P) {
 // of elementary functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990):
 // with R = RN(1/S) and q0 = RN(a R), the remainder r = a - q0 S is exact under an FMA and
 // q1 = RN(q0 + r R) is the correctly rounded a/S. Here S = c*s and a = vraw, so a/S = y/s.
-// The step is valid while S and 1/S are normal with headroom and |a| >= 2^-100 * max(1, S);
-// Smaller |a| give quotients below 2^-99, which every rounding rule here maps to a zero code
-// (stochastic rounding recomputes them with the IEEE division, see div_tiny_fix).
+// With S in [2^-60, 2^90] (the fast range) the step is exact for every quotient of at least
+// 2^-20: then |a| >= 2^-80, so the remainder is representable. Smaller quotients round to a
+// zero code under round-to-nearest; stochastic rounding and IF4 recompute them with the IEEE
+// division. Outside the fast range every quotient uses the IEEE division.
 struct Divider {
   float2 R2, nS2;   // (R, R), (-S, -S)
   float S, R;
@@ -101,7 +102,7 @@ struct Divider {
 __device__ __forceinline__ Divider make_divider(float s, float c) {
   Divider d;
   d.S = __fmul_rn(s, c);
-  d.fast = (d.S >= 0x1p-90f) && (d.S <= 0x1p+90f);
+  d.fast = (d.S >= 0x1p-60f) && (d.S <= 0x1p+90f);
   d.R = d.fast ? __frcp_rn(d.S) : 0.0f;
   d.R2 = make_float2(d.R, d.R);
   d.nS2 = make_float2(-d.S, -d.S);
@@ -159,6 +160,67 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// ------------------------------------------------------------------ bulk copies and barriers
+//
+// Global -> shared bulk copies (cp.async.bulk, no multicast) complete on an mbarrier with a
+// transaction count. Every wait is bounded by the global timer: a wait that gives up sets a
+// bit in the library's device status word and returns false, so no kernel can hang.
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete; false after kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 0u && global_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// bytes (multiple of 16) from global src (16-byte aligned) to shared dst (16-byte aligned).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
 
 // ------------------------------------------------------------------ stochastic rounding source

@@ -57,6 +57,11 @@ struct DualArgs {
   int grid_row, grid_col;
 };
 
+// Bits of the device status word (defined in fp4q_row.cu): bit 0 a bulk-copy / barrier wait in
+// a quantize kernel gave up, bit 1 the timeout self-test fired. Sticky until read with clear.
+constexpr int32_t kStatusWaitTimeout = 1;
+constexpr int32_t kStatusSelfTest = 2;
+
 // Host-side launchers (fp4q_row.cu / fp4q_dual.cu). Return the CUDA error of the launch.
 cudaError_t launch_quantize(int grid, int scale, int round, bool stats, const QuantArgs& a,
                             cudaStream_t st);
@@ -70,5 +75,7 @@ cudaError_t launch_stats_reduce(WsHeader* ws, const double* partials, cudaStream
 cudaError_t launch_dual(const DualArgs& a, cudaStream_t st);
 cudaError_t launch_division_check(uint64_t seed, uint64_t n, unsigned long long* bad,
                                   cudaStream_t st);
+cudaError_t launch_wait_timeout_check(unsigned long long limit_ns, cudaStream_t st);
+cudaError_t read_device_status(int32_t* out, bool clear, cudaStream_t st);
 
 }  // namespace fp4q

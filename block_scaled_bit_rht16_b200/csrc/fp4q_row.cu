@@ -25,6 +25,9 @@
 #include "fp4q_kernels.cuh"
 
 namespace fp4q {
+
+__device__ int32_t g_device_status = 0;
+
 namespace {
 
 __device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
@@ -302,6 +305,99 @@ __global__ void __launch_bounds__(kThreads) lean_kernel(const QuantArgs a) {
   }
 }
 
+// The hot path for contiguous tensors: a 4-stage ring of 8 KiB shared-memory stages filled by
+// bulk copies (one per 256 blocks of 16 elements). Thread 0 issues the copies and refills a
+// stage once all 256 threads have released it (mbarrier full/empty pairs); every thread
+// encodes one block per stage. Loads never occupy registers, so each CTA keeps up to 32 KiB
+// in flight regardless of occupancy.
+constexpr int kStages = 4;
+constexpr int kChunkBytes = kThreads * 32;
+
+template <int G>
+__global__ void __launch_bounds__(kThreads) lean_tma_kernel(const QuantArgs a) {
+  __shared__ __align__(128) uint8_t stage[kStages][kChunkBytes];
+  __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
+  const int t = threadIdx.x;
+  const int64_t nchunks = (a.nunits + kThreads - 1) / kThreads;
+  const uint8_t* xb = reinterpret_cast<const uint8_t*>(a.x);
+  auto issue = [&](int64_t c, int s) {
+    const int64_t u0 = c * kThreads;
+    const uint32_t bytes = (uint32_t)(min((int64_t)kThreads, a.nunits - u0) * 32);
+    mbar_arrive_expect_tx(&full[s], bytes);
+    bulk_load(stage[s], xb + u0 * 32, bytes, &full[s]);
+  };
+  if (t == 0) {
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kThreads);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (t == 0) {
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) {
+      const int64_t c = blockIdx.x + (int64_t)s * gridDim.x;
+      if (c < nchunks) issue(c, s);
+    }
+  }
+  bool ok = true;
+  int64_t k = 0;
+  for (;; ++k) {
+    const int64_t c = blockIdx.x + k * gridDim.x;
+    if (c >= nchunks) break;
+    const int s = (int)(k % kStages);
+    const uint32_t par = (uint32_t)((k / kStages) & 1);
+    if (!mbar_wait(&full[s], par)) {
+      ok = false;
+      break;
+    }
+    const int64_t u = c * kThreads + t;
+    if (u < a.nunits) {
+      const uint4* src = reinterpret_cast<const uint4*>(stage[s] + 32 * t);
+      float2 P[8];
+      unpack16(src[0], src[1], a.sw, P);
+      rotate_if(a, P);
+      const float sc = div_qmax<G>(__fmul_rn(absmax16(P), a.cinv));
+      const Divider dv = make_divider(sc, a.c);
+      const uint2 w = encode_lean<G>(P, sc, dv, a.cinv);
+      __stcs(reinterpret_cast<uint2*>(a.codes) + u, w);
+      __stcs(reinterpret_cast<float*>(a.scales) + u, sc);
+    }
+    mbar_arrive(&empty[s]);
+    if (t == 0) {
+      const int64_t cn = c + (int64_t)kStages * gridDim.x;
+      if (cn < nchunks) {
+        if (!mbar_wait(&empty[s], par)) {
+          ok = false;
+          break;
+        }
+        issue(cn, s);
+      }
+    }
+  }
+  if (!ok) {
+    atomicOr(&g_device_status, kStatusWaitTimeout);
+    // let copies this CTA issued and nobody consumed land before its shared memory goes away
+    if (t == 0) {
+      for (int64_t j = k; j < k + kStages; ++j) {
+        const int64_t cj = blockIdx.x + j * gridDim.x;
+        if (cj < nchunks) mbar_wait(&full[j % kStages], (uint32_t)((j / kStages) & 1), 100000000ull);
+      }
+    }
+  }
+}
+
+// Self-test of the bounded wait: one thread waits on a barrier nothing arrives on.
+__global__ void wait_timeout_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  if (!mbar_wait(&bar, 0u, limit_ns)) atomicOr(&g_device_status, kStatusSelfTest);
+  mbar_arrive(&bar);   // complete the phase so the barrier is left consistent
+}
+
 // Amax of the rotated tensor: per-warp maximum of the bit patterns (non-negative floats order
 // like unsigned integers), one atomicMax per warp into the workspace header.
 __global__ void __launch_bounds__(kThreads) amax_kernel(const QuantArgs a) {
@@ -532,8 +628,14 @@ cudaError_t launch_q_round(int round, bool stats, const QuantArgs& a, cudaStream
 
 template <int G>
 cudaError_t launch_lean(const QuantArgs& a, cudaStream_t st) {
-  auto k = lean_kernel<G>;
-  k<<<persistent_grid(k, (a.nunits + 1) / 2), kThreads, 0, st>>>(a);
+  if (a.contiguous) {
+    auto k = lean_tma_kernel<G>;
+    const int64_t chunks = (a.nunits + kThreads - 1) / kThreads;
+    k<<<(int)std::min<int64_t>(chunks, resident_ctas(k)), kThreads, 0, st>>>(a);
+  } else {
+    auto k = lean_kernel<G>;
+    k<<<persistent_grid(k, (a.nunits + 1) / 2), kThreads, 0, st>>>(a);
+  }
   return cudaGetLastError();
 }
 
@@ -622,6 +724,23 @@ cudaError_t launch_division_check(uint64_t seed, uint64_t n, unsigned long long*
   division_check_kernel<<<persistent_grid(division_check_kernel, (int64_t)std::min<uint64_t>(n, 1ull << 40)),
                           kThreads, 0, st>>>(seed, n, bad);
   return cudaGetLastError();
+}
+
+cudaError_t launch_wait_timeout_check(unsigned long long limit_ns, cudaStream_t st) {
+  wait_timeout_kernel<<<1, 1, 0, st>>>(limit_ns);
+  return cudaGetLastError();
+}
+
+cudaError_t read_device_status(int32_t* out, bool clear, cudaStream_t st) {
+  cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_device_status, sizeof(int32_t), 0,
+                                            cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return e;
+  if (clear) {
+    static const int32_t zero = 0;
+    e = cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(int32_t), 0, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaStreamSynchronize(st);
 }
 
 cudaError_t launch_stats_reduce(WsHeader* ws, const double* partials, cudaStream_t st) {

@@ -207,6 +207,17 @@ fp4q_status fp4q_rht16(const void* x, int64_t rows, int64_t cols, int64_t ld, ui
 fp4q_status fp4q_check_division(uint64_t seed, uint64_t n, unsigned long long* mismatches,
                                 fp4q_stream_t stream);
 
+/* Device status word of the library on the current device: bit 0 set when a bounded wait
+ * inside a quantize kernel (shared-memory stage copies) gave up after 2 s -- that launch's
+ * outputs are incomplete; bit 1 set by fp4q_check_wait_timeout. Copies the word to
+ * *status_bits (host), clears it when `clear` is 1, and synchronizes `stream`. */
+fp4q_status fp4q_device_status(int32_t* status_bits, int32_t clear, fp4q_stream_t stream);
+
+/* Diagnostic: launches one thread that waits, with a limit of limit_ns (1 ns .. 1 s), on a
+ * barrier nothing arrives on; when the limit runs out it sets bit 1 of the status word and
+ * returns. Exercises the timeout path of the kernels' bounded waits without any fault. */
+fp4q_status fp4q_check_wait_timeout(uint64_t limit_ns, fp4q_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
