@@ -11,6 +11,7 @@
 // (zhichai.net/topic/178208020), sections "E2M1" and "UFP4" (grids, recipe table).
 #pragma once
 #include <cstdint>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace fp4q {
@@ -99,11 +100,22 @@ struct Divider {
   bool fast;        // the block's S is in the range where the correction step is exact
 };
 
+// RN(1/S) for S in [2^-60, 2^90]: the hardware reciprocal approximation refined by one
+// Newton-Raphson step in FMA form, r1 = r0 + r0 (1 - S r0) (Markstein 1990; Cornea, Golliver
+// and Markstein, "Correctness proofs outline for Newton-Raphson based floating-point divide
+// and square root algorithms", ARITH 1999). fp4q_check_division compares it with the IEEE
+// reciprocal on every float of that range.
+__device__ __forceinline__ float rcp_rn_fast(float S) {
+  float r0;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(S));
+  return __fmaf_rn(__fmaf_rn(-S, r0, 1.0f), r0, r0);
+}
+
 __device__ __forceinline__ Divider make_divider(float s, float c) {
   Divider d;
   d.S = __fmul_rn(s, c);
   d.fast = (d.S >= 0x1p-60f) && (d.S <= 0x1p+90f);
-  d.R = d.fast ? __frcp_rn(d.S) : 0.0f;
+  d.R = d.fast ? rcp_rn_fast(d.S) : 0.0f;
   d.R2 = make_float2(d.R, d.R);
   d.nS2 = make_float2(-d.S, -d.S);
   return d;
@@ -139,6 +151,16 @@ __device__ __forceinline__ float2 e2m1x2_to_f32(uint32_t byte) {
   asm("{ .reg .b8 t; cvt.u8.u32 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }" : "=r"(h2) : "r"(byte));
   __half2 h = *reinterpret_cast<__half2*>(&h2);
   return __half22float2(h);
+}
+
+// E2M3 (FP6) codes of two values, round to nearest even, satfinite; each code in the low six
+// bits of a byte: sign << 5 | exponent << 3 | mantissa. Result: a in bits 8..13, b in 0..5.
+// Below 1 in magnitude E2M3 is subnormal with a uniform step of 1/8, so for |x| <= 7/8 the code
+// is sign << 5 | RNE(8 |x|) (ties to the even integer, the sign of zero kept).
+__device__ __forceinline__ uint32_t cvt_e2m3x2(float a, float b) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e2m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(a), "f"(b));
+  return r;
 }
 
 // E4M3 (satfinite, round to nearest even) of a non-negative float -> byte.

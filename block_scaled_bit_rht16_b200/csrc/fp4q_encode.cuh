@@ -77,12 +77,7 @@ __device__ __forceinline__ float with_sign_of(float q, float vraw) {
 
 // ------------------------------------------------------------------ lean encoder (hot path)
 //
-// FP32 1x16 scale, round to nearest even, codes only. Per element pair one packed FMA forms
-// t = 1.5 * 2^23 + v / step, whose float rounding is exactly round-half-even of v / step and
-// whose low four bits are that integer in two's complement. Funnel shifts pack the low nibbles
-// of eight such words (discarding the rest); E1M2 then turns the two's complement nibbles into
-// sign-magnitude with word-wide integer operations and takes each sign bit from the rotated
-// value itself (so a negative value that rounds to zero keeps its sign).
+// FP32 1x16 scale, round to nearest even, codes only.
 
 // Exact RN(a / qmax) for the grid's compile-time qmax: one multiply and two FMAs (the same
 // correction step as the element quotients, with the divisor's correctly rounded reciprocal
@@ -108,80 +103,85 @@ __device__ __forceinline__ uint32_t pack_low_nibbles(const uint32_t* t) {
   return w;
 }
 
-// Sign bits of f[0..7] at bit 4i+3.
-__device__ __forceinline__ uint32_t pack_signs(const float* f) {
-  uint32_t w = 0u;
-#pragma unroll
-  for (int i = 7; i >= 0; --i) w = __funnelshift_l(__float_as_uint(f[i]), w, 4);
-  return w & 0x88888888u;
-}
-
-// Two's complement nibbles (-7..7) -> magnitudes 0..7 in the same nibbles.
-__device__ __forceinline__ uint32_t nibble_magnitudes(uint32_t w) {
-  const uint32_t neg = (w >> 3) & 0x11111111u;
-  return (w ^ (neg * 15u)) + neg;
-}
-
-// Codes of one block on E1M2 / INT4 / E2M1 from the rotated raw values P (y = cinv * P) with
-// block scale s (already known nonzero or zero). Returns the two code words.
-template <int G>
-__device__ __forceinline__ uint2 encode_lean(const float2* P, float s, const Divider& dv,
-                                             float cinv) {
+// Codes of one block on E1M2 / INT4 / E2M1 from the (rotated) raw values P, y = P / c with
+// c = 4 under rotation and 1 without, and the block scale s. Returns the two code words.
+//
+// Signs: the element quotients carry the sign of P except for P = -0, where the correction step
+// returns +0. Under rotation a butterfly output is -0 only when all sixteen inputs are zeros,
+// i.e. in an all-zero block, which encodes as zeros anyway; without rotation the sign is copied
+// from P explicitly.
+//   E2M1: hardware round-to-nearest-even conversion of v (saturating at 6).
+//   E1M2: the FP6 E2M3 conversion of v/4: |v/4| <= 7/8 lies in E2M3's subnormal range, whose
+//         step 1/8 makes the code sign << 5 | RNE(2|v|) -- the E1M2 magnitude -- with ties to
+//         even and the sign of zero kept; a SIMD step moves the sign to bit 3 and pairs nibbles.
+//   INT4: t = 1.5 * 2^23 + v rounds v half-to-even into t's low bits in two's complement.
+template <int G, bool RHT>
+__device__ __forceinline__ uint2 encode_lean(const float2* P, float s) {
   if (s == 0.0f) return make_uint2(0u, 0u);
   constexpr float qmax = GridInfo<G>::qmax;
+  constexpr float kC = RHT ? 4.0f : 1.0f;
+  constexpr float kVScale = (G == kE1M2) ? 4.0f : 1.0f;   // quotients of v / kVScale
+  const Divider dv = make_divider(s, kC * kVScale);
   float2 Q[8];
   if (dv.fast) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) Q[i] = div2(dv, P[i]);
   } else {
-    // block scale outside the exact range of the correction step (tiny or huge data):
-    // IEEE division, then the saturation the fast range never needs
+    // scale outside the exact range of the correction step (tiny or huge data): IEEE division,
+    // then the saturation that the fast range never needs
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float qx = __fdiv_rn(__fmul_rn(P[i].x, cinv), s);
-      const float qy = __fdiv_rn(__fmul_rn(P[i].y, cinv), s);
-      Q[i] = make_float2(fminf(fmaxf(qx, -qmax), qmax), fminf(fmaxf(qy, -qmax), qmax));
+      const float qx = __fdiv_rn(__fmul_rn(P[i].x, 1.0f / kC), s);
+      const float qy = __fdiv_rn(__fmul_rn(P[i].y, 1.0f / kC), s);
+      Q[i] = make_float2(__fmul_rn(fminf(fmaxf(qx, -qmax), qmax), 1.0f / kVScale),
+                         __fmul_rn(fminf(fmaxf(qy, -qmax), qmax), 1.0f / kVScale));
     }
   }
+  if constexpr (!RHT && G != kINT4) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      Q[i] = make_float2(with_sign_of(Q[i].x, P[i].x), with_sign_of(Q[i].y, P[i].y));
+  }
+  uint32_t w[2];
   if constexpr (G == kE2M1) {
-    uint32_t w[2];
 #pragma unroll
     for (int l = 0; l < 2; ++l) {
       uint32_t b[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float lo = l ? with_sign_of(Q[2 * j].y, P[2 * j].y) : with_sign_of(Q[2 * j].x, P[2 * j].x);
-        const float hi = l ? with_sign_of(Q[2 * j + 1].y, P[2 * j + 1].y)
-                           : with_sign_of(Q[2 * j + 1].x, P[2 * j + 1].x);
+        const float lo = l ? Q[2 * j].y : Q[2 * j].x, hi = l ? Q[2 * j + 1].y : Q[2 * j + 1].x;
         b[j] = cvt_e2m1x2(hi, lo);
       }
       w[l] = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
     }
-    return make_uint2(w[0], w[1]);
+  } else if constexpr (G == kE1M2) {
+#pragma unroll
+    for (int l = 0; l < 2; ++l) {
+      uint32_t x[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {   // elements 4h .. 4h+3 of this word
+        const int j = 2 * h;
+        const float e0 = l ? Q[2 * j].y : Q[2 * j].x, e1 = l ? Q[2 * j + 1].y : Q[2 * j + 1].x;
+        const float e2 = l ? Q[2 * j + 2].y : Q[2 * j + 2].x, e3 = l ? Q[2 * j + 3].y : Q[2 * j + 3].x;
+        const uint32_t W = cvt_e2m3x2(e1, e0) | (cvt_e2m3x2(e3, e2) << 16);   // byte k = code k
+        const uint32_t N = W - 3u * ((W & 0x20202020u) >> 2);                  // sign to bit 3
+        x[h] = N + (N >> 4);                                                    // bytes 0, 2: pairs
+      }
+      w[l] = __byte_perm(x[0], x[1], 0x6420);
+    }
   } else {
-    constexpr float inv_step = (G == kE1M2) ? 2.0f : 1.0f;
-    const float2 m2 = make_float2(inv_step, inv_step);
     const float2 c2 = make_float2(12582912.0f, 12582912.0f);   // 1.5 * 2^23
     uint32_t t0[8], t1[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float2 t = __ffma2_rn(Q[i], m2, c2);
+      const float2 t = __fadd2_rn(Q[i], c2);
       t0[i] = __float_as_uint(t.x);
       t1[i] = __float_as_uint(t.y);
     }
-    uint32_t w0 = pack_low_nibbles(t0), w1 = pack_low_nibbles(t1);
-    if constexpr (G == kE1M2) {
-      float v0[8], v1[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        v0[i] = P[i].x;
-        v1[i] = P[i].y;
-      }
-      w0 = nibble_magnitudes(w0) | pack_signs(v0);
-      w1 = nibble_magnitudes(w1) | pack_signs(v1);
-    }
-    return make_uint2(w0, w1);
+    w[0] = pack_low_nibbles(t0);
+    w[1] = pack_low_nibbles(t1);
   }
+  return make_uint2(w[0], w[1]);
 }
 
 // ------------------------------------------------------------------ statistics accumulator

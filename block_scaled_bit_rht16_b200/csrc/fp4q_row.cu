@@ -278,113 +278,34 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantArgs a) {
   if constexpr (STATS) stats_finish(acc, a.partials);
 }
 
-// The hot path: FP32 1x16 scale, round to nearest even, codes and scales only.
-template <int G>
+// The hot path: FP32 1x16 scale, round to nearest even, codes and scales only. FLAT: the
+// tensor is contiguous and 32-byte aligned, so unit u is the 32 bytes at 32u (one 256-bit load).
+// Each thread keeps two blocks in flight; with 4+ resident CTAs per SM that saturates HBM.
+template <int G, bool RHT, bool FLAT>
 __global__ void __launch_bounds__(kThreads) lean_kernel(const QuantArgs a) {
-  const bool vec32 = a.vec32 != 0;
+  constexpr float kCinv = RHT ? 0.25f : 1.0f;
+  const uint32_t zero_sw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < a.nunits; u += 2 * stride) {
     uint4 lo[2], hi[2];
     const int64_t uu[2] = {u, u + stride};
     const bool has2 = uu[1] < a.nunits;
-    load16(a.x + unit_offset(a, uu[0], 16), vec32, lo[0], hi[0]);
-    if (has2) load16(a.x + unit_offset(a, uu[1], 16), vec32, lo[1], hi[1]);
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       if (k == 1 && !has2) break;
-      const int64_t un = uu[k];
-      float2 P[8];
-      unpack16(lo[k], hi[k], a.sw, P);
-      rotate_if(a, P);
-      const float s = div_qmax<G>(__fmul_rn(absmax16(P), a.cinv));
-      const Divider dv = make_divider(s, a.c);
-      const uint2 w = encode_lean<G>(P, s, dv, a.cinv);
-      __stcs(reinterpret_cast<uint2*>(a.codes) + un, w);
-      __stcs(reinterpret_cast<float*>(a.scales) + un, s);
+      if constexpr (FLAT) load16(a.x + uu[k] * 16, true, lo[k], hi[k]);
+      else load16(a.x + unit_offset(a, uu[k], 16), a.vec32 != 0, lo[k], hi[k]);
     }
-  }
-}
-
-// The hot path for contiguous tensors: a 4-stage ring of 8 KiB shared-memory stages filled by
-// bulk copies (one per 256 blocks of 16 elements). Thread 0 issues the copies and refills a
-// stage once all 256 threads have released it (mbarrier full/empty pairs); every thread
-// encodes one block per stage. Loads never occupy registers, so each CTA keeps up to 32 KiB
-// in flight regardless of occupancy.
-constexpr int kStages = 4;
-constexpr int kChunkBytes = kThreads * 32;
-
-template <int G>
-__global__ void __launch_bounds__(kThreads) lean_tma_kernel(const QuantArgs a) {
-  __shared__ __align__(128) uint8_t stage[kStages][kChunkBytes];
-  __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
-  const int t = threadIdx.x;
-  const int64_t nchunks = (a.nunits + kThreads - 1) / kThreads;
-  const uint8_t* xb = reinterpret_cast<const uint8_t*>(a.x);
-  auto issue = [&](int64_t c, int s) {
-    const int64_t u0 = c * kThreads;
-    const uint32_t bytes = (uint32_t)(min((int64_t)kThreads, a.nunits - u0) * 32);
-    mbar_arrive_expect_tx(&full[s], bytes);
-    bulk_load(stage[s], xb + u0 * 32, bytes, &full[s]);
-  };
-  if (t == 0) {
 #pragma unroll
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kThreads);
-    }
-    fence_mbar_init();
-  }
-  __syncthreads();
-  if (t == 0) {
-#pragma unroll
-    for (int s = 0; s < kStages; ++s) {
-      const int64_t c = blockIdx.x + (int64_t)s * gridDim.x;
-      if (c < nchunks) issue(c, s);
-    }
-  }
-  bool ok = true;
-  int64_t k = 0;
-  for (;; ++k) {
-    const int64_t c = blockIdx.x + k * gridDim.x;
-    if (c >= nchunks) break;
-    const int s = (int)(k % kStages);
-    const uint32_t par = (uint32_t)((k / kStages) & 1);
-    if (!mbar_wait(&full[s], par)) {
-      ok = false;
-      break;
-    }
-    const int64_t u = c * kThreads + t;
-    if (u < a.nunits) {
-      const uint4* src = reinterpret_cast<const uint4*>(stage[s] + 32 * t);
+    for (int k = 0; k < 2; ++k) {
+      if (k == 1 && !has2) break;
       float2 P[8];
-      unpack16(src[0], src[1], a.sw, P);
-      rotate_if(a, P);
-      const float sc = div_qmax<G>(__fmul_rn(absmax16(P), a.cinv));
-      const Divider dv = make_divider(sc, a.c);
-      const uint2 w = encode_lean<G>(P, sc, dv, a.cinv);
-      __stcs(reinterpret_cast<uint2*>(a.codes) + u, w);
-      __stcs(reinterpret_cast<float*>(a.scales) + u, sc);
-    }
-    mbar_arrive(&empty[s]);
-    if (t == 0) {
-      const int64_t cn = c + (int64_t)kStages * gridDim.x;
-      if (cn < nchunks) {
-        if (!mbar_wait(&empty[s], par)) {
-          ok = false;
-          break;
-        }
-        issue(cn, s);
-      }
-    }
-  }
-  if (!ok) {
-    atomicOr(&g_device_status, kStatusWaitTimeout);
-    // let copies this CTA issued and nobody consumed land before its shared memory goes away
-    if (t == 0) {
-      for (int64_t j = k; j < k + kStages; ++j) {
-        const int64_t cj = blockIdx.x + j * gridDim.x;
-        if (cj < nchunks) mbar_wait(&full[j % kStages], (uint32_t)((j / kStages) & 1), 100000000ull);
-      }
+      unpack16(lo[k], hi[k], RHT ? a.sw : zero_sw, P);
+      if constexpr (RHT) fwht16(P);
+      const float s = div_qmax<G>(__fmul_rn(absmax16(P), kCinv));
+      const uint2 w = encode_lean<G, RHT>(P, s);
+      __stcs(reinterpret_cast<uint2*>(a.codes) + uu[k], w);
+      __stcs(reinterpret_cast<float*>(a.scales) + uu[k], s);
     }
   }
 }
@@ -546,6 +467,11 @@ __global__ void __launch_bounds__(kThreads) division_check_kernel(uint64_t seed,
     else { got = div_qmax<kINT4>(a); want = __fdiv_rn(a, 7.0f); }
     if (__float_as_uint(got) != __float_as_uint(want)) ++local;
   }
+  // the block reciprocal: every float S in [2^-60, 2^91) (151 binades x 2^23 mantissas)
+  for (uint64_t i = (uint64_t)blockIdx.x * kThreads + threadIdx.x; i < (151ull << 23); i += stride) {
+    const float S = __uint_as_float(((uint32_t)(67 + (i >> 23)) << 23) | (uint32_t)(i & 0x7FFFFFu));
+    if (__float_as_uint(rcp_rn_fast(S)) != __float_as_uint(__frcp_rn(S))) ++local;
+  }
   for (uint64_t i = (uint64_t)blockIdx.x * kThreads + threadIdx.x; i < n; i += stride) {
     const uint64_t h = splitmix64(seed ^ (i * 0x9E3779B97F4A7C15ull));
     const uint64_t g = splitmix64(h);
@@ -626,17 +552,18 @@ cudaError_t launch_q_round(int round, bool stats, const QuantArgs& a, cudaStream
 
 }  // namespace
 
+template <int G, bool RHT, bool FLAT>
+cudaError_t launch_lean3(const QuantArgs& a, cudaStream_t st) {
+  auto k = lean_kernel<G, RHT, FLAT>;
+  k<<<persistent_grid(k, (a.nunits + 1) / 2), kThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
 template <int G>
 cudaError_t launch_lean(const QuantArgs& a, cudaStream_t st) {
-  if (a.contiguous) {
-    auto k = lean_tma_kernel<G>;
-    const int64_t chunks = (a.nunits + kThreads - 1) / kThreads;
-    k<<<(int)std::min<int64_t>(chunks, resident_ctas(k)), kThreads, 0, st>>>(a);
-  } else {
-    auto k = lean_kernel<G>;
-    k<<<persistent_grid(k, (a.nunits + 1) / 2), kThreads, 0, st>>>(a);
-  }
-  return cudaGetLastError();
+  const bool rht = a.c != 1.0f, flat = a.contiguous && a.vec32;
+  if (rht) return flat ? launch_lean3<G, true, true>(a, st) : launch_lean3<G, true, false>(a, st);
+  return flat ? launch_lean3<G, false, true>(a, st) : launch_lean3<G, false, false>(a, st);
 }
 
 cudaError_t launch_quantize(int grid, int scale, int round, bool stats, const QuantArgs& a,

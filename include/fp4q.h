@@ -200,10 +200,12 @@ fp4q_status fp4q_rht16(const void* x, int64_t rows, int64_t cols, int64_t ld, ui
 
 /* Diagnostic: checks the kernels' exact-quotient steps (one correctly rounded reciprocal plus
  * an FMA correction, after P. Markstein, IBM J. Res. Dev. 34(1), 1990) against IEEE division:
- * the scale quotient a / qmax for every mantissa of a in [1, 4) and qmax in {6, 3.5, 7}, and
- * the element quotient y / s on `n` pseudo-random pairs from `seed` with s in [2^-60, 2^90) and
- * |y/s| in [2^-20, 8), with and without the folded rotation normalisation. Writes the number
- * of quotients that differ in any bit to the device counter *mismatches (zeroed first). */
+ * the scale quotient a / qmax for every mantissa of a in [1, 4) and qmax in {6, 3.5, 7}; the
+ * block reciprocal (hardware approximation + one Newton-Raphson step) for every float in
+ * [2^-60, 2^91); and the element quotient y / s on `n` pseudo-random pairs from `seed` with s in
+ * [2^-60, 2^90) and |y/s| in [2^-20, 8), with and without the folded rotation normalisation.
+ * Writes the number of results that differ in any bit to the device counter *mismatches
+ * (zeroed first). */
 fp4q_status fp4q_check_division(uint64_t seed, uint64_t n, unsigned long long* mismatches,
                                 fp4q_stream_t stream);
 
