@@ -220,24 +220,28 @@ class RowWorkload(Workload):
         from dataclasses import replace
         return replace(self.cfg, rht=0, sign_mask=0)
 
-    # e2e through the public API with host buffers
+    # e2e through the public API with host buffers (device sets 0 and 1 double-buffer)
     def e2e_setup(self, device):
         import torch
         self.h_in = torch.from_numpy(self.host_bits.view("int16")).view(torch.bfloat16).pin_memory()
-        x, out, _ = self.sets[0]
-        self.h_codes = torch.empty(out.codes.shape, dtype=out.codes.dtype).pin_memory()
-        self.h_scales = torch.empty(out.scales.shape, dtype=out.scales.dtype).pin_memory()
-        return self.h_in.numel() * 2, self.h_codes.numel() + self.h_scales.numel() * self.h_scales.element_size()
+        self.h_out = []
+        for b in range(2):
+            _, out, _ = self.sets[b]
+            self.h_out.append([torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (out.codes, out.scales)])
+        return self.h_in.numel() * 2, sum(t.numel() * t.element_size() for t in self.h_out[0])
 
-    def e2e_step(self, stream):
-        import torch
-        x, out, _ = self.sets[0]
-        with torch.cuda.stream(stream):
-            x.copy_(self.h_in, non_blocking=True)
-            self.fq.rht_quantize(self.cfg, x, out=out, tensor_scale=out.tensor_scale,
-                                 tensor_scale_given=self.given, stream=stream)
-            self.h_codes.copy_(out.codes, non_blocking=True)
-            self.h_scales.copy_(out.scales, non_blocking=True)
+    def e2e_h2d(self, b):
+        self.sets[b][0].copy_(self.h_in, non_blocking=True)
+
+    def e2e_compute(self, b, stream):
+        x, out, _ = self.sets[b]
+        self.fq.rht_quantize(self.cfg, x, out=out, tensor_scale=out.tensor_scale,
+                             tensor_scale_given=self.given, stream=stream)
+
+    def e2e_d2h(self, b):
+        _, out, _ = self.sets[b]
+        for h, d in zip(self.h_out[b], (out.codes, out.scales)):
+            h.copy_(d, non_blocking=True)
 
 
 class DualWorkload(Workload):
@@ -280,19 +284,24 @@ class DualWorkload(Workload):
     def e2e_setup(self, device):
         import torch
         self.h_in = torch.from_numpy(self.host_bits.view("int16")).view(torch.bfloat16).pin_memory()
-        x, out = self.sets[0]
-        self.h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory()
-                      for t in (out.codes_row, out.scales_row, out.codes_col, out.scales_col)]
-        return self.h_in.numel() * 2, sum(t.numel() * t.element_size() for t in self.h_out)
+        self.h_out = []
+        for b in range(2):
+            _, out = self.sets[b]
+            self.h_out.append([torch.empty(t.shape, dtype=t.dtype).pin_memory()
+                               for t in (out.codes_row, out.scales_row, out.codes_col, out.scales_col)])
+        return self.h_in.numel() * 2, sum(t.numel() * t.element_size() for t in self.h_out[0])
 
-    def e2e_step(self, stream):
-        import torch
-        x, out = self.sets[0]
-        with torch.cuda.stream(stream):
-            x.copy_(self.h_in, non_blocking=True)
-            self.fq.quantize_dual(self.rc, self.cc, x, out=out, stream=stream)
-            for h, d in zip(self.h_out, (out.codes_row, out.scales_row, out.codes_col, out.scales_col)):
-                h.copy_(d, non_blocking=True)
+    def e2e_h2d(self, b):
+        self.sets[b][0].copy_(self.h_in, non_blocking=True)
+
+    def e2e_compute(self, b, stream):
+        x, out = self.sets[b]
+        self.fq.quantize_dual(self.rc, self.cc, x, out=out, stream=stream)
+
+    def e2e_d2h(self, b):
+        _, out = self.sets[b]
+        for h, d in zip(self.h_out[b], (out.codes_row, out.scales_row, out.codes_col, out.scales_col)):
+            h.copy_(d, non_blocking=True)
 
 
 def make_workload(name):
@@ -353,42 +362,28 @@ def make_workload(name):
 
 # ---------------------------------------------------------------------------- timing (ours)
 
-def time_graph(wl, steps, warmup, stream, per_launch_events=True):
-    """Warm up, capture a graph of G steps (with per-step event pairs), replay it to run exactly
-    `steps` steps. Returns (total_ms, per_step_kernel_ms or None)."""
+def time_graph(wl, steps, warmup, stream):
+    """Warm up, then capture a graph of G steps that the timed region replays (nothing between
+    the launches) and one with the remaining steps. Returns (g_main, g_rem, full_replays)."""
     import torch
     for i in range(warmup):
         wl.enqueue(i, stream)
     torch.cuda.synchronize()
     G = wl.R * max(1, min(steps, 64 * wl.R) // wl.R) if steps >= wl.R else steps
     full, rem = divmod(steps, G)
-    def ev():
-        try:   # an event recorded as a node of the captured graph
-            return torch.cuda.Event(enable_timing=True, external=True)
-        except TypeError:
-            return torch.cuda.Event(enable_timing=True)
-    evs = [(ev(), ev()) for _ in range(G)]
 
-    def capture(n, with_events):
+    def capture(n):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for i in range(n):
-                if with_events:
-                    evs[i][0].record(stream)
                 wl.enqueue(i, stream)
-                if with_events:
-                    evs[i][1].record(stream)
         return g
 
-    try:
-        g_main = capture(G, per_launch_events)
-    except Exception:
-        per_launch_events = False
-        g_main = capture(G, False)
-    g_rem = capture(rem, False) if rem else None
+    g_main = capture(G)
+    g_rem = capture(rem) if rem else None
     g_main.replay()
     torch.cuda.synchronize()
-    return g_main, g_rem, full, evs if per_launch_events else None
+    return g_main, g_rem, full
 
 
 def run_ours(args):
@@ -409,7 +404,7 @@ def run_ours(args):
     wl = make_workload(args.workload)
     wl.setup(dev, l2)
     stream = torch.cuda.Stream(device=dev)
-    g_main, g_rem, full, evs = time_graph(wl, args.steps, args.warmup, stream)
+    g_main, g_rem, full = time_graph(wl, args.steps, args.warmup, stream)
 
     sampler = ClockSampler("GPU-" + str(props.uuid)) if rank == 0 else None
     if sampler:
@@ -439,25 +434,21 @@ def run_ours(args):
     bytes_step = wl.bytes_per_step()
     value = world * bytes_step / (ms_per_step * 1e-3) / 1e9
 
-    kernel_ms = None
-    if evs is not None:
-        try:
-            kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-        except Exception:
-            kernel_ms = None
+    # per-launch duration: CUDA events around the timed region (launching stream) / launches
+    launch_ms = ms / (args.steps * wl.launches_per_step)
     peak, peak_src = hbm_peak()
-    achieved = bytes_step / wl.launches_per_step / ((kernel_ms if kernel_ms else ms_per_step) * 1e-3) / 1e9
+    achieved = bytes_step / wl.launches_per_step / (launch_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": profiled_traffic(wl.kernel_key),
                 "kernel": wl.kernel_key, "peak_source": peak_src,
-                "kernel_us": round((kernel_ms or ms_per_step) * 1e3, 3),
+                "launch_us": round(launch_ms * 1e3, 3),
                 "algorithmic_bytes_per_launch": bytes_step / wl.launches_per_step}
 
     extras = {}
     if not args.no_extras:
         extras["e2e"] = measure_e2e(wl, stream, world)
         if args.workload == "c2":
-            extras["ratios"] = measure_ratios(args, stream, dev, l2, kernel_ms or ms_per_step)
+            extras["ratios"] = measure_ratios(args, stream, dev, l2, ms_per_step)
     del g_main, g_rem
     if world > 1:
         dist.barrier()
@@ -470,7 +461,8 @@ def run_ours(args):
                    "algorithmic_bytes_per_step": bytes_step,
                    "l2": "rotating %d input/output sets (%.0f MiB total > 2x L2 of %.0f MiB)"
                          % (wl.R, wl.R * wl.set_bytes() / 2**20, l2 / 2**20),
-                   "launch": "CUDA graph replay, %d launch(es) per step" % wl.launches_per_step,
+                   "launch": "CUDA graph replay, %d launch(es) per step, programmatic dependent "
+                             "launch between steps" % wl.launches_per_step,
                    "parallelism": "dp%d (independent rows per rank, no collective)" % world},
         "hbm_frac": round(value / world / peak, 4),
         "roofline": roofline,
@@ -489,26 +481,54 @@ def run_ours(args):
 
 
 def measure_e2e(wl, stream, world, steps=30):
-    """Same metric through the public API with pinned host buffers: H2D copy of the step's
-    inputs, the quantize call, D2H copy of codes and scales, all inside the timed region."""
+    """Same metric through the public API with pinned host buffers: every step copies its
+    inputs host->device, quantizes, and copies codes and scales device->host, all inside the
+    timed region. Steps are pipelined over two device buffer sets: the upload of step i+1 and
+    the download of step i run on their own streams while step i+1 computes."""
     import torch
-    h2d, d2h = wl.e2e_setup(stream.device)
-    for _ in range(3):
-        wl.e2e_step(stream)
+    dev = stream.device
+    h2d, d2h = wl.e2e_setup(dev)
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    loaded = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    unloaded = [torch.cuda.Event() for _ in range(2)]
+    for e in computed + unloaded:
+        e.record(stream)
+
+    def step(i):
+        b = i % 2
+        s_in.wait_event(computed[b])        # the compute that last read set b is done
+        with torch.cuda.stream(s_in):
+            wl.e2e_h2d(b)
+            loaded[b].record(s_in)
+        stream.wait_event(loaded[b])
+        stream.wait_event(unloaded[b])      # the download that last read set b's outputs is done
+        wl.e2e_compute(b, stream)
+        computed[b].record(stream)
+        s_out.wait_event(computed[b])
+        with torch.cuda.stream(s_out):
+            wl.e2e_d2h(b)
+            unloaded[b].record(s_out)
+
+    for i in range(4):
+        step(i)
     torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        wl.e2e_step(stream)
-    b.record(stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(s_in)
+    stream.wait_event(t0)
+    s_out.wait_event(t0)
+    for i in range(steps):
+        step(i)
+    s_out.wait_event(computed[(steps - 1) % 2])
+    t1.record(s_out)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / steps
+    ms = t0.elapsed_time(t1) / steps
     return {"value": round(world * wl.bytes_per_step() / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "ms_per_step": round(ms, 4)}
+            "ms_per_step": round(ms, 4), "pipelined": "upload, compute, download on 3 streams"}
 
 
-def measure_ratios(args, stream, dev, l2, fused_kernel_ms):
+def measure_ratios(args, stream, dev, l2, fused_step_ms):
     """Time relative to quantize-only (rotation off), as the UFP4 pages report it: fused and
     unfused (rotation pass to bf16, then quantize-only), kernel time per step."""
     out = {}
@@ -517,7 +537,7 @@ def measure_ratios(args, stream, dev, l2, fused_kernel_ms):
         wl = make_workload(name)
         wl.setup(dev, l2)
         steps = 64 * wl.R
-        g, _, _, evs = time_graph(wl, steps, 20, stream)
+        g, _, _ = time_graph(wl, steps, 20, stream)
         g.replay()
         import torch
         torch.cuda.synchronize()
@@ -532,7 +552,7 @@ def measure_ratios(args, stream, dev, l2, fused_kernel_ms):
         torch.cuda.empty_cache()
     qo = per["c2-quant-only"]
     out["quant_only_us_per_step"] = round(qo * 1e3, 3)
-    out["fused_over_quant_only"] = round(fused_kernel_ms / qo, 4)
+    out["fused_over_quant_only"] = round(fused_step_ms / qo, 4)
     out["unfused_over_quant_only"] = round(per["c2-unfused"] / qo, 4)
     out["pages_sm100"] = {"fused": 1.07, "unfused": 1.41}
     return out

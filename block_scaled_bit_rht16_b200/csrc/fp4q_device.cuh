@@ -184,6 +184,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+//
+// Quantize kernels are launched with programmatic stream serialization: the next kernel in the
+// stream may become resident while this one drains. Each kernel first lets its dependents
+// launch, then waits for its own prerequisite grid to complete (and its memory to be visible)
+// before touching global memory, so stream order is preserved for inputs and outputs alike.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.launch_dependents;" :::);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ bulk copies and barriers
 //
 // Global -> shared bulk copies (cp.async.bulk, no multicast) complete on an mbarrier with a

@@ -184,6 +184,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantArgs a) {
   constexpr float qmax = GridInfo<G>::qmax;
   constexpr int kUnit = (S == kUE8M0) ? 32 : 16;
   constexpr int kVec = kUnit / 8;   // 16-byte loads per unit
+  pdl_enter();
 
   float alpha = 0.0f, denom = 0.0f;
   if constexpr (S == kE4M3) {
@@ -280,33 +281,35 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantArgs a) {
 
 // The hot path: FP32 1x16 scale, round to nearest even, codes and scales only. FLAT: the
 // tensor is contiguous and 32-byte aligned, so unit u is the 32 bytes at 32u (one 256-bit load).
-// Each thread keeps two blocks in flight; with 4+ resident CTAs per SM that saturates HBM.
+// Each thread encodes one block per iteration while the load of its next block is in flight.
+template <int G, bool RHT, bool FLAT>
+__device__ __forceinline__ void lean_load(const QuantArgs& a, int64_t u, uint4& lo, uint4& hi) {
+  if constexpr (FLAT) load16(a.x + u * 16, true, lo, hi);
+  else load16(a.x + unit_offset(a, u, 16), a.vec32 != 0, lo, hi);
+}
+
 template <int G, bool RHT, bool FLAT>
 __global__ void __launch_bounds__(kThreads) lean_kernel(const QuantArgs a) {
   constexpr float kCinv = RHT ? 0.25f : 1.0f;
   const uint32_t zero_sw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  pdl_enter();
   const int64_t stride = (int64_t)gridDim.x * kThreads;
-  for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < a.nunits; u += 2 * stride) {
-    uint4 lo[2], hi[2];
-    const int64_t uu[2] = {u, u + stride};
-    const bool has2 = uu[1] < a.nunits;
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      if (k == 1 && !has2) break;
-      if constexpr (FLAT) load16(a.x + uu[k] * 16, true, lo[k], hi[k]);
-      else load16(a.x + unit_offset(a, uu[k], 16), a.vec32 != 0, lo[k], hi[k]);
-    }
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      if (k == 1 && !has2) break;
-      float2 P[8];
-      unpack16(lo[k], hi[k], RHT ? a.sw : zero_sw, P);
-      if constexpr (RHT) fwht16(P);
-      const float s = div_qmax<G>(__fmul_rn(absmax16(P), kCinv));
-      const uint2 w = encode_lean<G, RHT>(P, s);
-      __stcs(reinterpret_cast<uint2*>(a.codes) + uu[k], w);
-      __stcs(reinterpret_cast<float*>(a.scales) + uu[k], s);
-    }
+  int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (u >= a.nunits) return;
+  uint4 lo, hi;
+  lean_load<G, RHT, FLAT>(a, u, lo, hi);
+  for (; u < a.nunits; u += stride) {
+    uint4 nlo = lo, nhi = hi;
+    if (u + stride < a.nunits) lean_load<G, RHT, FLAT>(a, u + stride, nlo, nhi);
+    float2 P[8];
+    unpack16(lo, hi, RHT ? a.sw : zero_sw, P);
+    if constexpr (RHT) fwht16(P);
+    const float s = div_qmax<G>(__fmul_rn(absmax16(P), kCinv));
+    const uint2 w = encode_lean<G, RHT>(P, s);
+    __stcs(reinterpret_cast<uint2*>(a.codes) + u, w);
+    __stcs(reinterpret_cast<float*>(a.scales) + u, s);
+    lo = nlo;
+    hi = nhi;
   }
 }
 
@@ -322,6 +325,7 @@ __global__ void wait_timeout_kernel(unsigned long long limit_ns) {
 // Amax of the rotated tensor: per-warp maximum of the bit patterns (non-negative floats order
 // like unsigned integers), one atomicMax per warp into the workspace header.
 __global__ void __launch_bounds__(kThreads) amax_kernel(const QuantArgs a) {
+  pdl_enter();
   uint32_t m = 0u;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < a.nunits; u += stride) {
@@ -519,6 +523,21 @@ int resident_ctas(K kernel) {
   return n;
 }
 
+// Launch with programmatic stream serialization (the kernels call pdl_enter() first).
+template <class... Args>
+cudaError_t launch_pdl(void (*kernel)(Args...), int grid, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <class K>
 int persistent_grid(K kernel, int64_t work_threads) {
   const int64_t need = (work_threads + kThreads - 1) / kThreads;
@@ -535,8 +554,8 @@ cudaError_t launch_q(const QuantArgs& a, cudaStream_t st) {
     // two units per thread per iteration
     grid = persistent_grid(k, (a.nunits + 1) / 2);
   }
-  k<<<grid, kThreads, 0, st>>>(a);
-  return cudaGetLastError();
+  const cudaError_t e = launch_pdl(k, grid, st, a);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int G, int S, int R>
@@ -555,8 +574,8 @@ cudaError_t launch_q_round(int round, bool stats, const QuantArgs& a, cudaStream
 template <int G, bool RHT, bool FLAT>
 cudaError_t launch_lean3(const QuantArgs& a, cudaStream_t st) {
   auto k = lean_kernel<G, RHT, FLAT>;
-  k<<<persistent_grid(k, (a.nunits + 1) / 2), kThreads, 0, st>>>(a);
-  return cudaGetLastError();
+  const cudaError_t e = launch_pdl(k, persistent_grid(k, a.nunits), st, a);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int G>
@@ -589,8 +608,8 @@ cudaError_t launch_quantize(int grid, int scale, int round, bool stats, const Qu
 }
 
 cudaError_t launch_amax(const QuantArgs& a, cudaStream_t st) {
-  amax_kernel<<<persistent_grid(amax_kernel, a.nunits), kThreads, 0, st>>>(a);
-  return cudaGetLastError();
+  const cudaError_t e = launch_pdl(amax_kernel, persistent_grid(amax_kernel, a.nunits), st, a);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_rht16(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
