@@ -381,7 +381,8 @@ def time_graph(wl, steps, warmup, stream):
 
     g_main = capture(G)
     g_rem = capture(rem) if rem else None
-    g_main.replay()
+    with torch.cuda.stream(stream):
+        g_main.replay()
     torch.cuda.synchronize()
     return g_main, g_rem, full
 
@@ -415,12 +416,13 @@ def run_ours(args):
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(full):
-        g_main.replay()
-    if g_rem is not None:
-        g_rem.replay()
-    t1.record(stream)
+    with torch.cuda.stream(stream):   # graphs replay on the current stream
+        t0.record(stream)
+        for _ in range(full):
+            g_main.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        t1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -538,14 +540,15 @@ def measure_ratios(args, stream, dev, l2, fused_step_ms):
         wl.setup(dev, l2)
         steps = 64 * wl.R
         g, _, _ = time_graph(wl, steps, 20, stream)
-        g.replay()
         import torch
-        torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(20):
+        with torch.cuda.stream(stream):
             g.replay()
-        b.record(stream)
+            torch.cuda.synchronize()
+            a.record(stream)
+            for _ in range(20):
+                g.replay()
+            b.record(stream)
         torch.cuda.synchronize()
         per[name] = a.elapsed_time(b) / (20 * steps)
         del g, wl
