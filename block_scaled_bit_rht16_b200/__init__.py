@@ -151,6 +151,21 @@ def rht_quantize(cfg: Config, x, *, out: Quantized = None, tensor_scale=None,
     return out
 
 
+def tensor_scale(cfg: Config, x, *, out=None, workspace=None, stream=None):
+    """fp4q_tensor_scale: the FP32 tensor scale alpha of x (E4M3 configurations) -> float32[1]."""
+    torch = _torch()
+    rows, cols, ld = _check_input(x)
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(256, dtype=torch.uint8, device=x.device)
+    c = cfg.c()
+    st = _lib.load().fp4q_tensor_scale(ctypes.byref(c), _ptr(x), rows, cols, ld, _ptr(out),
+                                       _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    _lib.check(st, "fp4q_tensor_scale")
+    return out
+
+
 def if4_select(cfg: Config, x, **kw) -> Quantized:
     """fp4q_if4_select: IF4 with NVFP4 scales (grid/scale in cfg are overridden)."""
     return rht_quantize(replace(cfg, grid=FP4Q_GRID_IF4, scale=FP4Q_SCALE_E4M3_1x16_TENSOR), x, **kw)

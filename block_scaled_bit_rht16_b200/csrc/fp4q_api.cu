@@ -155,6 +155,41 @@ fp4q_status fp4q_rht_quantize(const fp4q_config* cfg, const void* x, int64_t row
   return cuda_status(launch_quantize(cfg->grid, cfg->scale, cfg->round, want_stats, a, s));
 }
 
+fp4q_status fp4q_tensor_scale(const fp4q_config* cfg, const void* x, int64_t rows, int64_t cols,
+                              int64_t ld, float* tensor_scale, void* workspace,
+                              size_t workspace_bytes, fp4q_stream_t stream) {
+  fp4q_status st = check_cfg(cfg);
+  if (st != FP4Q_OK) return st;
+  if (cfg->scale != FP4Q_SCALE_E4M3_1x16_TENSOR) return FP4Q_ERR_UNSUPPORTED;
+  st = check_shape(rows, cols, ld, 16);
+  if (st != FP4Q_OK) return st;
+  const bool empty = rows == 0 || cols == 0;
+  if (tensor_scale == nullptr || (!empty && x == nullptr)) return FP4Q_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(tensor_scale, 4) || !aligned(workspace, 256)) return FP4Q_ERR_ALIGN;
+  if (workspace == nullptr || workspace_bytes < sizeof(WsHeader)) return FP4Q_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  WsHeader* ws = reinterpret_cast<WsHeader*>(workspace);
+  if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), s) != cudaSuccess) return FP4Q_ERR_CUDA;
+  if (!empty) {
+    QuantArgs a{};
+    a.x = static_cast<const uint16_t*>(x);
+    a.rows = rows;
+    a.cols = cols;
+    a.ld = ld;
+    a.units_per_row = cols / 16;
+    a.nunits = rows * a.units_per_row;
+    a.ws = ws;
+    sign_words(cfg->sign_mask, cfg->rht != 0, a.sw);
+    a.c = cfg->rht ? 4.0f : 1.0f;
+    a.cinv = cfg->rht ? 0.25f : 1.0f;
+    a.contiguous = (ld == cols) ? 1 : 0;
+    a.vec32 = (reinterpret_cast<uintptr_t>(x) % 32 == 0 && (rows == 1 || ld % 16 == 0)) ? 1 : 0;
+    if (launch_amax(a, s) != cudaSuccess) return FP4Q_ERR_CUDA;
+  }
+  const float qmax = cfg->grid == FP4Q_GRID_INT4 ? 7.0f : (cfg->grid == FP4Q_GRID_E1M2 ? 3.5f : 6.0f);
+  return cuda_status(launch_alpha(ws, qmax, tensor_scale, s));
+}
+
 fp4q_status fp4q_if4_select(const fp4q_config* cfg, const void* x, int64_t rows, int64_t cols,
                             int64_t ld, uint8_t* codes, uint8_t* scales_flagged,
                             float* tensor_scale, int32_t tensor_scale_given, void* dequant,

@@ -66,6 +66,7 @@ constexpr int32_t kStatusSelfTest = 2;
 cudaError_t launch_quantize(int grid, int scale, int round, bool stats, const QuantArgs& a,
                             cudaStream_t st);
 cudaError_t launch_amax(const QuantArgs& a, cudaStream_t st);
+cudaError_t launch_alpha(WsHeader* ws, float qmax, float* tensor_scale, cudaStream_t st);
 cudaError_t launch_rht16(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
                          const uint32_t* sw, void* out, bool out_fp32, cudaStream_t st);
 cudaError_t launch_dequant(int grid, int scale, const uint8_t* codes, const void* scales,

@@ -612,6 +612,15 @@ cudaError_t launch_amax(const QuantArgs& a, cudaStream_t st) {
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
+__global__ void alpha_kernel(const WsHeader* ws, float qmax, float* tensor_scale) {
+  *tensor_scale = __fdiv_rn(__uint_as_float(ws->amax_bits), __fmul_rn(qmax, 448.0f));
+}
+
+cudaError_t launch_alpha(WsHeader* ws, float qmax, float* tensor_scale, cudaStream_t st) {
+  alpha_kernel<<<1, 1, 0, st>>>(ws, qmax, tensor_scale);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_rht16(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
                          const uint32_t* sw, void* out, bool out_fp32, cudaStream_t st) {
   QuantArgs a{};

@@ -185,6 +185,16 @@ fp4q_status fp4q_if4_select(const fp4q_config* cfg, const void* x, int64_t rows,
                             float* tensor_scale, int32_t tensor_scale_given, void* dequant,
                             void* workspace, size_t workspace_bytes, fp4q_stream_t stream);
 
+/* The FP32 tensor scale alone (the first pass of the E4M3 two-level scale [IF4 section 3.2]):
+ * alpha = A / RN(qmax * 448), A the amax of the rotated x (cfg->grid, rht, sign_mask apply).
+ * Writes alpha to the device float *tensor_scale. For a tensor split by rows over ranks, the
+ * global alpha is the maximum of the ranks' alphas (rounding is monotonic), which is then passed
+ * to fp4q_rht_quantize with tensor_scale_given = 1. workspace: fp4q_workspace_size() of an
+ * E4M3 configuration (256 bytes). */
+fp4q_status fp4q_tensor_scale(const fp4q_config* cfg, const void* x, int64_t rows, int64_t cols,
+                              int64_t ld, float* tensor_scale, void* workspace,
+                              size_t workspace_bytes, fp4q_stream_t stream);
+
 /* Reduce the statistics a previous fp4q_rht_quantize / fp4q_if4_select call with
  * FP4Q_OUT_STATS left in `workspace` (in a fixed order, FP64), copy them to *host_out and
  * derive SQNR, alpha, MSE and the per-cell mean error [UFP4-A "E2M1", "复利效应的反向版本",

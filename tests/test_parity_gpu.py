@@ -300,3 +300,27 @@ def test_unfused_pipeline_equals_fused_on_fp32_intermediate():
     _, yref = O.rht16_rows(x, mask)
     ref = O.quantize(ocfg(cfg), yref)
     np.testing.assert_array_equal(host(q.codes), ref["codes"])
+
+
+# ------------------------------------------------------------------ tensor scale alone
+
+@pytest.mark.parametrize("grid", [E2M1, INT4, IF4, E1M2])
+@pytest.mark.parametrize("rht", [0, 1])
+def test_tensor_scale_and_row_shard_maximum(grid, rht):
+    cfg = fq.Config(grid=grid, scale=E4M3, rht=rht, sign_mask=0x6A6A)
+    x = synth.small(90 + grid, 200, 512, "laplace", 2.0)
+    a = host(fq.tensor_scale(cfg, to_dev(x)))[0]
+    qmax = {E2M1: 6.0, INT4: 7.0, IF4: 6.0, E1M2: 3.5}[grid]
+    want = np.float32(O.tensor_amax(ocfg(cfg), x)) / np.float32(qmax * 448)
+    assert a == want
+    # the whole tensor's scale is the maximum of its row shards' scales
+    parts = [host(fq.tensor_scale(cfg, to_dev(np.ascontiguousarray(x[r0:r1]))))[0]
+             for r0, r1 in [(0, 80), (80, 200)]]
+    assert max(parts) == a
+    # and quantizing with that scale given reproduces the computed-scale call
+    full = fq.rht_quantize(cfg, to_dev(x))
+    given = fq.rht_quantize(cfg, to_dev(x), tensor_scale=torch.tensor([a], device="cuda"),
+                            tensor_scale_given=True)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host(full.codes), host(given.codes))
+    np.testing.assert_array_equal(host(full.scales), host(given.scales))
