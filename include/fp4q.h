@@ -195,6 +195,25 @@ fp4q_status fp4q_tensor_scale(const fp4q_config* cfg, const void* x, int64_t row
                               int64_t ld, float* tensor_scale, void* workspace,
                               size_t workspace_bytes, fp4q_stream_t stream);
 
+/* fp4q_rht_quantize for callers that cannot allocate device memory (a runtime's plugin
+ * boundary that hands over only input and output buffers, a host framework that owns all
+ * device memory, or work where cudaMalloc is off limits). The pages have no counterpart: this
+ * is a calling convention of the library, not part of the method.
+ * Same arguments and results as fp4q_rht_quantize without the workspace: the scratch an E4M3
+ * tensor scale computed on the device needs (256 bytes) lives in a static array inside the
+ * library, which every GPU that loads the library keeps until the process exits. A
+ * configuration that needs more scratch than that -- statistics (FP4Q_OUT_STATS) -- is rejected
+ * with FP4Q_ERR_WORKSPACE before anything runs.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call outside any stream capture. All calls share the
+ * one array, which each call clears on its stream before use: calls that can overlap on the GPU
+ * (different streams, or different host threads, on the same device) race on it and must be
+ * ordered by the caller. No allocation happens in this call. */
+fp4q_status fp4q_rht_quantize_noalloc(const fp4q_config* cfg, const void* x, int64_t rows,
+                                      int64_t cols, int64_t ld, uint8_t* codes, void* scales,
+                                      float* tensor_scale, int32_t tensor_scale_given,
+                                      void* dequant, fp4q_stream_t stream);
+
 /* Reduce the statistics a previous fp4q_rht_quantize / fp4q_if4_select call with
  * FP4Q_OUT_STATS left in `workspace` (in a fixed order, FP64), copy them to *host_out and
  * derive SQNR, alpha, MSE and the per-cell mean error [UFP4-A "E2M1", "复利效应的反向版本",
