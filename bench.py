@@ -322,11 +322,11 @@ def make_workload(name):
         if name == "c2-quant-only":
             from dataclasses import replace
             return RowWorkload(name, desc + " -- rotation off (quantize only)", c2_input,
-                               replace(cfg, rht=0, sign_mask=0), "quantize_kernel<E1M2,FP32,RTNE>")
+                               replace(cfg, rht=0, sign_mask=0), "lean_kernel<E1M2,no-rotation,flat>")
         if name == "c2-unfused":
             return RowWorkload(name, desc + " -- unfused: rotation pass to bf16, then quantize",
-                               c2_input, cfg, "rht16_kernel+quantize_kernel", unfused=True)
-        return RowWorkload(name, desc, c2_input, cfg, "quantize_kernel<E1M2,FP32,RTNE>")
+                               c2_input, cfg, "rht16_kernel+lean_kernel", unfused=True)
+        return RowWorkload(name, desc, c2_input, cfg, "lean_kernel<E1M2,rotation,flat>")
     if name == "c3":
         mask = fq.sign_mask_from_seed(synth.sign_seed(3))
         rc = fq.recipe("ufp4", "bwd_dx", "dy", sign_mask=mask, sr_seed=synth.SR_SEED)
@@ -342,7 +342,7 @@ def make_workload(name):
         scale = fq.FP4Q_SCALE_UE8M0_1x32 if kind == "mxfp4" else fq.FP4Q_SCALE_E4M3_1x16_TENSOR
         cfg = fq.Config(grid=grid, scale=scale, rht=1, sign_mask=mask)
         return RowWorkload(name, "[16384,5120] Laplace(0,1), RHT16, %s" % kind, synth.workload4, cfg,
-                           "quantize_kernel<%s>" % kind)
+                           "quantize_kernel<%s>" % kind + ("" if kind in ("mxfp4", "nvfp4-given") else "+amax_kernel"))
     if name.startswith("c5"):
         mask = fq.sign_mask_from_seed(synth.sign_seed(5))
         ufp4 = name.endswith("ufp4")
@@ -356,7 +356,8 @@ def make_workload(name):
                 return synth.workload5_dense_rows(0, 32768)
             desc = "dense [32768,8192] N(0,1)"
         desc += ", %s fwd_y" % ("UFP4 RHT16+E1M2" if ufp4 else "E2M1 baseline (no rotation)")
-        return RowWorkload(name, desc, inp, cfg, "quantize_kernel")
+        return RowWorkload(name, desc, inp, cfg, "lean_kernel<%s,%s,flat>" % ("E1M2" if ufp4 else "E2M1",
+                                                                            "rotation" if ufp4 else "no-rotation"))
     raise ValueError(name)
 
 
