@@ -42,9 +42,6 @@ __global__ void __launch_bounds__(kThreads) dual_kernel(const DualArgs a) {
   }
   __syncthreads();
 
-  const EncCtx ctx_row{a.cinv_row, a.seedx_row};
-  const EncCtx ctx_col{a.cinv_col, a.seedx_col};
-
   // row blocks: rows t/4 and t/4 + 64, block t%4 (16 columns)
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
@@ -56,10 +53,10 @@ __global__ void __launch_bounds__(kThreads) dual_kernel(const DualArgs a) {
     unpack16(src[0], src[1], a.sw_row, P);
     if (a.c_row != 1.0f) fwht16(P);
     const float s = div_qmax<G>(__fmul_rn(absmax16(P), a.cinv_row));
-    const Divider dv = make_divider(s, a.c_row);
     const int64_t u = (m * a.N + n) >> 4;   // 16-block index in [M, N/16]
-    encode16<G, RR, false>(ctx_row, P, (uint64_t)u * 8u, a.codes_row + u * 8, nullptr, s, dv,
-                           nullptr);
+    const uint2 w = (RR == kSR) ? encode_sr<G>(P, s, a.c_row, a.seedx_row, (uint64_t)u * 8u)
+                                : encode_rtne_rt<G>(P, s, a.c_row != 1.0f);
+    __stcs(reinterpret_cast<uint2*>(a.codes_row) + u, w);
     __stcs(a.scales_row + u, s);
   }
 
@@ -83,10 +80,10 @@ __global__ void __launch_bounds__(kThreads) dual_kernel(const DualArgs a) {
              a.sw_col, P);
     if (a.c_col != 1.0f) fwht16(P);
     const float s = div_qmax<G>(__fmul_rn(absmax16(P), a.cinv_col));
-    const Divider dv = make_divider(s, a.c_col);
     const int64_t u = (n * a.M + m) >> 4;   // 16-block index in [N, M/16]
-    encode16<G, RC, false>(ctx_col, P, (uint64_t)u * 8u, a.codes_col + u * 8, nullptr, s, dv,
-                           nullptr);
+    const uint2 w = (RC == kSR) ? encode_sr<G>(P, s, a.c_col, a.seedx_col, (uint64_t)u * 8u)
+                                : encode_rtne_rt<G>(P, s, a.c_col != 1.0f);
+    __stcs(reinterpret_cast<uint2*>(a.codes_col) + u, w);
     __stcs(a.scales_col + u, s);
   }
 }

@@ -23,6 +23,9 @@ struct EncCtx {
 
 __device__ __forceinline__ uint32_t sign_bit(float x) { return __float_as_uint(x) >> 31; }
 
+// Element e (0..15) of a block held as P[i] = (v_i, v_{i+8}).
+__device__ __forceinline__ float elem_x(const float2* A, int e) { return e < 8 ? A[e].x : A[e - 8].y; }
+
 // Small exact integer m (0..15) as a float.
 __device__ __forceinline__ float small_int_f32(uint32_t m) {
   return __fadd_rn(__uint_as_float(0x4B000000u | m), -8388608.0f);
@@ -184,6 +187,109 @@ __device__ __forceinline__ uint2 encode_lean(const float2* P, float s) {
   return make_uint2(w[0], w[1]);
 }
 
+// Stochastic rounding, FP32 1x16 scale, codes only; runtime rotation factor c (4 or 1).
+// Element e (0..15) of the block has logical index 2*pair0 + e; pair j = (2j, 2j+1) shares one
+// SplitMix64 output (low half for 2j, high half for 2j+1), keys formed incrementally.
+// Per element: |v| clamped to qmax, t = |v| / step, fl = floor(t), frac = t - fl (all exact);
+// round up iff (u >> 8) < frac * 2^24; the chosen grid point is then encoded exactly like the
+// round-to-nearest path (E1M2 through E2M3 of value/4, E2M1 through its converter, INT4 by the
+// two's complement add), with the sign of the input value.
+template <int G>
+__device__ __forceinline__ uint2 encode_sr(const float2* P, float s, float c, uint64_t seedx,
+                                          uint64_t pair0) {
+  if (s == 0.0f) return make_uint2(0u, 0u);
+  constexpr float qmax = GridInfo<G>::qmax;
+  const float cinv = __frcp_rn(c);   // exact: c is 4 or 1
+  const Divider dv = make_divider(s, c);
+  float q[16];
+  if (dv.fast) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 r = div2(dv, P[i]);
+      q[i] = r.x;
+      q[i + 8] = r.y;
+    }
+    // the correction step is exact for quotients of at least 2^-20; smaller nonzero ones (rare)
+    // decide stochastic rounding through their exact value, so they take the IEEE division
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float pe = elem_x(P, e);
+      if (fabsf(q[e]) < 0x1p-19f && pe != 0.0f) q[e] = __fdiv_rn(__fmul_rn(pe, cinv), s);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) q[e] = __fdiv_rn(__fmul_rn(elem_x(P, e), cinv), s);
+  }
+  uint32_t rnd[16];
+  uint64_t key = pair0 * 0x9E3779B97F4A7C15ull;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint64_t h = splitmix64(seedx ^ key);
+    key += 0x9E3779B97F4A7C15ull;
+    rnd[2 * j] = (uint32_t)h;
+    rnd[2 * j + 1] = (uint32_t)(h >> 32);
+  }
+  // chosen grid point per element, signed like the input value (-0 keeps its sign)
+  float g[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const float a = fminf(fabsf(q[e]), qmax);
+    float mag;
+    if constexpr (G == kE2M1) {
+      const bool lo = a < 2.0f, mid = a < 4.0f;
+      const float inv_step = lo ? 2.0f : (mid ? 1.0f : 0.5f);
+      const float step = lo ? 0.5f : (mid ? 1.0f : 2.0f);
+      const float t = __fmul_rn(a, inv_step);
+      const float fl = floorf(t);
+      const float k = sr_up(rnd[e], __fsub_rn(t, fl)) ? __fadd_rn(fl, 1.0f) : fl;
+      mag = __fmul_rn(k, step);
+    } else {
+      constexpr float inv_step = (G == kE1M2) ? 2.0f : 1.0f;
+      const float t = __fmul_rn(a, inv_step);
+      const float fl = floorf(t);
+      mag = sr_up(rnd[e], __fsub_rn(t, fl)) ? __fadd_rn(fl, 1.0f) : fl;   // integer steps
+    }
+    g[e] = with_sign_of(mag, elem_x(P, e));
+  }
+  uint32_t w[2];
+  if constexpr (G == kE2M1) {
+#pragma unroll
+    for (int l = 0; l < 2; ++l) {
+      uint32_t b[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = cvt_e2m1x2(g[8 * l + 2 * j + 1], g[8 * l + 2 * j]);
+      w[l] = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+    }
+  } else if constexpr (G == kE1M2) {
+#pragma unroll
+    for (int l = 0; l < 2; ++l) {
+      uint32_t x[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int e = 8 * l + 4 * h;   // steps / 8 is the E2M3 subnormal code of value / 4
+        const uint32_t W = cvt_e2m3x2(__fmul_rn(g[e + 1], 0.125f), __fmul_rn(g[e], 0.125f)) |
+                           (cvt_e2m3x2(__fmul_rn(g[e + 3], 0.125f), __fmul_rn(g[e + 2], 0.125f)) << 16);
+        const uint32_t N = W - 3u * ((W & 0x20202020u) >> 2);
+        x[h] = N + (N >> 4);
+      }
+      w[l] = __byte_perm(x[0], x[1], 0x6420);
+    }
+  } else {
+    uint32_t t[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) t[e] = __float_as_uint(__fadd_rn(g[e], 12582912.0f));
+    w[0] = pack_low_nibbles(t);
+    w[1] = pack_low_nibbles(t + 8);
+  }
+  return make_uint2(w[0], w[1]);
+}
+
+// Round-to-nearest codes with a runtime rotation factor (signs always copied from the input).
+template <int G>
+__device__ __forceinline__ uint2 encode_rtne_rt(const float2* P, float s, bool rht) {
+  return rht ? encode_lean<G, true>(P, s) : encode_lean<G, false>(P, s);
+}
+
 // ------------------------------------------------------------------ statistics accumulator
 
 struct StatsAcc {
@@ -202,7 +308,6 @@ struct StatsAcc {
   }
 };
 
-__device__ __forceinline__ float elem_x(const float2* A, int e) { return e < 8 ? A[e].x : A[e - 8].y; }
 
 // Encodes one block. pair0 = (logical index of element 0) / 2 for the SR counter.
 // Returns the IF4 flag (0x80 for an INT4 block, else 0).

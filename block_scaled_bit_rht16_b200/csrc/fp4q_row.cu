@@ -288,7 +288,7 @@ __device__ __forceinline__ void lean_load(const QuantArgs& a, int64_t u, uint4& 
   else load16(a.x + unit_offset(a, u, 16), a.vec32 != 0, lo, hi);
 }
 
-template <int G, bool RHT, bool FLAT>
+template <int G, bool RHT, bool FLAT, int R>
 __global__ void __launch_bounds__(kThreads) lean_kernel(const QuantArgs a) {
   constexpr float kCinv = RHT ? 0.25f : 1.0f;
   const uint32_t zero_sw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
@@ -305,7 +305,9 @@ __global__ void __launch_bounds__(kThreads) lean_kernel(const QuantArgs a) {
     unpack16(lo, hi, RHT ? a.sw : zero_sw, P);
     if constexpr (RHT) fwht16(P);
     const float s = div_qmax<G>(__fmul_rn(absmax16(P), kCinv));
-    const uint2 w = encode_lean<G, RHT>(P, s);
+    uint2 w;
+    if constexpr (R == kSR) w = encode_sr<G>(P, s, RHT ? 4.0f : 1.0f, a.seedx, (uint64_t)u * 8u);
+    else w = encode_lean<G, RHT>(P, s);
     __stcs(reinterpret_cast<uint2*>(a.codes) + u, w);
     __stcs(reinterpret_cast<float*>(a.scales) + u, s);
     lo = nlo;
@@ -571,26 +573,32 @@ cudaError_t launch_q_round(int round, bool stats, const QuantArgs& a, cudaStream
 
 }  // namespace
 
-template <int G, bool RHT, bool FLAT>
+template <int G, bool RHT, bool FLAT, int R>
 cudaError_t launch_lean3(const QuantArgs& a, cudaStream_t st) {
-  auto k = lean_kernel<G, RHT, FLAT>;
+  auto k = lean_kernel<G, RHT, FLAT, R>;
   const cudaError_t e = launch_pdl(k, persistent_grid(k, a.nunits), st, a);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-template <int G>
+template <int G, int R>
 cudaError_t launch_lean(const QuantArgs& a, cudaStream_t st) {
   const bool rht = a.c != 1.0f, flat = a.contiguous && a.vec32;
-  if (rht) return flat ? launch_lean3<G, true, true>(a, st) : launch_lean3<G, true, false>(a, st);
-  return flat ? launch_lean3<G, false, true>(a, st) : launch_lean3<G, false, false>(a, st);
+  if (rht) return flat ? launch_lean3<G, true, true, R>(a, st) : launch_lean3<G, true, false, R>(a, st);
+  return flat ? launch_lean3<G, false, true, R>(a, st) : launch_lean3<G, false, false, R>(a, st);
 }
 
 cudaError_t launch_quantize(int grid, int scale, int round, bool stats, const QuantArgs& a,
                             cudaStream_t st) {
-  if (scale == kFP32 && round == kRTNE && !stats && a.deq == nullptr) {
-    if (grid == kE2M1) return launch_lean<kE2M1>(a, st);
-    if (grid == kE1M2) return launch_lean<kE1M2>(a, st);
-    if (grid == kINT4) return launch_lean<kINT4>(a, st);
+  if (scale == kFP32 && !stats && a.deq == nullptr) {
+    if (round == kSR) {
+      if (grid == kE2M1) return launch_lean<kE2M1, kSR>(a, st);
+      if (grid == kE1M2) return launch_lean<kE1M2, kSR>(a, st);
+      if (grid == kINT4) return launch_lean<kINT4, kSR>(a, st);
+    } else {
+      if (grid == kE2M1) return launch_lean<kE2M1, kRTNE>(a, st);
+      if (grid == kE1M2) return launch_lean<kE1M2, kRTNE>(a, st);
+      if (grid == kINT4) return launch_lean<kINT4, kRTNE>(a, st);
+    }
   }
   if (scale == kFP32) {
     if (grid == kE2M1) return launch_q_round<kE2M1, kFP32>(round, stats, a, st);
