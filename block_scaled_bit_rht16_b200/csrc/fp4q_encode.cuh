@@ -118,7 +118,9 @@ __device__ __forceinline__ uint32_t pack_low_nibbles(const uint32_t* t) {
 //         step 1/8 makes the code sign << 5 | RNE(2|v|) -- the E1M2 magnitude -- with ties to
 //         even and the sign of zero kept; a SIMD step moves the sign to bit 3 and pairs nibbles.
 //   INT4: t = 1.5 * 2^23 + v rounds v half-to-even into t's low bits in two's complement.
-template <int G, bool RHT>
+// CLAMP: saturate |v| at qmax before rounding. The FP32 scale needs none (|v| <= qmax up to an
+// ulp); E4M3 scales do (the rounded block scale, or a given tensor scale, can leave |v| > qmax).
+template <int G, bool RHT, bool CLAMP = false>
 __device__ __forceinline__ uint2 encode_lean(const float2* P, float s) {
   if (s == 0.0f) return make_uint2(0u, 0u);
   constexpr float qmax = GridInfo<G>::qmax;
@@ -129,6 +131,12 @@ __device__ __forceinline__ uint2 encode_lean(const float2* P, float s) {
   if (dv.fast) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) Q[i] = div2(dv, P[i]);
+    if constexpr (CLAMP && G != kE2M1) {   // the E2M1 conversion saturates by itself
+      constexpr float lim = qmax / kVScale;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        Q[i] = make_float2(fminf(fmaxf(Q[i].x, -lim), lim), fminf(fmaxf(Q[i].y, -lim), lim));
+    }
   } else {
     // scale outside the exact range of the correction step (tiny or huge data): IEEE division,
     // then the saturation that the fast range never needs

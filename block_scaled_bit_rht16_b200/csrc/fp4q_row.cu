@@ -324,6 +324,44 @@ __global__ void wait_timeout_kernel(unsigned long long limit_ns) {
   mbar_arrive(&bar);   // complete the phase so the barrier is left consistent
 }
 
+// E4M3 block scale + FP32 tensor scale, round to nearest even, codes and scale bytes only.
+template <int G, bool RHT, bool FLAT>
+__global__ void __launch_bounds__(kThreads) lean_nv_kernel(const QuantArgs a) {
+  constexpr float qmax = GridInfo<G>::qmax;
+  constexpr float kCinv = RHT ? 0.25f : 1.0f;
+  const uint32_t zero_sw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  pdl_enter();
+  float alpha;
+  if (a.ts_in != nullptr) {
+    alpha = *a.ts_in;
+  } else {
+    alpha = __fdiv_rn(__uint_as_float(a.ws->amax_bits), __fmul_rn(qmax, 448.0f));
+    if (a.ts_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *a.ts_out = alpha;
+  }
+  const float denom = __fmul_rn(alpha, qmax);
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (u >= a.nunits) return;
+  uint4 lo, hi;
+  lean_load<G, RHT, FLAT>(a, u, lo, hi);
+  for (; u < a.nunits; u += stride) {
+    uint4 nlo = lo, nhi = hi;
+    if (u + stride < a.nunits) lean_load<G, RHT, FLAT>(a, u + stride, nlo, nhi);
+    float2 P[8];
+    unpack16(lo, hi, RHT ? a.sw : zero_sw, P);
+    if constexpr (RHT) fwht16(P);
+    const float amax_y = __fmul_rn(absmax16(P), kCinv);
+    const float delta = denom > 0.0f ? __fdiv_rn(amax_y, denom) : 0.0f;
+    const uint32_t sbyte = cvt_e4m3(delta);
+    const float s = __fmul_rn(e4m3_to_f32(sbyte), alpha);
+    const uint2 w = encode_lean<G, RHT, true>(P, s);
+    __stcs(reinterpret_cast<uint2*>(a.codes) + u, w);
+    reinterpret_cast<uint8_t*>(a.scales)[u] = (uint8_t)sbyte;
+    lo = nlo;
+    hi = nhi;
+  }
+}
+
 // Amax of the rotated tensor: per-warp maximum of the bit patterns (non-negative floats order
 // like unsigned integers), one atomicMax per warp into the workspace header.
 __global__ void __launch_bounds__(kThreads) amax_kernel(const QuantArgs a) {
@@ -580,6 +618,20 @@ cudaError_t launch_lean3(const QuantArgs& a, cudaStream_t st) {
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
+template <int G, bool RHT, bool FLAT>
+cudaError_t launch_lean_nv3(const QuantArgs& a, cudaStream_t st) {
+  auto k = lean_nv_kernel<G, RHT, FLAT>;
+  const cudaError_t e = launch_pdl(k, persistent_grid(k, a.nunits), st, a);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+template <int G>
+cudaError_t launch_lean_nv(const QuantArgs& a, cudaStream_t st) {
+  const bool rht = a.c != 1.0f, flat = a.contiguous && a.vec32;
+  if (rht) return flat ? launch_lean_nv3<G, true, true>(a, st) : launch_lean_nv3<G, true, false>(a, st);
+  return flat ? launch_lean_nv3<G, false, true>(a, st) : launch_lean_nv3<G, false, false>(a, st);
+}
+
 template <int G, int R>
 cudaError_t launch_lean(const QuantArgs& a, cudaStream_t st) {
   const bool rht = a.c != 1.0f, flat = a.contiguous && a.vec32;
@@ -599,6 +651,11 @@ cudaError_t launch_quantize(int grid, int scale, int round, bool stats, const Qu
       if (grid == kE1M2) return launch_lean<kE1M2, kRTNE>(a, st);
       if (grid == kINT4) return launch_lean<kINT4, kRTNE>(a, st);
     }
+  }
+  if (scale == kE4M3 && round == kRTNE && !stats && a.deq == nullptr) {
+    if (grid == kE2M1) return launch_lean_nv<kE2M1>(a, st);
+    if (grid == kE1M2) return launch_lean_nv<kE1M2>(a, st);
+    if (grid == kINT4) return launch_lean_nv<kINT4>(a, st);
   }
   if (scale == kFP32) {
     if (grid == kE2M1) return launch_q_round<kE2M1, kFP32>(round, stats, a, st);
