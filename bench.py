@@ -38,7 +38,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=400)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="c2",
-                   choices=["c2", "c2-quant-only", "c2-unfused", "c3", "c4-nvfp4", "c4-nvfp4-given",
+                   choices=["c2", "c2-quant-only", "c2-unfused", "c3", "c3-rtne", "c3-row-sr",
+                            "c4-nvfp4", "c4-nvfp4-given",
                             "c4-nvint4", "c4-mxfp4", "c4-if4", "c5-moe-ufp4", "c5-moe-e2m1",
                             "c5-dense-ufp4", "c5-dense-e2m1"])
     p.add_argument("--no-extras", action="store_true", help="skip e2e, ratios and CPU baseline")
@@ -327,10 +328,20 @@ def make_workload(name):
             return RowWorkload(name, desc + " -- unfused: rotation pass to bf16, then quantize",
                                c2_input, cfg, "rht16_kernel+lean_kernel", unfused=True)
         return RowWorkload(name, desc, c2_input, cfg, "lean_kernel<E1M2,rotation,flat>")
-    if name == "c3":
+    if name == "c3-row-sr":
+        mask = fq.sign_mask_from_seed(synth.sign_seed(3))
+        rc = fq.recipe("ufp4", "bwd_dx", "dy", sign_mask=mask, sr_seed=synth.SR_SEED)
+        return RowWorkload(name, "dY[8192,8192] row orientation only, RHT16 + E1M2 SR", synth.workload3,
+                           rc, "lean_kernel<E1M2,rotation,flat,SR>")
+    if name in ("c3", "c3-rtne"):
         mask = fq.sign_mask_from_seed(synth.sign_seed(3))
         rc = fq.recipe("ufp4", "bwd_dx", "dy", sign_mask=mask, sr_seed=synth.SR_SEED)
         cc = fq.recipe("ufp4", "bwd_dw", "dy", sign_mask=mask, sr_seed=synth.SR_SEED)
+        if name == "c3-rtne":
+            from dataclasses import replace
+            rc, cc = replace(rc, round=fq.FP4Q_ROUND_RTNE), replace(cc, round=fq.FP4Q_ROUND_RTNE)
+            return DualWorkload(name, "dY[8192,8192] dual orientation, RHT16 + E1M2 round-to-nearest "
+                                "(diagnostic)", synth.workload3, rc, cc, "dual_kernel<E1M2,RTNE,RTNE>")
         return DualWorkload(name, "backward dY[8192,8192] N(0,1e-3) with 0.01% x100, RHT16 + E1M2 "
                             "SR in row and column orientation from one read", synth.workload3, rc, cc,
                             "dual_kernel<E1M2,SR,SR>")

@@ -198,8 +198,10 @@ __device__ __forceinline__ uint2 encode_lean(const float2* P, float s) {
 // Stochastic rounding, FP32 1x16 scale, codes only; runtime rotation factor c (4 or 1).
 // Element e (0..15) of the block has logical index 2*pair0 + e; pair j = (2j, 2j+1) shares one
 // SplitMix64 output (low half for 2j, high half for 2j+1), keys formed incrementally.
-// Per element: |v| clamped to qmax, t = |v| / step, fl = floor(t), frac = t - fl (all exact);
-// round up iff (u >> 8) < frac * 2^24; the chosen grid point is then encoded exactly like the
+// Per element: |v| clamped to qmax, t = |v| / step (exact), r = (u >> 8) * 2^-24 (exact). The
+// rule "round up iff r < t - floor(t)" picks k = floor(t) + [r < t - floor(t)] = ceil(t - r):
+// t - r lies in (k-1, k]. Computing t - r rounded toward +inf keeps it in (k-1, k] (k is a
+// float), so ceil of that is k exactly. The chosen grid point is then encoded like the
 // round-to-nearest path (E1M2 through E2M3 of value/4, E2M1 through its converter, INT4 by the
 // two's complement add), with the sign of the input value.
 template <int G>
@@ -243,19 +245,15 @@ __device__ __forceinline__ uint2 encode_sr(const float2* P, float s, float c, ui
   for (int e = 0; e < 16; ++e) {
     const float a = fminf(fabsf(q[e]), qmax);
     float mag;
+    const float r = __fmul_rn(__uint2float_rn(rnd[e] >> 8), 0x1p-24f);
     if constexpr (G == kE2M1) {
       const bool lo = a < 2.0f, mid = a < 4.0f;
       const float inv_step = lo ? 2.0f : (mid ? 1.0f : 0.5f);
       const float step = lo ? 0.5f : (mid ? 1.0f : 2.0f);
-      const float t = __fmul_rn(a, inv_step);
-      const float fl = floorf(t);
-      const float k = sr_up(rnd[e], __fsub_rn(t, fl)) ? __fadd_rn(fl, 1.0f) : fl;
-      mag = __fmul_rn(k, step);
+      mag = __fmul_rn(ceilf(__fsub_ru(__fmul_rn(a, inv_step), r)), step);
     } else {
       constexpr float inv_step = (G == kE1M2) ? 2.0f : 1.0f;
-      const float t = __fmul_rn(a, inv_step);
-      const float fl = floorf(t);
-      mag = sr_up(rnd[e], __fsub_rn(t, fl)) ? __fadd_rn(fl, 1.0f) : fl;   // integer steps
+      mag = ceilf(__fsub_ru(__fmul_rn(a, inv_step), r));   // integer steps
     }
     g[e] = with_sign_of(mag, elem_x(P, e));
   }
