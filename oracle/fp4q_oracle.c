@@ -170,14 +170,15 @@ uint8_t orc_round_rtne(int grid, float v) {
 
 /* Stochastic rounding [IF4 section 6.1 pseudo-code: floor(x) + (random() < frac)], applied on
  * the non-uniform grids by its meaning: between the adjacent grid points lo <= |v| <= hi,
- * round away from zero iff r < (|v| - lo) / (hi - lo), with r = (u >> 8) * 2^-24 from the
- * counter hash (R12). |v| is first clamped to the largest magnitude (R4, R13). */
+ * round away from zero iff r < (|v| - lo) / (hi - lo), with r = u * 2^-16 for the element's
+ * 16-bit draw u from the counter hash (R12). |v| is first clamped to the largest magnitude
+ * (R4, R13). */
 static int sr_magnitude_code(const double* g, double a, uint32_t u) {
   if (a >= g[7]) return 7;
   int c = 0;
   while (g[c + 1] <= a) ++c;
   double frac = (a - g[c]) / (g[c + 1] - g[c]);
-  double r = (double)(u >> 8) * 0x1p-24;
+  double r = (double)(u & 0xFFFFu) * 0x1p-16;
   return (r < frac) ? c + 1 : c;
 }
 
@@ -200,12 +201,12 @@ uint64_t orc_splitmix64(uint64_t x) {
   return z ^ (z >> 31);
 }
 
-/* 32 random bits for element `idx` (linear index in its output orientation). Elements 2k and
- * 2k+1 share one hash: the even one takes its low half, the odd one its high half. */
+/* The 16-bit draw u of element `idx` (linear index in its output orientation). Elements
+ * 4k .. 4k+3 share one hash: element 4k + l takes bits 16l .. 16l+15 of it. */
 uint32_t orc_sr_bits(uint64_t seed, uint32_t stream, uint64_t idx) {
-  uint64_t key = seed ^ ((uint64_t)(stream & 1u) << 63) ^ ((idx >> 1) * 0x9E3779B97F4A7C15ull);
+  uint64_t key = seed ^ ((uint64_t)(stream & 1u) << 63) ^ ((idx >> 2) * 0x9E3779B97F4A7C15ull);
   uint64_t h = orc_splitmix64(key);
-  return (idx & 1u) ? (uint32_t)(h >> 32) : (uint32_t)h;
+  return (uint32_t)((h >> (16u * (unsigned)(idx & 3u))) & 0xFFFFu);
 }
 
 /* Sign diagonal from a seed (R1): low 16 bits of SplitMix64(seed). */

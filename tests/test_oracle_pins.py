@@ -216,10 +216,11 @@ def test_splitmix64_published_vectors():
 
 
 def test_sr_probability_exact_by_enumeration():
-    # P(round up) = ceil(frac * 2^24) / 2^24, counted over every r = k * 2^-24
-    k = np.arange(1 << 24, dtype=np.uint32) << np.uint32(8)
+    # P(round up) = ceil(frac * 2^16) / 2^16, counted over every draw u (r = u * 2^-16)
+    k = np.arange(1 << 16, dtype=np.uint32)
     for grid, v in [(O.GRID_E1M2, 1.3), (O.GRID_E1M2, 0.0001), (O.GRID_E2M1, 2.7),
-                    (O.GRID_E2M1, 4.5), (O.GRID_INT4, 3.999), (O.GRID_E1M2, 3.4999)]:
+                    (O.GRID_E2M1, 4.5), (O.GRID_INT4, 3.999), (O.GRID_E1M2, 3.4999),
+                    (O.GRID_E2M1, 0.74), (O.GRID_INT4, 6.0000005), (O.GRID_E1M2, 1e-30)]:
         v32 = np.float32(v)
         g = O.grid_magnitudes(grid)
         lo = g[np.searchsorted(g, v32, side="right") - 1]
@@ -227,7 +228,7 @@ def test_sr_probability_exact_by_enumeration():
         frac = (float(v32) - lo) / (hi - lo)
         codes = O.round_sr(grid, np.full(k.shape, v32), k)
         ups = int(np.count_nonzero(_value_of(grid, codes) == hi))
-        assert ups == math.ceil(frac * 2**24), (grid, v)
+        assert ups == math.ceil(frac * 2**16), (grid, v)
         assert np.all((_value_of(grid, codes) == hi) | (_value_of(grid, codes) == lo))
 
 
@@ -246,14 +247,19 @@ def test_sr_keeps_grid_points_and_is_unbiased():
         assert abs(vals.mean() - float(np.float32(v))) < 4 * sigma + 1e-12
 
 
-def test_sr_bits_pairing_and_streams():
-    # elements 2k and 2k+1 take the two halves of one 64-bit hash; streams differ
-    for idx in (0, 2, 1000, 2**40):
-        lo, hi = O.sr_bits(1, 0, idx), O.sr_bits(1, 0, idx + 1)
-        assert lo != hi
-        assert O.sr_bits(1, 1, idx) != lo
+def test_sr_bits_lanes_and_streams():
+    # elements 4k .. 4k+3 take the four 16-bit lanes of one SplitMix64 output (low lane first);
+    # the column stream flips the key's top bit
+    gamma, mask = 0x9E3779B97F4A7C15, 2**64 - 1
+    for seed, k in ((1, 0), (1, 250), (0x5A5A0003, 2**38 + 5)):
+        for stream in (0, 1):
+            h = O.splitmix64(seed ^ (stream << 63) ^ ((k * gamma) & mask))
+            lanes = [(h >> (16 * l)) & 0xFFFF for l in range(4)]
+            assert [O.sr_bits(seed, stream, 4 * k + l) for l in range(4)] == lanes
+    assert O.sr_bits(1, 1, 1000) != O.sr_bits(1, 0, 1000)
     bits = np.array([O.sr_bits(123, 0, i) for i in range(200_000)], dtype=np.uint64)
-    for b in range(32):
+    assert int(bits.max()) < 2**16
+    for b in range(16):
         frac = np.mean((bits >> np.uint64(b)) & np.uint64(1))
         assert abs(frac - 0.5) < 0.01
 
