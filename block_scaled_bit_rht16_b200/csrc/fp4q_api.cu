@@ -239,7 +239,9 @@ fp4q_status fp4q_quantize_dual(const fp4q_config* row_cfg, const fp4q_config* co
   a.codes_col = codes_col;
   a.scales_col = static_cast<float*>(scales_col);
   sign_words(row_cfg->sign_mask, row_cfg->rht != 0, a.sw_row);
-  sign_words(col_cfg->sign_mask, col_cfg->rht != 0, a.sw_col);
+  for (int i = 0; i < 16; ++i)
+    a.sc_col[i] = (col_cfg->rht != 0 && ((col_cfg->sign_mask >> i) & 1u)) ? 0x80008000u : 0u;
+  a.vec32 = ((reinterpret_cast<uintptr_t>(dy) & 31u) == 0 && ld % 16 == 0) ? 1 : 0;
   a.c_row = row_cfg->rht ? 4.0f : 1.0f;
   a.cinv_row = row_cfg->rht ? 0.25f : 1.0f;
   a.c_col = col_cfg->rht ? 4.0f : 1.0f;

@@ -45,6 +45,24 @@ __device__ __forceinline__ void unpack16(const uint4& lo, const uint4& hi, const
   }
 }
 
+__device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
+  return __ldcs(reinterpret_cast<const uint4*>(p));
+}
+
+// 16 bf16 (32 bytes): one 256-bit load when the address is 32-byte aligned (callers pass vec32
+// only when every block start is), else two 128-bit loads. Read-only, streamed past L1.
+__device__ __forceinline__ void load16(const uint16_t* p, bool vec32, uint4& lo, uint4& hi) {
+  if (vec32) {
+    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w),
+                   "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+                 : "l"(p));
+  } else {
+    lo = ld_stream(p);
+    hi = ld_stream(p + 8);
+  }
+}
+
 // v <- H16 v in natural (Sylvester) order, stages h = 1, 2, 4, 8. No 1/4 here: callers fold the
 // exact power-of-two normalisation into the scale.
 __device__ __forceinline__ void fwht16(float2* P) {
@@ -69,6 +87,12 @@ __device__ __forceinline__ void fwht16(float2* P) {
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+__device__ __forceinline__ float min3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
 
@@ -265,15 +289,29 @@ __device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
   return z ^ (z >> 31);
 }
 
-// 64 random bits for the element pair (2p, 2p+1); seedx = seed ^ (stream << 63).
-__device__ __forceinline__ uint64_t sr_pair_bits(uint64_t seedx, uint64_t pair) {
-  return splitmix64(seedx ^ (pair * 0x9E3779B97F4A7C15ull));
+constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;
+
+// 16-bit draws u[e] for the sixteen consecutive elements whose first has logical index
+// 4 * quad0 (a multiple of 4): element 4j + l takes bits 16l .. 16l+15 of
+// SplitMix64(seedx ^ ((quad0 + j) * gamma)); seedx = seed ^ (stream << 63).
+__device__ __forceinline__ void sr_draws16(uint64_t seedx, uint64_t quad0, uint32_t* u) {
+  uint64_t key = quad0 * kGamma;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint64_t h = splitmix64(seedx ^ key);
+    key += kGamma;
+    const uint32_t lo = (uint32_t)h, hi = (uint32_t)(h >> 32);
+    u[4 * j] = lo & 0xFFFFu;
+    u[4 * j + 1] = lo >> 16;
+    u[4 * j + 2] = hi & 0xFFFFu;
+    u[4 * j + 3] = hi >> 16;
+  }
 }
 
-// Round-up decision r < frac with r = (u >> 8) * 2^-24, taken exactly as
-// (u >> 8) < frac * 2^24 (both sides exact in FP32).
+// Round-up decision r < frac with r = u * 2^-16, taken exactly as u < frac * 2^16 (both sides
+// exact in FP32).
 __device__ __forceinline__ bool sr_up(uint32_t u, float frac) {
-  return __uint2float_rn(u >> 8) < __fmul_rn(frac, 16777216.0f);
+  return __uint2float_rn(u) < __fmul_rn(frac, 65536.0f);
 }
 
 }  // namespace fp4q

@@ -6,11 +6,13 @@
 // 178208020, recipe table of section "UFP4：换一把尺子"; "蚂蚁集团揭秘…", techwalker.com,
 // section 三 on bwd_dx / bwd_dw).
 //
-// A CTA stages a 128 x 64 bf16 tile in shared memory (padded pitch: conflict-free 16-byte row
-// reads and 2-byte column reads), then each of its 256 threads encodes two row blocks and two
-// column blocks with the same per-block encoder as the row kernel. A column's codes for the
-// tile are 64 contiguous bytes of codes_col and its scales 32 contiguous bytes of scales_col,
-// so every 32-byte sector of both outputs is written whole by one CTA.
+// A CTA owns a 128 x 64 tile of dY. Each of its 256 threads loads two row blocks (16
+// consecutive bf16 of one row, 32 bytes), encodes them from registers and parks them in a
+// padded shared tile; after one barrier, warp g encodes the column blocks of rows
+// 16g .. 16g+15, each lane the two adjacent columns 2l, 2l+1 whose elements share one 32-bit
+// shared-memory word per row. A column's codes for the tile are 64 contiguous bytes of
+// codes_col and its scales 32 contiguous bytes of scales_col; every 32-byte sector of both
+// outputs is written whole by one CTA.
 #include <cuda_fp16.h>
 
 #include "fp4q_device.cuh"
@@ -21,68 +23,74 @@ namespace fp4q {
 namespace {
 
 constexpr int kTileM = 128, kTileN = 64;
-constexpr int kPitch = kTileN + 8;   // elements; 144-byte rows
+constexpr int kPitch = kTileN + 8;   // elements; 144-byte rows (conflict-free 16-byte stores)
 
-template <int G, int RR, int RC>
+// ROT: both orientations rotated (c = 4 at compile time); otherwise per-orientation flags.
+template <int G, int RR, int RC, bool ROT>
 __global__ void __launch_bounds__(kThreads) dual_kernel(const DualArgs a) {
   __shared__ __align__(16) uint16_t tile[kTileM * kPitch];
   const int64_t m0 = (int64_t)blockIdx.y * kTileM;
   const int64_t n0 = (int64_t)blockIdx.x * kTileN;
   const int t = threadIdx.x;
+  const bool rot_row = ROT || a.c_row != 1.0f;
+  const bool rot_col = ROT || a.c_col != 1.0f;
+  const float c_row = ROT ? 4.0f : a.c_row, c_col = ROT ? 4.0f : a.c_col;
+  const float cinv_row = ROT ? 0.25f : a.cinv_row, cinv_col = ROT ? 0.25f : a.cinv_col;
 
-  // stage: 1024 chunks of 16 bytes (8 per tile row), four per thread, zero outside the tensor
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int c = t + k * kThreads;
-    const int r = c >> 3, cc = c & 7;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (m0 + r < a.M && n0 + 8 * cc < a.N)
-      v = __ldcs(reinterpret_cast<const uint4*>(a.dy + (m0 + r) * a.ld + n0 + 8 * cc));
-    *reinterpret_cast<uint4*>(&tile[r * kPitch + 8 * cc]) = v;
-  }
-  __syncthreads();
-
-  // row blocks: rows t/4 and t/4 + 64, block t%4 (16 columns)
+  // row blocks rb = t, t + 256: row rb / 4, columns 16 * (rb % 4) .. +15 (zeros outside)
+  uint4 v[2][2];
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
-    const int r = (t >> 2) + 64 * k, b = t & 3;
+    const int rb = t + k * kThreads, r = rb >> 2, b = rb & 3;
+    v[k][0] = v[k][1] = make_uint4(0u, 0u, 0u, 0u);
+    if (m0 + r < a.M && n0 + 16 * b < a.N)
+      load16(a.dy + (m0 + r) * a.ld + n0 + 16 * b, a.vec32 != 0, v[k][0], v[k][1]);
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int rb = t + k * kThreads, r = rb >> 2, b = rb & 3;
+    uint4* dst = reinterpret_cast<uint4*>(&tile[r * kPitch + 16 * b]);
+    dst[0] = v[k][0];
+    dst[1] = v[k][1];
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int rb = t + k * kThreads, r = rb >> 2, b = rb & 3;
     const int64_t m = m0 + r, n = n0 + 16 * b;
     if (m >= a.M || n >= a.N) continue;
-    const uint4* src = reinterpret_cast<const uint4*>(&tile[r * kPitch + 16 * b]);
     float2 P[8];
-    unpack16(src[0], src[1], a.sw_row, P);
-    if (a.c_row != 1.0f) fwht16(P);
-    const float s = div_qmax<G>(__fmul_rn(absmax16(P), a.cinv_row));
+    unpack16(v[k][0], v[k][1], a.sw_row, P);
+    if (rot_row) fwht16(P);
+    const float s = div_qmax<G>(__fmul_rn(absmax16(P), cinv_row));
     const int64_t u = (m * a.N + n) >> 4;   // 16-block index in [M, N/16]
-    const uint2 w = (RR == kSR) ? encode_sr<G>(P, s, a.c_row, a.seedx_row, (uint64_t)u * 8u)
-                                : encode_rtne_rt<G>(P, s, a.c_row != 1.0f);
+    uint2 w;
+    if constexpr (RR == kSR) w = encode_sr<G>(P, s, c_row, a.seedx_row, (uint64_t)u * 4u);
+    else w = ROT ? encode_lean<G, true>(P, s) : encode_rtne_rt<G>(P, s, rot_row);
     __stcs(reinterpret_cast<uint2*>(a.codes_row) + u, w);
     __stcs(a.scales_row + u, s);
   }
+  __syncthreads();
 
-  // column blocks: column (w & 1) * 32 + lane, row groups (w >> 1) and (w >> 1) + 4
-  const int w = t >> 5, lane = t & 31;
-  const int c = (w & 1) * 32 + lane;
+  // column blocks: rows 16g .. 16g+15, columns 2 * lane + h
+  const int g = t >> 5, lane = t & 31;
+  const int64_t m = m0 + 16 * g, nA = n0 + 2 * lane;
+  if (m >= a.M || nA >= a.N) return;   // N % 16 == 0: column nA + 1 exists too
+  uint32_t wd[16];
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int g = (w >> 1) + 4 * k;
-    const int64_t n = n0 + c, m = m0 + 16 * g;
-    if (n >= a.N || m >= a.M) continue;
-    uint32_t wd[8];
+  for (int i = 0; i < 16; ++i)
+    wd[i] = *reinterpret_cast<const uint32_t*>(&tile[(16 * g + i) * kPitch + 2 * lane]) ^ a.sc_col[i];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t lo = tile[(16 * g + 2 * j) * kPitch + c];
-      const uint32_t hi = tile[(16 * g + 2 * j + 1) * kPitch + c];
-      wd[j] = lo | (hi << 16);
-    }
+  for (int h = 0; h < 2; ++h) {
     float2 P[8];
-    unpack16(make_uint4(wd[0], wd[1], wd[2], wd[3]), make_uint4(wd[4], wd[5], wd[6], wd[7]),
-             a.sw_col, P);
-    if (a.c_col != 1.0f) fwht16(P);
-    const float s = div_qmax<G>(__fmul_rn(absmax16(P), a.cinv_col));
-    const int64_t u = (n * a.M + m) >> 4;   // 16-block index in [N, M/16]
-    const uint2 w = (RC == kSR) ? encode_sr<G>(P, s, a.c_col, a.seedx_col, (uint64_t)u * 8u)
-                                : encode_rtne_rt<G>(P, s, a.c_col != 1.0f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      P[i] = h ? make_float2(bf_hi(wd[i]), bf_hi(wd[i + 8])) : make_float2(bf_lo(wd[i]), bf_lo(wd[i + 8]));
+    if (rot_col) fwht16(P);
+    const float s = div_qmax<G>(__fmul_rn(absmax16(P), cinv_col));
+    const int64_t u = ((nA + h) * a.M + m) >> 4;   // 16-block index in [N, M/16]
+    uint2 w;
+    if constexpr (RC == kSR) w = encode_sr<G>(P, s, c_col, a.seedx_col, (uint64_t)u * 4u);
+    else w = ROT ? encode_lean<G, true>(P, s) : encode_rtne_rt<G>(P, s, rot_col);
     __stcs(reinterpret_cast<uint2*>(a.codes_col) + u, w);
     __stcs(a.scales_col + u, s);
   }
@@ -91,7 +99,8 @@ __global__ void __launch_bounds__(kThreads) dual_kernel(const DualArgs a) {
 template <int G, int RR, int RC>
 cudaError_t launch_d(const DualArgs& a, cudaStream_t st) {
   const dim3 grid((unsigned)((a.N + kTileN - 1) / kTileN), (unsigned)((a.M + kTileM - 1) / kTileM));
-  dual_kernel<G, RR, RC><<<grid, kThreads, 0, st>>>(a);
+  if (a.c_row != 1.0f && a.c_col != 1.0f) dual_kernel<G, RR, RC, true><<<grid, kThreads, 0, st>>>(a);
+  else dual_kernel<G, RR, RC, false><<<grid, kThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -196,17 +196,23 @@ __device__ __forceinline__ uint2 encode_lean(const float2* P, float s) {
 }
 
 // Stochastic rounding, FP32 1x16 scale, codes only; runtime rotation factor c (4 or 1).
-// Element e (0..15) of the block has logical index 2*pair0 + e; pair j = (2j, 2j+1) shares one
-// SplitMix64 output (low half for 2j, high half for 2j+1), keys formed incrementally.
-// Per element: |v| clamped to qmax, t = |v| / step (exact), r = (u >> 8) * 2^-24 (exact). The
-// rule "round up iff r < t - floor(t)" picks k = floor(t) + [r < t - floor(t)] = ceil(t - r):
-// t - r lies in (k-1, k]. Computing t - r rounded toward +inf keeps it in (k-1, k] (k is a
-// float), so ceil of that is k exactly. The chosen grid point is then encoded like the
-// round-to-nearest path (E1M2 through E2M3 of value/4, E2M1 through its converter, INT4 by the
-// two's complement add), with the sign of the input value.
+// Element e (0..15) of the block has logical index 4*quad0 + e and the 16-bit draw u_e.
+//
+// Per element, with a = min(|v|, qmax) and t = a / step in [0, 8) (exact): the rule "round up
+// iff u * 2^-16 < t - floor(t)" picks k = floor(t) + [u < ceil(frac * 2^16)]. Y = RU(t + 192)
+// is 192 + T * 2^-16 with T = ceil(t * 2^16) (the binade [128, 256) has ulp 2^-16), and T is
+// the bit pattern of Y minus that of 192 (0x43400000, whose low 16 bits are zero). Then
+//   Z = bits(Y) + 0xFFFF - u  has  Z >> 16 = 0x4340 + floor((T - u + 0xFFFF) / 2^16)
+//                                          = 0x4340 + k,
+// because T - u + 0xFFFF = floor(t) * 2^16 + 2^16 + (ceil(frac * 2^16) - u - 1) and the last
+// term lies in [0, 2^16) exactly when the element rounds up and in [-2^16, 0) otherwise. As
+// 0x4340 ends in a zero nibble and k <= 7, the low nibble of Z >> 16 is k. On E2M1 the step
+// is 1/2, 1 or 2 on [0, 2), [2, 4), [4, 6], and the code is k, k + 2 or k + 4.
+// Codes: sign-magnitude (E1M2, E2M1) takes the input's sign bit as bit 3; INT4 takes -k in
+// two's complement for a negative input.
 template <int G>
 __device__ __forceinline__ uint2 encode_sr(const float2* P, float s, float c, uint64_t seedx,
-                                          uint64_t pair0) {
+                                          uint64_t quad0) {
   if (s == 0.0f) return make_uint2(0u, 0u);
   constexpr float qmax = GridInfo<G>::qmax;
   const float cinv = __frcp_rn(c);   // exact: c is 4 or 1
@@ -220,72 +226,56 @@ __device__ __forceinline__ uint2 encode_sr(const float2* P, float s, float c, ui
       q[i + 8] = r.y;
     }
     // the correction step is exact for quotients of at least 2^-20; smaller nonzero ones (rare)
-    // decide stochastic rounding through their exact value, so they take the IEEE division
+    // decide stochastic rounding through their exact value, so they take the IEEE division.
+    // One block-wide minimum keeps the per-element test off the common path.
+    float qmin = fabsf(q[0]);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const float pe = elem_x(P, e);
-      if (fabsf(q[e]) < 0x1p-19f && pe != 0.0f) q[e] = __fdiv_rn(__fmul_rn(pe, cinv), s);
+    for (int e = 1; e < 15; e += 2) qmin = min3(qmin, fabsf(q[e]), fabsf(q[e + 1]));
+    qmin = fminf(qmin, fabsf(q[15]));
+    if (qmin < 0x1p-19f) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float pe = elem_x(P, e);
+        if (fabsf(q[e]) < 0x1p-19f && pe != 0.0f) q[e] = __fdiv_rn(__fmul_rn(pe, cinv), s);
+      }
     }
   } else {
 #pragma unroll
     for (int e = 0; e < 16; ++e) q[e] = __fdiv_rn(__fmul_rn(elem_x(P, e), cinv), s);
   }
-  uint32_t rnd[16];
-  uint64_t key = pair0 * 0x9E3779B97F4A7C15ull;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint64_t h = splitmix64(seedx ^ key);
-    key += 0x9E3779B97F4A7C15ull;
-    rnd[2 * j] = (uint32_t)h;
-    rnd[2 * j + 1] = (uint32_t)(h >> 32);
-  }
-  // chosen grid point per element, signed like the input value (-0 keeps its sign)
-  float g[16];
-#pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    const float a = fminf(fabsf(q[e]), qmax);
-    float mag;
-    const float r = __fmul_rn(__uint2float_rn(rnd[e] >> 8), 0x1p-24f);
-    if constexpr (G == kE2M1) {
-      const bool lo = a < 2.0f, mid = a < 4.0f;
-      const float inv_step = lo ? 2.0f : (mid ? 1.0f : 0.5f);
-      const float step = lo ? 0.5f : (mid ? 1.0f : 2.0f);
-      mag = __fmul_rn(ceilf(__fsub_ru(__fmul_rn(a, inv_step), r)), step);
-    } else {
-      constexpr float inv_step = (G == kE1M2) ? 2.0f : 1.0f;
-      mag = ceilf(__fsub_ru(__fmul_rn(a, inv_step), r));   // integer steps
-    }
-    g[e] = with_sign_of(mag, elem_x(P, e));
-  }
+  uint32_t u[16];
+  sr_draws16(seedx, quad0, u);
   uint32_t w[2];
-  if constexpr (G == kE2M1) {
 #pragma unroll
-    for (int l = 0; l < 2; ++l) {
-      uint32_t b[4];
+  for (int l = 0; l < 2; ++l) {
+    uint32_t mags = 0u, signs = 0u;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = cvt_e2m1x2(g[8 * l + 2 * j + 1], g[8 * l + 2 * j]);
-      w[l] = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-    }
-  } else if constexpr (G == kE1M2) {
-#pragma unroll
-    for (int l = 0; l < 2; ++l) {
-      uint32_t x[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int e = 8 * l + 4 * h;   // steps / 8 is the E2M3 subnormal code of value / 4
-        const uint32_t W = cvt_e2m3x2(__fmul_rn(g[e + 1], 0.125f), __fmul_rn(g[e], 0.125f)) |
-                           (cvt_e2m3x2(__fmul_rn(g[e + 3], 0.125f), __fmul_rn(g[e + 2], 0.125f)) << 16);
-        const uint32_t N = W - 3u * ((W & 0x20202020u) >> 2);
-        x[h] = N + (N >> 4);
+    for (int j = 0; j < 8; ++j) {
+      const int e = 8 * l + j;
+      const float a = fminf(fabsf(q[e]), qmax);
+      uint32_t z;
+      if constexpr (G == kE2M1) {
+        const bool lo = a < 2.0f, mid = a < 4.0f;
+        const float inv_step = lo ? 2.0f : (mid ? 1.0f : 0.5f);
+        const uint32_t off = lo ? 0u : (mid ? 0x20000u : 0x40000u);
+        z = __float_as_uint(__fmaf_ru(a, inv_step, 192.0f)) + off + 0xFFFFu - u[e];
+      } else {
+        constexpr float inv_step = (G == kE1M2) ? 2.0f : 1.0f;
+        z = __float_as_uint(__fmaf_ru(a, inv_step, 192.0f)) + 0xFFFFu - u[e];
       }
-      w[l] = __byte_perm(x[0], x[1], 0x6420);
+      uint32_t nib = z >> 16;   // low nibble: the magnitude code
+      if constexpr (G == kINT4) {
+        const uint32_t m = (uint32_t)((int32_t)__float_as_uint(elem_x(P, e)) >> 31);
+        nib = (nib ^ m) - m;
+      }
+      mags = __funnelshift_r(mags, nib, 4);   // element 8l ends in bits 0..3
     }
-  } else {
-    uint32_t t[16];
+    if constexpr (G != kINT4) {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) t[e] = __float_as_uint(__fadd_rn(g[e], 12582912.0f));
-    w[0] = pack_low_nibbles(t);
-    w[1] = pack_low_nibbles(t + 8);
+      for (int j = 7; j >= 0; --j) signs = __funnelshift_l(__float_as_uint(elem_x(P, 8 * l + j)), signs, 4);
+      mags |= signs & 0x88888888u;
+    }
+    w[l] = mags;
   }
   return make_uint2(w[0], w[1]);
 }
@@ -315,10 +305,10 @@ struct StatsAcc {
 };
 
 
-// Encodes one block. pair0 = (logical index of element 0) / 2 for the SR counter.
+// Encodes one block. quad0 = (logical index of element 0) / 4 for the SR counter.
 // Returns the IF4 flag (0x80 for an INT4 block, else 0).
 template <int G, int R, bool STATS>
-__device__ __forceinline__ uint32_t encode16(const EncCtx& ctx, const float2* P, uint64_t pair0,
+__device__ __forceinline__ uint32_t encode16(const EncCtx& ctx, const float2* P, uint64_t quad0,
                                              uint8_t* codes, uint16_t* deq, float s,
                                              const Divider& dv, StatsAcc* acc) {
   const bool zero = (s == 0.0f);
@@ -346,15 +336,10 @@ __device__ __forceinline__ uint32_t encode16(const EncCtx& ctx, const float2* P,
                          __fdiv_rn(__fmul_rn(P[i].y, ctx.cinv), s));
   }
 
-  // 32 random bits per element: pair j covers elements 2j (low half) and 2j+1 (high half)
+  // one 16-bit draw per element
   uint32_t rnd[16];
   if constexpr (R == kSR) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint64_t h = sr_pair_bits(ctx.seedx, pair0 + (uint64_t)j);
-      rnd[2 * j] = (uint32_t)h;
-      rnd[2 * j + 1] = (uint32_t)(h >> 32);
-    }
+    sr_draws16(ctx.seedx, quad0, rnd);
   } else {
 #pragma unroll
     for (int j = 0; j < 16; ++j) rnd[j] = 0u;

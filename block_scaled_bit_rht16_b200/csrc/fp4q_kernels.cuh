@@ -50,7 +50,9 @@ struct DualArgs {
   int64_t M, N, ld;
   uint8_t* codes_row; float* scales_row;
   uint8_t* codes_col; float* scales_col;
-  uint32_t sw_row[8], sw_col[8];
+  uint32_t sw_row[8];       // row blocks: sign flips per bf16 pair (elements 2j, 2j+1)
+  uint32_t sc_col[16];      // column blocks: flip of element i in both halves of a bf16 pair
+  int vec32;                // dy 32-byte aligned and ld % 16 == 0: 256-bit row-block loads
   float c_row, cinv_row, c_col, cinv_col;
   uint64_t seedx_row, seedx_col;
   int round_row, round_col;   // per orientation

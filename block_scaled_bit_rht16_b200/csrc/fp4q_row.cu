@@ -30,24 +30,6 @@ __device__ int32_t g_device_status = 0;
 
 namespace {
 
-__device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
-  return __ldcs(reinterpret_cast<const uint4*>(p));
-}
-
-// 16 bf16 (32 bytes): one 256-bit load when the address is 32-byte aligned (the host sets
-// vec32 only when every unit start is), else two 128-bit loads. Read-only, streamed past L1.
-__device__ __forceinline__ void load16(const uint16_t* p, bool vec32, uint4& lo, uint4& hi) {
-  if (vec32) {
-    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w),
-                   "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
-                 : "l"(p));
-  } else {
-    lo = ld_stream(p);
-    hi = ld_stream(p + 8);
-  }
-}
-
 __device__ __forceinline__ int64_t unit_offset(const QuantArgs& a, int64_t u, int unit) {
   if (a.contiguous) return u * unit;
   const int64_t r = u / a.units_per_row;
@@ -96,7 +78,7 @@ __device__ void stats_finish(const StatsAcc& acc, double* partials) {
 // `mult` = 2^-e * cinv), E2M1 with saturation.
 template <int R, bool STATS>
 __device__ __forceinline__ void encode_mx(const EncCtx& ctx, const float2* P, const float2* Q,
-                                          uint64_t pair0, uint8_t* codes, uint16_t* deq, float s,
+                                          uint64_t quad0, uint8_t* codes, uint16_t* deq, float s,
                                           float mult, bool zero, StatsAcc* acc) {
   const float2 m2 = make_float2(mult, mult);
   uint32_t w[4];
@@ -113,14 +95,7 @@ __device__ __forceinline__ void encode_mx(const EncCtx& ctx, const float2* P, co
       vq[16 * half + 8 + i] = V[i].y;
     }
     uint32_t rnd[16];
-    if constexpr (R == kSR) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint64_t h = sr_pair_bits(ctx.seedx, pair0 + 8u * half + (uint64_t)j);
-        rnd[2 * j] = (uint32_t)h;
-        rnd[2 * j + 1] = (uint32_t)(h >> 32);
-      }
-    }
+    if constexpr (R == kSR) sr_draws16(ctx.seedx, quad0 + 4u * half, rnd);
     uint32_t wa = 0u, wb = 0u;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -249,7 +224,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantArgs a) {
           s = __fmul_rn(e4m3_to_f32(sbyte), alpha);
         }
         const Divider dv = make_divider(s, a.c);
-        const uint32_t flag = encode16<G, R, STATS>(ctx, P, (uint64_t)un * 8u, a.codes + un * 8,
+        const uint32_t flag = encode16<G, R, STATS>(ctx, P, (uint64_t)un * 4u, a.codes + un * 8,
                                                     deq, s, dv, STATS ? &acc : nullptr);
         if constexpr (S == kFP32) {
           __stcs(reinterpret_cast<float*>(a.scales) + un, s);
@@ -270,7 +245,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantArgs a) {
         }
         const float s = (e >= -126) ? __uint_as_float((uint32_t)(127 + e) << 23) : 0x1p-127f;
         const float mult = __fmul_rn(__uint_as_float((uint32_t)(127 - e) << 23), a.cinv);
-        encode_mx<R, STATS>(ctx, P, Q, (uint64_t)un * 16u, a.codes + un * 16, deq, s, mult,
+        encode_mx<R, STATS>(ctx, P, Q, (uint64_t)un * 8u, a.codes + un * 16, deq, s, mult,
                             amax_y == 0.0f, STATS ? &acc : nullptr);
         reinterpret_cast<uint8_t*>(a.scales)[un] = (uint8_t)(e + 127);
       }
@@ -306,7 +281,7 @@ __global__ void __launch_bounds__(kThreads) lean_kernel(const QuantArgs a) {
     if constexpr (RHT) fwht16(P);
     const float s = div_qmax<G>(__fmul_rn(absmax16(P), kCinv));
     uint2 w;
-    if constexpr (R == kSR) w = encode_sr<G>(P, s, RHT ? 4.0f : 1.0f, a.seedx, (uint64_t)u * 8u);
+    if constexpr (R == kSR) w = encode_sr<G>(P, s, RHT ? 4.0f : 1.0f, a.seedx, (uint64_t)u * 4u);
     else w = encode_lean<G, RHT>(P, s);
     __stcs(reinterpret_cast<uint2*>(a.codes) + u, w);
     __stcs(reinterpret_cast<float*>(a.scales) + u, s);
