@@ -86,10 +86,10 @@ typedef enum {
 
 /* Rounding [UFP4-B section 二 (RTNE); IF4 section 6.1 (stochastic rounding); UFP4-A recipe
  * table (SR on dY only)]. SR rounds |v| up between adjacent grid points lo <= |v| < hi iff
- * r < (|v|-lo)/(hi-lo), r = u * 2^-16, u = bits 16l .. 16l+15 of
- * SplitMix64(sr_seed ^ (sr_stream << 63) ^ (idx>>2) * 0x9E3779B97F4A7C15) with l = idx & 3;
- * idx = row * cols + col in the output orientation. The expected code then differs from |v| by
- * at most 2^-16 of the cell width. */
+ * r < (|v|-lo)/(hi-lo), r = u * 2^-16, u = bits 16l .. 16l+15 (l = idx & 3) of output idx>>2
+ * of the SplitMix64 stream seeded with sr_seed ^ (sr_stream << 63), i.e. of the finalizer of
+ * state seed + ((idx>>2) + 1) * 0x9E3779B97F4A7C15; idx = row * cols + col in the output
+ * orientation. The expected code differs from |v| by at most 2^-16 of the cell width. */
 typedef enum { FP4Q_ROUND_RTNE = 0, FP4Q_ROUND_SR = 1 } fp4q_round;
 
 /* Output bits of fp4q_config.outputs. Codes and scales are always written. */

@@ -201,11 +201,13 @@ uint64_t orc_splitmix64(uint64_t x) {
   return z ^ (z >> 31);
 }
 
-/* The 16-bit draw u of element `idx` (linear index in its output orientation). Elements
- * 4k .. 4k+3 share one hash: element 4k + l takes bits 16l .. 16l+15 of it. */
+/* The 16-bit draw u of element `idx` (linear index in its output orientation). The draws are
+ * the output stream of the SplitMix64 generator seeded with seed ^ (stream << 63): output k is
+ * the finalizer of state seed' + (k + 1) * gamma, i.e. orc_splitmix64(seed' + k * gamma).
+ * Elements 4k .. 4k+3 share output k: element 4k + l takes bits 16l .. 16l+15 of it. */
 uint32_t orc_sr_bits(uint64_t seed, uint32_t stream, uint64_t idx) {
-  uint64_t key = seed ^ ((uint64_t)(stream & 1u) << 63) ^ ((idx >> 2) * 0x9E3779B97F4A7C15ull);
-  uint64_t h = orc_splitmix64(key);
+  uint64_t seed_s = seed ^ ((uint64_t)(stream & 1u) << 63);
+  uint64_t h = orc_splitmix64(seed_s + (idx >> 2) * 0x9E3779B97F4A7C15ull);
   return (uint32_t)((h >> (16u * (unsigned)(idx & 3u))) & 0xFFFFu);
 }
 

@@ -248,12 +248,19 @@ def test_sr_keeps_grid_points_and_is_unbiased():
 
 
 def test_sr_bits_lanes_and_streams():
-    # elements 4k .. 4k+3 take the four 16-bit lanes of one SplitMix64 output (low lane first);
-    # the column stream flips the key's top bit
+    # elements 4k .. 4k+3 take the four 16-bit lanes (low lane first) of output k of the
+    # SplitMix64 stream seeded with seed ^ (stream << 63): the finalizer of state
+    # seed' + (k+1) * gamma, stepped here one gamma at a time from the seed
     gamma, mask = 0x9E3779B97F4A7C15, 2**64 - 1
     for seed, k in ((1, 0), (1, 250), (0x5A5A0003, 2**38 + 5)):
         for stream in (0, 1):
-            h = O.splitmix64(seed ^ (stream << 63) ^ ((k * gamma) & mask))
+            state = seed ^ (stream << 63)
+            if k < 1000:
+                for _ in range(k):
+                    state = (state + gamma) & mask
+            else:
+                state = (state + k * gamma) & mask
+            h = O.splitmix64(state)
             lanes = [(h >> (16 * l)) & 0xFFFF for l in range(4)]
             assert [O.sr_bits(seed, stream, 4 * k + l) for l in range(4)] == lanes
     assert O.sr_bits(1, 1, 1000) != O.sr_bits(1, 0, 1000)
