@@ -242,6 +242,7 @@ fp4q_status fp4q_quantize_dual(const fp4q_config* row_cfg, const fp4q_config* co
   for (int i = 0; i < 16; ++i)
     a.sc_col[i] = (col_cfg->rht != 0 && ((col_cfg->sign_mask >> i) & 1u)) ? 0x80008000u : 0u;
   a.vec32 = ((reinterpret_cast<uintptr_t>(dy) & 31u) == 0 && ld % 16 == 0) ? 1 : 0;
+  a.col16 = (M % 64 == 0 && aligned(codes_col, 16) && aligned(scales_col, 16)) ? 1 : 0;
   a.c_row = row_cfg->rht ? 4.0f : 1.0f;
   a.cinv_row = row_cfg->rht ? 0.25f : 1.0f;
   a.c_col = col_cfg->rht ? 4.0f : 1.0f;

@@ -282,8 +282,9 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 
 // ------------------------------------------------------------------ stochastic rounding source
 
-__device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
-  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+// SplitMix64 (Steele, Lea & Flood, OOPSLA 2014): the finalizer of a state, and the output for
+// state x + gamma (the generator's next output from state x).
+__device__ __forceinline__ uint64_t splitmix64_mix(uint64_t z) {
   z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
   z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
   return z ^ (z >> 31);
@@ -291,15 +292,18 @@ __device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
 
 constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;
 
+__device__ __forceinline__ uint64_t splitmix64(uint64_t x) { return splitmix64_mix(x + kGamma); }
+
 // 16-bit draws u[e] for the sixteen consecutive elements whose first has logical index
-// 4 * quad0 (a multiple of 4): element 4j + l takes bits 16l .. 16l+15 of
-// SplitMix64(seedx ^ ((quad0 + j) * gamma)); seedx = seed ^ (stream << 63).
+// 4 * quad0 (a multiple of 4): element 4j + l takes bits 16l .. 16l+15 of output quad0 + j of
+// the SplitMix64 stream seeded with seedx = seed ^ (stream << 63), whose state for output k is
+// seedx + (k + 1) * gamma.
 __device__ __forceinline__ void sr_draws16(uint64_t seedx, uint64_t quad0, uint32_t* u) {
-  uint64_t key = quad0 * kGamma;
+  uint64_t state = seedx + (quad0 + 1u) * kGamma;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const uint64_t h = splitmix64(seedx ^ key);
-    key += kGamma;
+    const uint64_t h = splitmix64_mix(state);
+    state += kGamma;
     const uint32_t lo = (uint32_t)h, hi = (uint32_t)(h >> 32);
     u[4 * j] = lo & 0xFFFFu;
     u[4 * j + 1] = lo >> 16;

@@ -10,9 +10,10 @@
 // consecutive bf16 of one row, 32 bytes), encodes them from registers and parks them in a
 // padded shared tile; after one barrier, warp g encodes the column blocks of rows
 // 16g .. 16g+15, each lane the two adjacent columns 2l, 2l+1 whose elements share one 32-bit
-// shared-memory word per row. A column's codes for the tile are 64 contiguous bytes of
-// codes_col and its scales 32 contiguous bytes of scales_col; every 32-byte sector of both
-// outputs is written whole by one CTA.
+// shared-memory word per row. The column results are staged in shared memory and leave as
+// 16-byte stores, each column's 64 bytes of codes and 32 bytes of scales contiguous: the
+// transposed outputs are the pass's costly writes (every CTA in flight scatters them over the
+// whole of codes_col), and per-element 8-byte stores made them costlier still.
 #include <cuda_fp16.h>
 
 #include "fp4q_device.cuh"
@@ -24,11 +25,16 @@ namespace {
 
 constexpr int kTileM = 128, kTileN = 64;
 constexpr int kPitch = kTileN + 8;   // elements; 144-byte rows (conflict-free 16-byte stores)
+constexpr int kGroups = kTileM / 16;  // column blocks per column of a tile
+constexpr int kCodePitch = 10;        // uint2 per staged column (8 used; 16-byte aligned rows)
+constexpr int kScalePitch = 12;       // floats per staged column (8 used)
 
 // ROT: both orientations rotated (c = 4 at compile time); otherwise per-orientation flags.
 template <int G, int RR, int RC, bool ROT>
-__global__ void __launch_bounds__(kThreads) dual_kernel(const DualArgs a) {
+__global__ void __launch_bounds__(kThreads, 4) dual_kernel(const DualArgs a) {
   __shared__ __align__(16) uint16_t tile[kTileM * kPitch];
+  __shared__ __align__(16) uint2 stage_codes[kTileN * kCodePitch];
+  __shared__ __align__(16) float stage_scales[kTileN * kScalePitch];
   const int64_t m0 = (int64_t)blockIdx.y * kTileM;
   const int64_t n0 = (int64_t)blockIdx.x * kTileN;
   const int t = threadIdx.x;
@@ -71,28 +77,67 @@ __global__ void __launch_bounds__(kThreads) dual_kernel(const DualArgs a) {
   }
   __syncthreads();
 
-  // column blocks: rows 16g .. 16g+15, columns 2 * lane + h
+  // column blocks: rows 16g .. 16g+15, columns 2 * lane + h (N % 16 == 0, M % 16 == 0: a
+  // column pair and a group of 16 rows are in range or out of range as a whole)
   const int g = t >> 5, lane = t & 31;
   const int64_t m = m0 + 16 * g, nA = n0 + 2 * lane;
-  if (m >= a.M || nA >= a.N) return;   // N % 16 == 0: column nA + 1 exists too
-  uint32_t wd[16];
+  if (m < a.M && nA < a.N) {
+    uint32_t wd[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i)
-    wd[i] = *reinterpret_cast<const uint32_t*>(&tile[(16 * g + i) * kPitch + 2 * lane]) ^ a.sc_col[i];
+    for (int i = 0; i < 16; ++i)
+      wd[i] = *reinterpret_cast<const uint32_t*>(&tile[(16 * g + i) * kPitch + 2 * lane]) ^ a.sc_col[i];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    float2 P[8];
+    for (int h = 0; h < 2; ++h) {
+      float2 P[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      P[i] = h ? make_float2(bf_hi(wd[i]), bf_hi(wd[i + 8])) : make_float2(bf_lo(wd[i]), bf_lo(wd[i + 8]));
-    if (rot_col) fwht16(P);
-    const float s = div_qmax<G>(__fmul_rn(absmax16(P), cinv_col));
-    const int64_t u = ((nA + h) * a.M + m) >> 4;   // 16-block index in [N, M/16]
-    uint2 w;
-    if constexpr (RC == kSR) w = encode_sr<G>(P, s, c_col, a.seedx_col, (uint64_t)u * 4u);
-    else w = ROT ? encode_lean<G, true>(P, s) : encode_rtne_rt<G>(P, s, rot_col);
-    __stcs(reinterpret_cast<uint2*>(a.codes_col) + u, w);
-    __stcs(a.scales_col + u, s);
+      for (int i = 0; i < 8; ++i)
+        P[i] = h ? make_float2(bf_hi(wd[i]), bf_hi(wd[i + 8])) : make_float2(bf_lo(wd[i]), bf_lo(wd[i + 8]));
+      if (rot_col) fwht16(P);
+      const float s = div_qmax<G>(__fmul_rn(absmax16(P), cinv_col));
+      const int64_t u = ((nA + h) * a.M + m) >> 4;   // 16-block index in [N, M/16]
+      uint2 w;
+      if constexpr (RC == kSR) w = encode_sr<G>(P, s, c_col, a.seedx_col, (uint64_t)u * 4u);
+      else w = ROT ? encode_lean<G, true>(P, s) : encode_rtne_rt<G>(P, s, rot_col);
+      const int c = 2 * lane + h;
+      stage_codes[c * kCodePitch + g] = w;
+      stage_scales[c * kScalePitch + g] = s;
+    }
+  }
+  __syncthreads();
+
+  // column c's blocks for rows m0 .. m0+127 are kGroups consecutive entries of codes_col /
+  // scales_col starting at block (n0 + c) * M/16 + m0/16
+  const int64_t rows_left = (a.M - m0) >> 4, cols_left = a.N - n0;
+  const int ng = rows_left < kGroups ? (int)rows_left : kGroups;
+  const int nc = cols_left < kTileN ? (int)cols_left : kTileN;
+  if (a.col16 && ng == kGroups) {
+    // 16-byte stores: codes as 4 chunks of 2 blocks, scales as 2 chunks of 4 blocks per column
+    {
+      const int c = t >> 2, q = t & 3;
+      if (c < nc) {
+        const uint2 lo = stage_codes[c * kCodePitch + 2 * q], hi = stage_codes[c * kCodePitch + 2 * q + 1];
+        uint2* dst = reinterpret_cast<uint2*>(a.codes_col) + (((n0 + c) * a.M + m0) >> 4) + 2 * q;
+        __stcs(reinterpret_cast<uint4*>(dst), make_uint4(lo.x, lo.y, hi.x, hi.y));
+      }
+    }
+    if (t < 2 * kTileN) {
+      const int c = t >> 1, q = t & 1;
+      if (c < nc) {
+        const float4 v4 = *reinterpret_cast<const float4*>(&stage_scales[c * kScalePitch + 4 * q]);
+        float* dst = a.scales_col + (((n0 + c) * a.M + m0) >> 4) + 4 * q;
+        __stcs(reinterpret_cast<float4*>(dst), v4);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int e = t + k * kThreads, c = e >> 3, gg = e & 7;
+      if (c < nc && gg < ng) {
+        const int64_t u = (((n0 + c) * a.M + m0) >> 4) + gg;
+        __stcs(reinterpret_cast<uint2*>(a.codes_col) + u, stage_codes[c * kCodePitch + gg]);
+        __stcs(a.scales_col + u, stage_scales[c * kScalePitch + gg]);
+      }
+    }
   }
 }
 

@@ -198,26 +198,22 @@ __device__ __forceinline__ uint2 encode_lean(const float2* P, float s) {
 // Stochastic rounding, FP32 1x16 scale, codes only; runtime rotation factor c (4 or 1).
 // Element e (0..15) of the block has logical index 4*quad0 + e and the 16-bit draw u_e.
 //
-// Per element, with a = min(|v|, qmax) and t = a / step in [0, 8) (exact): the rule "round up
-// iff u * 2^-16 < t - floor(t)" picks k = floor(t) + [u < ceil(frac * 2^16)]. Y = RU(t + 192)
-// is 192 + T * 2^-16 with T = ceil(t * 2^16) (the binade [128, 256) has ulp 2^-16), and T is
-// the bit pattern of Y minus that of 192 (0x43400000, whose low 16 bits are zero). Then
-//   Z = bits(Y) + 0xFFFF - u  has  Z >> 16 = 0x4340 + floor((T - u + 0xFFFF) / 2^16)
-//                                          = 0x4340 + k,
-// because T - u + 0xFFFF = floor(t) * 2^16 + 2^16 + (ceil(frac * 2^16) - u - 1) and the last
-// term lies in [0, 2^16) exactly when the element rounds up and in [-2^16, 0) otherwise. As
-// 0x4340 ends in a zero nibble and k <= 7, the low nibble of Z >> 16 is k. On E2M1 the step
-// is 1/2, 1 or 2 on [0, 2), [2, 4), [4, 6], and the code is k, k + 2 or k + 4.
+// Per element, with a = min(|v|, qmax) and t = a / step in [0, 8) (exact), the rule "round up
+// iff r < t - floor(t)" with r = u * 2^-16 picks k = floor(t) + [r < t - floor(t)] =
+// ceil(t - r): t - r lies in (k-1, k]. r is formed exactly as the float with bits
+// 0x3F800000 + 128u (that is 1 + u * 2^-16) minus 1. D = t - r rounded toward +inf stays in
+// (k-1, k] (k is a float), so K = RU(D + 1.5 * 2^23) = 1.5 * 2^23 + k exactly: the binade
+// [2^23, 2^24) has unit spacing, and K's bit pattern is 0x4B400000 + k. On E2M1 the step is
+// 1/2, 1 or 2 on [0, 2), [2, 4), [4, 6], and the code is k, k + 2 or k + 4, added to the
+// constant. The decision runs on the floating-point pipe; the bit patterns of eight elements
+// accumulate as sum(bits_j * 16^j), from which the constant part is subtracted once.
 // Codes: sign-magnitude (E1M2, E2M1) takes the input's sign bit as bit 3; INT4 takes -k in
 // two's complement for a negative input.
-template <int G>
-__device__ __forceinline__ uint2 encode_sr(const float2* P, float s, float c, uint64_t seedx,
-                                          uint64_t quad0) {
-  if (s == 0.0f) return make_uint2(0u, 0u);
-  constexpr float qmax = GridInfo<G>::qmax;
+
+// Quotients v_e = RN(P_e / (c * s)) of a nonzero block, exact.
+__device__ __forceinline__ void sr_quotients(const float2* P, float s, float c, float* q) {
   const float cinv = __frcp_rn(c);   // exact: c is 4 or 1
   const Divider dv = make_divider(s, c);
-  float q[16];
   if (dv.fast) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -243,41 +239,62 @@ __device__ __forceinline__ uint2 encode_sr(const float2* P, float s, float c, ui
 #pragma unroll
     for (int e = 0; e < 16; ++e) q[e] = __fdiv_rn(__fmul_rn(elem_x(P, e), cinv), s);
   }
-  uint32_t u[16];
-  sr_draws16(seedx, quad0, u);
+}
+
+// Codes of a nonzero block from its quotients q, draws u and raw values P (for the signs).
+template <int G>
+__device__ __forceinline__ uint2 sr_codes(const float* q, const uint32_t* u, const float2* P) {
+  constexpr float qmax = GridInfo<G>::qmax;
+  // sum over j = 0..7 of 0x4B400000 * 16^j, modulo 2^32
+  constexpr uint32_t kBias = 0x4B400000u + (0x4B400000u << 4) + (0x4B400000u << 8) +
+                             (0x4B400000u << 12) + (0x4B400000u << 16) + (0x4B400000u << 20) +
+                             (0x4B400000u << 24) + (0x4B400000u << 28);
   uint32_t w[2];
 #pragma unroll
   for (int l = 0; l < 2; ++l) {
     uint32_t mags = 0u, signs = 0u;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 7; j >= 0; --j) {
       const int e = 8 * l + j;
       const float a = fminf(fabsf(q[e]), qmax);
-      uint32_t z;
+      const float r = __fadd_rn(__uint_as_float(u[e] * 128u + 0x3F800000u), -1.0f);   // exact
+      float K;
       if constexpr (G == kE2M1) {
         const bool lo = a < 2.0f, mid = a < 4.0f;
         const float inv_step = lo ? 2.0f : (mid ? 1.0f : 0.5f);
-        const uint32_t off = lo ? 0u : (mid ? 0x20000u : 0x40000u);
-        z = __float_as_uint(__fmaf_ru(a, inv_step, 192.0f)) + off + 0xFFFFu - u[e];
+        const float base = lo ? 12582912.0f : (mid ? 12582914.0f : 12582916.0f);
+        K = __fadd_ru(__fmaf_ru(a, inv_step, -r), base);
       } else {
         constexpr float inv_step = (G == kE1M2) ? 2.0f : 1.0f;
-        z = __float_as_uint(__fmaf_ru(a, inv_step, 192.0f)) + 0xFFFFu - u[e];
+        K = __fadd_ru(__fmaf_ru(a, inv_step, -r), 12582912.0f);
       }
-      uint32_t nib = z >> 16;   // low nibble: the magnitude code
+      const uint32_t bits = __float_as_uint(K);   // 0x4B400000 + magnitude code
       if constexpr (G == kINT4) {
         const uint32_t m = (uint32_t)((int32_t)__float_as_uint(elem_x(P, e)) >> 31);
-        nib = (nib ^ m) - m;
+        mags = mags * 16u + (((bits ^ m) - m) & 0xFu);   // two's complement nibble
+      } else {
+        mags = mags * 16u + bits;
+        signs = __funnelshift_l(__float_as_uint(elem_x(P, e)), signs, 4);
       }
-      mags = __funnelshift_r(mags, nib, 4);   // element 8l ends in bits 0..3
     }
-    if constexpr (G != kINT4) {
-#pragma unroll
-      for (int j = 7; j >= 0; --j) signs = __funnelshift_l(__float_as_uint(elem_x(P, 8 * l + j)), signs, 4);
-      mags |= signs & 0x88888888u;
+    if constexpr (G == kINT4) {
+      w[l] = mags;
+    } else {
+      w[l] = (mags - kBias) | (signs & 0x88888888u);
     }
-    w[l] = mags;
   }
   return make_uint2(w[0], w[1]);
+}
+
+template <int G>
+__device__ __forceinline__ uint2 encode_sr(const float2* P, float s, float c, uint64_t seedx,
+                                          uint64_t quad0) {
+  if (s == 0.0f) return make_uint2(0u, 0u);
+  float q[16];
+  sr_quotients(P, s, c, q);
+  uint32_t u[16];
+  sr_draws16(seedx, quad0, u);
+  return sr_codes<G>(q, u, P);
 }
 
 // Round-to-nearest codes with a runtime rotation factor (signs always copied from the input).

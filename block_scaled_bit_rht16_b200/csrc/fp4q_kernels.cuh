@@ -53,6 +53,7 @@ struct DualArgs {
   uint32_t sw_row[8];       // row blocks: sign flips per bf16 pair (elements 2j, 2j+1)
   uint32_t sc_col[16];      // column blocks: flip of element i in both halves of a bf16 pair
   int vec32;                // dy 32-byte aligned and ld % 16 == 0: 256-bit row-block loads
+  int col16;                // M % 64 == 0 and codes_col, scales_col 16-byte aligned
   float c_row, cinv_row, c_col, cinv_col;
   uint64_t seedx_row, seedx_col;
   int round_row, round_col;   // per orientation
