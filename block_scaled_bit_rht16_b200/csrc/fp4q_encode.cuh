@@ -297,6 +297,78 @@ __device__ __forceinline__ uint2 encode_sr(const float2* P, float s, float c, ui
   return sr_codes<G>(q, u, P);
 }
 
+// IF4 block, E4M3 block scale (NVFP4's), codes only: the E2M1 candidate (round to nearest even,
+// saturating) and the INT4 candidate k = RNE(RN(v * RN(7/6))) clamped to +-7 with value
+// RN(k * RN(6/7)); INT4 is kept iff its squared error, summed in FP32 over the balanced pairwise
+// tree of elements 0..15, is strictly smaller ("低精度量化技术：IF4…", sections 3.1-3.2).
+// The errors RN(value - v) are formed on magnitudes: a nonzero candidate has the sign of v and
+// RN is symmetric, so each square equals the signed one. Returns the code words; flag = 0x80 for
+// an INT4 block.
+template <bool RHT>
+__device__ __forceinline__ uint2 encode_if4(const float2* P, float s, uint32_t& flag) {
+  flag = 0u;
+  if (s == 0.0f) return make_uint2(0u, 0u);
+  float q[16];
+  sr_quotients(P, s, RHT ? 4.0f : 1.0f, q);   // exact quotients, small ones included
+  const float r76 = __fdiv_rn(7.0f, 6.0f), r67 = __fdiv_rn(6.0f, 7.0f);
+  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+  uint32_t fw[2], iw[2];
+  float2 Efp[8], Eint[8];
+#pragma unroll
+  for (int l = 0; l < 2; ++l) {
+    uint32_t bytes = 0u;
+    uint32_t t[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = 8 * l + 2 * j;
+      // E2M1 candidate: codes from the signed quotients (-0 keeps its sign), values decoded
+      const float v0 = RHT ? q[e] : with_sign_of(q[e], elem_x(P, e));
+      const float v1 = RHT ? q[e + 1] : with_sign_of(q[e + 1], elem_x(P, e + 1));
+      const uint32_t b = cvt_e2m1x2(v1, v0);
+      bytes |= b << (8 * j);
+      const float2 g = e2m1x2_to_f32(b);
+      const float2 a2 = make_float2(fabsf(q[e]), fabsf(q[e + 1]));
+      const float2 dfp = sub2(make_float2(fabsf(g.x), fabsf(g.y)), a2);
+      // INT4 candidate: w = RN(v * 7/6) clamped to +-7, rounded half-even by the 1.5 * 2^23 add
+      // (its low nibble is the two's complement code); magnitude k back as an exact float
+      const float w0 = __fmul_rn(q[e], r76), w1 = __fmul_rn(q[e + 1], r76);
+      const float2 tw = add2(make_float2(fminf(fmaxf(w0, -7.0f), 7.0f), fminf(fmaxf(w1, -7.0f), 7.0f)),
+                             make_float2(kMagic, kMagic));
+      t[2 * j] = __float_as_uint(tw.x);
+      t[2 * j + 1] = __float_as_uint(tw.y);
+      const float2 k = add2(tw, make_float2(-kMagic, -kMagic));   // exact
+      const float2 vint = __fmul2_rn(make_float2(fabsf(k.x), fabsf(k.y)), make_float2(r67, r67));
+      const float2 dint = sub2(vint, a2);
+      const float2 sfp = __fmul2_rn(dfp, dfp), sint = __fmul2_rn(dint, dint);
+      // pairwise leaves (e, e+1) of elements 8l + 2j: stored as Efp[4l + j] (x: e, y: e+1)
+      Efp[4 * l + j] = sfp;
+      Eint[4 * l + j] = sint;
+    }
+    fw[l] = bytes;
+    iw[l] = pack_low_nibbles(t);
+  }
+  // balanced tree over elements 0..15: leaves pairs (2i, 2i+1), then 4, 8, 16
+  float fsum[8], isum[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    fsum[i] = __fadd_rn(Efp[i].x, Efp[i].y);
+    isum[i] = __fadd_rn(Eint[i].x, Eint[i].y);
+  }
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 8; i += 2 * h) {
+      fsum[i] = __fadd_rn(fsum[i], fsum[i + h]);
+      isum[i] = __fadd_rn(isum[i], isum[i + h]);
+    }
+  }
+  if (isum[0] < fsum[0]) {
+    flag = 0x80u;
+    return make_uint2(iw[0], iw[1]);
+  }
+  return make_uint2(fw[0], fw[1]);
+}
+
 // Round-to-nearest codes with a runtime rotation factor (signs always copied from the input).
 template <int G>
 __device__ __forceinline__ uint2 encode_rtne_rt(const float2* P, float s, bool rht) {

@@ -300,6 +300,7 @@ __global__ void wait_timeout_kernel(unsigned long long limit_ns) {
 }
 
 // E4M3 block scale + FP32 tensor scale, round to nearest even, codes and scale bytes only.
+// G = kIF4: the per-block FP4 / INT4 choice, flagged in bit 7 of the scale byte.
 template <int G, bool RHT, bool FLAT>
 __global__ void __launch_bounds__(kThreads) lean_nv_kernel(const QuantArgs a) {
   constexpr float qmax = GridInfo<G>::qmax;
@@ -314,6 +315,9 @@ __global__ void __launch_bounds__(kThreads) lean_nv_kernel(const QuantArgs a) {
     if (a.ts_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *a.ts_out = alpha;
   }
   const float denom = __fmul_rn(alpha, qmax);
+  // RN(amax / denom) for every block through the correction step on one reciprocal (exact for
+  // quotients in [2^-20, 2^64); the E4M3 conversion sends anything below 2^-11 to 0 either way)
+  const Divider dd = make_divider(denom, 1.0f);
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x;
   if (u >= a.nunits) return;
@@ -326,12 +330,19 @@ __global__ void __launch_bounds__(kThreads) lean_nv_kernel(const QuantArgs a) {
     unpack16(lo, hi, RHT ? a.sw : zero_sw, P);
     if constexpr (RHT) fwht16(P);
     const float amax_y = __fmul_rn(absmax16(P), kCinv);
-    const float delta = denom > 0.0f ? __fdiv_rn(amax_y, denom) : 0.0f;
+    float delta = 0.0f;
+    if (dd.fast) delta = div2(dd, make_float2(amax_y, 0.0f)).x;
+    // outside the fast range, and for quotients too large for the correction step (a given
+    // tensor scale may be tiny), the IEEE division
+    if ((!dd.fast || !(delta < 0x1p+64f)) && denom > 0.0f) delta = __fdiv_rn(amax_y, denom);
     const uint32_t sbyte = cvt_e4m3(delta);
     const float s = __fmul_rn(e4m3_to_f32(sbyte), alpha);
-    const uint2 w = encode_lean<G, RHT, true>(P, s);
+    uint2 w;
+    uint32_t flag = 0u;
+    if constexpr (G == kIF4) w = encode_if4<RHT>(P, s, flag);
+    else w = encode_lean<G, RHT, true>(P, s);
     __stcs(reinterpret_cast<uint2*>(a.codes) + u, w);
-    reinterpret_cast<uint8_t*>(a.scales)[u] = (uint8_t)sbyte;
+    reinterpret_cast<uint8_t*>(a.scales)[u] = (uint8_t)(sbyte | flag);
     lo = nlo;
     hi = nhi;
   }
@@ -631,6 +642,7 @@ cudaError_t launch_quantize(int grid, int scale, int round, bool stats, const Qu
     if (grid == kE2M1) return launch_lean_nv<kE2M1>(a, st);
     if (grid == kE1M2) return launch_lean_nv<kE1M2>(a, st);
     if (grid == kINT4) return launch_lean_nv<kINT4>(a, st);
+    if (grid == kIF4) return launch_lean_nv<kIF4>(a, st);
   }
   if (scale == kFP32) {
     if (grid == kE2M1) return launch_q_round<kE2M1, kFP32>(round, stats, a, st);

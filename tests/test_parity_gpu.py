@@ -190,9 +190,10 @@ def test_edge_blocks(combo, rht, unit, outs):
     cfg = fq.Config(grid=grid, scale=scale, round=rnd, rht=rht, sign_mask=0x5A5A, sr_seed=3,
                     dequant=full, stats=full)
     compare_quant(cfg, x, gpu_quantize(cfg, x))
-    if scale == E4M3:   # the same blocks under a given (stale, too small) tensor scale
-        ts = np.float32(1e-4)
-        compare_quant(cfg, x, gpu_quantize(cfg, x, tensor_scale=ts), tensor_scale=ts)
+    if scale == E4M3:   # the same blocks under given (stale, too small) tensor scales; 1e-30
+        # makes amax / (alpha * qmax) overflow FP32 in the huge rows
+        for ts in (np.float32(1e-4), np.float32(1e-30)):
+            compare_quant(cfg, x, gpu_quantize(cfg, x, tensor_scale=ts), tensor_scale=ts)
 
 
 def test_edge_blocks_inside_random_data():
