@@ -352,8 +352,12 @@ def make_workload(name):
                 "mxfp4": fq.FP4Q_GRID_E2M1, "if4": fq.FP4Q_GRID_IF4}[kind]
         scale = fq.FP4Q_SCALE_UE8M0_1x32 if kind == "mxfp4" else fq.FP4Q_SCALE_E4M3_1x16_TENSOR
         cfg = fq.Config(grid=grid, scale=scale, rht=1, sign_mask=mask)
-        return RowWorkload(name, "[16384,5120] Laplace(0,1), RHT16, %s" % kind, synth.workload4, cfg,
-                           "quantize_kernel<%s>" % kind + ("" if kind in ("mxfp4", "nvfp4-given") else "+amax_kernel"))
+        key = {"nvfp4": "lean_nv_kernel<E2M1,rotation,flat>", "nvfp4-given": "lean_nv_kernel<E2M1,rotation,flat>",
+               "nvint4": "lean_nv_kernel<INT4,rotation,flat>", "if4": "lean_nv_kernel<IF4,rotation,flat>",
+               "mxfp4": "quantize_kernel<E2M1,UE8M0>"}[kind]
+        if kind in ("nvfp4", "nvint4", "if4"):
+            key += "+amax_kernel<rotation,flat>"
+        return RowWorkload(name, "[16384,5120] Laplace(0,1), RHT16, %s" % kind, synth.workload4, cfg, key)
     if name.startswith("c5"):
         mask = fq.sign_mask_from_seed(synth.sign_seed(5))
         ufp4 = name.endswith("ufp4")

@@ -349,18 +349,29 @@ __global__ void __launch_bounds__(kThreads) lean_nv_kernel(const QuantArgs a) {
 }
 
 // Amax of the rotated tensor: per-warp maximum of the bit patterns (non-negative floats order
-// like unsigned integers), one atomicMax per warp into the workspace header.
+// like unsigned integers), one atomicMax per warp into the workspace header. Like the lean
+// kernels: rotation and layout fixed at compile time, the next block's load in flight.
+template <bool RHT, bool FLAT>
 __global__ void __launch_bounds__(kThreads) amax_kernel(const QuantArgs a) {
+  constexpr float kCinv = RHT ? 0.25f : 1.0f;
+  const uint32_t zero_sw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
   pdl_enter();
   uint32_t m = 0u;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
-  for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < a.nunits; u += stride) {
+  int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  if (u < a.nunits) {
     uint4 lo, hi;
-    load16(a.x + unit_offset(a, u, 16), a.vec32 != 0, lo, hi);
-    float2 P[8];
-    unpack16(lo, hi, a.sw, P);
-    rotate_if(a, P);
-    m = max(m, __float_as_uint(__fmul_rn(absmax16(P), a.cinv)));
+    lean_load<0, RHT, FLAT>(a, u, lo, hi);
+    for (; u < a.nunits; u += stride) {
+      uint4 nlo = lo, nhi = hi;
+      if (u + stride < a.nunits) lean_load<0, RHT, FLAT>(a, u + stride, nlo, nhi);
+      float2 P[8];
+      unpack16(lo, hi, RHT ? a.sw : zero_sw, P);
+      if constexpr (RHT) fwht16(P);
+      m = max(m, __float_as_uint(__fmul_rn(absmax16(P), kCinv)));
+      lo = nlo;
+      hi = nhi;
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
@@ -659,9 +670,17 @@ cudaError_t launch_quantize(int grid, int scale, int round, bool stats, const Qu
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_amax(const QuantArgs& a, cudaStream_t st) {
-  const cudaError_t e = launch_pdl(amax_kernel, persistent_grid(amax_kernel, a.nunits), st, a);
+template <bool RHT, bool FLAT>
+cudaError_t launch_amax2(const QuantArgs& a, cudaStream_t st) {
+  auto k = amax_kernel<RHT, FLAT>;
+  const cudaError_t e = launch_pdl(k, persistent_grid(k, a.nunits), st, a);
   return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_amax(const QuantArgs& a, cudaStream_t st) {
+  const bool rht = a.c != 1.0f, flat = a.contiguous && a.vec32;
+  if (rht) return flat ? launch_amax2<true, true>(a, st) : launch_amax2<true, false>(a, st);
+  return flat ? launch_amax2<false, true>(a, st) : launch_amax2<false, false>(a, st);
 }
 
 __global__ void alpha_kernel(const WsHeader* ws, float qmax, float* tensor_scale) {
