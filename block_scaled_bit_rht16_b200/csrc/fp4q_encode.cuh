@@ -312,59 +312,57 @@ __device__ __forceinline__ uint2 encode_if4(const float2* P, float s, uint32_t& 
   sr_quotients(P, s, RHT ? 4.0f : 1.0f, q);   // exact quotients, small ones included
   const float r76 = __fdiv_rn(7.0f, 6.0f), r67 = __fdiv_rn(6.0f, 7.0f);
   constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
-  uint32_t fw[2], iw[2];
-  float2 Efp[8], Eint[8];
+  // E2M1 candidate: codes from the signed quotients (-0 keeps its sign), magnitudes decoded.
+  // Byte j of word l holds elements 8l + 2j (low nibble) and 8l + 2j + 1.
+  uint32_t fw[2] = {0u, 0u};
+  float gabs[16];
 #pragma unroll
   for (int l = 0; l < 2; ++l) {
-    uint32_t bytes = 0u;
-    uint32_t t[8];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int e = 8 * l + 2 * j;
-      // E2M1 candidate: codes from the signed quotients (-0 keeps its sign), values decoded
       const float v0 = RHT ? q[e] : with_sign_of(q[e], elem_x(P, e));
       const float v1 = RHT ? q[e + 1] : with_sign_of(q[e + 1], elem_x(P, e + 1));
       const uint32_t b = cvt_e2m1x2(v1, v0);
-      bytes |= b << (8 * j);
+      fw[l] |= b << (8 * j);
       const float2 g = e2m1x2_to_f32(b);
-      const float2 a2 = make_float2(fabsf(q[e]), fabsf(q[e + 1]));
-      const float2 dfp = sub2(make_float2(fabsf(g.x), fabsf(g.y)), a2);
-      // INT4 candidate: w = RN(v * 7/6) clamped to +-7, rounded half-even by the 1.5 * 2^23 add
-      // (its low nibble is the two's complement code); magnitude k back as an exact float
-      const float w0 = __fmul_rn(q[e], r76), w1 = __fmul_rn(q[e + 1], r76);
-      const float2 tw = add2(make_float2(fminf(fmaxf(w0, -7.0f), 7.0f), fminf(fmaxf(w1, -7.0f), 7.0f)),
-                             make_float2(kMagic, kMagic));
-      t[2 * j] = __float_as_uint(tw.x);
-      t[2 * j + 1] = __float_as_uint(tw.y);
-      const float2 k = add2(tw, make_float2(-kMagic, -kMagic));   // exact
-      const float2 vint = __fmul2_rn(make_float2(fabsf(k.x), fabsf(k.y)), make_float2(r67, r67));
-      const float2 dint = sub2(vint, a2);
-      const float2 sfp = __fmul2_rn(dfp, dfp), sint = __fmul2_rn(dint, dint);
-      // pairwise leaves (e, e+1) of elements 8l + 2j: stored as Efp[4l + j] (x: e, y: e+1)
-      Efp[4 * l + j] = sfp;
-      Eint[4 * l + j] = sint;
+      gabs[e] = fabsf(g.x);
+      gabs[e + 1] = fabsf(g.y);
     }
-    fw[l] = bytes;
-    iw[l] = pack_low_nibbles(t);
   }
-  // balanced tree over elements 0..15: leaves pairs (2i, 2i+1), then 4, 8, 16
-  float fsum[8], isum[8];
+  // INT4 candidate and both squared errors, two elements (i, i+8) per float2: w = RN(v * 7/6)
+  // clamped to +-7 and rounded half-even by the 1.5 * 2^23 add (its low nibble is the two's
+  // complement code), the magnitude k back as an exact float.
+  uint32_t t0[8], t1[8];
+  float2 Sf[8], Si[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    fsum[i] = __fadd_rn(Efp[i].x, Efp[i].y);
-    isum[i] = __fadd_rn(Eint[i].x, Eint[i].y);
+    const float2 a2 = make_float2(fabsf(q[i]), fabsf(q[i + 8]));
+    const float2 w = __fmul2_rn(make_float2(q[i], q[i + 8]), make_float2(r76, r76));
+    const float2 tw = add2(make_float2(fminf(fmaxf(w.x, -7.0f), 7.0f), fminf(fmaxf(w.y, -7.0f), 7.0f)),
+                           make_float2(kMagic, kMagic));
+    t0[i] = __float_as_uint(tw.x);
+    t1[i] = __float_as_uint(tw.y);
+    const float2 k = add2(tw, make_float2(-kMagic, -kMagic));   // exact
+    const float2 vint = __fmul2_rn(make_float2(fabsf(k.x), fabsf(k.y)), make_float2(r67, r67));
+    const float2 dint = sub2(vint, a2);
+    const float2 dfp = sub2(make_float2(gabs[i], gabs[i + 8]), a2);
+    Sf[i] = __fmul2_rn(dfp, dfp);
+    Si[i] = __fmul2_rn(dint, dint);
   }
+  // balanced tree over elements 0..15 with both halves at once: lanes (e_i, e_{i+8})
 #pragma unroll
   for (int h = 1; h < 8; h <<= 1) {
 #pragma unroll
     for (int i = 0; i < 8; i += 2 * h) {
-      fsum[i] = __fadd_rn(fsum[i], fsum[i + h]);
-      isum[i] = __fadd_rn(isum[i], isum[i + h]);
+      Sf[i] = add2(Sf[i], Sf[i + h]);
+      Si[i] = add2(Si[i], Si[i + h]);
     }
   }
-  if (isum[0] < fsum[0]) {
+  const float sse_fp = __fadd_rn(Sf[0].x, Sf[0].y), sse_int = __fadd_rn(Si[0].x, Si[0].y);
+  if (sse_int < sse_fp) {
     flag = 0x80u;
-    return make_uint2(iw[0], iw[1]);
+    return make_uint2(pack_low_nibbles(t0), pack_low_nibbles(t1));
   }
   return make_uint2(fw[0], fw[1]);
 }
