@@ -175,8 +175,10 @@ __device__ __forceinline__ uint2 encode_lean(const float2* P, float s) {
         const float e0 = l ? Q[2 * j].y : Q[2 * j].x, e1 = l ? Q[2 * j + 1].y : Q[2 * j + 1].x;
         const float e2 = l ? Q[2 * j + 2].y : Q[2 * j + 2].x, e3 = l ? Q[2 * j + 3].y : Q[2 * j + 3].x;
         const uint32_t W = cvt_e2m3x2(e1, e0) | (cvt_e2m3x2(e3, e2) << 16);   // byte k = code k
-        const uint32_t N = W - 3u * ((W & 0x20202020u) >> 2);                  // sign to bit 3
-        x[h] = N + (N >> 4);                                                    // bytes 0, 2: pairs
+        // byte k of W is 00s00mmm (v/4 is an E2M3 subnormal): N's low nibbles s mmm (bits 4..7
+        // of each byte are don't-care), then X's bytes 0 and 2 pair nibbles 0|1 and 2|3
+        const uint32_t N = (W & 0x07070707u) | ((W >> 2) & 0xF8F8F8F8u);
+        x[h] = (N & 0x0F0F0F0Fu) | ((N >> 4) & 0xF0F0F0F0u);
       }
       w[l] = __byte_perm(x[0], x[1], 0x6420);
     }

@@ -257,25 +257,31 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantArgs a) {
 // The hot path: FP32 1x16 scale, round to nearest even, codes and scales only. FLAT: the
 // tensor is contiguous and 32-byte aligned, so unit u is the 32 bytes at 32u (one 256-bit load).
 // Each thread encodes one block per iteration while the load of its next block is in flight.
+// FLAT launches also have fewer than 2^31 units, so their block counters are 32-bit.
 template <int G, bool RHT, bool FLAT>
 __device__ __forceinline__ void lean_load(const QuantArgs& a, int64_t u, uint4& lo, uint4& hi) {
   if constexpr (FLAT) load16(a.x + u * 16, true, lo, hi);
   else load16(a.x + unit_offset(a, u, 16), a.vec32 != 0, lo, hi);
 }
 
+template <bool FLAT> struct UnitIdx { using T = int64_t; };
+template <> struct UnitIdx<true> { using T = uint32_t; };
+
 template <int G, bool RHT, bool FLAT, int R>
 __global__ void __launch_bounds__(kThreads) lean_kernel(const QuantArgs a) {
   constexpr float kCinv = RHT ? 0.25f : 1.0f;
   const uint32_t zero_sw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
   pdl_enter();
-  const int64_t stride = (int64_t)gridDim.x * kThreads;
-  int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  if (u >= a.nunits) return;
+  using Idx = typename UnitIdx<FLAT>::T;
+  const Idx n = (Idx)a.nunits;
+  const Idx stride = (Idx)gridDim.x * kThreads;
+  Idx u = (Idx)blockIdx.x * kThreads + threadIdx.x;
+  if (u >= n) return;
   uint4 lo, hi;
   lean_load<G, RHT, FLAT>(a, u, lo, hi);
-  for (; u < a.nunits; u += stride) {
+  for (; u < n; u += stride) {
     uint4 nlo = lo, nhi = hi;
-    if (u + stride < a.nunits) lean_load<G, RHT, FLAT>(a, u + stride, nlo, nhi);
+    if (u + stride < n) lean_load<G, RHT, FLAT>(a, u + stride, nlo, nhi);
     float2 P[8];
     unpack16(lo, hi, RHT ? a.sw : zero_sw, P);
     if constexpr (RHT) fwht16(P);
@@ -318,14 +324,16 @@ __global__ void __launch_bounds__(kThreads) lean_nv_kernel(const QuantArgs a) {
   // RN(amax / denom) for every block through the correction step on one reciprocal (exact for
   // quotients in [2^-20, 2^64); the E4M3 conversion sends anything below 2^-11 to 0 either way)
   const Divider dd = make_divider(denom, 1.0f);
-  const int64_t stride = (int64_t)gridDim.x * kThreads;
-  int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  if (u >= a.nunits) return;
+  using Idx = typename UnitIdx<FLAT>::T;
+  const Idx n = (Idx)a.nunits;
+  const Idx stride = (Idx)gridDim.x * kThreads;
+  Idx u = (Idx)blockIdx.x * kThreads + threadIdx.x;
+  if (u >= n) return;
   uint4 lo, hi;
   lean_load<G, RHT, FLAT>(a, u, lo, hi);
-  for (; u < a.nunits; u += stride) {
+  for (; u < n; u += stride) {
     uint4 nlo = lo, nhi = hi;
-    if (u + stride < a.nunits) lean_load<G, RHT, FLAT>(a, u + stride, nlo, nhi);
+    if (u + stride < n) lean_load<G, RHT, FLAT>(a, u + stride, nlo, nhi);
     float2 P[8];
     unpack16(lo, hi, RHT ? a.sw : zero_sw, P);
     if constexpr (RHT) fwht16(P);
@@ -357,14 +365,16 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const QuantArgs a) {
   const uint32_t zero_sw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
   pdl_enter();
   uint32_t m = 0u;
-  const int64_t stride = (int64_t)gridDim.x * kThreads;
-  int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  if (u < a.nunits) {
+  using Idx = typename UnitIdx<FLAT>::T;
+  const Idx n = (Idx)a.nunits;
+  const Idx stride = (Idx)gridDim.x * kThreads;
+  Idx u = (Idx)blockIdx.x * kThreads + threadIdx.x;
+  if (u < n) {
     uint4 lo, hi;
     lean_load<0, RHT, FLAT>(a, u, lo, hi);
-    for (; u < a.nunits; u += stride) {
+    for (; u < n; u += stride) {
       uint4 nlo = lo, nhi = hi;
-      if (u + stride < a.nunits) lean_load<0, RHT, FLAT>(a, u + stride, nlo, nhi);
+      if (u + stride < n) lean_load<0, RHT, FLAT>(a, u + stride, nlo, nhi);
       float2 P[8];
       unpack16(lo, hi, RHT ? a.sw : zero_sw, P);
       if constexpr (RHT) fwht16(P);
@@ -624,14 +634,14 @@ cudaError_t launch_lean_nv3(const QuantArgs& a, cudaStream_t st) {
 
 template <int G>
 cudaError_t launch_lean_nv(const QuantArgs& a, cudaStream_t st) {
-  const bool rht = a.c != 1.0f, flat = a.contiguous && a.vec32;
+  const bool rht = a.c != 1.0f, flat = a.contiguous && a.vec32 && a.nunits < (int64_t(1) << 31);
   if (rht) return flat ? launch_lean_nv3<G, true, true>(a, st) : launch_lean_nv3<G, true, false>(a, st);
   return flat ? launch_lean_nv3<G, false, true>(a, st) : launch_lean_nv3<G, false, false>(a, st);
 }
 
 template <int G, int R>
 cudaError_t launch_lean(const QuantArgs& a, cudaStream_t st) {
-  const bool rht = a.c != 1.0f, flat = a.contiguous && a.vec32;
+  const bool rht = a.c != 1.0f, flat = a.contiguous && a.vec32 && a.nunits < (int64_t(1) << 31);
   if (rht) return flat ? launch_lean3<G, true, true, R>(a, st) : launch_lean3<G, true, false, R>(a, st);
   return flat ? launch_lean3<G, false, true, R>(a, st) : launch_lean3<G, false, false, R>(a, st);
 }
@@ -678,7 +688,7 @@ cudaError_t launch_amax2(const QuantArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_amax(const QuantArgs& a, cudaStream_t st) {
-  const bool rht = a.c != 1.0f, flat = a.contiguous && a.vec32;
+  const bool rht = a.c != 1.0f, flat = a.contiguous && a.vec32 && a.nunits < (int64_t(1) << 31);
   if (rht) return flat ? launch_amax2<true, true>(a, st) : launch_amax2<true, false>(a, st);
   return flat ? launch_amax2<false, true>(a, st) : launch_amax2<false, false>(a, st);
 }
