@@ -15,6 +15,7 @@ barrier + synchronize around the timed region, max over ranks. Prints one JSON l
 """
 import argparse
 import concurrent.futures as cf
+import datetime
 import hashlib
 import json
 import math
@@ -62,7 +63,7 @@ def hbm_peak():
 
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
-    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -80,7 +81,9 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def stop(self, t_begin=None, t_end=None):
+        """Summary of the samples whose timestamps fall in [t_begin, t_end] (host wall-clock
+        seconds bracketing the timed region); all samples if none do."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -89,24 +92,26 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        sm, mx, reasons = [], [], set()
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in out.splitlines():
             parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 7:
+            if len(parts) < 8:
                 continue
             try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[1]), float(parts[2]),
+                             [n for n, v in zip(names, parts[4:8]) if v.lower().startswith("active")]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[3:7]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
+        if not rows:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        inside = [r for r in rows if t_begin is not None and t_begin <= r[0] <= t_end]
+        use = inside or rows
+        reasons = sorted({n for r in use for n in r[3]})
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "reasons": reasons, "samples": len(use),
+                "window": "timed region" if inside else "whole run (no sample fell in the timed region)"}
 
 
 def kernel_source_sha():
@@ -432,6 +437,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    host_begin = time.time()
     with torch.cuda.stream(stream):   # graphs replay on the current stream
         t0.record(stream)
         for _ in range(full):
@@ -440,9 +446,10 @@ def run_ours(args):
             g_rem.replay()
         t1.record(stream)
     torch.cuda.synchronize()
+    host_end = time.time()
     if world > 1:
         dist.barrier()
-    clocks = sampler.stop() if sampler else None
+    clocks = sampler.stop(host_begin, host_end) if sampler else None
     ms = t0.elapsed_time(t1)
     if world > 1:
         t = torch.tensor([ms], device=dev, dtype=torch.float64)
