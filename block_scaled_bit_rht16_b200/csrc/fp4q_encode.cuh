@@ -202,13 +202,14 @@ __device__ __forceinline__ uint2 encode_lean(const float2* P, float s) {
 //
 // Per element, with a = min(|v|, qmax) and t = a / step in [0, 8) (exact), the rule "round up
 // iff r < t - floor(t)" with r = u * 2^-16 picks k = floor(t) + [r < t - floor(t)] =
-// ceil(t - r): t - r lies in (k-1, k]. r is formed exactly as the float with bits
-// 0x3F800000 + 128u (that is 1 + u * 2^-16) minus 1. D = t - r rounded toward +inf stays in
-// (k-1, k] (k is a float), so K = RU(D + 1.5 * 2^23) = 1.5 * 2^23 + k exactly: the binade
-// [2^23, 2^24) has unit spacing, and K's bit pattern is 0x4B400000 + k. On E2M1 the step is
-// 1/2, 1 or 2 on [0, 2), [2, 4), [4, 6], and the code is k, k + 2 or k + 4, added to the
-// constant. The decision runs on the floating-point pipe; the bit patterns of eight elements
-// accumulate as sum(bits_j * 16^j), from which the constant part is subtracted once.
+// ceil(t - r): t - r lies in (k-1, k]. Every k is read off K = 1.5 * 2^23 + k, exact in the
+// unit-spaced binade [2^23, 2^24), whose bit pattern is 0x4B400000 + k. On E2M1, r is formed
+// exactly as the float with bits 0x3F800000 + 128u (1 + u * 2^-16) minus 1, D = t - r rounded
+// toward +inf stays in (k-1, k] (k is a float), and K = RU(D + 1.5 * 2^23); the step is 1/2, 1
+// or 2 on [0, 2), [2, 4), [4, 6] and the code k, k + 2 or k + 4. The uniform grids fold the
+// clamp at qmax into a saturating FMA (below). The decision runs on the floating-point pipe;
+// the bit patterns of eight elements accumulate as sum(bits_j * 16^j), from which the constant
+// part is subtracted once.
 // Codes: sign-magnitude (E1M2, E2M1) takes the input's sign bit as bit 3; INT4 takes -k in
 // two's complement for a negative input.
 
@@ -258,17 +259,27 @@ __device__ __forceinline__ uint2 sr_codes(const float* q, const uint32_t* u, con
 #pragma unroll
     for (int j = 7; j >= 0; --j) {
       const int e = 8 * l + j;
-      const float a = fminf(fabsf(q[e]), qmax);
-      const float r = __fadd_rn(__uint_as_float(u[e] * 128u + 0x3F800000u), -1.0f);   // exact
       float K;
       if constexpr (G == kE2M1) {
+        const float a = fminf(fabsf(q[e]), qmax);
+        const float r = __fadd_rn(__uint_as_float(u[e] * 128u + 0x3F800000u), -1.0f);   // exact
         const bool lo = a < 2.0f, mid = a < 4.0f;
         const float inv_step = lo ? 2.0f : (mid ? 1.0f : 0.5f);
         const float base = lo ? 12582912.0f : (mid ? 12582914.0f : 12582916.0f);
         K = __fadd_ru(__fmaf_ru(a, inv_step, -r), base);
       } else {
-        constexpr float inv_step = (G == kE1M2) ? 2.0f : 1.0f;
-        K = __fadd_ru(__fmaf_ru(a, inv_step, -r), 12582912.0f);
+        // uniform grids, t = |v| / step with qmax = 7 steps: F = 1 + u * 2^-23 (the draw in the
+        // low mantissa bits, one byte permute), c = 16.125 - 16 F = (1 - r) / 8 exactly;
+        // w = min(RU((t - r + 1) / 8), 1) (the saturation is the clamp at qmax: t' = min(t, 7));
+        // 8w = RU(t' - r + 1), whose ceiling is ceil(t' - r) + 1 (no integer up to 8 lies
+        // between a real and its upward rounding), so K = RU(8w + 1.5 * 2^23 - 1) is
+        // 1.5 * 2^23 + ceil(t' - r).
+        const float F = __uint_as_float(__byte_perm(u[e], 0x3F800000u, 0x7610));
+        const float c = __fmaf_rn(F, -16.0f, 16.125f);
+        constexpr float inv8step = (G == kE1M2) ? 0.25f : 0.125f;
+        float w;
+        asm("fma.rp.sat.f32 %0, %1, %2, %3;" : "=f"(w) : "f"(fabsf(q[e])), "f"(inv8step), "f"(c));
+        K = __fmaf_ru(w, 8.0f, 12582911.0f);
       }
       const uint32_t bits = __float_as_uint(K);   // 0x4B400000 + magnitude code
       if constexpr (G == kINT4) {
