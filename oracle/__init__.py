@@ -17,6 +17,7 @@ import numpy as np
 from . import build as _build
 
 GRID_E2M1, GRID_E1M2, GRID_INT4, GRID_IF4 = 0, 1, 2, 3
+GRID_E2M1_MAX4, GRID_E2M1_MAX3, GRID_E2M1_MAX2 = 4, 5, 6   # range-restricted E2M1
 SCALE_FP32_1x16, SCALE_E4M3_1x16, SCALE_UE8M0_1x32 = 0, 1, 2
 ROUND_RTNE, ROUND_SR = 0, 1
 
@@ -97,9 +98,11 @@ def sign_mask_from_seed(seed: int) -> int:
 
 
 def grid_magnitudes(grid: int) -> np.ndarray:
+    """The magnitudes a grid rounds to, by magnitude code (8; 7, 6, 5 for restricted E2M1)."""
     g = np.zeros(8, dtype=np.float64)
-    assert _lib.orc_grid_magnitudes(grid, _ptr(g)) == 8
-    return g
+    n = _lib.orc_grid_magnitudes(grid, _ptr(g))
+    assert n > 0
+    return g[:n]
 
 
 def decode_nibble(grid: int, nib: int) -> float:

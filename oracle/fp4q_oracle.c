@@ -33,7 +33,9 @@
 /* ------------------------------------------------------------------------------------ */
 /* Configuration (the oracle's own encoding; the test layer maps the library's onto it). */
 
-enum { ORC_GRID_E2M1 = 0, ORC_GRID_E1M2 = 1, ORC_GRID_INT4 = 2, ORC_GRID_IF4 = 3 };
+enum { ORC_GRID_E2M1 = 0, ORC_GRID_E1M2 = 1, ORC_GRID_INT4 = 2, ORC_GRID_IF4 = 3,
+       /* E2M1 with the largest magnitude restricted to 4, 3 or 2 (codes above it unused) */
+       ORC_GRID_E2M1_MAX4 = 4, ORC_GRID_E2M1_MAX3 = 5, ORC_GRID_E2M1_MAX2 = 6 };
 enum { ORC_SCALE_FP32_1x16 = 0, ORC_SCALE_E4M3_1x16 = 1, ORC_SCALE_UE8M0_1x32 = 2 };
 enum { ORC_ROUND_RTNE = 0, ORC_ROUND_SR = 1 };
 
@@ -100,11 +102,20 @@ static double minifloat_magnitude(int mbits, int bias, int e, int m) {
   return ldexp(1.0 + frac, e - bias);          /* normal */
 }
 
-/* Fills g[0..7] with the non-negative magnitudes of `grid`, indexed by magnitude code.
- * IF4 uses the E2M1 table for its FP4 blocks. Returns 8, or 0 for an unknown grid. */
+/* Fills g[0..7] with the non-negative magnitudes of `grid`, indexed by magnitude code, and
+ * returns how many codes the grid rounds to (8; 0 for an unknown grid). IF4 uses the E2M1
+ * table for its FP4 blocks.
+ * Range-restricted E2M1 ["当你的 GPU 学不会算账", section "124B MoE 上的验证": E2M1 limited
+ * to a largest value of 2, i.e. {0, .5, 1, 1.5, 2}; "蚂蚁集团揭秘…", section 六: largest
+ * value 6 lowered to 4, 3 or 2]: the E2M1 table, of which only the codes up to the new largest
+ * magnitude are used (7, 6 or 5 codes); the rest keep their E2M1 values for decoding. */
 int orc_grid_magnitudes(int grid, double* g) {
-  if (grid == ORC_GRID_E2M1 || grid == ORC_GRID_IF4) {
+  if (grid == ORC_GRID_E2M1 || grid == ORC_GRID_IF4 || grid == ORC_GRID_E2M1_MAX4 ||
+      grid == ORC_GRID_E2M1_MAX3 || grid == ORC_GRID_E2M1_MAX2) {
     for (int c = 0; c < 8; ++c) g[c] = minifloat_magnitude(1, 1, c >> 1, c & 1);
+    if (grid == ORC_GRID_E2M1_MAX4) return 7;   /* ... 3, 4 */
+    if (grid == ORC_GRID_E2M1_MAX3) return 6;   /* ... 2, 3 */
+    if (grid == ORC_GRID_E2M1_MAX2) return 5;   /* ... 1.5, 2 */
     return 8;
   }
   if (grid == ORC_GRID_E1M2) {
@@ -150,11 +161,11 @@ double orc_decode_nibble(int grid, uint8_t nib) {
  * (a float under 8 minus a grid point of few bits); far above it they would not be, which is
  * why saturation is decided first. */
 
-static int nearest_magnitude_code(const double* g, double a) {
-  if (a >= g[7]) return 7;
+static int nearest_magnitude_code(const double* g, int n, double a) {
+  if (a >= g[n - 1]) return n - 1;
   int best = 0;
   double bd = fabs(a - g[0]);
-  for (int c = 1; c < 8; ++c) {
+  for (int c = 1; c < n; ++c) {
     double d = fabs(a - g[c]);
     if (d < bd || (d == bd && (c & 1) == 0)) { best = c; bd = d; }
   }
@@ -163,9 +174,9 @@ static int nearest_magnitude_code(const double* g, double a) {
 
 uint8_t orc_round_rtne(int grid, float v) {
   double g[8];
-  orc_grid_magnitudes(grid, g);
+  int n = orc_grid_magnitudes(grid, g);
   int neg = signbit(v) ? 1 : 0;
-  return encode_nibble(grid, neg, nearest_magnitude_code(g, fabs((double)v)));
+  return encode_nibble(grid, neg, nearest_magnitude_code(g, n, fabs((double)v)));
 }
 
 /* Stochastic rounding [IF4 section 6.1 pseudo-code: floor(x) + (random() < frac)], applied on
@@ -173,8 +184,8 @@ uint8_t orc_round_rtne(int grid, float v) {
  * round away from zero iff r < (|v| - lo) / (hi - lo), with r = u * 2^-16 for the element's
  * 16-bit draw u from the counter hash (R12). |v| is first clamped to the largest magnitude
  * (R4, R13). */
-static int sr_magnitude_code(const double* g, double a, uint32_t u) {
-  if (a >= g[7]) return 7;
+static int sr_magnitude_code(const double* g, int n, double a, uint32_t u) {
+  if (a >= g[n - 1]) return n - 1;
   int c = 0;
   while (g[c + 1] <= a) ++c;
   double frac = (a - g[c]) / (g[c + 1] - g[c]);
@@ -184,9 +195,9 @@ static int sr_magnitude_code(const double* g, double a, uint32_t u) {
 
 uint8_t orc_round_sr(int grid, float v, uint32_t u) {
   double g[8];
-  orc_grid_magnitudes(grid, g);
+  int n = orc_grid_magnitudes(grid, g);
   int neg = signbit(v) ? 1 : 0;
-  return encode_nibble(grid, neg, sr_magnitude_code(g, fabs((double)v), u));
+  return encode_nibble(grid, neg, sr_magnitude_code(g, n, fabs((double)v), u));
 }
 
 /* ------------------------------------------------------------------------------------ */
@@ -376,13 +387,14 @@ int orc_quantize(const orc_cfg* cfg, const uint16_t* x, int64_t rows, int64_t co
   const int grid = cfg->grid, scale = cfg->scale;
   const int bs = (scale == ORC_SCALE_UE8M0_1x32) ? 32 : 16;
   if (rows < 0 || cols < 0 || cols % bs != 0 || ld < cols) return -1;
-  if (grid < 0 || grid > 3 || scale < 0 || scale > 2 || cfg->round < 0 || cfg->round > 1) return -1;
+  if (grid < 0 || grid > 6 || scale < 0 || scale > 2 || cfg->round < 0 || cfg->round > 1) return -1;
   if (grid == ORC_GRID_IF4 && (scale != ORC_SCALE_E4M3_1x16 || cfg->round != ORC_ROUND_RTNE)) return -1;
   if (scale == ORC_SCALE_UE8M0_1x32 && grid != ORC_GRID_E2M1) return -1;
+  if (grid >= ORC_GRID_E2M1_MAX4 && scale != ORC_SCALE_FP32_1x16) return -1;
 
   double g[8];
-  orc_grid_magnitudes(grid, g);
-  const float qmax = (float)g[7];
+  const int ncodes = orc_grid_magnitudes(grid, g);
+  const float qmax = (float)g[ncodes - 1];
   const int elem_grid = (grid == ORC_GRID_IF4) ? ORC_GRID_E2M1 : grid;
 
   float alpha = 0.0f;

@@ -23,7 +23,8 @@ def _golden_lines(name):
         return [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
 
 
-GRID_IDS = {"E2M1": O.GRID_E2M1, "E1M2": O.GRID_E1M2, "INT4": O.GRID_INT4}
+GRID_IDS = {"E2M1": O.GRID_E2M1, "E1M2": O.GRID_E1M2, "INT4": O.GRID_INT4,
+            "E2M1_MAX2": O.GRID_E2M1_MAX2}
 
 
 # ------------------------------------------------------------------ number formats
@@ -31,6 +32,57 @@ GRID_IDS = {"E2M1": O.GRID_E2M1, "E1M2": O.GRID_E1M2, "INT4": O.GRID_INT4}
 def test_grids_match_printed_tables():
     for name, *vals in _golden_lines("grids.txt"):
         np.testing.assert_array_equal(O.grid_magnitudes(GRID_IDS[name]), np.array(vals, float))
+
+
+def test_restricted_e2m1_grids_are_prefixes_of_e2m1():
+    # the page's limits 4, 3, 2: the E2M1 magnitudes up to the limit, codes unchanged
+    full = O.grid_magnitudes(O.GRID_E2M1)
+    for grid, top in [(O.GRID_E2M1_MAX4, 4.0), (O.GRID_E2M1_MAX3, 3.0), (O.GRID_E2M1_MAX2, 2.0)]:
+        g = O.grid_magnitudes(grid)
+        np.testing.assert_array_equal(g, full[full <= top])
+        # decoding is E2M1's for every code, also the unused ones
+        for nib in range(16):
+            assert O.decode_nibble(grid, nib) == O.decode_nibble(O.GRID_E2M1, nib)
+
+
+def _restricted_rtne_brute(v, top):
+    """Nearest value of {E2M1 magnitudes <= top}, ties to the even code, saturating; sign kept."""
+    full = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    cand = [(c, m) for c, m in enumerate(full) if m <= top]
+    a = abs(float(v))
+    if a >= top:
+        code = cand[-1][0]
+    else:
+        code = min(cand, key=lambda cm: (abs(a - cm[1]), cm[0] & 1))[0]
+    return (8 if math.copysign(1.0, float(v)) < 0 else 0) | code
+
+
+def test_restricted_e2m1_rtne_brute_force():
+    vals = np.concatenate([np.arange(-8, 8.0001, 0.125), [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0],
+                           np.random.default_rng(3).uniform(-7, 7, 2000)]).astype(np.float32)
+    vals = np.concatenate([vals, -np.zeros(1, np.float32)])
+    for grid, top in [(O.GRID_E2M1_MAX4, 4.0), (O.GRID_E2M1_MAX3, 3.0), (O.GRID_E2M1_MAX2, 2.0)]:
+        got = O.round_rtne(grid, vals)
+        want = np.array([_restricted_rtne_brute(v, top) for v in vals], np.uint8)
+        np.testing.assert_array_equal(got, want)
+
+
+def test_restricted_e2m1_block_scale_and_saturation():
+    # FP32 1x16 scale s = RN(amax / top): in every nonzero block the largest element lands on
+    # the top code, and no code above it is ever produced
+    x = synth.small(17, 64, 128, "laplace")
+    for grid, top, topcode in [(O.GRID_E2M1_MAX4, 4.0, 6), (O.GRID_E2M1_MAX3, 3.0, 5),
+                               (O.GRID_E2M1_MAX2, 2.0, 4)]:
+        cfg = O.OracleConfig(grid=grid, scale=O.SCALE_FP32_1x16, rht=0)
+        out = O.quantize(cfg, x)
+        codes = out["codes"]
+        nib = np.stack([codes & 0xF, codes >> 4], axis=-1).reshape(x.shape[0], -1)
+        assert int((nib & 7).max()) == topcode
+        s = out["scales"].reshape(x.shape[0], -1)
+        blocks_top = (nib & 7).reshape(x.shape[0], -1, 16).max(axis=-1)
+        assert np.all(blocks_top[s > 0] == topcode)
+    with pytest.raises(Exception):
+        O.quantize(O.OracleConfig(grid=O.GRID_E2M1_MAX4, scale=O.SCALE_E4M3_1x16, rht=0), x)
 
 
 def test_e1m2_grid_is_uniform_and_e2m1_is_not():
@@ -220,7 +272,8 @@ def test_sr_probability_exact_by_enumeration():
     k = np.arange(1 << 16, dtype=np.uint32)
     for grid, v in [(O.GRID_E1M2, 1.3), (O.GRID_E1M2, 0.0001), (O.GRID_E2M1, 2.7),
                     (O.GRID_E2M1, 4.5), (O.GRID_INT4, 3.999), (O.GRID_E1M2, 3.4999),
-                    (O.GRID_E2M1, 0.74), (O.GRID_INT4, 6.0000005), (O.GRID_E1M2, 1e-30)]:
+                    (O.GRID_E2M1, 0.74), (O.GRID_INT4, 6.0000005), (O.GRID_E1M2, 1e-30),
+                    (O.GRID_E2M1_MAX4, 3.3), (O.GRID_E2M1_MAX3, 2.7), (O.GRID_E2M1_MAX2, 1.9)]:
         v32 = np.float32(v)
         g = O.grid_magnitudes(grid)
         lo = g[np.searchsorted(g, v32, side="right") - 1]
