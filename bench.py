@@ -45,7 +45,8 @@ def parse():
                    choices=["c2", "c2-quant-only", "c2-unfused", "c3", "c3-rtne", "c3-row-sr",
                             "c4-nvfp4", "c4-nvfp4-given",
                             "c4-nvint4", "c4-mxfp4", "c4-if4", "c5-moe-ufp4", "c5-moe-e2m1",
-                            "c5-dense-ufp4", "c5-dense-e2m1"])
+                            "c5-dense-ufp4", "c5-dense-e2m1", "c2-e2m1", "c2-e2m1-max4",
+                            "c2-e2m1-max3", "c2-e2m1-max2"])
     p.add_argument("--no-extras", action="store_true", help="skip e2e, ratios and CPU baseline")
     a = p.parse_args()
     if a.warmup < 3:
@@ -332,6 +333,15 @@ def make_workload(name):
             from dataclasses import replace
             return RowWorkload(name, desc + " -- rotation off (quantize only)", c2_input,
                                replace(cfg, rht=0, sign_mask=0), "lean_kernel<E1M2,no-rotation,flat>")
+        if name.startswith("c2-e2m1"):
+            # the E2M1 baseline recipe's fwd_y operand (no rotation), full table or range-restricted
+            from dataclasses import replace
+            top = int(name[-1]) if name.endswith(("max4", "max3", "max2")) else 0
+            ec = replace(fq.recipe("e2m1", "fwd_y", "x", sign_mask=mask), e2m1_max=top)
+            what = "E2M1 limited to a largest value of %d" % top if top else "E2M1"
+            return RowWorkload(name, desc.split(", UFP4")[0] + ", E2M1 baseline fwd_y: %s RTNE, no "
+                               "rotation, FP32 1x16 scales" % what, c2_input, ec,
+                               "lean_kernel<%s,no-rotation,flat>" % ("E2M1max%d" % top if top else "E2M1"))
         if name == "c2-unfused":
             return RowWorkload(name, desc + " -- unfused: rotation pass to bf16, then quantize",
                                c2_input, cfg, "rht16_kernel+lean_kernel", unfused=True)
@@ -594,6 +604,8 @@ def _oracle_cfg(cfg):
     import block_scaled_bit_rht16_b200 as fq
     g = {fq.FP4Q_GRID_E2M1: O.GRID_E2M1, fq.FP4Q_GRID_E1M2: O.GRID_E1M2, fq.FP4Q_GRID_INT4: O.GRID_INT4,
          fq.FP4Q_GRID_IF4: O.GRID_IF4}[cfg.grid]
+    if cfg.e2m1_max:
+        g = {4: O.GRID_E2M1_MAX4, 3: O.GRID_E2M1_MAX3, 2: O.GRID_E2M1_MAX2}[cfg.e2m1_max]
     s = {fq.FP4Q_SCALE_FP32_1x16: O.SCALE_FP32_1x16, fq.FP4Q_SCALE_E4M3_1x16_TENSOR: O.SCALE_E4M3_1x16,
          fq.FP4Q_SCALE_UE8M0_1x32: O.SCALE_UE8M0_1x32}[cfg.scale]
     return O.OracleConfig(grid=g, scale=s, round=O.ROUND_SR if cfg.round else O.ROUND_RTNE, rht=cfg.rht,

@@ -35,12 +35,14 @@ class Config:
     sr_seed: int = 0
     dequant: bool = False
     stats: bool = False
+    e2m1_max: int = 0   # 4, 3, 2: range-restricted E2M1 (grid E2M1, FP32 1x16 scale)
 
     def c(self) -> _lib.fp4q_config:
         outputs = FP4Q_OUT_CODES | (FP4Q_OUT_DEQUANT if self.dequant else 0) | \
             (FP4Q_OUT_STATS if self.stats else 0)
         return _lib.fp4q_config(self.grid, self.scale, self.round, self.rht, self.sign_mask,
-                                self.sr_stream, self.sr_seed & 0xFFFFFFFFFFFFFFFF, outputs, 0)
+                                self.sr_stream, self.sr_seed & 0xFFFFFFFFFFFFFFFF, outputs,
+                                self.e2m1_max)
 
     @property
     def block(self) -> int:

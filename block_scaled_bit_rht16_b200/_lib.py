@@ -26,7 +26,7 @@ class fp4q_config(ctypes.Structure):
     _fields_ = [("grid", ctypes.c_int32), ("scale", ctypes.c_int32), ("round", ctypes.c_int32),
                 ("rht", ctypes.c_int32), ("sign_mask", ctypes.c_uint32),
                 ("sr_stream", ctypes.c_uint32), ("sr_seed", ctypes.c_uint64),
-                ("outputs", ctypes.c_uint32), ("reserved", ctypes.c_uint32)]
+                ("outputs", ctypes.c_uint32), ("e2m1_max", ctypes.c_uint32)]
 
 
 class fp4q_stats_t(ctypes.Structure):

@@ -38,12 +38,24 @@ fp4q_status check_cfg(const fp4q_config* cfg) {
   if (cfg->rht != 0 && cfg->rht != 1) return FP4Q_ERR_INVALID_ARG;
   if (cfg->sign_mask > 0xFFFFu) return FP4Q_ERR_INVALID_ARG;
   if (cfg->outputs & ~(uint32_t)(FP4Q_OUT_CODES | FP4Q_OUT_DEQUANT | FP4Q_OUT_STATS)) return FP4Q_ERR_INVALID_ARG;
-  if (cfg->reserved != 0u) return FP4Q_ERR_INVALID_ARG;
+  if (cfg->e2m1_max != 0u && cfg->e2m1_max != 4u && cfg->e2m1_max != 3u && cfg->e2m1_max != 2u)
+    return FP4Q_ERR_INVALID_ARG;
+  if (cfg->e2m1_max != 0u &&
+      (cfg->grid != FP4Q_GRID_E2M1 || cfg->scale != FP4Q_SCALE_FP32_1x16))
+    return FP4Q_ERR_UNSUPPORTED;
   if (cfg->grid == FP4Q_GRID_IF4 &&
       (cfg->scale != FP4Q_SCALE_E4M3_1x16_TENSOR || cfg->round != FP4Q_ROUND_RTNE))
     return FP4Q_ERR_UNSUPPORTED;
   if (cfg->scale == FP4Q_SCALE_UE8M0_1x32 && cfg->grid != FP4Q_GRID_E2M1) return FP4Q_ERR_UNSUPPORTED;
   return FP4Q_OK;
+}
+
+// Kernel grid id: the ABI grid, or the range-restricted E2M1 table selected by e2m1_max.
+int kernel_grid(const fp4q_config* cfg) {
+  if (cfg->e2m1_max == 4u) return kE2M1Max4;
+  if (cfg->e2m1_max == 3u) return kE2M1Max3;
+  if (cfg->e2m1_max == 2u) return kE2M1Max2;
+  return cfg->grid;
 }
 
 int block_elems(const fp4q_config* cfg) { return cfg->scale == FP4Q_SCALE_UE8M0_1x32 ? 32 : 16; }
@@ -152,7 +164,7 @@ fp4q_status fp4q_rht_quantize(const fp4q_config* cfg, const void* x, int64_t row
     }
     if (launch_amax(am, s) != cudaSuccess) return FP4Q_ERR_CUDA;
   }
-  return cuda_status(launch_quantize(cfg->grid, cfg->scale, cfg->round, want_stats, a, s));
+  return cuda_status(launch_quantize(kernel_grid(cfg), cfg->scale, cfg->round, want_stats, a, s));
 }
 
 fp4q_status fp4q_tensor_scale(const fp4q_config* cfg, const void* x, int64_t rows, int64_t cols,
@@ -218,6 +230,7 @@ fp4q_status fp4q_quantize_dual(const fp4q_config* row_cfg, const fp4q_config* co
     if (c->outputs & (FP4Q_OUT_DEQUANT | FP4Q_OUT_STATS)) return FP4Q_ERR_UNSUPPORTED;
   }
   if (row_cfg->grid != col_cfg->grid) return FP4Q_ERR_UNSUPPORTED;
+  if (row_cfg->e2m1_max != 0u || col_cfg->e2m1_max != 0u) return FP4Q_ERR_UNSUPPORTED;
   if (M < 0 || N < 0 || M % 16 != 0 || N % 16 != 0) return FP4Q_ERR_SHAPE;
   if (M > 0 && N > 0 && ld < N) return FP4Q_ERR_SHAPE;
   if (M > 1 && N > 0 && ld % 8 != 0) return FP4Q_ERR_ALIGN;

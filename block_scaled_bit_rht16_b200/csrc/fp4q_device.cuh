@@ -14,11 +14,10 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "fp4q_kernels.cuh"
+
 namespace fp4q {
 
-enum Grid { kE2M1 = 0, kE1M2 = 1, kINT4 = 2, kIF4 = 3 };
-enum Scale { kFP32 = 0, kE4M3 = 1, kUE8M0 = 2 };
-enum Round { kRTNE = 0, kSR = 1 };
 
 // ------------------------------------------------------------------ bf16 / packed helpers
 
@@ -159,6 +158,9 @@ template <> struct GridInfo<kE2M1> { static constexpr float qmax = 6.0f; };
 template <> struct GridInfo<kE1M2> { static constexpr float qmax = 3.5f; };
 template <> struct GridInfo<kINT4> { static constexpr float qmax = 7.0f; };
 template <> struct GridInfo<kIF4> { static constexpr float qmax = 6.0f; };
+template <> struct GridInfo<kE2M1Max4> { static constexpr float qmax = 4.0f; };
+template <> struct GridInfo<kE2M1Max3> { static constexpr float qmax = 3.0f; };
+template <> struct GridInfo<kE2M1Max2> { static constexpr float qmax = 2.0f; };
 
 // E2M1 codes of two values, hardware round-to-nearest-even with saturation to +-6; the sign of
 // each input (including -0) is kept. Result: a in bits 4..7, b in bits 0..3.

@@ -60,9 +60,10 @@ __device__ __forceinline__ uint32_t round_uniform(float q, float vraw, uint32_t 
   }
 }
 
-// E2M1 stochastic rounding of one value: the chosen grid point, signed like vraw.
-__device__ __forceinline__ float e2m1_sr_value(float q, float vraw, uint32_t rnd) {
-  const float a = fminf(fabsf(q), 6.0f);
+// E2M1 stochastic rounding of one value: the chosen grid point, signed like vraw. qmax: 6, or
+// the largest value of a range-restricted E2M1 table (4, 3, 2).
+__device__ __forceinline__ float e2m1_sr_value(float q, float vraw, uint32_t rnd, float qmax = 6.0f) {
+  const float a = fminf(fabsf(q), qmax);
   const bool lo = a < 2.0f, mid = a < 4.0f;
   const float inv_step = lo ? 2.0f : (mid ? 1.0f : 0.5f);
   const float step = lo ? 0.5f : (mid ? 1.0f : 2.0f);
@@ -131,7 +132,7 @@ __device__ __forceinline__ uint2 encode_lean(const float2* P, float s) {
   if (dv.fast) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) Q[i] = div2(dv, P[i]);
-    if constexpr (CLAMP && G != kE2M1) {   // the E2M1 conversion saturates by itself
+    if constexpr (CLAMP && !kIsE2M1<G>) {   // the E2M1 conversion saturates by itself
       constexpr float lim = qmax / kVScale;
 #pragma unroll
       for (int i = 0; i < 8; ++i)
@@ -154,7 +155,7 @@ __device__ __forceinline__ uint2 encode_lean(const float2* P, float s) {
       Q[i] = make_float2(with_sign_of(Q[i].x, P[i].x), with_sign_of(Q[i].y, P[i].y));
   }
   uint32_t w[2];
-  if constexpr (G == kE2M1) {
+  if constexpr (kIsE2M1<G>) {
 #pragma unroll
     for (int l = 0; l < 2; ++l) {
       uint32_t b[4];
@@ -260,7 +261,7 @@ __device__ __forceinline__ uint2 sr_codes(const float* q, const uint32_t* u, con
     for (int j = 7; j >= 0; --j) {
       const int e = 8 * l + j;
       float K;
-      if constexpr (G == kE2M1) {
+      if constexpr (kIsE2M1<G>) {
         const float a = fminf(fabsf(q[e]), qmax);
         const float r = __fadd_rn(__uint_as_float(u[e] * 128u + 0x3F800000u), -1.0f);   // exact
         const bool lo = a < 2.0f, mid = a < 4.0f;
@@ -461,10 +462,11 @@ __device__ __forceinline__ uint32_t encode16(const EncCtx& ctx, const float2* P,
     for (int j = 0; j < 4; ++j) {
       float e0, e1, f0, f1;   // elements 2j, 2j+1 (word 0) and 8+2j, 9+2j (word 1)
       if constexpr (R == kSR) {
-        e0 = e2m1_sr_value(Q[2 * j].x, P[2 * j].x, rnd[2 * j]);
-        e1 = e2m1_sr_value(Q[2 * j + 1].x, P[2 * j + 1].x, rnd[2 * j + 1]);
-        f0 = e2m1_sr_value(Q[2 * j].y, P[2 * j].y, rnd[2 * j + 8]);
-        f1 = e2m1_sr_value(Q[2 * j + 1].y, P[2 * j + 1].y, rnd[2 * j + 9]);
+        constexpr float qm = GridInfo<G>::qmax;
+        e0 = e2m1_sr_value(Q[2 * j].x, P[2 * j].x, rnd[2 * j], qm);
+        e1 = e2m1_sr_value(Q[2 * j + 1].x, P[2 * j + 1].x, rnd[2 * j + 1], qm);
+        f0 = e2m1_sr_value(Q[2 * j].y, P[2 * j].y, rnd[2 * j + 8], qm);
+        f1 = e2m1_sr_value(Q[2 * j + 1].y, P[2 * j + 1].y, rnd[2 * j + 9], qm);
       } else {
         e0 = with_sign_of(Q[2 * j].x, P[2 * j].x);
         e1 = with_sign_of(Q[2 * j + 1].x, P[2 * j + 1].x);

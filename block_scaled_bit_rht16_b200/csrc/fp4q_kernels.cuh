@@ -6,6 +6,15 @@
 
 namespace fp4q {
 
+// kE2M1Max4/3/2: E2M1 with the largest magnitude lowered to 4, 3 or 2 (internal ids; the C
+// ABI selects them with fp4q_config.e2m1_max). Codes and decoding are E2M1's.
+enum Grid { kE2M1 = 0, kE1M2 = 1, kINT4 = 2, kIF4 = 3, kE2M1Max4 = 4, kE2M1Max3 = 5, kE2M1Max2 = 6 };
+
+// Grids encoded by the E2M1 converter (the full table or a range-restricted one).
+template <int G> constexpr bool kIsE2M1 = (G == kE2M1 || G == kE2M1Max4 || G == kE2M1Max3 || G == kE2M1Max2);
+enum Scale { kFP32 = 0, kE4M3 = 1, kUE8M0 = 2 };
+enum Round { kRTNE = 0, kSR = 1 };
+
 // Raw statistics record (doubles), one per CTA in the workspace and once reduced.
 enum {
   ST_SUM_Y2 = 0, ST_SUM_ERR2 = 1, ST_SUM_YXHAT = 2, ST_N = 3, ST_CELL_N = 4, ST_CELL_ERR = 12,

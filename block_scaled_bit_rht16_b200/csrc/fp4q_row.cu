@@ -506,16 +506,19 @@ __global__ void __launch_bounds__(kThreads) division_check_kernel(uint64_t seed,
                                                                   unsigned long long* bad) {
   unsigned long long local = 0;
   const uint64_t stride = (uint64_t)gridDim.x * kThreads;
-  // every mantissa of a in [1, 4) for the three compile-time divisors (the scale quotient
+  // every mantissa of a in [1, 4) for the six compile-time divisors (the scale quotient
   // a / qmax); by scale invariance this covers all a in [2^-100, 2^100]
-  for (uint64_t i = (uint64_t)blockIdx.x * kThreads + threadIdx.x; i < (3ull << 24); i += stride) {
+  for (uint64_t i = (uint64_t)blockIdx.x * kThreads + threadIdx.x; i < (6ull << 24); i += stride) {
     const uint32_t m = (uint32_t)(i & 0xFFFFFFu);
     const float a = __uint_as_float(((127u + (m >> 23)) << 23) | (m & 0x7FFFFFu));
     const int g = (int)(i >> 24);
     float got, want;
     if (g == 0) { got = div_qmax<kE2M1>(a); want = __fdiv_rn(a, 6.0f); }
     else if (g == 1) { got = div_qmax<kE1M2>(a); want = __fdiv_rn(a, 3.5f); }
-    else { got = div_qmax<kINT4>(a); want = __fdiv_rn(a, 7.0f); }
+    else if (g == 2) { got = div_qmax<kINT4>(a); want = __fdiv_rn(a, 7.0f); }
+    else if (g == 3) { got = div_qmax<kE2M1Max4>(a); want = __fdiv_rn(a, 4.0f); }
+    else if (g == 4) { got = div_qmax<kE2M1Max3>(a); want = __fdiv_rn(a, 3.0f); }
+    else { got = div_qmax<kE2M1Max2>(a); want = __fdiv_rn(a, 2.0f); }
     if (__float_as_uint(got) != __float_as_uint(want)) ++local;
   }
   // the block reciprocal: every float S in [2^-60, 2^91) (151 binades x 2^23 mantissas)
@@ -646,8 +649,23 @@ cudaError_t launch_lean(const QuantArgs& a, cudaStream_t st) {
   return flat ? launch_lean3<G, false, true, R>(a, st) : launch_lean3<G, false, false, R>(a, st);
 }
 
+// Range-restricted E2M1 (FP32 scale only): the lean kernel for codes only, else the generic one.
+template <int G>
+cudaError_t launch_restricted(int round, bool stats, const QuantArgs& a, cudaStream_t st) {
+  if (!stats && a.deq == nullptr)
+    return round == kSR ? launch_lean<G, kSR>(a, st) : launch_lean<G, kRTNE>(a, st);
+  return launch_q_round<G, kFP32>(round, stats, a, st);
+}
+
 cudaError_t launch_quantize(int grid, int scale, int round, bool stats, const QuantArgs& a,
                             cudaStream_t st) {
+  if (grid >= kE2M1Max4) {
+    if (scale != kFP32) return cudaErrorInvalidValue;
+    if (grid == kE2M1Max4) return launch_restricted<kE2M1Max4>(round, stats, a, st);
+    if (grid == kE2M1Max3) return launch_restricted<kE2M1Max3>(round, stats, a, st);
+    if (grid == kE2M1Max2) return launch_restricted<kE2M1Max2>(round, stats, a, st);
+    return cudaErrorInvalidValue;
+  }
   if (scale == kFP32 && !stats && a.deq == nullptr) {
     if (round == kSR) {
       if (grid == kE2M1) return launch_lean<kE2M1, kSR>(a, st);

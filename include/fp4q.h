@@ -104,7 +104,13 @@ typedef struct {
   uint32_t sr_stream;  /* SR counter stream: 0 row orientation, 1 column orientation */
   uint64_t sr_seed;    /* SR counter seed */
   uint32_t outputs;    /* FP4Q_OUT_* bits */
-  uint32_t reserved;   /* must be 0 */
+  uint32_t e2m1_max;   /* 0: the grid as named. 4, 3 or 2: range-restricted E2M1, the E2M1 table
+                          up to that largest value ("当你的 GPU 学不会算账", section "124B MoE 上的
+                          验证"; "蚂蚁集团揭秘…", section 六) -- grid E2M1 with the FP32 1x16
+                          scale only, s = amax / e2m1_max, RTNE or SR onto the restricted table,
+                          E2M1 codes (dequantize as E2M1). Other values: FP4Q_ERR_INVALID_ARG;
+                          with another grid or scale, or in fp4q_quantize_dual:
+                          FP4Q_ERR_UNSUPPORTED. */
 } fp4q_config;
 
 /* Statistics of one quantizer call, in the rotated domain (y vs the FP32 xhat). */

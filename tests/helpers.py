@@ -11,8 +11,12 @@ SCALE = {fq.FP4Q_SCALE_FP32_1x16: O.SCALE_FP32_1x16, fq.FP4Q_SCALE_E4M3_1x16_TEN
 ROUND = {fq.FP4Q_ROUND_RTNE: O.ROUND_RTNE, fq.FP4Q_ROUND_SR: O.ROUND_SR}
 
 
+RESTRICTED = {4: O.GRID_E2M1_MAX4, 3: O.GRID_E2M1_MAX3, 2: O.GRID_E2M1_MAX2}
+
+
 def ocfg(cfg: "fq.Config") -> O.OracleConfig:
-    return O.OracleConfig(grid=GRID[cfg.grid], scale=SCALE[cfg.scale], round=ROUND[cfg.round],
+    grid = RESTRICTED[cfg.e2m1_max] if cfg.e2m1_max else GRID[cfg.grid]
+    return O.OracleConfig(grid=grid, scale=SCALE[cfg.scale], round=ROUND[cfg.round],
                           rht=cfg.rht, sign_mask=cfg.sign_mask, sr_stream=cfg.sr_stream,
                           sr_seed=cfg.sr_seed)
 

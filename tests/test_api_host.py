@@ -112,10 +112,17 @@ def test_rejects_bad_arguments_before_launch():
     mx = fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=fq.FP4Q_SCALE_UE8M0_1x32)
     assert _q(mx, cols=48, ld=48) == _lib.FP4Q_ERR_SHAPE
     assert _q(mx, codes=FAKE + 8) == _lib.FP4Q_ERR_ALIGN
-    c = fq.Config().c()
-    c.reserved = 1
-    assert _lib.load().fp4q_rht_quantize(ctypes.byref(c), FAKE, 4, 32, 32, FAKE, FAKE, None, 0, None,
-                                         None, 0, None) == _lib.FP4Q_ERR_INVALID_ARG
+    for bad in (1, 5, 6, 7):   # e2m1_max takes 0, 4, 3, 2
+        c = fq.Config(grid=fq.FP4Q_GRID_E2M1).c()
+        c.e2m1_max = bad
+        assert _lib.load().fp4q_rht_quantize(ctypes.byref(c), FAKE, 4, 32, 32, FAKE, FAKE, None, 0,
+                                             None, None, 0, None) == _lib.FP4Q_ERR_INVALID_ARG
+    # range restriction is for E2M1 with the FP32 1x16 scale only
+    assert _q(fq.Config(grid=fq.FP4Q_GRID_E1M2, e2m1_max=4)) == _lib.FP4Q_ERR_UNSUPPORTED
+    assert _q(fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=fq.FP4Q_SCALE_E4M3_1x16_TENSOR,
+                        e2m1_max=3)) == _lib.FP4Q_ERR_UNSUPPORTED
+    assert _q(fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=fq.FP4Q_SCALE_UE8M0_1x32,
+                        e2m1_max=2)) == _lib.FP4Q_ERR_UNSUPPORTED
     assert _lib.load().fp4q_rht_quantize(None, FAKE, 4, 32, 32, FAKE, FAKE, None, 0, None, None, 0,
                                          None) == _lib.FP4Q_ERR_INVALID_ARG
 
@@ -134,6 +141,9 @@ def test_dual_dequant_rht_stats_validation():
     nv = fq.Config(scale=fq.FP4Q_SCALE_E4M3_1x16_TENSOR).c()
     assert dual(rc=nv) == _lib.FP4Q_ERR_UNSUPPORTED
     assert dual(rc=fq.Config(dequant=True).c()) == _lib.FP4Q_ERR_UNSUPPORTED
+    r4 = fq.Config(grid=fq.FP4Q_GRID_E2M1, round=fq.FP4Q_ROUND_SR, e2m1_max=4).c()
+    c4 = fq.Config(grid=fq.FP4Q_GRID_E2M1, round=fq.FP4Q_ROUND_SR, sr_stream=1, e2m1_max=4).c()
+    assert dual(rc=r4, cc=c4) == _lib.FP4Q_ERR_UNSUPPORTED
     d = fq.Config().c()
     assert lib.fp4q_dequantize(ctypes.byref(d), None, FAKE, None, 4, 32, 0, FAKE, None) == _lib.FP4Q_ERR_INVALID_ARG
     assert lib.fp4q_dequantize(ctypes.byref(d), FAKE, FAKE, None, 4, 24, 0, FAKE, None) == _lib.FP4Q_ERR_SHAPE

@@ -95,6 +95,25 @@ def test_small_ragged(combo, rht, outs):
         compare_quant(cfg, x, gpu_quantize(cfg, x))
 
 
+@pytest.mark.parametrize("top", [4, 3, 2])
+@pytest.mark.parametrize("rnd", [RTNE, SR])
+@pytest.mark.parametrize("rht", [0, 1])
+@pytest.mark.parametrize("outs", ["all", "codes"])
+def test_range_restricted_e2m1(top, rnd, rht, outs):
+    # E2M1 limited to a largest value of 4, 3 or 2: lean kernel for codes only, generic with
+    # dequant and statistics; ragged shapes, many iterations, and the edge blocks
+    full = outs == "all"
+    cfg = fq.Config(grid=E2M1, scale=FP32, round=rnd, rht=rht, sign_mask=MASK, sr_seed=0x77,
+                    dequant=full, stats=full, e2m1_max=top)
+    for rows, cols, kind in [(1, 32, "normal"), (37, 96, "t4"), (130, 1056, "laplace"),
+                             (2048, 2048, "t4")]:
+        x = synth.small(rows * 11 + cols + top, rows, cols, kind)
+        compare_quant(cfg, x, gpu_quantize(cfg, x))
+    for unit in (1.0, 2.0 ** -100, 2.0 ** 40):
+        x = _edge_matrix(unit)
+        compare_quant(cfg, x, gpu_quantize(cfg, x))
+
+
 @pytest.mark.parametrize("combo", COMBOS, ids=_cid)
 def test_many_grid_iterations(combo):
     # 4M elements: each thread of the persistent grid runs several iterations (and a ragged
