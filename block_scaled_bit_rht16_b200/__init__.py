@@ -16,7 +16,7 @@ from dataclasses import dataclass, replace
 
 from . import _lib
 from ._lib import (FP4Q_GRID_E1M2, FP4Q_GRID_E2M1, FP4Q_GRID_IF4, FP4Q_GRID_INT4,  # noqa: F401
-                   FP4Q_OUT_CODES, FP4Q_OUT_DEQUANT, FP4Q_OUT_STATS, FP4Q_ROUND_RTNE,
+                   FP4Q_OUT_CODES, FP4Q_OUT_DEQUANT, FP4Q_OUT_SCALES_MMA, FP4Q_OUT_STATS, FP4Q_ROUND_RTNE,
                    FP4Q_ROUND_SR, FP4Q_SCALE_E4M3_1x16_TENSOR, FP4Q_SCALE_FP32_1x16,
                    FP4Q_SCALE_UE8M0_1x32, Fp4qError)
 
@@ -36,10 +36,11 @@ class Config:
     dequant: bool = False
     stats: bool = False
     e2m1_max: int = 0   # 4, 3, 2: range-restricted E2M1 (grid E2M1, FP32 1x16 scale)
+    mma_scales: bool = False   # E4M3 / UE8M0 scales in the block-scaled MMA tile layout
 
     def c(self) -> _lib.fp4q_config:
         outputs = FP4Q_OUT_CODES | (FP4Q_OUT_DEQUANT if self.dequant else 0) | \
-            (FP4Q_OUT_STATS if self.stats else 0)
+            (FP4Q_OUT_STATS if self.stats else 0) | (FP4Q_OUT_SCALES_MMA if self.mma_scales else 0)
         return _lib.fp4q_config(self.grid, self.scale, self.round, self.rht, self.sign_mask,
                                 self.sr_stream, self.sr_seed & 0xFFFFFFFFFFFFFFFF, outputs,
                                 self.e2m1_max)

@@ -13,7 +13,7 @@ FP4Q_ERR_UNSUPPORTED, FP4Q_ERR_WORKSPACE, FP4Q_ERR_CUDA, FP4Q_ERR_TIMEOUT = 4, 5
 FP4Q_GRID_E2M1, FP4Q_GRID_E1M2, FP4Q_GRID_INT4, FP4Q_GRID_IF4 = 0, 1, 2, 3
 FP4Q_SCALE_FP32_1x16, FP4Q_SCALE_E4M3_1x16_TENSOR, FP4Q_SCALE_UE8M0_1x32 = 0, 1, 2
 FP4Q_ROUND_RTNE, FP4Q_ROUND_SR = 0, 1
-FP4Q_OUT_CODES, FP4Q_OUT_DEQUANT, FP4Q_OUT_STATS = 1, 2, 4
+FP4Q_OUT_CODES, FP4Q_OUT_DEQUANT, FP4Q_OUT_STATS, FP4Q_OUT_SCALES_MMA = 1, 2, 4, 8
 
 # Every function include/fp4q.h declares (checked by the host tests against the header).
 EXPORTS = ["fp4q_status_string", "fp4q_sign_mask_from_seed", "fp4q_workspace_size",

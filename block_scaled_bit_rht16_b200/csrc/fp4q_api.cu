@@ -37,7 +37,11 @@ fp4q_status check_cfg(const fp4q_config* cfg) {
   if (cfg->round != FP4Q_ROUND_RTNE && cfg->round != FP4Q_ROUND_SR) return FP4Q_ERR_INVALID_ARG;
   if (cfg->rht != 0 && cfg->rht != 1) return FP4Q_ERR_INVALID_ARG;
   if (cfg->sign_mask > 0xFFFFu) return FP4Q_ERR_INVALID_ARG;
-  if (cfg->outputs & ~(uint32_t)(FP4Q_OUT_CODES | FP4Q_OUT_DEQUANT | FP4Q_OUT_STATS)) return FP4Q_ERR_INVALID_ARG;
+  if (cfg->outputs & ~(uint32_t)(FP4Q_OUT_CODES | FP4Q_OUT_DEQUANT | FP4Q_OUT_STATS | FP4Q_OUT_SCALES_MMA))
+    return FP4Q_ERR_INVALID_ARG;
+  if ((cfg->outputs & FP4Q_OUT_SCALES_MMA) &&
+      (cfg->scale == FP4Q_SCALE_FP32_1x16 || cfg->grid == FP4Q_GRID_IF4))
+    return FP4Q_ERR_UNSUPPORTED;
   if (cfg->e2m1_max != 0u && cfg->e2m1_max != 4u && cfg->e2m1_max != 3u && cfg->e2m1_max != 2u)
     return FP4Q_ERR_INVALID_ARG;
   if (cfg->e2m1_max != 0u &&
@@ -56,6 +60,13 @@ int kernel_grid(const fp4q_config* cfg) {
   if (cfg->e2m1_max == 3u) return kE2M1Max3;
   if (cfg->e2m1_max == 2u) return kE2M1Max2;
   return cfg->grid;
+}
+
+// The block-scaled MMA scale layout tiles 128 rows x 4 scale columns.
+fp4q_status check_mma_shape(const fp4q_config* cfg, int64_t rows, int64_t cols) {
+  if (!(cfg->outputs & FP4Q_OUT_SCALES_MMA) || rows == 0 || cols == 0) return FP4Q_OK;
+  const int64_t scale_cols = cols / (cfg->scale == FP4Q_SCALE_UE8M0_1x32 ? 32 : 16);
+  return (rows % 128 == 0 && scale_cols % 4 == 0) ? FP4Q_OK : FP4Q_ERR_SHAPE;
 }
 
 int block_elems(const fp4q_config* cfg) { return cfg->scale == FP4Q_SCALE_UE8M0_1x32 ? 32 : 16; }
@@ -110,6 +121,8 @@ fp4q_status fp4q_rht_quantize(const fp4q_config* cfg, const void* x, int64_t row
   const int unit = block_elems(cfg);
   st = check_shape(rows, cols, ld, unit);
   if (st != FP4Q_OK) return st;
+  st = check_mma_shape(cfg, rows, cols);
+  if (st != FP4Q_OK) return st;
   const bool want_deq = (cfg->outputs & FP4Q_OUT_DEQUANT) != 0;
   const bool want_stats = (cfg->outputs & FP4Q_OUT_STATS) != 0;
   const bool nv = cfg->scale == FP4Q_SCALE_E4M3_1x16_TENSOR;
@@ -155,6 +168,7 @@ fp4q_status fp4q_rht_quantize(const fp4q_config* cfg, const void* x, int64_t row
   a.seedx = cfg->sr_seed ^ ((uint64_t)(cfg->sr_stream & 1u) << 63);
   a.contiguous = (ld == cols) ? 1 : 0;
   a.vec32 = (reinterpret_cast<uintptr_t>(x) % 32 == 0 && (rows == 1 || ld % 16 == 0)) ? 1 : 0;
+  a.mma_scales = (cfg->outputs & FP4Q_OUT_SCALES_MMA) ? 1 : 0;
 
   if (compute_alpha) {
     QuantArgs am = a;
@@ -277,6 +291,8 @@ fp4q_status fp4q_dequantize(const fp4q_config* cfg, const uint8_t* codes, const 
   if (inverse_rht != 0 && inverse_rht != 1) return FP4Q_ERR_INVALID_ARG;
   st = check_shape(rows, cols, cols, block_elems(cfg));
   if (st != FP4Q_OK) return st;
+  st = check_mma_shape(cfg, rows, cols);
+  if (st != FP4Q_OK) return st;
   const bool empty = rows == 0 || cols == 0;
   const bool nv = cfg->scale == FP4Q_SCALE_E4M3_1x16_TENSOR;
   if (!empty && (codes == nullptr || scales == nullptr || out == nullptr)) return FP4Q_ERR_INVALID_ARG;
@@ -287,7 +303,8 @@ fp4q_status fp4q_dequantize(const fp4q_config* cfg, const uint8_t* codes, const 
   uint32_t sw[8];
   sign_words(cfg->sign_mask, true, sw);
   return cuda_status(launch_dequant(cfg->grid, cfg->scale, codes, scales, tensor_scale, rows, cols,
-                                    sw, inverse_rht != 0, static_cast<uint16_t*>(out),
+                                    sw, inverse_rht != 0, (cfg->outputs & FP4Q_OUT_SCALES_MMA) != 0,
+                                    static_cast<uint16_t*>(out),
                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 

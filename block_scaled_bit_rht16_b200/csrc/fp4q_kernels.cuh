@@ -52,7 +52,23 @@ struct QuantArgs {
   uint64_t seedx;          // SR: seed ^ (stream << 63)
   int contiguous;          // ld == cols
   int vec32;               // every unit starts 32-byte aligned: one 256-bit load per 16 elements
+  int mma_scales;          // E4M3 / UE8M0 scales in the block-scaled MMA tile layout
 };
+
+// Byte position of scale (r, c) of a [rows, C] scale matrix in the scale-factor layout that
+// sm_100 block-scaled MMA (NVFP4 / MXFP4) consumes: 512-byte tiles of 128 rows x 4 columns,
+// row-major over tiles (C / 4 tiles per tile row); inside a tile, row r and column c sit at
+// (r % 32) * 16 + (r / 32 % 4) * 4 + c % 4. Needs rows % 128 == 0 and C % 4 == 0.
+__host__ __device__ inline int64_t mma_scale_slot(int64_t r, int64_t c, int64_t C) {
+  return ((r >> 7) * (C >> 2) + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
+}
+
+// Slot of block u (row-major block index, C scale columns per row) in either layout.
+__host__ __device__ inline int64_t scale_slot(int64_t u, int64_t C, int mma) {
+  if (!mma) return u;
+  const int64_t r = u / C;
+  return mma_scale_slot(r, u - r * C, C);
+}
 
 struct DualArgs {
   const uint16_t* dy;
@@ -83,7 +99,7 @@ cudaError_t launch_rht16(const uint16_t* x, int64_t rows, int64_t cols, int64_t 
                          const uint32_t* sw, void* out, bool out_fp32, cudaStream_t st);
 cudaError_t launch_dequant(int grid, int scale, const uint8_t* codes, const void* scales,
                            const float* ts, int64_t rows, int64_t cols, const uint32_t* sw,
-                           bool inverse, uint16_t* out, cudaStream_t st);
+                           bool inverse, bool mma_scales, uint16_t* out, cudaStream_t st);
 cudaError_t launch_stats_reduce(WsHeader* ws, const double* partials, cudaStream_t st);
 cudaError_t launch_dual(const DualArgs& a, cudaStream_t st);
 cudaError_t launch_division_check(uint64_t seed, uint64_t n, unsigned long long* bad,

@@ -229,7 +229,8 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantArgs a) {
         if constexpr (S == kFP32) {
           __stcs(reinterpret_cast<float*>(a.scales) + un, s);
         } else {
-          reinterpret_cast<uint8_t*>(a.scales)[un] = (uint8_t)(sbyte | flag);
+          reinterpret_cast<uint8_t*>(a.scales)[scale_slot(un, a.units_per_row, a.mma_scales)] =
+              (uint8_t)(sbyte | flag);
         }
       } else {
         float2 P[8], Q[8];
@@ -247,7 +248,8 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantArgs a) {
         const float mult = __fmul_rn(__uint_as_float((uint32_t)(127 - e) << 23), a.cinv);
         encode_mx<R, STATS>(ctx, P, Q, (uint64_t)un * 8u, a.codes + un * 16, deq, s, mult,
                             amax_y == 0.0f, STATS ? &acc : nullptr);
-        reinterpret_cast<uint8_t*>(a.scales)[un] = (uint8_t)(e + 127);
+        reinterpret_cast<uint8_t*>(a.scales)[scale_slot(un, a.units_per_row, a.mma_scales)] =
+            (uint8_t)(e + 127);
       }
     }
   }
@@ -350,7 +352,8 @@ __global__ void __launch_bounds__(kThreads) lean_nv_kernel(const QuantArgs a) {
     if constexpr (G == kIF4) w = encode_if4<RHT>(P, s, flag);
     else w = encode_lean<G, RHT, true>(P, s);
     __stcs(reinterpret_cast<uint2*>(a.codes) + u, w);
-    reinterpret_cast<uint8_t*>(a.scales)[u] = (uint8_t)(sbyte | flag);
+    reinterpret_cast<uint8_t*>(a.scales)[scale_slot((int64_t)u, a.units_per_row, a.mma_scales)] =
+        (uint8_t)(sbyte | flag);
     lo = nlo;
     hi = nhi;
   }
@@ -424,8 +427,10 @@ struct DeqArgs {
   const float* ts;
   uint16_t* out;
   int64_t nunits;    // 16-element blocks
+  int64_t scale_cols;  // scale columns per row (cols/16, MX cols/32)
   uint32_t sw[8];
   int inverse;
+  int mma_scales;    // E4M3 / UE8M0 scales in the block-scaled MMA tile layout
 };
 
 template <int G, int S>
@@ -440,11 +445,12 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const DeqArgs a) {
     if constexpr (S == kFP32) {
       s = reinterpret_cast<const float*>(a.scales)[u];
     } else if constexpr (S == kE4M3) {
-      const uint32_t b = reinterpret_cast<const uint8_t*>(a.scales)[u];
+      const uint32_t b = reinterpret_cast<const uint8_t*>(a.scales)[scale_slot(u, a.scale_cols, a.mma_scales)];
       int_block = (G == kIF4) && (b & 0x80u);
       s = __fmul_rn(e4m3_to_f32(b & 0x7Fu), alpha);
     } else {
-      const int e = (int)reinterpret_cast<const uint8_t*>(a.scales)[u >> 1] - 127;
+      const int e =
+          (int)reinterpret_cast<const uint8_t*>(a.scales)[scale_slot(u >> 1, a.scale_cols, a.mma_scales)] - 127;
       s = (e >= -126) ? __uint_as_float((uint32_t)(127 + e) << 23) : 0x1p-127f;
     }
     float v[16];
@@ -748,13 +754,15 @@ cudaError_t launch_dq(const DeqArgs& a, cudaStream_t st) {
 
 cudaError_t launch_dequant(int grid, int scale, const uint8_t* codes, const void* scales,
                            const float* ts, int64_t rows, int64_t cols, const uint32_t* sw,
-                           bool inverse, uint16_t* out, cudaStream_t st) {
+                           bool inverse, bool mma_scales, uint16_t* out, cudaStream_t st) {
   DeqArgs a{};
   a.codes = codes;
   a.scales = scales;
   a.ts = ts;
   a.out = out;
   a.nunits = rows * (cols / 16);
+  a.scale_cols = scale == kUE8M0 ? cols / 32 : cols / 16;
+  a.mma_scales = mma_scales ? 1 : 0;
   for (int k = 0; k < 8; ++k) a.sw[k] = sw[k];
   a.inverse = inverse ? 1 : 0;
   if (a.nunits == 0) return cudaSuccess;

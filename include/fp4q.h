@@ -92,8 +92,16 @@ typedef enum {
  * orientation. The expected code differs from |v| by at most 2^-16 of the cell width. */
 typedef enum { FP4Q_ROUND_RTNE = 0, FP4Q_ROUND_SR = 1 } fp4q_round;
 
-/* Output bits of fp4q_config.outputs. Codes and scales are always written. */
-enum { FP4Q_OUT_CODES = 1u, FP4Q_OUT_DEQUANT = 2u, FP4Q_OUT_STATS = 4u };
+/* Output bits of fp4q_config.outputs. Codes and scales are always written.
+ * FP4Q_OUT_SCALES_MMA: E4M3 / UE8M0 block scales in the scale-factor layout that sm_100
+ *   block-scaled tensor-core MMA (NVFP4, MXFP4) consumes, instead of row-major: the [rows, C]
+ *   scale matrix (C = cols/16, MX cols/32) as 512-byte tiles of 128 rows x 4 columns, row-major
+ *   over tiles, with row r, column c of a tile at byte (r % 32) * 16 + (r / 32 % 4) * 4 + c % 4.
+ *   The buffer size is unchanged. Needs rows % 128 == 0 and C % 4 == 0 (else FP4Q_ERR_SHAPE);
+ *   FP32 scales and IF4 (flagged scale bytes): FP4Q_ERR_UNSUPPORTED. fp4q_dequantize reads the
+ *   scales in the layout the same bit names. The pages give no interface; this serves the
+ *   hardware FP4 GEMM path the NVFP4 recipe targets ("低精度量化技术：IF4…", section 3.2). */
+enum { FP4Q_OUT_CODES = 1u, FP4Q_OUT_DEQUANT = 2u, FP4Q_OUT_STATS = 4u, FP4Q_OUT_SCALES_MMA = 8u };
 
 typedef struct {
   int32_t grid;        /* fp4q_grid */

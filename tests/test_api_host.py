@@ -117,6 +117,13 @@ def test_rejects_bad_arguments_before_launch():
         c.e2m1_max = bad
         assert _lib.load().fp4q_rht_quantize(ctypes.byref(c), FAKE, 4, 32, 32, FAKE, FAKE, None, 0,
                                              None, None, 0, None) == _lib.FP4Q_ERR_INVALID_ARG
+    # block-scaled MMA scale layout: E4M3 / UE8M0 scales only, 128-row and 4-column tiles
+    nvm = fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=fq.FP4Q_SCALE_E4M3_1x16_TENSOR, mma_scales=True)
+    assert _q(fq.Config(mma_scales=True)) == _lib.FP4Q_ERR_UNSUPPORTED          # FP32 scales
+    assert _q(fq.Config(grid=fq.FP4Q_GRID_IF4, scale=fq.FP4Q_SCALE_E4M3_1x16_TENSOR,
+                        mma_scales=True), ts=FAKE) == _lib.FP4Q_ERR_UNSUPPORTED
+    assert _q(nvm, rows=4, cols=64, ld=64, ts=FAKE) == _lib.FP4Q_ERR_SHAPE        # rows % 128
+    assert _q(nvm, rows=128, cols=32, ld=32, ts=FAKE) == _lib.FP4Q_ERR_SHAPE      # 2 scale columns
     # range restriction is for E2M1 with the FP32 1x16 scale only
     assert _q(fq.Config(grid=fq.FP4Q_GRID_E1M2, e2m1_max=4)) == _lib.FP4Q_ERR_UNSUPPORTED
     assert _q(fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=fq.FP4Q_SCALE_E4M3_1x16_TENSOR,
