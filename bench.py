@@ -46,7 +46,7 @@ def parse():
                             "c4-nvfp4", "c4-nvfp4-given",
                             "c4-nvint4", "c4-mxfp4", "c4-if4", "c5-moe-ufp4", "c5-moe-e2m1",
                             "c5-dense-ufp4", "c5-dense-e2m1", "c2-e2m1", "c2-e2m1-max4",
-                            "c2-e2m1-max3", "c2-e2m1-max2"])
+                            "c2-e2m1-max3", "c2-e2m1-max2", "c5-moe-nvfp4-grouped"])
     p.add_argument("--no-extras", action="store_true", help="skip e2e, ratios and CPU baseline")
     a = p.parse_args()
     if a.warmup < 3:
@@ -254,6 +254,34 @@ class RowWorkload(Workload):
             h.copy_(d, non_blocking=True)
 
 
+class GroupedWorkload(RowWorkload):
+    """fp4q_rht_quantize_grouped over [rows, cols] with row groups of the given sizes: per-group
+    E4M3 tensor scales computed every step (amax pass, alpha, quantize pass)."""
+
+    def __init__(self, name, desc, make_input, cfg, kernel_key, group_rows):
+        super().__init__(name, desc, make_input, cfg, kernel_key)
+        self.group_rows = list(group_rows)
+
+    def setup(self, device, l2_bytes):
+        import numpy as np
+        import torch
+        super().setup(device, l2_bytes)
+        offs = np.concatenate([[0], np.cumsum(self.group_rows)]).astype(np.int64)
+        assert offs[-1] == self.rows
+        self.offsets = torch.from_numpy(offs).to(device)
+        n = len(self.group_rows)
+        c = self.cfg.c()
+        nws = self.fq._lib.load().fp4q_grouped_workspace_size(__import__("ctypes").byref(c), n)
+        for _, out, _ in self.sets:
+            out.tensor_scale = torch.zeros(n, dtype=torch.float32, device=device)
+            out.workspace = torch.empty(nws, dtype=torch.uint8, device=device)
+        self.launches_per_step = 3   # grouped amax, per-group alpha, quantize
+
+    def enqueue(self, i, stream):
+        x, out, _ = self.sets[i % self.R]
+        self.fq.rht_quantize_grouped(self.cfg, x, self.offsets, out=out, stream=stream)
+
+
 class DualWorkload(Workload):
     def __init__(self, name, desc, make_input, rc, cc, kernel_key):
         self.name, self.desc, self.rc, self.cc, self.kernel_key = name, desc, rc, cc, kernel_key
@@ -376,6 +404,18 @@ def make_workload(name):
         if kind in ("nvfp4", "nvint4", "if4"):
             key += "+amax_kernel<rotation,flat>"
         return RowWorkload(name, "[16384,5120] Laplace(0,1), RHT16, %s" % kind, synth.workload4, cfg, key)
+    if name == "c5-moe-nvfp4-grouped":
+        mask = fq.sign_mask_from_seed(synth.sign_seed(5))
+        cfg = fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=fq.FP4Q_SCALE_E4M3_1x16_TENSOR, rht=1,
+                        sign_mask=mask)
+
+        def inp():
+            return np.concatenate([synth.workload5_expert(e) for e in range(64)], axis=0)
+        return GroupedWorkload(name, "MoE experts [64,2048,7168] as [131072,7168], sigma_e log-uniform "
+                               "[0.1,10], NVFP4 (RHT16, E4M3 1x16 + one FP32 tensor scale per expert, "
+                               "computed each step)", inp, cfg,
+                               "lean_nv_kernel<E2M1,rotation,flat,grouped>+grouped_amax_kernel",
+                               [2048] * 64)
     if name.startswith("c5"):
         mask = fq.sign_mask_from_seed(synth.sign_seed(5))
         ufp4 = name.endswith("ufp4")

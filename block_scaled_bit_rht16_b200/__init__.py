@@ -154,6 +154,34 @@ def rht_quantize(cfg: Config, x, *, out: Quantized = None, tensor_scale=None,
     return out
 
 
+def rht_quantize_grouped(cfg: Config, x, group_offsets, *, out: Quantized = None,
+                         tensor_scales=None, tensor_scales_given: bool = False,
+                         stream=None) -> Quantized:
+    """fp4q_rht_quantize_grouped. group_offsets: device int64[n_groups + 1] row offsets.
+    tensor_scales (E4M3 scales): device float32[n_groups], read when tensor_scales_given, else
+    written with each group's computed alpha; returned as Quantized.tensor_scale."""
+    torch = _torch()
+    rows, cols, ld = _check_input(x)
+    n_groups = int(group_offsets.numel()) - 1
+    c = cfg.c()
+    if out is None:
+        codes, scales = _alloc_outputs(cfg, rows, cols, x.device)
+        nws = _lib.load().fp4q_grouped_workspace_size(ctypes.byref(c), n_groups)
+        ws = torch.empty(nws, dtype=torch.uint8, device=x.device) if nws else None
+        out = Quantized(codes, scales, None, None, ws)
+    if tensor_scales is not None:
+        out.tensor_scale = tensor_scales
+    if cfg.scale == FP4Q_SCALE_E4M3_1x16_TENSOR and out.tensor_scale is None:
+        out.tensor_scale = torch.zeros(max(n_groups, 1), dtype=torch.float32, device=x.device)
+    ws = out.workspace
+    st = _lib.load().fp4q_rht_quantize_grouped(
+        ctypes.byref(c), _ptr(x), rows, cols, ld, _ptr(group_offsets), n_groups, _ptr(out.codes),
+        _ptr(out.scales), _ptr(out.tensor_scale), int(bool(tensor_scales_given)), _ptr(ws),
+        0 if ws is None else ws.numel(), _stream_ptr(stream))
+    _lib.check(st, "fp4q_rht_quantize_grouped")
+    return out
+
+
 def tensor_scale(cfg: Config, x, *, out=None, workspace=None, stream=None):
     """fp4q_tensor_scale: the FP32 tensor scale alpha of x (E4M3 configurations) -> float32[1]."""
     torch = _torch()

@@ -19,7 +19,8 @@ FP4Q_OUT_CODES, FP4Q_OUT_DEQUANT, FP4Q_OUT_STATS, FP4Q_OUT_SCALES_MMA = 1, 2, 4,
 EXPORTS = ["fp4q_status_string", "fp4q_sign_mask_from_seed", "fp4q_workspace_size",
            "fp4q_rht_quantize", "fp4q_quantize_dual", "fp4q_dequantize", "fp4q_if4_select",
            "fp4q_stats", "fp4q_rht16", "fp4q_check_division", "fp4q_device_status",
-           "fp4q_check_wait_timeout", "fp4q_tensor_scale", "fp4q_rht_quantize_noalloc"]
+           "fp4q_check_wait_timeout", "fp4q_tensor_scale", "fp4q_rht_quantize_noalloc",
+           "fp4q_grouped_workspace_size", "fp4q_rht_quantize_grouped"]
 
 
 class fp4q_config(ctypes.Structure):
@@ -62,6 +63,10 @@ SIGNATURES = {
     "fp4q_tensor_scale": (ctypes.c_int, [_CFG, _P, _I64, _I64, _I64, _P, _P, ctypes.c_size_t, _P]),
     "fp4q_rht_quantize_noalloc": (ctypes.c_int, [_CFG, _P, _I64, _I64, _I64, _P, _P, _P,
                                                  ctypes.c_int32, _P, _P]),
+    "fp4q_grouped_workspace_size": (ctypes.c_size_t, [_CFG, ctypes.c_int32]),
+    "fp4q_rht_quantize_grouped": (ctypes.c_int, [_CFG, _P, _I64, _I64, _I64, _P, ctypes.c_int32,
+                                                 _P, _P, _P, ctypes.c_int32, _P, ctypes.c_size_t,
+                                                 _P]),
 }
 
 _lib = None

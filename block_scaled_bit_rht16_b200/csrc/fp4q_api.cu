@@ -84,6 +84,27 @@ fp4q_status check_shape(int64_t rows, int64_t cols, int64_t ld, int unit) {
 
 fp4q_status cuda_status(cudaError_t e) { return e == cudaSuccess ? FP4Q_OK : FP4Q_ERR_CUDA; }
 
+// Kernel arguments common to the row quantizers (a valid configuration and shape).
+QuantArgs base_args(const fp4q_config* cfg, const void* x, int64_t rows, int64_t cols, int64_t ld,
+                    uint8_t* codes, void* scales) {
+  QuantArgs a{};
+  a.x = static_cast<const uint16_t*>(x);
+  a.rows = rows;
+  a.cols = cols;
+  a.ld = ld;
+  a.units_per_row = cols / block_elems(cfg);
+  a.nunits = rows * a.units_per_row;
+  a.codes = codes;
+  a.scales = scales;
+  sign_words(cfg->sign_mask, cfg->rht != 0, a.sw);
+  a.c = cfg->rht ? 4.0f : 1.0f;
+  a.cinv = cfg->rht ? 0.25f : 1.0f;
+  a.seedx = cfg->sr_seed ^ ((uint64_t)(cfg->sr_stream & 1u) << 63);
+  a.contiguous = (ld == cols) ? 1 : 0;
+  a.vec32 = (reinterpret_cast<uintptr_t>(x) % 32 == 0 && (rows == 1 || ld % 16 == 0)) ? 1 : 0;
+  a.mma_scales = (cfg->outputs & FP4Q_OUT_SCALES_MMA) ? 1 : 0;
+  return a;
+}
 }  // namespace
 
 extern "C" {
@@ -111,6 +132,7 @@ size_t fp4q_workspace_size(const fp4q_config* cfg, int64_t rows, int64_t cols) {
   if (!stats && !nv) return 0;
   return sizeof(WsHeader) + (stats ? stats_bytes() : 0);
 }
+
 
 fp4q_status fp4q_rht_quantize(const fp4q_config* cfg, const void* x, int64_t rows, int64_t cols,
                               int64_t ld, uint8_t* codes, void* scales, float* tensor_scale,
@@ -148,27 +170,12 @@ fp4q_status fp4q_rht_quantize(const fp4q_config* cfg, const void* x, int64_t row
     return FP4Q_OK;
   }
 
-  QuantArgs a{};
-  a.x = static_cast<const uint16_t*>(x);
-  a.rows = rows;
-  a.cols = cols;
-  a.ld = ld;
-  a.units_per_row = cols / unit;
-  a.nunits = rows * a.units_per_row;
-  a.codes = codes;
-  a.scales = scales;
+  QuantArgs a = base_args(cfg, x, rows, cols, ld, codes, scales);
   a.deq = want_deq ? static_cast<uint16_t*>(dequant) : nullptr;
   a.ts_in = (nv && tensor_scale_given) ? tensor_scale : nullptr;
   a.ts_out = compute_alpha ? tensor_scale : nullptr;
   a.ws = need > 0 ? ws : nullptr;
   a.partials = want_stats ? reinterpret_cast<double*>(static_cast<char*>(workspace) + sizeof(WsHeader)) : nullptr;
-  sign_words(cfg->sign_mask, cfg->rht != 0, a.sw);
-  a.c = cfg->rht ? 4.0f : 1.0f;
-  a.cinv = cfg->rht ? 0.25f : 1.0f;
-  a.seedx = cfg->sr_seed ^ ((uint64_t)(cfg->sr_stream & 1u) << 63);
-  a.contiguous = (ld == cols) ? 1 : 0;
-  a.vec32 = (reinterpret_cast<uintptr_t>(x) % 32 == 0 && (rows == 1 || ld % 16 == 0)) ? 1 : 0;
-  a.mma_scales = (cfg->outputs & FP4Q_OUT_SCALES_MMA) ? 1 : 0;
 
   if (compute_alpha) {
     QuantArgs am = a;
@@ -179,6 +186,56 @@ fp4q_status fp4q_rht_quantize(const fp4q_config* cfg, const void* x, int64_t row
     if (launch_amax(am, s) != cudaSuccess) return FP4Q_ERR_CUDA;
   }
   return cuda_status(launch_quantize(kernel_grid(cfg), cfg->scale, cfg->round, want_stats, a, s));
+}
+
+size_t fp4q_grouped_workspace_size(const fp4q_config* cfg, int32_t n_groups) {
+  if (cfg == nullptr || n_groups < 1 || n_groups > (1 << 24)) return 0;
+  if (cfg->scale != FP4Q_SCALE_E4M3_1x16_TENSOR) return 0;
+  return ((size_t)n_groups * sizeof(uint32_t) + 255) / 256 * 256;
+}
+
+fp4q_status fp4q_rht_quantize_grouped(const fp4q_config* cfg, const void* x, int64_t rows,
+                                      int64_t cols, int64_t ld, const int64_t* group_offsets,
+                                      int32_t n_groups, uint8_t* codes, void* scales,
+                                      float* tensor_scales, int32_t tensor_scales_given,
+                                      void* workspace, size_t workspace_bytes,
+                                      fp4q_stream_t stream) {
+  fp4q_status st = check_cfg(cfg);
+  if (st != FP4Q_OK) return st;
+  if (cfg->outputs & (FP4Q_OUT_DEQUANT | FP4Q_OUT_STATS)) return FP4Q_ERR_UNSUPPORTED;
+  if (n_groups < 1 || n_groups > (1 << 24)) return FP4Q_ERR_INVALID_ARG;
+  if (tensor_scales_given != 0 && tensor_scales_given != 1) return FP4Q_ERR_INVALID_ARG;
+  if (cfg->scale != FP4Q_SCALE_E4M3_1x16_TENSOR)   // no per-group state
+    return fp4q_rht_quantize(cfg, x, rows, cols, ld, codes, scales, nullptr, 0, nullptr, nullptr,
+                             0, stream);
+  st = check_shape(rows, cols, ld, 16);
+  if (st != FP4Q_OK) return st;
+  st = check_mma_shape(cfg, rows, cols);
+  if (st != FP4Q_OK) return st;
+  const bool empty = rows == 0 || cols == 0;
+  if (group_offsets == nullptr || tensor_scales == nullptr) return FP4Q_ERR_INVALID_ARG;
+  if (!empty && (x == nullptr || codes == nullptr || scales == nullptr)) return FP4Q_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(codes, 8) || !aligned(scales, 4) || !aligned(group_offsets, 8) ||
+      !aligned(tensor_scales, 4) || !aligned(workspace, 256))
+    return FP4Q_ERR_ALIGN;
+  const bool given = tensor_scales_given != 0;
+  const size_t need = given ? 0 : fp4q_grouped_workspace_size(cfg, n_groups);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return FP4Q_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!given && cudaMemsetAsync(workspace, 0, need, s) != cudaSuccess) return FP4Q_ERR_CUDA;
+  QuantArgs a = base_args(cfg, x, rows, cols, ld, codes, scales);
+  a.group_off = group_offsets;
+  a.n_groups = n_groups;
+  a.group_ts = tensor_scales;
+  a.group_amax = static_cast<uint32_t*>(workspace);
+  if (!given) {
+    // every group's alpha, 0 for the empty ones (all of them when the tensor is empty)
+    if (!empty && launch_grouped_amax(a, s) != cudaSuccess) return FP4Q_ERR_CUDA;
+    const float qmax = cfg->grid == FP4Q_GRID_INT4 ? 7.0f : (cfg->grid == FP4Q_GRID_E1M2 ? 3.5f : 6.0f);
+    if (launch_grouped_alpha(a, qmax, s) != cudaSuccess) return FP4Q_ERR_CUDA;
+  }
+  if (empty) return FP4Q_OK;
+  return cuda_status(launch_quantize_grouped(cfg->grid, a, s));
 }
 
 fp4q_status fp4q_tensor_scale(const fp4q_config* cfg, const void* x, int64_t rows, int64_t cols,

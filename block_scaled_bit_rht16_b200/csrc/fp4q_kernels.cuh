@@ -53,6 +53,12 @@ struct QuantArgs {
   int contiguous;          // ld == cols
   int vec32;               // every unit starts 32-byte aligned: one 256-bit load per 16 elements
   int mma_scales;          // E4M3 / UE8M0 scales in the block-scaled MMA tile layout
+  // grouped (E4M3): rows [group_off[g], group_off[g+1]) form group g, with tensor scale
+  // group_ts[g]; group_amax: per-group rotated amax bits (workspace) for the computed scales
+  const int64_t* group_off;
+  int32_t n_groups;
+  float* group_ts;
+  uint32_t* group_amax;
 };
 
 // Byte position of scale (r, c) of a [rows, C] scale matrix in the scale-factor layout that
@@ -94,6 +100,9 @@ constexpr int32_t kStatusSelfTest = 2;
 cudaError_t launch_quantize(int grid, int scale, int round, bool stats, const QuantArgs& a,
                             cudaStream_t st);
 cudaError_t launch_amax(const QuantArgs& a, cudaStream_t st);
+cudaError_t launch_grouped_amax(const QuantArgs& a, cudaStream_t st);
+cudaError_t launch_grouped_alpha(const QuantArgs& a, float qmax, cudaStream_t st);
+cudaError_t launch_quantize_grouped(int grid, const QuantArgs& a, cudaStream_t st);
 cudaError_t launch_alpha(WsHeader* ws, float qmax, float* tensor_scale, cudaStream_t st);
 cudaError_t launch_rht16(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
                          const uint32_t* sw, void* out, bool out_fp32, cudaStream_t st);

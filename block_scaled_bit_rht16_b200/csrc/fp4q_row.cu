@@ -307,25 +307,41 @@ __global__ void wait_timeout_kernel(unsigned long long limit_ns) {
   mbar_arrive(&bar);   // complete the phase so the barrier is left consistent
 }
 
+// Group of row r: the last g in [0, n) with off[g] <= r (offsets nondecreasing; empty groups
+// are skipped). The result is always a valid index, whatever the offsets hold.
+__device__ __forceinline__ int group_of(const int64_t* off, int n, int64_t r) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(off + mid) <= r) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
 // E4M3 block scale + FP32 tensor scale, round to nearest even, codes and scale bytes only.
 // G = kIF4: the per-block FP4 / INT4 choice, flagged in bit 7 of the scale byte.
-template <int G, bool RHT, bool FLAT>
+// GROUPED: the tensor scale is that of the block's row group (group_ts), looked up again only
+// when a thread's block leaves the rows of the group it last used.
+template <int G, bool RHT, bool FLAT, bool GROUPED = false>
 __global__ void __launch_bounds__(kThreads) lean_nv_kernel(const QuantArgs a) {
   constexpr float qmax = GridInfo<G>::qmax;
   constexpr float kCinv = RHT ? 0.25f : 1.0f;
   const uint32_t zero_sw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
   pdl_enter();
-  float alpha;
-  if (a.ts_in != nullptr) {
-    alpha = *a.ts_in;
-  } else {
-    alpha = __fdiv_rn(__uint_as_float(a.ws->amax_bits), __fmul_rn(qmax, 448.0f));
-    if (a.ts_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *a.ts_out = alpha;
+  float alpha = 0.0f;
+  if constexpr (!GROUPED) {
+    if (a.ts_in != nullptr) {
+      alpha = *a.ts_in;
+    } else {
+      alpha = __fdiv_rn(__uint_as_float(a.ws->amax_bits), __fmul_rn(qmax, 448.0f));
+      if (a.ts_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *a.ts_out = alpha;
+    }
   }
-  const float denom = __fmul_rn(alpha, qmax);
+  float denom = __fmul_rn(alpha, qmax);
   // RN(amax / denom) for every block through the correction step on one reciprocal (exact for
   // quotients in [2^-20, 2^64); the E4M3 conversion sends anything below 2^-11 to 0 either way)
-  const Divider dd = make_divider(denom, 1.0f);
+  Divider dd = make_divider(denom, 1.0f);
+  int64_t g_lo = 0, g_hi = 0;   // rows of the group whose scale is loaded (none yet)
   using Idx = typename UnitIdx<FLAT>::T;
   const Idx n = (Idx)a.nunits;
   const Idx stride = (Idx)gridDim.x * kThreads;
@@ -340,6 +356,17 @@ __global__ void __launch_bounds__(kThreads) lean_nv_kernel(const QuantArgs a) {
     unpack16(lo, hi, RHT ? a.sw : zero_sw, P);
     if constexpr (RHT) fwht16(P);
     const float amax_y = __fmul_rn(absmax16(P), kCinv);
+    if constexpr (GROUPED) {
+      const int64_t r = (int64_t)u / a.units_per_row;
+      if (r < g_lo || r >= g_hi) {
+        const int g = group_of(a.group_off, a.n_groups, r);
+        g_lo = __ldg(a.group_off + g);
+        g_hi = __ldg(a.group_off + g + 1);
+        alpha = a.group_ts[g];
+        denom = __fmul_rn(alpha, qmax);
+        dd = make_divider(denom, 1.0f);
+      }
+    }
     float delta = 0.0f;
     if (dd.fast) delta = div2(dd, make_float2(amax_y, 0.0f)).x;
     // outside the fast range, and for quotients too large for the correction step (a given
@@ -389,6 +416,38 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const QuantArgs a) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   if ((threadIdx.x & 31) == 0 && m != 0u) atomicMax(&a.ws->amax_bits, m);
+}
+
+// Per-group amax of the rotated tensor: one warp per row (a row lies in one group), the
+// row's blocks strided over the lanes, a warp maximum, one atomicMax per row into the group's
+// slot.
+template <bool RHT>
+__global__ void __launch_bounds__(kThreads) grouped_amax_kernel(const QuantArgs a) {
+  constexpr float kCinv = RHT ? 0.25f : 1.0f;
+  const uint32_t zero_sw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
+  for (int64_t r = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); r < a.rows; r += warps) {
+    uint32_t m = 0u;
+    for (int64_t b = lane; b < a.units_per_row; b += 32) {
+      uint4 lo, hi;
+      load16(a.x + r * a.ld + b * 16, a.vec32 != 0, lo, hi);
+      float2 P[8];
+      unpack16(lo, hi, RHT ? a.sw : zero_sw, P);
+      if constexpr (RHT) fwht16(P);
+      m = max(m, __float_as_uint(__fmul_rn(absmax16(P), kCinv)));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (lane == 0 && m != 0u) atomicMax(a.group_amax + group_of(a.group_off, a.n_groups, r), m);
+  }
+}
+
+// alpha_g = RN(amax_g / RN(qmax * 448)) for every group (0 for an empty or all-zero group).
+__global__ void grouped_alpha_kernel(const uint32_t* amax, int n, float qmax, float* ts) {
+  for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < n; g += gridDim.x * blockDim.x)
+    ts[g] = __fdiv_rn(__uint_as_float(amax[g]), __fmul_rn(qmax, 448.0f));
 }
 
 // The rotation alone: y = 1/4 H16 D x, stored bf16 (RNE) or FP32.
@@ -634,18 +693,18 @@ cudaError_t launch_lean3(const QuantArgs& a, cudaStream_t st) {
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-template <int G, bool RHT, bool FLAT>
-cudaError_t launch_lean_nv3(const QuantArgs& a, cudaStream_t st) {
-  auto k = lean_nv_kernel<G, RHT, FLAT>;
+template <int G, bool RHT, bool FLAT, bool GROUPED>
+cudaError_t launch_lean_nv4(const QuantArgs& a, cudaStream_t st) {
+  auto k = lean_nv_kernel<G, RHT, FLAT, GROUPED>;
   const cudaError_t e = launch_pdl(k, persistent_grid(k, a.nunits), st, a);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-template <int G>
+template <int G, bool GROUPED = false>
 cudaError_t launch_lean_nv(const QuantArgs& a, cudaStream_t st) {
   const bool rht = a.c != 1.0f, flat = a.contiguous && a.vec32 && a.nunits < (int64_t(1) << 31);
-  if (rht) return flat ? launch_lean_nv3<G, true, true>(a, st) : launch_lean_nv3<G, true, false>(a, st);
-  return flat ? launch_lean_nv3<G, false, true>(a, st) : launch_lean_nv3<G, false, false>(a, st);
+  if (rht) return flat ? launch_lean_nv4<G, true, true, GROUPED>(a, st) : launch_lean_nv4<G, true, false, GROUPED>(a, st);
+  return flat ? launch_lean_nv4<G, false, true, GROUPED>(a, st) : launch_lean_nv4<G, false, false, GROUPED>(a, st);
 }
 
 template <int G, int R>
@@ -702,6 +761,25 @@ cudaError_t launch_quantize(int grid, int scale, int round, bool stats, const Qu
     if (grid == kE2M1) return launch_q_round<kE2M1, kUE8M0>(round, stats, a, st);
   }
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_quantize_grouped(int grid, const QuantArgs& a, cudaStream_t st) {
+  if (grid == kE2M1) return launch_lean_nv<kE2M1, true>(a, st);
+  if (grid == kE1M2) return launch_lean_nv<kE1M2, true>(a, st);
+  if (grid == kINT4) return launch_lean_nv<kINT4, true>(a, st);
+  if (grid == kIF4) return launch_lean_nv<kIF4, true>(a, st);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_grouped_amax(const QuantArgs& a, cudaStream_t st) {
+  auto k = a.c != 1.0f ? grouped_amax_kernel<true> : grouped_amax_kernel<false>;
+  const cudaError_t e = launch_pdl(k, persistent_grid(k, a.rows * 32), st, a);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+cudaError_t launch_grouped_alpha(const QuantArgs& a, float qmax, cudaStream_t st) {
+  grouped_alpha_kernel<<<(a.n_groups + 255) / 256, 256, 0, st>>>(a.group_amax, a.n_groups, qmax, a.group_ts);
+  return cudaGetLastError();
 }
 
 template <bool RHT, bool FLAT>

@@ -229,6 +229,30 @@ fp4q_status fp4q_rht_quantize_noalloc(const fp4q_config* cfg, const void* x, int
                                       float* tensor_scale, int32_t tensor_scale_given,
                                       void* dequant, fp4q_stream_t stream);
 
+/* Grouped quantization of the rows of x as n_groups consecutive tensors, e.g. the experts of an
+ * MoE layer with variable token counts ("当你的 GPU 学不会算账", section "124B MoE 上的验证"
+ * and the MoE rows of the scale table): group g is rows [group_offsets[g], group_offsets[g+1]).
+ * With the E4M3 scale (NVFP4, NVINT4, IF4) every group has its own FP32 tensor scale
+ * alpha_g = RN(A_g / RN(qmax * 448)), A_g the amax of the group's rotated rows: tensor_scales
+ * (device float[n_groups]) receives the alpha_g, or supplies them when tensor_scales_given; an
+ * empty or all-zero group gets alpha 0. Codes and scales are laid out as for one
+ * fp4q_rht_quantize call over all rows (FP4Q_OUT_SCALES_MMA included); SR indices are global.
+ * With the FP32 or UE8M0 scale no state is per group, and the call is fp4q_rht_quantize over all
+ * rows (group_offsets and tensor_scales are not read).
+ *   group_offsets: device int64[n_groups + 1], nondecreasing, [0] = 0, [n_groups] = rows. Other
+ *   values give an unspecified grouping but never an out-of-bounds access.
+ *   workspace: fp4q_grouped_workspace_size(cfg, n_groups) bytes, 256-byte aligned (per-group
+ *   amax slots; zeroed by the call on its stream).
+ * Errors as fp4q_rht_quantize; n_groups < 1 or > 2^24, or a null group_offsets / tensor_scales
+ * that is needed: FP4Q_ERR_INVALID_ARG; FP4Q_OUT_DEQUANT / FP4Q_OUT_STATS: FP4Q_ERR_UNSUPPORTED. */
+size_t fp4q_grouped_workspace_size(const fp4q_config* cfg, int32_t n_groups);
+fp4q_status fp4q_rht_quantize_grouped(const fp4q_config* cfg, const void* x, int64_t rows,
+                                      int64_t cols, int64_t ld, const int64_t* group_offsets,
+                                      int32_t n_groups, uint8_t* codes, void* scales,
+                                      float* tensor_scales, int32_t tensor_scales_given,
+                                      void* workspace, size_t workspace_bytes,
+                                      fp4q_stream_t stream);
+
 /* Reduce the statistics a previous fp4q_rht_quantize / fp4q_if4_select call with
  * FP4Q_OUT_STATS left in `workspace` (in a fixed order, FP64), copy them to *host_out and
  * derive SQNR, alpha, MSE and the per-cell mean error [UFP4-A "E2M1", "复利效应的反向版本",

@@ -174,3 +174,27 @@ def test_recipe_presets():
     dy = fq.recipe("ufp4", "bwd_dw", "dy", sr_seed=5)
     assert dy.round == fq.FP4Q_ROUND_SR and dy.sr_stream == 1
     assert fq.recipe("ufp4", "bwd_dx", "dy").sr_stream == 0
+
+
+def test_grouped_validation():
+    lib = _lib.load()
+    nv = fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=fq.FP4Q_SCALE_E4M3_1x16_TENSOR).c()
+    assert lib.fp4q_grouped_workspace_size(ctypes.byref(nv), 64) == 256
+    assert lib.fp4q_grouped_workspace_size(ctypes.byref(nv), 65) == 512
+    assert lib.fp4q_grouped_workspace_size(ctypes.byref(nv), 0) == 0
+    assert lib.fp4q_grouped_workspace_size(ctypes.byref(fq.Config().c()), 64) == 0   # FP32 scales
+
+    def g(cfg=nv, offs=FAKE, n=4, ts=FAKE, given=0, ws=FAKE, wsb=256, rows=4, cols=32):
+        return lib.fp4q_rht_quantize_grouped(ctypes.byref(cfg), FAKE, rows, cols, cols, offs, n, FAKE,
+                                             FAKE, ts, given, ws, wsb, None)
+    assert g(n=0) == _lib.FP4Q_ERR_INVALID_ARG
+    assert g(n=(1 << 24) + 1) == _lib.FP4Q_ERR_INVALID_ARG
+    assert g(offs=None) == _lib.FP4Q_ERR_INVALID_ARG
+    assert g(ts=None) == _lib.FP4Q_ERR_INVALID_ARG
+    assert g(given=2) == _lib.FP4Q_ERR_INVALID_ARG
+    assert g(offs=FAKE + 4) == _lib.FP4Q_ERR_ALIGN
+    assert g(ws=None) == _lib.FP4Q_ERR_WORKSPACE
+    assert g(wsb=128) == _lib.FP4Q_ERR_WORKSPACE
+    assert g(cols=24) == _lib.FP4Q_ERR_SHAPE
+    deq = fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=fq.FP4Q_SCALE_E4M3_1x16_TENSOR, dequant=True).c()
+    assert g(cfg=deq) == _lib.FP4Q_ERR_UNSUPPORTED
