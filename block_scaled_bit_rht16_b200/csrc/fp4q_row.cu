@@ -341,7 +341,7 @@ __global__ void __launch_bounds__(kThreads) lean_nv_kernel(const QuantArgs a) {
   // RN(amax / denom) for every block through the correction step on one reciprocal (exact for
   // quotients in [2^-20, 2^64); the E4M3 conversion sends anything below 2^-11 to 0 either way)
   Divider dd = make_divider(denom, 1.0f);
-  int64_t g_lo = 0, g_hi = 0;   // rows of the group whose scale is loaded (none yet)
+  int64_t g_lo = 0, g_hi = 0;   // blocks of the group whose scale is loaded (none yet)
   using Idx = typename UnitIdx<FLAT>::T;
   const Idx n = (Idx)a.nunits;
   const Idx stride = (Idx)gridDim.x * kThreads;
@@ -357,11 +357,10 @@ __global__ void __launch_bounds__(kThreads) lean_nv_kernel(const QuantArgs a) {
     if constexpr (RHT) fwht16(P);
     const float amax_y = __fmul_rn(absmax16(P), kCinv);
     if constexpr (GROUPED) {
-      const int64_t r = (int64_t)u / a.units_per_row;
-      if (r < g_lo || r >= g_hi) {
-        const int g = group_of(a.group_off, a.n_groups, r);
-        g_lo = __ldg(a.group_off + g);
-        g_hi = __ldg(a.group_off + g + 1);
+      if ((int64_t)u < g_lo || (int64_t)u >= g_hi) {
+        const int g = group_of(a.group_off, a.n_groups, (int64_t)u / a.units_per_row);
+        g_lo = __ldg(a.group_off + g) * a.units_per_row;
+        g_hi = __ldg(a.group_off + g + 1) * a.units_per_row;
         alpha = a.group_ts[g];
         denom = __fmul_rn(alpha, qmax);
         dd = make_divider(denom, 1.0f);
