@@ -331,7 +331,7 @@ def _cell_lattice(grid, q):
     g = O.grid_magnitudes(grid)
     c = int(np.where(g == q)[0][0])
     left = (g[c] - g[c - 1]) / 2 if c > 0 else 0.0
-    right = (g[c + 1] - g[c]) / 2 if c < 7 else 0.0
+    right = (g[c + 1] - g[c]) / 2 if c < len(g) - 1 else 0.0
     h = 1.0 / 16
     n = int(round((left + right) / h))
     return q - left + (np.arange(n) + 0.5) * h, left, right
@@ -341,7 +341,7 @@ def _bias_blocks(grid, q):
     """Blocks of 16 with element 0 = qmax (so the FP32 scale is exactly 1 and v = y) and 15
     points of the cell lattice of q (the lattice repeated 15 times, so the mean is exact)."""
     lat, _, _ = _cell_lattice(grid, q)
-    qmax = O.grid_magnitudes(grid)[7]
+    qmax = O.grid_magnitudes(grid)[-1]
     blocks = np.tile(lat, 15).reshape(-1, 15)
     x = np.concatenate([np.full((blocks.shape[0], 1), qmax), blocks], axis=1).astype(np.float32)
     return synth.to_bf16_bits(x), x
@@ -372,6 +372,24 @@ def test_shrinkage_bias_closed_form_every_cell(grid):
         assert st["cell_mean_err"][c] == pytest.approx((left - right) / 2, abs=1e-9)
         if grid != O.GRID_E2M1:
             assert st["cell_mean_err"][c] == pytest.approx(0.0, abs=1e-9)
+
+
+@pytest.mark.parametrize("grid", [O.GRID_E2M1_MAX4, O.GRID_E2M1_MAX3, O.GRID_E2M1_MAX2])
+def test_shrinkage_bias_closed_form_restricted_e2m1(grid):
+    # interior cells (L - R) / 2 as for E2M1; the new top cell is clipped on the right (values
+    # never exceed the limit), so its lattice has mean signed error +L / 2 -- diluted to
+    # 15/16 of that by each block's scale-setting element, which sits at the limit with error 0
+    g = O.grid_magnitudes(grid)
+    top = len(g) - 1
+    for c in range(1, len(g)):
+        bits, _ = _bias_blocks(grid, g[c])
+        st = O.finalize_stats(O.quantize(O.OracleConfig(grid=grid, rht=0), bits, stats=True)["stats_raw"])
+        left = (g[c] - g[c - 1]) / 2
+        if c < top:
+            want = (left - (g[c + 1] - g[c]) / 2) / 2
+        else:
+            want = (15.0 / 16.0) * left / 2
+        assert st["cell_mean_err"][c] == pytest.approx(want, abs=1e-9)
 
 
 # ------------------------------------------------------------------ quantizer invariants
