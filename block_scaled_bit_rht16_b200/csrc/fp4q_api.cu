@@ -203,6 +203,8 @@ fp4q_status fp4q_rht_quantize_grouped(const fp4q_config* cfg, const void* x, int
   fp4q_status st = check_cfg(cfg);
   if (st != FP4Q_OK) return st;
   if (cfg->outputs & (FP4Q_OUT_DEQUANT | FP4Q_OUT_STATS)) return FP4Q_ERR_UNSUPPORTED;
+  if (cfg->scale == FP4Q_SCALE_E4M3_1x16_TENSOR && cfg->round != FP4Q_ROUND_RTNE)
+    return FP4Q_ERR_UNSUPPORTED;   // the grouped E4M3 kernel rounds to nearest
   if (n_groups < 1 || n_groups > (1 << 24)) return FP4Q_ERR_INVALID_ARG;
   if (tensor_scales_given != 0 && tensor_scales_given != 1) return FP4Q_ERR_INVALID_ARG;
   if (cfg->scale != FP4Q_SCALE_E4M3_1x16_TENSOR)   // no per-group state

@@ -244,7 +244,8 @@ fp4q_status fp4q_rht_quantize_noalloc(const fp4q_config* cfg, const void* x, int
  *   workspace: fp4q_grouped_workspace_size(cfg, n_groups) bytes, 256-byte aligned (per-group
  *   amax slots; zeroed by the call on its stream).
  * Errors as fp4q_rht_quantize; n_groups < 1 or > 2^24, or a null group_offsets / tensor_scales
- * that is needed: FP4Q_ERR_INVALID_ARG; FP4Q_OUT_DEQUANT / FP4Q_OUT_STATS: FP4Q_ERR_UNSUPPORTED. */
+ * that is needed: FP4Q_ERR_INVALID_ARG; FP4Q_OUT_DEQUANT / FP4Q_OUT_STATS, or stochastic
+ * rounding with the E4M3 scale: FP4Q_ERR_UNSUPPORTED. */
 size_t fp4q_grouped_workspace_size(const fp4q_config* cfg, int32_t n_groups);
 fp4q_status fp4q_rht_quantize_grouped(const fp4q_config* cfg, const void* x, int64_t rows,
                                       int64_t cols, int64_t ld, const int64_t* group_offsets,

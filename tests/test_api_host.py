@@ -198,3 +198,6 @@ def test_grouped_validation():
     assert g(cols=24) == _lib.FP4Q_ERR_SHAPE
     deq = fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=fq.FP4Q_SCALE_E4M3_1x16_TENSOR, dequant=True).c()
     assert g(cfg=deq) == _lib.FP4Q_ERR_UNSUPPORTED
+    sr = fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=fq.FP4Q_SCALE_E4M3_1x16_TENSOR,
+                   round=fq.FP4Q_ROUND_SR).c()
+    assert g(cfg=sr) == _lib.FP4Q_ERR_UNSUPPORTED
