@@ -695,9 +695,25 @@ def cpu_baseline(wl, budget_s=12.0):
     t = oracle_pass(cfg, bits, rows, cores)
     per_elem = wl.bytes_per_step() / wl.elements()
     gbs = rows * bits.shape[1] * per_elem / t / 1e9
+    # one thread on a short sample, for the per-core figure
+    t1 = oracle_pass(cfg, bits, probe_rows, 1)
+    gbs1 = probe_rows * bits.shape[1] * per_elem / t1 / 1e9
     return {"value": round(gbs, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": "%d of %d rows of the step's tensor (%.1f s wall on %d threads)"
-                      % (rows, bits.shape[0], t, cores)}
+                      % (rows, bits.shape[0], t, cores),
+            "single_thread": {"value": round(gbs1, 4), "sample": "%d rows" % probe_rows},
+            "cpu_model": _cpu_model()}
+
+
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 def run_reference(args):
