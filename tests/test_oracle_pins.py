@@ -290,6 +290,7 @@ def test_sr_keeps_grid_points_and_is_unbiased():
     for grid in (O.GRID_E1M2, O.GRID_E2M1, O.GRID_INT4):
         g = O.grid_magnitudes(grid)
         u = rng.integers(0, 2**32, size=(8, 4096), dtype=np.uint64).astype(np.uint32)
+        u[0, :] = 0                    # r = 0: a grid point (frac = 0) must still stay put
         on = np.repeat(np.concatenate([g, -g]).astype(np.float32), 512)[: u.size]
         np.testing.assert_array_equal(_value_of(grid, O.round_sr(grid, on, u.reshape(-1)[: on.size])), on)
     n = 1_000_000
