@@ -45,3 +45,30 @@ def test_clock_summary_falls_back_to_all_samples():
     c = smp.stop(_t("2026/12/02 21:00:00.000"), _t("2026/12/02 21:00:01.000"))
     assert c["samples"] == 4 and c["window"].startswith("whole run")
     assert c["reasons"] == ["sw_power_cap"]
+
+
+def _workload_choices():
+    """The --workload choices, read from bench.py's argument parser definition."""
+    import re
+    with open(bench.__file__) as f:
+        src = f.read()
+    block = src[src.index('p.add_argument("--workload"'):]
+    block = block[block.index("choices="):block.index("])") + 2]
+    return re.findall(r'"([a-z0-9-]+)"', block)
+
+
+def test_every_workload_constructs():
+    # make_workload only builds configurations (no device work): every --workload choice must
+    # name a workload with a description and a kernel key
+    import json
+    names = _workload_choices()
+    assert "c2" in names and len(names) > 10
+    keys = set()
+    for name in names:
+        wl = bench.make_workload(name)
+        assert wl.desc and wl.kernel_key
+        keys.add(wl.kernel_key)
+    # the committed ncu traffic record names kernels that the bench reports
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    with open(os.path.join(root, "profiles", "traffic.json")) as f:
+        assert set(json.load(f)) <= keys
