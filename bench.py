@@ -7,7 +7,7 @@ on the UFP4 fwd_y path -- RHT16 + E1M2 round-to-nearest-even, FP32 1x16 scales, 
 as one launch over the stacked [16384, 2048] operands. Algorithmic bytes: 2 (bf16 in) + 0.5
 (codes) + 0.25 (FP32 scale) per element.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload c2|...]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload linear1.5b-ufp4|...]
 
 Timing: inputs resident in HBM, rotating through enough buffer sets that every launch reads
 data evicted from L2; steps replayed from a CUDA graph; CUDA events on the launching stream,
@@ -41,12 +41,14 @@ def parse():
     p.add_argument("--steps", type=int, default=3000)
     p.add_argument("--warmup", type=int, default=400)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    p.add_argument("--workload", default="c2",
-                   choices=["c2", "c2-quant-only", "c2-unfused", "c3", "c3-rtne", "c3-row-sr",
-                            "c4-nvfp4", "c4-nvfp4-given",
-                            "c4-nvint4", "c4-mxfp4", "c4-if4", "c5-moe-ufp4", "c5-moe-e2m1",
-                            "c5-dense-ufp4", "c5-dense-e2m1", "c2-e2m1", "c2-e2m1-max4",
-                            "c2-e2m1-max3", "c2-e2m1-max2", "c5-moe-nvfp4-grouped"])
+    p.add_argument("--workload", default="linear1.5b-ufp4",
+                   choices=["linear1.5b-ufp4", "linear1.5b-ufp4-quant-only", "linear1.5b-ufp4-unfused",
+                            "linear1.5b-e2m1", "linear1.5b-e2m1-max4", "linear1.5b-e2m1-max3",
+                            "linear1.5b-e2m1-max2", "dy8192-dual-sr", "dy8192-dual-rtne",
+                            "dy8192-row-sr", "laplace16k-nvfp4", "laplace16k-nvfp4-given",
+                            "laplace16k-nvint4", "laplace16k-mxfp4", "laplace16k-if4",
+                            "moe-experts-ufp4", "moe-experts-e2m1", "moe-experts-nvfp4-grouped",
+                            "dense32k-ufp4", "dense32k-e2m1"])
     p.add_argument("--no-extras", action="store_true", help="skip e2e, ratios and CPU baseline")
     a = p.parse_args()
     if a.warmup < 3:
@@ -352,51 +354,51 @@ def make_workload(name):
     import block_scaled_bit_rht16_b200 as fq
     from block_scaled_bit_rht16_b200 import synth
 
-    def c2_input():
-        x, w = synth.workload2()
+    def stacked_operands():
+        x, w = synth.dense_linear_operands()
         return np.concatenate([x, w], axis=0)
 
-    if name.startswith("c2"):
+    if name.startswith("linear1.5b-"):
         mask = fq.sign_mask_from_seed(synth.sign_seed(2))
         cfg = fq.recipe("ufp4", "fwd_y", "x", sign_mask=mask)
         desc = ("dense-1.5B-like operands X[8192,2048] Student-t(4) + W[8192,2048] N(0,0.02), "
                 "UFP4 fwd_y: RHT16 + E1M2 RTNE, FP32 1x16 scales along K=2048, one launch over "
                 "the stacked [16384,2048]")
-        if name == "c2-quant-only":
+        if name == "linear1.5b-ufp4-quant-only":
             from dataclasses import replace
-            return RowWorkload(name, desc + " -- rotation off (quantize only)", c2_input,
+            return RowWorkload(name, desc + " -- rotation off (quantize only)", stacked_operands,
                                replace(cfg, rht=0, sign_mask=0), "lean_kernel<E1M2,no-rotation,flat>")
-        if name.startswith("c2-e2m1"):
+        if name.startswith("linear1.5b-e2m1"):
             # the E2M1 baseline recipe's fwd_y operand (no rotation), full table or range-restricted
             from dataclasses import replace
             top = int(name[-1]) if name.endswith(("max4", "max3", "max2")) else 0
             ec = replace(fq.recipe("e2m1", "fwd_y", "x", sign_mask=mask), e2m1_max=top)
             what = "E2M1 limited to a largest value of %d" % top if top else "E2M1"
             return RowWorkload(name, desc.split(", UFP4")[0] + ", E2M1 baseline fwd_y: %s RTNE, no "
-                               "rotation, FP32 1x16 scales" % what, c2_input, ec,
+                               "rotation, FP32 1x16 scales" % what, stacked_operands, ec,
                                "lean_kernel<%s,no-rotation,flat>" % ("E2M1max%d" % top if top else "E2M1"))
-        if name == "c2-unfused":
+        if name == "linear1.5b-ufp4-unfused":
             return RowWorkload(name, desc + " -- unfused: rotation pass to bf16, then quantize",
-                               c2_input, cfg, "rht16_kernel+lean_kernel", unfused=True)
-        return RowWorkload(name, desc, c2_input, cfg, "lean_kernel<E1M2,rotation,flat>")
-    if name == "c3-row-sr":
+                               stacked_operands, cfg, "rht16_kernel+lean_kernel", unfused=True)
+        return RowWorkload(name, desc, stacked_operands, cfg, "lean_kernel<E1M2,rotation,flat>")
+    if name == "dy8192-row-sr":
         mask = fq.sign_mask_from_seed(synth.sign_seed(3))
         rc = fq.recipe("ufp4", "bwd_dx", "dy", sign_mask=mask, sr_seed=synth.SR_SEED)
-        return RowWorkload(name, "dY[8192,8192] row orientation only, RHT16 + E1M2 SR", synth.workload3,
+        return RowWorkload(name, "dY[8192,8192] row orientation only, RHT16 + E1M2 SR", synth.backward_dy,
                            rc, "lean_kernel<E1M2,rotation,flat,SR>")
-    if name in ("c3", "c3-rtne"):
+    if name in ("dy8192-dual-sr", "dy8192-dual-rtne"):
         mask = fq.sign_mask_from_seed(synth.sign_seed(3))
         rc = fq.recipe("ufp4", "bwd_dx", "dy", sign_mask=mask, sr_seed=synth.SR_SEED)
         cc = fq.recipe("ufp4", "bwd_dw", "dy", sign_mask=mask, sr_seed=synth.SR_SEED)
-        if name == "c3-rtne":
+        if name == "dy8192-dual-rtne":
             from dataclasses import replace
             rc, cc = replace(rc, round=fq.FP4Q_ROUND_RTNE), replace(cc, round=fq.FP4Q_ROUND_RTNE)
             return DualWorkload(name, "dY[8192,8192] dual orientation, RHT16 + E1M2 round-to-nearest "
-                                "(diagnostic)", synth.workload3, rc, cc, "dual_kernel<E1M2,RTNE,RTNE>")
+                                "(diagnostic)", synth.backward_dy, rc, cc, "dual_kernel<E1M2,RTNE,RTNE>")
         return DualWorkload(name, "backward dY[8192,8192] N(0,1e-3) with 0.01% x100, RHT16 + E1M2 "
-                            "SR in row and column orientation from one read", synth.workload3, rc, cc,
+                            "SR in row and column orientation from one read", synth.backward_dy, rc, cc,
                             "dual_kernel<E1M2,SR,SR>")
-    if name.startswith("c4"):
+    if name.startswith("laplace16k-"):
         mask = fq.sign_mask_from_seed(synth.sign_seed(4))
         kind = name.split("-", 1)[1]
         grid = {"nvfp4": fq.FP4Q_GRID_E2M1, "nvfp4-given": fq.FP4Q_GRID_E2M1, "nvint4": fq.FP4Q_GRID_INT4,
@@ -408,30 +410,30 @@ def make_workload(name):
                "mxfp4": "quantize_kernel<E2M1,UE8M0>"}[kind]
         if kind in ("nvfp4", "nvint4", "if4"):
             key += "+amax_kernel<rotation,flat>"
-        return RowWorkload(name, "[16384,5120] Laplace(0,1), RHT16, %s" % kind, synth.workload4, cfg, key)
-    if name == "c5-moe-nvfp4-grouped":
+        return RowWorkload(name, "[16384,5120] Laplace(0,1), RHT16, %s" % kind, synth.laplace_format_tensor, cfg, key)
+    if name == "moe-experts-nvfp4-grouped":
         mask = fq.sign_mask_from_seed(synth.sign_seed(5))
         cfg = fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=fq.FP4Q_SCALE_E4M3_1x16_TENSOR, rht=1,
                         sign_mask=mask)
 
         def inp():
-            return np.concatenate([synth.workload5_expert(e) for e in range(64)], axis=0)
+            return np.concatenate([synth.moe_expert(e) for e in range(64)], axis=0)
         return GroupedWorkload(name, "MoE experts [64,2048,7168] as [131072,7168], sigma_e log-uniform "
                                "[0.1,10], NVFP4 (RHT16, E4M3 1x16 + one FP32 tensor scale per expert, "
                                "computed each step)", inp, cfg,
                                "lean_nv_kernel<E2M1,rotation,flat,grouped>+grouped_amax_kernel",
                                [2048] * 64)
-    if name.startswith("c5"):
+    if name in ("moe-experts-ufp4", "moe-experts-e2m1", "dense32k-ufp4", "dense32k-e2m1"):
         mask = fq.sign_mask_from_seed(synth.sign_seed(5))
         ufp4 = name.endswith("ufp4")
         cfg = fq.recipe("ufp4" if ufp4 else "e2m1", "fwd_y", "x", sign_mask=mask)
         if "moe" in name:
             def inp():
-                return np.concatenate([synth.workload5_expert(e) for e in range(64)], axis=0)
+                return np.concatenate([synth.moe_expert(e) for e in range(64)], axis=0)
             desc = "MoE experts [64,2048,7168] as [131072,7168], sigma_e log-uniform [0.1,10]"
         else:
             def inp():
-                return synth.workload5_dense_rows(0, 32768)
+                return synth.dense_layer_rows(0, 32768)
             desc = "dense [32768,8192] N(0,1)"
         desc += ", %s fwd_y" % ("UFP4 RHT16+E1M2" if ufp4 else "E2M1 baseline (no rotation)")
         return RowWorkload(name, desc, inp, cfg, "lean_kernel<%s,%s,flat>" % ("E1M2" if ufp4 else "E2M1",
@@ -530,7 +532,7 @@ def run_ours(args):
     extras = {}
     if not args.no_extras:
         extras["e2e"] = measure_e2e(wl, stream, world)
-        if args.workload == "c2":
+        if args.workload == "linear1.5b-ufp4":
             extras["ratios"] = measure_ratios(args, stream, dev, l2, ms_per_step)
     del g_main, g_rem
     if world > 1:
@@ -621,7 +623,7 @@ def measure_ratios(args, stream, dev, l2, fused_step_ms):
     unfused (rotation pass to bf16, then quantize-only), kernel time per step."""
     out = {}
     per = {}
-    for name in ("c2-quant-only", "c2-unfused"):
+    for name in ("linear1.5b-ufp4-quant-only", "linear1.5b-ufp4-unfused"):
         wl = make_workload(name)
         wl.setup(dev, l2)
         steps = 64 * wl.R
@@ -639,10 +641,10 @@ def measure_ratios(args, stream, dev, l2, fused_step_ms):
         per[name] = a.elapsed_time(b) / (20 * steps)
         del g, wl
         torch.cuda.empty_cache()
-    qo = per["c2-quant-only"]
+    qo = per["linear1.5b-ufp4-quant-only"]
     out["quant_only_us_per_step"] = round(qo * 1e3, 3)
     out["fused_over_quant_only"] = round(fused_step_ms / qo, 4)
-    out["unfused_over_quant_only"] = round(per["c2-unfused"] / qo, 4)
+    out["unfused_over_quant_only"] = round(per["linear1.5b-ufp4-unfused"] / qo, 4)
     out["pages_sm100"] = {"fused": 1.07, "unfused": 1.41}
     return out
 
@@ -727,7 +729,7 @@ def run_reference(args):
     import block_scaled_bit_rht16_b200 as fq
     mask = fq.sign_mask_from_seed(synth.sign_seed(2))
     cfg = fq.recipe("ufp4", "fwd_y", "x", sign_mask=mask)
-    x, w = synth.workload2()
+    x, w = synth.dense_linear_operands()
     bits = np.concatenate([x, w], axis=0)
     cores = len(os.sched_getaffinity(0))
     t1 = oracle_pass(cfg, bits, 64, 1)   # rows per second on one core

@@ -54,7 +54,7 @@ def _workload_choices():
         src = f.read()
     block = src[src.index('p.add_argument("--workload"'):]
     block = block[block.index("choices="):block.index("])") + 2]
-    return re.findall(r'"([a-z0-9-]+)"', block)
+    return re.findall(r'"([a-z0-9.-]+)"', block)
 
 
 def test_every_workload_constructs():
@@ -62,7 +62,7 @@ def test_every_workload_constructs():
     # name a workload with a description and a kernel key
     import json
     names = _workload_choices()
-    assert "c2" in names and len(names) > 10
+    assert "linear1.5b-ufp4" in names and len(names) > 10
     keys = set()
     for name in names:
         wl = bench.make_workload(name)

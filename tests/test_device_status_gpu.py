@@ -29,7 +29,7 @@ def test_wait_timeout_is_reported_and_cleared():
 
 def test_pipelined_launches_report_no_timeouts():
     fq.device_status(clear=True)
-    x, w = synth.workload2(rows=2048)
+    x, w = synth.dense_linear_operands(rows=2048)
     t = to_dev(np.concatenate([x, w], axis=0))
     for grid in (fq.FP4Q_GRID_E1M2, fq.FP4Q_GRID_E2M1, fq.FP4Q_GRID_INT4):
         for _ in range(3):

@@ -595,7 +595,7 @@ def test_stats_on_grid_input_and_direct_formulas():
 def test_sqnr_direction_on_outlier_workload():
     # the pages' qualitative reversal across the rotation on an outlier-heavy tensor:
     # without RHT E2M1 >= E1M2; with RHT E1M2 > E2M1 (UFP4 page, RHT section; values unpinned)
-    x = synth.workload1(rows=128)
+    x = synth.outlier_activation(rows=128)
     mask = O.sign_mask_from_seed(synth.sign_seed(1))
     sq = {}
     for grid in (O.GRID_E2M1, O.GRID_E1M2):

@@ -36,8 +36,8 @@ def _check_rows(cfg, bits, out, rows, tensor_scale=None):
         np.testing.assert_array_equal(scales[r], ref["scales"][0], err_msg="row %d" % r)
 
 
-def test_workload1_activation_with_outliers():
-    x = synth.workload1()
+def test_outlier_activation_512x2048():
+    x = synth.outlier_activation()
     mask = fq.sign_mask_from_seed(synth.sign_seed(1))
     sq = {}
     for grid in (fq.FP4Q_GRID_E2M1, fq.FP4Q_GRID_E1M2):
@@ -56,8 +56,8 @@ def test_workload1_activation_with_outliers():
     assert sq[fq.FP4Q_GRID_E2M1, 0] >= sq[fq.FP4Q_GRID_E1M2, 0]
 
 
-def test_workload2_stacked_operands():
-    x, w = synth.workload2()
+def test_dense_linear_operands_stacked_16384x2048():
+    x, w = synth.dense_linear_operands()
     bits = np.concatenate([x, w], axis=0)
     mask = fq.sign_mask_from_seed(synth.sign_seed(2))
     cfg = fq.recipe("ufp4", "fwd_y", "x", sign_mask=mask)
@@ -68,8 +68,8 @@ def test_workload2_stacked_operands():
     _check_rows(cfg, bits, out, _sample_rows(bits.shape[0], 192, 2) + [8191, 8192])
 
 
-def test_workload3_dual_orientation():
-    dy = synth.workload3()
+def test_backward_dy_8192x8192_dual_orientation():
+    dy = synth.backward_dy()
     mask = fq.sign_mask_from_seed(synth.sign_seed(3))
     rc = fq.recipe("ufp4", "bwd_dx", "dy", sign_mask=mask, sr_seed=synth.SR_SEED)
     cc = fq.recipe("ufp4", "bwd_dw", "dy", sign_mask=mask, sr_seed=synth.SR_SEED)
@@ -89,8 +89,8 @@ def test_workload3_dual_orientation():
 
 
 @pytest.mark.parametrize("kind", ["nvfp4", "nvint4", "mxfp4", "if4"])
-def test_workload4_formats(kind):
-    x = synth.workload4()
+def test_laplace_16384x5120_formats(kind):
+    x = synth.laplace_format_tensor()
     mask = fq.sign_mask_from_seed(synth.sign_seed(4))
     grid = {"nvfp4": fq.FP4Q_GRID_E2M1, "nvint4": fq.FP4Q_GRID_INT4, "mxfp4": fq.FP4Q_GRID_E2M1,
             "if4": fq.FP4Q_GRID_IF4}[kind]
@@ -108,17 +108,17 @@ def test_workload4_formats(kind):
 
 
 @pytest.mark.parametrize("recipe", ["ufp4", "e2m1"])
-def test_workload5_moe_and_dense(recipe):
+def test_moe_experts_and_dense_layer(recipe):
     mask = fq.sign_mask_from_seed(synth.sign_seed(5))
     cfg = fq.recipe(recipe, "fwd_y", "x", sign_mask=mask)
-    experts = [synth.workload5_expert(e) for e in range(64)]
+    experts = [synth.moe_expert(e) for e in range(64)]
     moe = np.concatenate(experts, axis=0)
     del experts
     out = fq.rht_quantize(cfg, to_dev(moe))
     torch.cuda.synchronize()
     _check_rows(cfg, moe, out, _sample_rows(moe.shape[0], 96, 6))
     del out, moe
-    dense = synth.workload5_dense_rows(0, 32768)
+    dense = synth.dense_layer_rows(0, 32768)
     out = fq.rht_quantize(cfg, to_dev(dense))
     torch.cuda.synchronize()
     _check_rows(cfg, dense, out, _sample_rows(dense.shape[0], 64, 7))
