@@ -73,6 +73,10 @@ int block_elems(const fp4q_config* cfg) { return cfg->scale == FP4Q_SCALE_UE8M0_
 
 size_t stats_bytes() { return (size_t)kStatsCtas * ST_LEN * sizeof(double); }
 
+// Largest M of fp4q_quantize_dual: its kernel puts the 128-row tiles of dY on the grid's y axis,
+// which holds at most 65535 blocks.
+constexpr int64_t kDualMaxRows = 65535ll * 128;
+
 fp4q_status check_shape(int64_t rows, int64_t cols, int64_t ld, int unit) {
   if (rows < 0 || cols < 0) return FP4Q_ERR_SHAPE;
   if (cols % unit != 0) return FP4Q_ERR_SHAPE;
@@ -305,6 +309,7 @@ fp4q_status fp4q_quantize_dual(const fp4q_config* row_cfg, const fp4q_config* co
   if (row_cfg->grid != col_cfg->grid) return FP4Q_ERR_UNSUPPORTED;
   if (row_cfg->e2m1_max != 0u || col_cfg->e2m1_max != 0u) return FP4Q_ERR_UNSUPPORTED;
   if (M < 0 || N < 0 || M % 16 != 0 || N % 16 != 0) return FP4Q_ERR_SHAPE;
+  if (M > kDualMaxRows) return FP4Q_ERR_SHAPE;   // 128-row tiles on the grid's y axis
   if (M > 0 && N > 0 && ld < N) return FP4Q_ERR_SHAPE;
   if (M > 1 && N > 0 && ld % 8 != 0) return FP4Q_ERR_ALIGN;
   const bool empty = M == 0 || N == 0;

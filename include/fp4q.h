@@ -176,7 +176,8 @@ fp4q_status fp4q_rht_quantize(const fp4q_config* cfg, const void* x, int64_t row
  *  codes_col  uint8 [N, M/2], scales_col float [N, M/16]: blocks along M, i.e. dy^T
  *             quantized along its rows (col_cfg; SR index n * M + m).
  * Both configs must use FP4Q_SCALE_FP32_1x16 and no dequant/stats outputs; M and N must be
- * multiples of 16. workspace may be NULL. */
+ * multiples of 16 and M at most 65535 * 128 = 8388480 (else FP4Q_ERR_SHAPE; quantize taller dY
+ * in row slices). workspace may be NULL. */
 fp4q_status fp4q_quantize_dual(const fp4q_config* row_cfg, const fp4q_config* col_cfg,
                                const void* dy, int64_t M, int64_t N, int64_t ld,
                                uint8_t* codes_row, void* scales_row, uint8_t* codes_col,
