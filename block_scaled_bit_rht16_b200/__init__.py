@@ -72,9 +72,10 @@ def _torch():
     return torch
 
 
-def _stream_ptr(stream):
+def _stream_ptr(stream, device=None):
+    """The stream handle: `stream`, else torch's current stream on `device`."""
     torch = _torch()
-    s = stream if stream is not None else torch.cuda.current_stream()
+    s = stream if stream is not None else torch.cuda.current_stream(device)
     return ctypes.c_void_p(s.cuda_stream)
 
 
@@ -90,6 +91,37 @@ def _check_input(x, name="x"):
         raise ValueError("%s must have unit column stride" % name)
     ld = x.stride(0) if (x.shape[0] > 1 and x.numel() > 0) else x.shape[1]
     return x.shape[0], x.shape[1], ld
+
+
+def _check_buf(t, name, dtype, numel, device):
+    """A buffer the library reads or writes through a raw pointer: a contiguous CUDA tensor of
+    `dtype` on `device` with at least `numel` elements. Checked here because the C ABI cannot
+    tell a host pointer or a short buffer from a good one."""
+    torch = _torch()
+    if not (isinstance(t, torch.Tensor) and t.is_cuda):
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.device != device:
+        raise ValueError("%s is on %s but the input is on %s" % (name, t.device, device))
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, not %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if t.numel() < numel:
+        raise ValueError("%s holds %d elements, %d needed" % (name, t.numel(), numel))
+
+
+def _scale_dtype(cfg):
+    torch = _torch()
+    return torch.float32 if cfg.scale == FP4Q_SCALE_FP32_1x16 else torch.uint8
+
+
+def _check_quantized(cfg, out, rows, cols, device, dequant=False):
+    """The code and scale buffers (and the dequant buffer when requested) of a row quantizer."""
+    torch = _torch()
+    _check_buf(out.codes, "codes", torch.uint8, rows * (cols // 2), device)
+    _check_buf(out.scales, "scales", _scale_dtype(cfg), rows * (cols // cfg.block), device)
+    if dequant:
+        _check_buf(out.dequant, "dequant", torch.bfloat16, rows * cols, device)
 
 
 def sign_mask_from_seed(seed: int) -> int:
@@ -144,12 +176,17 @@ def rht_quantize(cfg: Config, x, *, out: Quantized = None, tensor_scale=None,
             tensor_scale = out.tensor_scale if out.tensor_scale is not None else \
                 torch.zeros(1, dtype=torch.float32, device=x.device)
         out.tensor_scale = tensor_scale
+        _check_buf(out.tensor_scale, "tensor_scale", torch.float32, 1, x.device)
+    _check_quantized(cfg, out, rows, cols, x.device, dequant=cfg.dequant)
     c = cfg.c()
     ws = out.workspace
+    if ws is not None:
+        _check_buf(ws, "workspace", torch.uint8, 0, x.device)
     fn = _lib.load().fp4q_if4_select if cfg.grid == FP4Q_GRID_IF4 else _lib.load().fp4q_rht_quantize
-    st = fn(ctypes.byref(c), _ptr(x), rows, cols, ld, _ptr(out.codes), _ptr(out.scales),
-            _ptr(out.tensor_scale), int(bool(tensor_scale_given)), _ptr(out.dequant), _ptr(ws),
-            0 if ws is None else ws.numel(), _stream_ptr(stream))
+    with torch.cuda.device(x.device):
+        st = fn(ctypes.byref(c), _ptr(x), rows, cols, ld, _ptr(out.codes), _ptr(out.scales),
+                _ptr(out.tensor_scale), int(bool(tensor_scale_given)), _ptr(out.dequant), _ptr(ws),
+                0 if ws is None else ws.numel(), _stream_ptr(stream, x.device))
     _lib.check(st, "fp4q_rht_quantize")
     return out
 
@@ -162,6 +199,7 @@ def rht_quantize_grouped(cfg: Config, x, group_offsets, *, out: Quantized = None
     written with each group's computed alpha; returned as Quantized.tensor_scale."""
     torch = _torch()
     rows, cols, ld = _check_input(x)
+    _check_buf(group_offsets, "group_offsets", torch.int64, 2, x.device)
     n_groups = int(group_offsets.numel()) - 1
     c = cfg.c()
     if out is None:
@@ -173,11 +211,17 @@ def rht_quantize_grouped(cfg: Config, x, group_offsets, *, out: Quantized = None
         out.tensor_scale = tensor_scales
     if cfg.scale == FP4Q_SCALE_E4M3_1x16_TENSOR and out.tensor_scale is None:
         out.tensor_scale = torch.zeros(max(n_groups, 1), dtype=torch.float32, device=x.device)
+    if cfg.scale == FP4Q_SCALE_E4M3_1x16_TENSOR:
+        _check_buf(out.tensor_scale, "tensor_scales", torch.float32, n_groups, x.device)
+    _check_quantized(cfg, out, rows, cols, x.device)
     ws = out.workspace
-    st = _lib.load().fp4q_rht_quantize_grouped(
-        ctypes.byref(c), _ptr(x), rows, cols, ld, _ptr(group_offsets), n_groups, _ptr(out.codes),
-        _ptr(out.scales), _ptr(out.tensor_scale), int(bool(tensor_scales_given)), _ptr(ws),
-        0 if ws is None else ws.numel(), _stream_ptr(stream))
+    if ws is not None:
+        _check_buf(ws, "workspace", torch.uint8, 0, x.device)
+    with torch.cuda.device(x.device):
+        st = _lib.load().fp4q_rht_quantize_grouped(
+            ctypes.byref(c), _ptr(x), rows, cols, ld, _ptr(group_offsets), n_groups,
+            _ptr(out.codes), _ptr(out.scales), _ptr(out.tensor_scale), int(bool(tensor_scales_given)),
+            _ptr(ws), 0 if ws is None else ws.numel(), _stream_ptr(stream, x.device))
     _lib.check(st, "fp4q_rht_quantize_grouped")
     return out
 
@@ -190,9 +234,13 @@ def tensor_scale(cfg: Config, x, *, out=None, workspace=None, stream=None):
         out = torch.empty(1, dtype=torch.float32, device=x.device)
     if workspace is None:
         workspace = torch.empty(256, dtype=torch.uint8, device=x.device)
+    _check_buf(out, "out", torch.float32, 1, x.device)
+    _check_buf(workspace, "workspace", torch.uint8, 0, x.device)
     c = cfg.c()
-    st = _lib.load().fp4q_tensor_scale(ctypes.byref(c), _ptr(x), rows, cols, ld, _ptr(out),
-                                       _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    with torch.cuda.device(x.device):
+        st = _lib.load().fp4q_tensor_scale(ctypes.byref(c), _ptr(x), rows, cols, ld, _ptr(out),
+                                           _ptr(workspace), workspace.numel(),
+                                           _stream_ptr(stream, x.device))
     _lib.check(st, "fp4q_tensor_scale")
     return out
 
@@ -220,11 +268,15 @@ def quantize_dual(row_cfg: Config, col_cfg: Config, dy, *, out: Dual = None, str
                    torch.empty((M, N // 16), dtype=torch.float32, device=dev),
                    torch.empty((N, M // 2), dtype=torch.uint8, device=dev),
                    torch.empty((N, M // 16), dtype=torch.float32, device=dev))
+    for name, dt, n in (("codes_row", torch.uint8, M * (N // 2)), ("scales_row", torch.float32, M * (N // 16)),
+                        ("codes_col", torch.uint8, N * (M // 2)), ("scales_col", torch.float32, N * (M // 16))):
+        _check_buf(getattr(out, name), name, dt, n, dy.device)
     rc, cc = row_cfg.c(), col_cfg.c()
-    st = _lib.load().fp4q_quantize_dual(ctypes.byref(rc), ctypes.byref(cc), _ptr(dy), M, N, ld,
-                                        _ptr(out.codes_row), _ptr(out.scales_row),
-                                        _ptr(out.codes_col), _ptr(out.scales_col), None, 0,
-                                        _stream_ptr(stream))
+    with torch.cuda.device(dy.device):
+        st = _lib.load().fp4q_quantize_dual(ctypes.byref(rc), ctypes.byref(cc), _ptr(dy), M, N, ld,
+                                            _ptr(out.codes_row), _ptr(out.scales_row),
+                                            _ptr(out.codes_col), _ptr(out.scales_col), None, 0,
+                                            _stream_ptr(stream, dy.device))
     _lib.check(st, "fp4q_quantize_dual")
     return out
 
@@ -233,12 +285,22 @@ def dequantize(cfg: Config, codes, scales, tensor_scale=None, *, inverse_rht: bo
                out=None, stream=None):
     """fp4q_dequantize: codes [rows, cols/2] -> bf16 [rows, cols]."""
     torch = _torch()
+    if not (isinstance(codes, torch.Tensor) and codes.dim() == 2):
+        raise TypeError("codes must be a 2-D uint8 CUDA tensor [rows, cols/2]")
     rows, cols = codes.shape[0], codes.shape[1] * 2
+    dev = codes.device
+    _check_buf(codes, "codes", torch.uint8, rows * (cols // 2), dev)
+    _check_buf(scales, "scales", _scale_dtype(cfg), rows * (cols // cfg.block), dev)
+    if cfg.scale == FP4Q_SCALE_E4M3_1x16_TENSOR:
+        _check_buf(tensor_scale, "tensor_scale", torch.float32, 1, dev)
     if out is None:
-        out = torch.empty((rows, cols), dtype=torch.bfloat16, device=codes.device)
+        out = torch.empty((rows, cols), dtype=torch.bfloat16, device=dev)
+    _check_buf(out, "out", torch.bfloat16, rows * cols, dev)
     c = cfg.c()
-    st = _lib.load().fp4q_dequantize(ctypes.byref(c), _ptr(codes), _ptr(scales), _ptr(tensor_scale),
-                                     rows, cols, int(bool(inverse_rht)), _ptr(out), _stream_ptr(stream))
+    with torch.cuda.device(dev):
+        st = _lib.load().fp4q_dequantize(ctypes.byref(c), _ptr(codes), _ptr(scales), _ptr(tensor_scale),
+                                         rows, cols, int(bool(inverse_rht)), _ptr(out),
+                                         _stream_ptr(stream, dev))
     _lib.check(st, "fp4q_dequantize")
     return out
 
@@ -250,8 +312,10 @@ def rht16(x, sign_mask: int, *, out_fp32: bool = False, out=None, stream=None):
     if out is None:
         out = torch.empty((rows, cols), dtype=torch.float32 if out_fp32 else torch.bfloat16,
                           device=x.device)
-    st = _lib.load().fp4q_rht16(_ptr(x), rows, cols, ld, sign_mask, _ptr(out), int(bool(out_fp32)),
-                                _stream_ptr(stream))
+    _check_buf(out, "out", torch.float32 if out_fp32 else torch.bfloat16, rows * cols, x.device)
+    with torch.cuda.device(x.device):
+        st = _lib.load().fp4q_rht16(_ptr(x), rows, cols, ld, sign_mask, _ptr(out), int(bool(out_fp32)),
+                                    _stream_ptr(stream, x.device))
     _lib.check(st, "fp4q_rht16")
     return out
 
@@ -266,9 +330,12 @@ def device_status(clear: bool = False, stream=None) -> int:
 
 def stats(workspace, stream=None) -> dict:
     """fp4q_stats: reduce and fetch the statistics a stats-enabled call left in `workspace`."""
+    torch = _torch()
+    _check_buf(workspace, "workspace", torch.uint8, 0, getattr(workspace, "device", None))
     res = _lib.fp4q_stats_t()
-    st = _lib.load().fp4q_stats(_ptr(workspace), workspace.numel(), ctypes.byref(res),
-                                _stream_ptr(stream))
+    with torch.cuda.device(workspace.device):
+        st = _lib.load().fp4q_stats(_ptr(workspace), workspace.numel(), ctypes.byref(res),
+                                    _stream_ptr(stream, workspace.device))
     _lib.check(st, "fp4q_stats")
     out = {}
     for name, _ in _lib.fp4q_stats_t._fields_:
