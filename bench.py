@@ -664,46 +664,68 @@ def _oracle_cfg(cfg):
                           sign_mask=cfg.sign_mask, sr_stream=cfg.sr_stream, sr_seed=cfg.sr_seed)
 
 
-def oracle_pass(cfg, bits, rows_total, threads):
-    """The oracle over `rows_total` rows of `bits` (cycled), chunked over a thread pool (the
-    ctypes call releases the GIL). Returns seconds."""
+def oracle_pass(wl, units, threads):
+    """The oracle over `units` sample units of the workload's tensor (cycled), chunked over a
+    thread pool (the ctypes call releases the GIL). A unit is one row of the input for the row
+    quantizers; for the dual pass it is one row of dY quantized in row orientation plus one
+    column of dY in column orientation, i.e. (M + N) / 2 elements of dY in both orientations.
+    An E4M3 tensor scale that the workload computes every step is computed by the oracle too
+    (per chunk of rows: the same amax work per element); a given one is passed in.
+    Returns (seconds, elements of the workload the sample stands for)."""
+    import numpy as np
     import oracle as O
-    oc = _oracle_cfg(cfg)
+    bits = wl.host_bits
+    M, N = bits.shape
     chunk = 64
-    starts = [(r % bits.shape[0]) for r in range(0, rows_total, chunk)]
+    starts = list(range(0, units, chunk))
+    if isinstance(wl, DualWorkload):
+        orc, occ = _oracle_cfg(wl.rc), _oracle_cfg(wl.cc)
 
-    def one(r0):
-        r1 = min(r0 + chunk, bits.shape[0])
-        O.quantize(oc, bits[r0:r1], row0=r0,
-                   tensor_scale=0.01 if oc.scale == O.SCALE_E4M3_1x16 else None)
+        def one(k):
+            r0, c0 = k % M, k % N
+            r1, c1 = min(r0 + chunk, M, r0 + units - k), min(c0 + chunk, N, c0 + units - k)
+            O.quantize(orc, bits[r0:r1], row0=r0)
+            O.quantize(occ, np.ascontiguousarray(bits[:, c0:c1].T), row0=c0)
+            return ((r1 - r0) * N + (c1 - c0) * M) / 2.0
+    else:
+        oc = _oracle_cfg(wl.cfg)
+        given = oc.scale == O.SCALE_E4M3_1x16 and getattr(wl, "given", False)
+
+        def one(k):
+            r0 = k % M
+            r1 = min(r0 + chunk, M, r0 + units - k)
+            O.quantize(oc, bits[r0:r1], row0=r0, tensor_scale=0.01 if given else None)
+            return float((r1 - r0) * N)
 
     t = time.perf_counter()
     if threads > 1:
         with cf.ThreadPoolExecutor(max_workers=threads) as ex:
-            list(ex.map(one, starts))
+            elems = sum(ex.map(one, starts))
     else:
-        for r0 in starts:
-            one(r0)
-    return time.perf_counter() - t
+        elems = sum(one(k) for k in starts)
+    return time.perf_counter() - t, elems
+
+
+def _unit_name(wl):
+    return "rows + columns of dY" if isinstance(wl, DualWorkload) else "rows"
 
 
 def cpu_baseline(wl, budget_s=12.0):
     cores = len(os.sched_getaffinity(0))
-    cfg = getattr(wl, "cfg", None) or wl.rc
-    bits = wl.host_bits
-    probe_rows = 256
-    t = oracle_pass(cfg, bits, probe_rows, cores)
-    rows = int(min(bits.shape[0], max(probe_rows, probe_rows * budget_s / max(t, 1e-6) / 4)))
-    t = oracle_pass(cfg, bits, rows, cores)
+    total = wl.host_bits.shape[0]
     per_elem = wl.bytes_per_step() / wl.elements()
-    gbs = rows * bits.shape[1] * per_elem / t / 1e9
+    probe = 256
+    t, _ = oracle_pass(wl, probe, cores)
+    units = int(min(total, max(probe, probe * budget_s / max(t, 1e-6) / 4)))
+    t, elems = oracle_pass(wl, units, cores)
+    gbs = elems * per_elem / t / 1e9
     # one thread on a short sample, for the per-core figure
-    t1 = oracle_pass(cfg, bits, probe_rows, 1)
-    gbs1 = probe_rows * bits.shape[1] * per_elem / t1 / 1e9
+    t1, elems1 = oracle_pass(wl, probe, 1)
+    gbs1 = elems1 * per_elem / t1 / 1e9
     return {"value": round(gbs, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": "%d of %d rows of the step's tensor (%.1f s wall on %d threads)"
-                      % (rows, bits.shape[0], t, cores),
-            "single_thread": {"value": round(gbs1, 4), "sample": "%d rows" % probe_rows},
+            "sample": "%d of %d %s of the step's tensor (%.1f s wall on %d threads)"
+                      % (units, total, _unit_name(wl), t, cores),
+            "single_thread": {"value": round(gbs1, 4), "sample": "%d %s" % (probe, _unit_name(wl))},
             "cpu_model": _cpu_model()}
 
 
@@ -724,34 +746,35 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    from block_scaled_bit_rht16_b200 import synth
-    import numpy as np
-    import block_scaled_bit_rht16_b200 as fq
-    mask = fq.sign_mask_from_seed(synth.sign_seed(2))
-    cfg = fq.recipe("ufp4", "fwd_y", "x", sign_mask=mask)
-    x, w = synth.dense_linear_operands()
-    bits = np.concatenate([x, w], axis=0)
+    wl = make_workload(args.workload)
+    wl.host_bits = wl.make_input()
+    wl.rows, wl.cols = wl.host_bits.shape
     cores = len(os.sched_getaffinity(0))
-    t1 = oracle_pass(cfg, bits, 64, 1)   # rows per second on one core
+    per_elem = wl.bytes_per_step() / wl.elements()
+    t1, _ = oracle_pass(wl, 64, 1)   # units per second on one core
     rate = 64 / max(t1, 1e-6) * max(1, cores) * 0.7
     budget = 120.0
-    rows = max(1, min(bits.shape[0], int(rate * budget / (args.steps + args.warmup))))
-    threads = cores if rows >= 64 * cores else 1
+    units = max(1, min(wl.rows, int(rate * budget / (args.steps + args.warmup))))
+    threads = cores if units >= 64 * cores else 1
     for i in range(args.warmup):
-        oracle_pass(cfg, bits, rows, threads)
-    t = 0.0
+        oracle_pass(wl, units, threads)
+    t, elems = 0.0, 0.0
     for i in range(args.steps):
-        t += oracle_pass(cfg, bits, rows, threads)
-    bytes_per_elem = 2.75
-    value = args.steps * rows * bits.shape[1] * bytes_per_elem / t / 1e9
+        dt, de = oracle_pass(wl, units, threads)
+        t += dt
+        elems += de
+    value = elems * per_elem / t / 1e9
+    sample = "%d of %d %s per step (the oracle's bounded share of one step)" % (
+        units, wl.rows, _unit_name(wl))
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(t / args.steps * 1e3, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": "dense-1.5B-like operands X[8192,2048] + W[8192,2048], UFP4 fwd_y "
-                                   "(RHT16 + E1M2 RTNE, FP32 1x16), CPU oracle on %d rows per step" % rows},
+            "config": {"workload": wl.desc, "elements_per_step": wl.elements(),
+                       "algorithmic_bytes_per_step": wl.bytes_per_step(),
+                       "parallelism": "CPU oracle, %d host thread(s)" % threads},
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
-                             "sample": "%d rows x 2048 per step, cycled through the stacked X,W" % rows},
+                             "sample": sample, "cpu_model": _cpu_model()},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

@@ -72,3 +72,52 @@ def test_every_workload_constructs():
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     with open(os.path.join(root, "profiles", "traffic.json")) as f:
         assert set(json.load(f)) <= keys
+
+
+_MAKE_WORKLOAD = bench.make_workload
+
+
+def _small_row_workload():
+    from block_scaled_bit_rht16_b200 import synth
+    wl = _MAKE_WORKLOAD("linear1.5b-ufp4")
+    wl.make_input = lambda: synth.small(5, 256, 512, "t4")
+    return wl
+
+
+def _small_dual_workload():
+    from block_scaled_bit_rht16_b200 import synth
+    wl = _MAKE_WORKLOAD("dy8192-dual-sr")
+    wl.make_input = lambda: synth.small(6, 192, 128, "normal", 1e-3)
+    return wl
+
+
+def test_oracle_sample_counts_the_elements_it_quantizes():
+    # the row quantizer: one unit is one row; a partial last chunk counts only its rows
+    wl = _small_row_workload()
+    wl.host_bits = wl.make_input()
+    t, elems = bench.oracle_pass(wl, 100, 2)
+    assert t > 0 and elems == 100 * 512
+    # the dual pass: a unit is a row of dY in row orientation plus a column in column
+    # orientation, (M + N) / 2 elements of dY in both orientations
+    wl = _small_dual_workload()
+    wl.host_bits = wl.make_input()
+    t, elems = bench.oracle_pass(wl, 96, 1)
+    assert t > 0 and elems == 96 * (192 + 128) / 2
+
+
+def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
+    import json
+    import types
+    for make in (_small_row_workload, _small_dual_workload):
+        monkeypatch.setattr(bench, "make_workload", lambda name, make=make: make())
+        args = types.SimpleNamespace(workload="any", steps=2, warmup=3, gpus=1)
+        bench.run_reference(args)
+        line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+        assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+        assert line["unit"] == "GB/s" and line["higher_is_better"] is True and line["value"] > 0
+        assert line["steps"] == 2 and line["warmup"] == 3 and line["n_gpus"] == 1
+        assert line["config"]["workload"] == make().desc
+        cb = line["cpu_baseline"]
+        assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
+        assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                               "d2h_bytes_per_step": 0}
