@@ -490,7 +490,23 @@ def test_nv_scales_follow_the_tensor_amax():
     assert abs(xh - A) <= A * 2 ** -7                       # largest dequant value ~ A
     # NVINT4: same two-level rule with 7 in place of 6 (reading R9)
     c4 = O.OracleConfig(grid=O.GRID_INT4, scale=O.SCALE_E4M3_1x16, sign_mask=0x3C3C)
-    assert O.quantize(c4, x)["tensor_scale"] == np.float32(np.float32(A) / np.float32(7 * 448))
+    r4 = O.quantize(c4, x)
+    assert r4["tensor_scale"] == np.float32(np.float32(A) / np.float32(7 * 448))
+    # every block's scale maps its own amax onto qmax: E4M3 keeps 3 mantissa bits, so in its
+    # normal range RNE moves the block scale by at most 2^-4 relative, and amax_b / s lies in
+    # qmax * [1/(1 + 2^-4), 1/(1 - 2^-4)] (IF4 page, section 3.2: the block scale is amax_b
+    # over qmax in units of the tensor scale); blocks that saturate at 448 or fall below
+    # E4M3's normal range are left out
+    xf = synth.bf16_bits_to_f32(x).reshape(-1, 16)
+    amax_b = np.abs(np.stack([O.rht16(b, 0x3C3C) for b in xf])).max(-1).astype(np.float64)
+    dec = np.array([O.e4m3_decode(b) for b in range(128)], np.float64)
+    for res, qmax in ((r, 6.0), (r4, 7.0)):
+        d8 = dec[res["scales"].reshape(-1)]
+        s_b = d8 * float(res["tensor_scale"])
+        ok = (d8 >= 2.0 ** -6) & (d8 < 448)
+        assert ok.sum() > 500
+        ratio = amax_b[ok] / s_b[ok]
+        assert np.all((ratio >= qmax / (1 + 2 ** -4) * (1 - 1e-6)) & (ratio <= qmax / (1 - 2 ** -4) * (1 + 1e-6)))
 
 
 def test_mx_block_scale_powers_of_two():
