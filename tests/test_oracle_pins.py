@@ -633,3 +633,161 @@ def test_sr_index_is_logical_row_major():
     np.testing.assert_array_equal(full["codes"][10:20], part["codes"])
     other = O.quantize(cfg, np.ascontiguousarray(x[10:20]), row0=0)
     assert not np.array_equal(other["codes"], part["codes"])
+
+
+# ------------------------------------------------------------------ pins from decoded outputs
+
+_E4M3_TABLE = None
+
+
+def _e4m3_table():
+    global _E4M3_TABLE
+    if _E4M3_TABLE is None:
+        _E4M3_TABLE = np.array([O.e4m3_decode(b) for b in range(128)], np.float32)
+    return _E4M3_TABLE
+
+
+def _decoded_blocks(cfg, r, x):
+    """From the input and the oracle's codes and scales alone: per element y (rotated, FP32),
+    v = y / s (FP32 IEEE division, the scaled value), the decoded value in scaled units, its
+    magnitude cell, and xhat = value * s (FP32); per block the IF4 INT4 flag."""
+    rows, cols = x.shape
+    bs = 32 if cfg.scale == O.SCALE_UE8M0_1x32 else 16
+    xf = synth.bf16_bits_to_f32(x).reshape(-1, 16)
+    y = np.stack([O.rht16(b, cfg.sign_mask) if cfg.rht else b for b in xf]).reshape(rows, cols)
+    y = y.astype(np.float32)
+    sc = r["scales"]
+    flag = np.zeros(sc.shape, bool)
+    if cfg.scale == O.SCALE_FP32_1x16:
+        s = sc.astype(np.float32)
+    elif cfg.scale == O.SCALE_E4M3_1x16:
+        s = _e4m3_table()[sc & 0x7F] * np.float32(r["tensor_scale"])
+        flag = (sc >> 7).astype(bool) if cfg.grid == O.GRID_IF4 else flag
+    else:
+        s = np.ldexp(np.float32(1), sc.astype(np.int32) - 127).astype(np.float32)
+    s_el = np.repeat(s, bs, axis=1)
+    int_el = np.repeat(flag, bs, axis=1)
+    nib = _nib(r["codes"])
+    fp_grid = O.GRID_E2M1 if cfg.grid == O.GRID_IF4 else cfg.grid
+    k = _value_of(O.GRID_INT4, nib).astype(np.float32)
+    if cfg.grid == O.GRID_INT4:
+        val, cell = k, np.abs(k).astype(int)
+    else:
+        val, cell = _value_of(fp_grid, nib).astype(np.float32), (nib & 7).astype(int)
+    val = np.where(int_el, k * np.float32(6 / 7), val).astype(np.float32)
+    cell = np.where(int_el, np.abs(k).astype(int), cell)
+    zero = s_el == 0
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.where(zero, np.float32(0), y / np.where(zero, np.float32(1), s_el)).astype(np.float32)
+    xhat = np.where(zero, np.float32(0), val * s_el).astype(np.float32)
+    return y, v, val, cell, xhat, flag
+
+
+@pytest.mark.parametrize("name,cfg", [
+    ("e1m2_fp32_rht", O.OracleConfig(grid=O.GRID_E1M2, sign_mask=0x1111)),
+    ("int4_fp32_sr", O.OracleConfig(grid=O.GRID_INT4, round=O.ROUND_SR, sign_mask=0x0FF0, sr_seed=17)),
+    ("e2m1max3_fp32", O.OracleConfig(grid=O.GRID_E2M1_MAX3, rht=0)),
+    ("nvint4", O.OracleConfig(grid=O.GRID_INT4, scale=O.SCALE_E4M3_1x16, sign_mask=0x3003)),
+    ("if4", O.OracleConfig(grid=O.GRID_IF4, scale=O.SCALE_E4M3_1x16, sign_mask=0x5A5A)),
+    ("mxfp4", O.OracleConfig(grid=O.GRID_E2M1, scale=O.SCALE_UE8M0_1x32, sign_mask=0x0001)),
+])
+def test_stats_are_the_sums_over_decoded_codes(name, cfg):
+    # UFP4-A (RHT and compounding sections) defines SQNR from sum y^2 / sum (y - xhat)^2 and the
+    # attenuation from <xhat, y> / |y|^2; the E2M1 section the per-cell signed error in scaled
+    # units; IF4 6.2 the share of blocks that keep FP4. Every raw sum is recomputed here from
+    # the codes and scales, so a sum over the wrong operand or cell cannot pass.
+    x = synth.small(97, 48, 256, "t4")
+    r = O.quantize(cfg, x, stats=True)
+    raw = r["stats_raw"]
+    y, v, val, cell, xhat, flag = _decoded_blocks(cfg, r, x)
+    y64, xh64 = y.astype(np.float64), xhat.astype(np.float64)
+    np.testing.assert_allclose(raw[O.ST_SUM_Y2], (y64 ** 2).sum(), rtol=1e-12)
+    np.testing.assert_allclose(raw[O.ST_SUM_ERR2], ((y64 - xh64) ** 2).sum(), rtol=1e-12)
+    np.testing.assert_allclose(raw[O.ST_SUM_YXHAT], (y64 * xh64).sum(), rtol=1e-12)
+    assert raw[O.ST_N] == x.size
+    err = np.abs(val.astype(np.float64)) - np.abs(v.astype(np.float64))
+    for c in range(8):
+        assert raw[O.ST_CELL_N + c] == (cell == c).sum(), c
+        np.testing.assert_allclose(raw[O.ST_CELL_ERR + c], err[cell == c].sum(), rtol=1e-9, atol=1e-9)
+    assert raw[O.ST_BLOCKS] == r["scales"].size
+    if cfg.grid == O.GRID_IF4:
+        assert 0 < flag.sum() < flag.size
+        assert raw[O.ST_IF4_FP4] == (~flag).sum()
+
+
+def test_if4_picks_the_smaller_squared_error_brute_force():
+    # IF4 sections 3.1 / 3.1.1: each block keeps the candidate with the smaller mean squared
+    # error; INT4 only when strictly smaller (R11). Both candidates are formed here from v by
+    # brute force: E2M1 by the exponent/step rule, INT4 as round-half-even(v * RN(7/6)) clamped to
+    # 7 and valued k * RN(6/7); errors in FP64.
+    cfg = O.OracleConfig(grid=O.GRID_IF4, scale=O.SCALE_E4M3_1x16, sign_mask=0x6C6C)
+    checked = separated = 0
+    for seed, kind in [(101, "uniform"), (102, "normal"), (103, "laplace"), (104, "t4")]:
+        x = synth.small(seed, 128, 256, kind)
+        r = O.quantize(cfg, x)
+        _, v, _, _, _, flag = _decoded_blocks(cfg, r, x)
+        v = v.reshape(-1, 16)
+        fp = np.copysign(_e2m1_by_exponent(np.abs(v.astype(np.float64))), v)
+        w = (v * np.float32(7 / 6)).astype(np.float32)
+        k = np.clip(np.rint(w), -7, 7).astype(np.float32)
+        it = (k * np.float32(6 / 7)).astype(np.float64)
+        sse_fp = ((fp - v) ** 2).sum(-1)
+        sse_int = ((it - v) ** 2).sum(-1)
+        decided = np.abs(sse_int - sse_fp) > 1e-4 * np.maximum(sse_fp, 1e-30)
+        want = sse_int < sse_fp
+        got = flag.reshape(-1)
+        np.testing.assert_array_equal(got[decided], want[decided])
+        checked += decided.sum()
+        # blocks where the absolute error would choose the other way
+        l1 = np.abs(it - v).sum(-1) < np.abs(fp - v).sum(-1)
+        separated += (decided & (l1 != want)).sum()
+    assert checked > 1500 and separated > 0
+    # an exact tie: scaled values in {0, +-6} lie on both candidates (7 * RN(6/7) rounds to 6),
+    # both errors are 0, and the block keeps FP4
+    tie = np.array([6, 0, -6, 0] * 4, np.float32)
+    assert np.float32(7) * np.float32(6 / 7) == np.float32(6)
+    r = O.quantize(O.OracleConfig(grid=O.GRID_IF4, scale=O.SCALE_E4M3_1x16, rht=0),
+                   synth.to_bf16_bits(tie[None]), tensor_scale=np.float32(1 / 64))
+    # Delta = 6 / (6/64) = 64 = 2^6: E4M3 exponent field 6 + 7 = 13, mantissa 0 -> 0x68; bit 7
+    # clear: FP4 kept
+    assert r["scales"][0, 0] == 0x68
+
+
+def test_sr_rounds_each_element_with_its_own_draw():
+    # R12: element (m, n) draws u = sr_bits(seed, stream, m * cols + n). With every element half
+    # way between two E1M2 points (v = 1.25, s = 1) it rounds up to 1.5 exactly when
+    # u * 2^-16 < 1/2; the block's first element (3.5) sets s and is a grid point.
+    rows, cols, row0 = 6, 64, 5
+    row = np.full(cols, 1.25, np.float32)
+    row[::16] = 3.5
+    x = synth.to_bf16_bits(np.tile(row, (rows, 1)))
+    for stream in (0, 1):
+        cfg = O.OracleConfig(grid=O.GRID_E1M2, round=O.ROUND_SR, rht=0, sr_seed=1234, sr_stream=stream)
+        nib = _nib(O.quantize(cfg, x, row0=row0)["codes"])
+        want = np.empty((rows, cols), np.uint8)
+        for m in range(rows):
+            for n in range(cols):
+                u = O.sr_bits(1234, stream, (row0 + m) * cols + n)
+                want[m, n] = 7 if n % 16 == 0 else (3 if u < 2 ** 15 else 2)
+        np.testing.assert_array_equal(nib, want)
+        assert 0.3 < (want == 3).mean() < 0.7
+
+
+def test_sign_mask_is_the_low_bits_of_the_published_outputs():
+    # R1: the sign mask of a seed is the low 16 bits of SplitMix64's first output from that
+    # state; from states 0 and gamma these are the first two published outputs
+    outs = [int(ln[0], 16) for ln in _golden_lines("splitmix64.txt")]
+    assert O.sign_mask_from_seed(0) == outs[0] & 0xFFFF
+    assert O.sign_mask_from_seed(0x9E3779B97F4A7C15) == outs[1] & 0xFFFF
+
+
+def test_nv_block_below_the_e4m3_range_encodes_zero():
+    # R8: a block whose Delta = amax_b / (alpha * 6) rounds to E4M3 zero (below 2^-10, half the
+    # smallest subnormal) has s = 0 and encodes as zeros, whatever its signs
+    big = np.full(16, 448.0 * 6, np.float32)              # alpha = A / (6 * 448) = 1
+    tiny = np.array([1e-4, -2e-4, 3e-4, -1e-4] * 4, np.float32)
+    x = synth.to_bf16_bits(np.stack([big, tiny]))
+    r = O.quantize(O.OracleConfig(grid=O.GRID_E2M1, scale=O.SCALE_E4M3_1x16, rht=0), x, dequant=True)
+    assert r["tensor_scale"] == 1.0 and r["scales"][0, 0] == 0x7E
+    assert r["scales"][1, 0] == 0
+    assert np.all(r["codes"][1] == 0) and np.all(r["dequant"][1] == 0)
