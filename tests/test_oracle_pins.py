@@ -791,3 +791,24 @@ def test_nv_block_below_the_e4m3_range_encodes_zero():
     assert r["tensor_scale"] == 1.0 and r["scales"][0, 0] == 0x7E
     assert r["scales"][1, 0] == 0
     assert np.all(r["codes"][1] == 0) and np.all(r["dequant"][1] == 0)
+
+
+def test_row_pitch_is_layout_only():
+    # a row pitch larger than the row (ld > cols) changes where rows start, not what is
+    # quantized: a view into a wider array gives the outputs of its contiguous copy, with the
+    # padding columns (filled with large values) never read
+    wide = synth.small(111, 40, 320, "laplace", 2.0)
+    wide[:, 256:] = synth.to_bf16_bits(np.full((40, 64), 1e4, np.float32))
+    view = wide[:, :256]
+    dense = np.ascontiguousarray(view)
+    assert view.strides[0] == 640 and dense.strides[0] == 512
+    for cfg in (O.OracleConfig(grid=O.GRID_E1M2, sign_mask=0x4321),
+                O.OracleConfig(grid=O.GRID_E2M1, scale=O.SCALE_E4M3_1x16, sign_mask=0x4321),
+                O.OracleConfig(grid=O.GRID_E2M1, scale=O.SCALE_UE8M0_1x32, sign_mask=0x4321)):
+        a, b = O.quantize(cfg, view, dequant=True), O.quantize(cfg, dense, dequant=True)
+        for key in ("codes", "scales", "dequant"):
+            np.testing.assert_array_equal(a[key], b[key])
+        assert a["tensor_scale"] == b["tensor_scale"]
+        assert O.tensor_amax(cfg, view) == O.tensor_amax(cfg, dense)
+    for ya, yb in zip(O.rht16_rows(view, 0x4321), O.rht16_rows(dense, 0x4321)):
+        np.testing.assert_array_equal(ya, yb)
