@@ -483,6 +483,14 @@ def test_nv_scales_follow_the_tensor_amax():
     cfg = O.OracleConfig(grid=O.GRID_E2M1, scale=O.SCALE_E4M3_1x16, sign_mask=0x3C3C)
     r = O.quantize(cfg, x, dequant=True)
     A = O.tensor_amax(cfg, x)
+    # A is the largest magnitude of the rotated tensor, also when that element is negative
+    yall = np.stack([O.rht16(b, 0x3C3C) for b in synth.bf16_bits_to_f32(x).reshape(-1, 16)])
+    assert A == np.abs(yall).max()
+    neg = synth.bf16_bits_to_f32(x).copy()
+    neg[3, 17] = -1000.0
+    ny = np.stack([O.rht16(b, 0x3C3C) for b in neg.reshape(-1, 16)])
+    assert ny.max() < -ny.min()
+    assert O.tensor_amax(cfg, synth.to_bf16_bits(neg)) == np.abs(ny).max()
     assert r["tensor_scale"] == np.float32(np.float32(A) / np.float32(6 * 448))
     assert r["scales"].max() == 0x7E                       # the block holding A gets 448
     assert np.all(r["scales"] <= 0x7E)
@@ -738,6 +746,12 @@ def test_if4_picks_the_smaller_squared_error_brute_force():
         got = flag.reshape(-1)
         np.testing.assert_array_equal(got[decided], want[decided])
         checked += decided.sum()
+        # and each block carries the codes of the candidate it chose
+        nib = _nib(r["codes"]).reshape(-1, 16)
+        k_codes = (k.astype(np.int64) & 0xF).astype(np.uint8)
+        np.testing.assert_array_equal(nib[got], k_codes[got])
+        fp_vals = np.array([O.decode_nibble(O.GRID_E2M1, c) for c in range(16)])[nib[~got]]
+        np.testing.assert_array_equal(np.abs(fp_vals), np.abs(fp[~got]))
         # blocks where the absolute error would choose the other way
         l1 = np.abs(it - v).sum(-1) < np.abs(fp - v).sum(-1)
         separated += (decided & (l1 != want)).sum()
