@@ -7,8 +7,12 @@ with no data exchange, except for two reductions:
     monotonic, so max_r alpha_r is exactly the alpha of the whole tensor -- one all-reduce(MAX)
     of a single float, after which every rank quantizes with the tensor scale given;
   * statistics: the raw FP64 records add up (all-reduce(SUM) of 24 doubles).
-Stochastic rounding stays identical to the unsharded tensor because its counter uses the
-global element index (row offset r0 passed in).
+Stochastic rounding stays identical to the unsharded tensor: a shard quantizes its rows as a
+tensor of their own (element indices from 0) with the seed from shard_sr_seed, which starts
+the counter stream where those rows start in the whole tensor. This holds for the row
+orientation. The column orientation of the dual dY pass indexes element (m, n) as n * M + m,
+which depends on the whole tensor's M; a row-sharded dual pass with stochastic rounding on the
+column orientation therefore draws differently from the unsharded one.
 
 The compute steps are passed in as callables so the same logic runs with the CUDA library on
 GPUs and, in the tests, with the CPU oracle on gloo ranks.
@@ -30,6 +34,23 @@ def row_range(rows: int, rank: int, world: int, multiple: int = 1):
     u0 = rank * per + min(rank, extra)
     u1 = u0 + per + (1 if rank < extra else 0)
     return u0 * multiple, u1 * multiple
+
+
+GAMMA = 0x9E3779B97F4A7C15   # SplitMix64's state increment (Steele, Lea & Flood 2014)
+
+
+def shard_sr_seed(sr_seed: int, r0: int, cols: int) -> int:
+    """The stochastic-rounding seed for rows [r0, ...) of a [rows, cols] tensor quantized on
+    their own, such that every element draws what it draws inside the whole tensor.
+
+    Element idx (row-major) takes 16-bit lane idx & 3 of output idx >> 2 of the SplitMix64
+    stream whose state starts at the seed (with the stream number in bit 63) and advances by
+    GAMMA per output. Row r0 starts at output r0 * cols / 4 (cols is a multiple of 4), so the
+    shard's stream must start r0 * cols / 4 increments later. Flipping bit 63 equals adding
+    2^63 modulo 2^64, so the same shift serves both streams."""
+    if cols % 4 or r0 < 0:
+        raise ValueError("cols must be a multiple of 4 and r0 non-negative")
+    return (int(sr_seed) + (r0 * cols // 4) * GAMMA) % (1 << 64)
 
 
 def global_tensor_scale(local_alpha: float, group=None) -> float:

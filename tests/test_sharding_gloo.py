@@ -36,9 +36,13 @@ def _worker(rank, port, case, out_dir):
         }[case]
         r0, r1 = sharding.row_range(x.shape[0], rank, WORLD, multiple=16)
         xs = np.ascontiguousarray(x[r0:r1])
+        # the shard is quantized as a tensor of its own, as the library's call sees it: element
+        # indices from 0, with the stochastic-rounding seed shifted to where its rows start
+        from dataclasses import replace
+        scfg = replace(cfg, sr_seed=sharding.shard_sr_seed(cfg.sr_seed, r0, x.shape[1]))
         steps = sharding.ShardSteps(
             tensor_scale=lambda: np.float32(O.tensor_amax(cfg, xs)) / np.float32(6.0 * 448.0),
-            quantize=lambda alpha: O.quantize(cfg, xs, row0=r0, tensor_scale=alpha, stats=True))
+            quantize=lambda alpha: O.quantize(scfg, xs, row0=0, tensor_scale=alpha, stats=True))
         res = sharding.quantize_rows_sharded(steps, cfg.scale == O.SCALE_E4M3_1x16)
         stats = sharding.global_stats_raw(res["stats_raw"])
         np.savez(os.path.join(out_dir, "r%d.npz" % rank), codes=res["codes"], scales=res["scales"],
@@ -79,3 +83,24 @@ def test_row_range_partitions():
         assert all(s[0] % mult == 0 for s in spans)
     with pytest.raises(ValueError):
         sharding.row_range(20, 0, 2, 16)
+
+
+def test_shard_seed_reproduces_the_draws_of_every_row_range():
+    # without any communication, a row range quantized on its own with the shifted seed gives
+    # the rows of the whole tensor's result, in both counter streams and for ragged starts
+    import oracle as O
+    from dataclasses import replace
+    from block_scaled_bit_rht16_b200 import sharding, synth
+    x = synth.small(78, 40, 96, "normal")
+    for stream in (0, 1):
+        cfg = O.OracleConfig(grid=O.GRID_INT4, round=O.ROUND_SR, sign_mask=0x0F0F,
+                             sr_seed=0xFFFF_FFFF_FFFF_FFF0, sr_stream=stream)
+        full = O.quantize(cfg, x)["codes"]
+        for r0 in (0, 1, 7, 39):
+            part = O.quantize(replace(cfg, sr_seed=sharding.shard_sr_seed(cfg.sr_seed, r0, 96)),
+                              np.ascontiguousarray(x[r0:]))["codes"]
+            np.testing.assert_array_equal(part, full[r0:])
+        # the unshifted seed does not: the shift is what makes the shard agree
+        assert not np.array_equal(O.quantize(cfg, np.ascontiguousarray(x[7:]))["codes"], full[7:])
+    with pytest.raises(ValueError):
+        sharding.shard_sr_seed(1, 3, 6)
