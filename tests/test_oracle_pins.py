@@ -826,3 +826,22 @@ def test_row_pitch_is_layout_only():
         assert O.tensor_amax(cfg, view) == O.tensor_amax(cfg, dense)
     for ya, yb in zip(O.rht16_rows(view, 0x4321), O.rht16_rows(dense, 0x4321)):
         np.testing.assert_array_equal(ya, yb)
+
+
+def test_format_error_ranking_on_laplace():
+    # IF4 page, section 2.2 table: MXFP4 > NVFP4 > NVINT4 > IF4 in quantization MSE (values
+    # printed without their data, so only the order is pinned), and IF4 keeps FP4 on part of
+    # the blocks (section 6.2); on a Laplace sample with the rotation
+    x = synth.laplace_format_tensor(rows=512)
+    mask = O.sign_mask_from_seed(synth.sign_seed(4))
+    nmse = {}
+    for name, grid, scale in (("MXFP4", O.GRID_E2M1, O.SCALE_UE8M0_1x32),
+                              ("NVFP4", O.GRID_E2M1, O.SCALE_E4M3_1x16),
+                              ("NVINT4", O.GRID_INT4, O.SCALE_E4M3_1x16),
+                              ("IF4", O.GRID_IF4, O.SCALE_E4M3_1x16)):
+        st = O.finalize_stats(O.quantize(O.OracleConfig(grid=grid, scale=scale, sign_mask=mask), x,
+                                         stats=True)["stats_raw"])
+        nmse[name] = st["nmse"]
+        if grid == O.GRID_IF4:
+            assert 0.1 < st["if4_fp4_fraction"] < 0.9
+    assert nmse["MXFP4"] > nmse["NVFP4"] > nmse["NVINT4"] > nmse["IF4"]
