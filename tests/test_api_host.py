@@ -202,3 +202,42 @@ def test_grouped_validation():
     sr = fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=fq.FP4Q_SCALE_E4M3_1x16_TENSOR,
                    round=fq.FP4Q_ROUND_SR).c()
     assert g(cfg=sr) == _lib.FP4Q_ERR_UNSUPPORTED
+
+
+def test_plain_c_program_uses_the_library(tmp_path):
+    # the ABI is usable from C alone: a program built against include/fp4q.h and linked with
+    # libfp4q.so calls the host-side entry points and gets the documented statuses (no GPU work:
+    # every quantize call here is rejected by validation)
+    prog = tmp_path / "consumer.c"
+    prog.write_text(r'''#include <stdio.h>
+#include <string.h>
+#include "fp4q.h"
+int main(void) {
+  fp4q_config c;
+  memset(&c, 0, sizeof c);
+  c.grid = FP4Q_GRID_E1M2; c.scale = FP4Q_SCALE_FP32_1x16; c.round = FP4Q_ROUND_RTNE; c.rht = 1;
+  c.sign_mask = fp4q_sign_mask_from_seed(7); c.outputs = FP4Q_OUT_CODES;
+  void* fake = (void*)(uintptr_t)(1u << 20);
+  printf("%u\n", c.sign_mask);
+  printf("%zu\n", fp4q_workspace_size(&c, 128, 256));
+  c.outputs |= FP4Q_OUT_STATS;
+  printf("%zu\n", fp4q_workspace_size(&c, 128, 256));
+  c.outputs = FP4Q_OUT_CODES;
+  printf("%d\n", (int)fp4q_rht_quantize(&c, fake, 4, 24, 24, fake, fake, NULL, 0, NULL, NULL, 0, NULL));
+  printf("%d\n", (int)fp4q_rht_quantize(&c, NULL, 4, 32, 32, fake, fake, NULL, 0, NULL, NULL, 0, NULL));
+  printf("%d\n", (int)fp4q_quantize_dual(&c, &c, fake, 24, 32, 32, fake, fake, fake, fake, NULL, 0, NULL));
+  printf("%d\n", (int)fp4q_rht_quantize_noalloc(&c, (char*)fake + 8, 4, 32, 32, fake, fake, NULL, 0, NULL, NULL));
+  printf("%s\n", fp4q_status_string(FP4Q_ERR_ALIGN));
+  return 0;
+}
+''')
+    exe = tmp_path / "consumer"
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(prog),
+                    "-L", libdir, "-lfp4q", "-Wl,-rpath," + libdir, "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    assert int(out[0]) == O.sign_mask_from_seed(7)
+    assert int(out[1]) == 0 and int(out[2]) == fq.workspace_size(fq.Config(stats=True), 128, 256)
+    assert [int(v) for v in out[3:7]] == [_lib.FP4Q_ERR_SHAPE, _lib.FP4Q_ERR_INVALID_ARG,
+                                          _lib.FP4Q_ERR_SHAPE, _lib.FP4Q_ERR_ALIGN]
+    assert out[7] == "misaligned pointer or row pitch"
