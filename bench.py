@@ -124,14 +124,50 @@ class ClockSampler:
 HOST_ONLY_SOURCES = ("fp4q_api.cu", "fp4q_noalloc.cu")
 
 
-def kernel_source_sha():
-    """Fingerprint of the device sources, to tell whether committed ncu counters still apply."""
+def strip_c_comments(src):
+    """C/C++ source text without its // and /* */ comments (string and character literals are
+    kept whole); each comment leaves one space, line breaks inside block comments are kept."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+            out.append(" ")
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            j = n if j < 0 else j + 2
+            out.append(" " + "\n" * src.count("\n", i, j))
+            i = j
+        else:
+            out.append(c)
+            i += 1
+    return "".join(out)
+
+
+def canonical_code(src):
+    """The source's code alone: comments removed, every run of blanks made one space, blank
+    lines dropped. Two sources that differ only in comments and layout map to the same text."""
+    lines = (" ".join(ln.split()) for ln in strip_c_comments(src).split("\n"))
+    return "\n".join(ln for ln in lines if ln)
+
+
+def kernel_source_sha(csrc=None):
+    """Fingerprint of the device sources, to tell whether committed ncu counters still apply.
+    Comments and layout are left out: they cannot change what a kernel does."""
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "block_scaled_bit_rht16_b200", "csrc")
+    csrc = csrc or os.path.join(ROOT, "block_scaled_bit_rht16_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh")) and name not in HOST_ONLY_SOURCES:
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+            with open(os.path.join(csrc, name), encoding="utf-8") as f:
+                code = canonical_code(f.read())
+            h.update(name.encode() + b"\0" + code.encode())
     return h.hexdigest()[:16]
 
 

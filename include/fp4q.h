@@ -138,7 +138,8 @@ typedef struct {
   double nmse;              /* sum_err2 / sum_y2 */
   double cell_mean_err[8];  /* cell_err / cell_count (NaN for an empty cell): shrinkage bias */
   double if4_fp4_fraction;  /* if4_fp4_blocks / blocks */
-  int32_t status;           /* FP4Q_OK, or FP4Q_ERR_TIMEOUT if a device wait gave up */
+  int32_t status;           /* FP4Q_OK, or FP4Q_ERR_TIMEOUT if a device wait gave up (no
+                               current kernel waits: always FP4Q_OK) */
   int32_t reserved;
 } fp4q_stats_t;
 
@@ -279,10 +280,11 @@ fp4q_status fp4q_rht16(const void* x, int64_t rows, int64_t cols, int64_t ld, ui
 fp4q_status fp4q_check_division(uint64_t seed, uint64_t n, unsigned long long* mismatches,
                                 fp4q_stream_t stream);
 
-/* Device status word of the library on the current device: bit 0 set when a bounded wait
- * inside a quantize kernel (shared-memory stage copies) gave up after 2 s -- that launch's
- * outputs are incomplete; bit 1 set by fp4q_check_wait_timeout. Copies the word to
- * *status_bits (host), clears it when `clear` is 1, and synchronizes `stream`. */
+/* Device status word of the library on the current device: bit 0 is reserved for a bounded
+ * wait inside a quantize kernel that gives up (that launch's outputs would be incomplete); the
+ * current kernels read their inputs with plain loads and never wait, so it stays clear. Bit 1 is
+ * set by fp4q_check_wait_timeout. Copies the word to *status_bits (host), clears it when
+ * `clear` is 1, and synchronizes `stream`. */
 fp4q_status fp4q_device_status(int32_t* status_bits, int32_t clear, fp4q_stream_t stream);
 
 /* Diagnostic: launches one thread that waits, with a limit of limit_ns (1 ns .. 1 s), on a

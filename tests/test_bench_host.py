@@ -121,3 +121,11 @@ def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
         assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
         assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
                                "d2h_bytes_per_step": 0}
+
+
+def test_kernel_fingerprint_ignores_comments_and_layout_only():
+    a = 'int f(int x) {  // scale\n  return x * 2; /* twice */\n}\nconst char* s = "a // b /* c */";\n'
+    b = '/* new header\n   comment */\nint f(int x) {\n\n  return x * 2;\n}\nconst char* s = "a // b /* c */";'
+    assert bench.canonical_code(a) == bench.canonical_code(b)
+    assert "a // b /* c */" in bench.canonical_code(a)           # string literals kept whole
+    assert bench.canonical_code(a) != bench.canonical_code(a.replace("x * 2", "x * 3"))
