@@ -1,7 +1,7 @@
 // fp4q_row.cu -- row-orientation kernels of the fused RHT16 + block-scaled 4-bit quantizer.
 //
-// One thread owns one scale block (16 elements; 32 for UE8M0) end to end: two (four) 128-bit
-// coalesced loads, sign flips on the bf16 bits, the 16-point butterfly in registers (packed
+// One thread owns one scale block (16 elements; 32 for UE8M0) end to end: one 256-bit load per
+// 16 elements when rows are 32-byte aligned (else two 128-bit loads), sign flips on the bf16 bits, the 16-point butterfly in registers (packed
 // f32x2), block absmax, the scale, exact quotients, rounding, nibble packing, one 8-byte
 // (16-byte) code store and the scale store. Consecutive threads own consecutive blocks, so a
 // warp reads 1 KiB and writes 256 B of codes contiguously. The grid is persistent (SM count x
