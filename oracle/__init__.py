@@ -9,7 +9,6 @@ Configuration constants here are the oracle's own; callers map the library's con
 """
 import ctypes
 import math
-import os
 from dataclasses import dataclass
 
 import numpy as np

@@ -6,8 +6,6 @@ import os
 import re
 import subprocess
 
-import numpy as np
-import pytest
 
 import oracle as O
 import block_scaled_bit_rht16_b200 as fq

@@ -26,7 +26,6 @@ RESULTS = {}
 
 
 def _gemm_case(grid, rht):
-    import torch
     x_bits, w_bits = synth.dense_linear_operands()
     mask = fq.sign_mask_from_seed(synth.sign_seed(2)) if rht else 0
     cfg = fq.Config(grid=grid, scale=fq.FP4Q_SCALE_FP32_1x16, rht=rht, sign_mask=mask, stats=True)
