@@ -239,3 +239,27 @@ int main(void) {
     assert [int(v) for v in out[3:7]] == [_lib.FP4Q_ERR_SHAPE, _lib.FP4Q_ERR_INVALID_ARG,
                                           _lib.FP4Q_ERR_SHAPE, _lib.FP4Q_ERR_ALIGN]
     assert out[7] == "misaligned pointer or row pitch"
+
+
+def test_binding_rejects_host_tensors_before_any_call():
+    # every public function checks its tensors first: host memory never reaches the library
+    import pytest
+    import torch
+    x = torch.zeros((4, 32), dtype=torch.bfloat16)
+    cfg = fq.Config()
+    with pytest.raises(TypeError):
+        fq.rht_quantize(cfg, x)
+    with pytest.raises(TypeError):
+        fq.rht_quantize_grouped(cfg, x, torch.tensor([0, 4]))
+    with pytest.raises(TypeError):
+        fq.quantize_dual(cfg, cfg, torch.zeros((16, 32), dtype=torch.bfloat16))
+    with pytest.raises(TypeError):
+        fq.dequantize(cfg, torch.zeros((4, 16), dtype=torch.uint8), torch.zeros((4, 2)))
+    with pytest.raises(TypeError):
+        fq.rht16(x, 0)
+    with pytest.raises(TypeError):
+        fq.tensor_scale(fq.Config(scale=fq.FP4Q_SCALE_E4M3_1x16_TENSOR), x)
+    with pytest.raises(TypeError):
+        fq.stats(torch.zeros(256, dtype=torch.uint8))
+    with pytest.raises(TypeError):
+        fq.rht_quantize(cfg, torch.zeros((4, 32), dtype=torch.float32))
