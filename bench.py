@@ -171,16 +171,46 @@ def kernel_source_sha(csrc=None):
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel_key):
-    """DRAM bytes per launch from the committed ncu summary, if taken on the current sources."""
+def profiled_record(kernel_key):
+    """The committed ncu record of a kernel (profiles/traffic.json), if it was taken on the
+    current device sources; else None."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f).get(kernel_key)
         if rec and rec.get("source_sha") == kernel_source_sha():
-            return rec["bytes_per_launch"]
+            return rec
     except Exception:
         pass
     return None
+
+
+def profiled_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current sources."""
+    rec = profiled_record(kernel_key)
+    return rec["bytes_per_launch"] if rec else None
+
+
+SCHEDULERS_PER_SM = 4   # warp schedulers per SM, each issuing at most one instruction per clock
+
+
+def issue_roofline(warp_instructions, launch_ms, sms, sm_mhz):
+    """The instruction-issue roofline of one launch: the recorded warp instructions over the
+    launch's time against SMs x schedulers x clock."""
+    peak = sms * SCHEDULERS_PER_SM * sm_mhz * 1e6
+    achieved = warp_instructions / (launch_ms * 1e-3)
+    return {"warp_instructions_per_launch": int(warp_instructions),
+            "achieved_per_s": round(achieved / 1e9, 1), "peak_per_s": round(peak / 1e9, 1),
+            "unit": "G warp instructions/s", "frac": round(achieved / peak, 4),
+            "peak_source": "%d SMs x %d schedulers x %.0f MHz" % (sms, SCHEDULERS_PER_SM, sm_mhz)}
+
+
+def max_sm_mhz(clocks):
+    """The SM clock ceiling: MEASURED_PEAKS.json's sm_max_mhz, else the sampled maximum."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["sm_max_mhz"])
+    except Exception:
+        return float((clocks or {}).get("sm_max_mhz") or 1965.0)
 
 
 # ---------------------------------------------------------------------------- workloads
@@ -564,6 +594,13 @@ def run_ours(args):
                 "kernel": wl.kernel_key, "peak_source": peak_src,
                 "launch_us": round(launch_ms * 1e3, 3),
                 "algorithmic_bytes_per_launch": bytes_step / wl.launches_per_step}
+    try:   # the second roofline, where the committed capture recorded the instruction count
+        rec = profiled_record(wl.kernel_key)
+        if rec and rec.get("warp_instructions_per_launch"):
+            roofline["issue"] = issue_roofline(rec["warp_instructions_per_launch"], launch_ms,
+                                               props.multi_processor_count, max_sm_mhz(clocks))
+    except Exception:
+        pass
 
     extras = {}
     if not args.no_extras:

@@ -129,3 +129,11 @@ def test_kernel_fingerprint_ignores_comments_and_layout_only():
     assert bench.canonical_code(a) == bench.canonical_code(b)
     assert "a // b /* c */" in bench.canonical_code(a)           # string literals kept whole
     assert bench.canonical_code(a) != bench.canonical_code(a.replace("x * 2", "x * 3"))
+
+
+def test_issue_roofline_arithmetic():
+    r = bench.issue_roofline(115174472, 0.1396, 148, 1965.0)
+    assert r["peak_per_s"] == round(148 * 4 * 1965e6 / 1e9, 1)
+    assert abs(r["frac"] - 115174472 / 0.1396e-3 / (148 * 4 * 1965e6)) < 1e-4
+    assert r["warp_instructions_per_launch"] == 115174472
+    assert bench.max_sm_mhz({"sm_max_mhz": 1800.0}) > 0
