@@ -182,6 +182,21 @@ def test_e4m3_encoder_matches_torch_in_range():
     np.testing.assert_array_equal(O.e4m3_encode(x), ref)
 
 
+def test_e4m3_every_code_midpoint_and_its_neighbours():
+    # the decode table of all 127 finite non-negative codes equals torch's float8_e4m3fn values,
+    # and at every midpoint between adjacent values (a tie: to the even code) and at the FP32
+    # neighbours on either side of it the encoder agrees with torch's conversion
+    codes = torch.arange(127, dtype=torch.uint8)
+    vals = codes.view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    np.testing.assert_array_equal(np.array([O.e4m3_decode(c) for c in range(127)], np.float32), vals)
+    mids = ((vals[1:].astype(np.float64) + vals[:-1]) / 2).astype(np.float32)
+    assert np.all(mids.astype(np.float64) == (vals[1:].astype(np.float64) + vals[:-1]) / 2)  # exact
+    probe = np.concatenate([mids, np.nextafter(mids, np.float32(0)), np.nextafter(mids, np.float32(1e9)),
+                            vals]).astype(np.float32)
+    ref = torch.from_numpy(probe).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(O.e4m3_encode(probe), ref)
+
+
 def test_e4m3_saturates_and_decodes():
     assert O.e4m3_encode(np.float32([448.0, 500.0, 1e30, np.inf])).tolist() == [0x7E] * 4
     assert O.e4m3_decode(0x7E) == 448.0
