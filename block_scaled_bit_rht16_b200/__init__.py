@@ -20,7 +20,6 @@ from ._lib import (FP4Q_GRID_E1M2, FP4Q_GRID_E2M1, FP4Q_GRID_IF4, FP4Q_GRID_INT4
                    FP4Q_ROUND_SR, FP4Q_SCALE_E4M3_1x16_TENSOR, FP4Q_SCALE_FP32_1x16,
                    FP4Q_SCALE_UE8M0_1x32, Fp4qError)
 
-GRID_QMAX = {FP4Q_GRID_E2M1: 6.0, FP4Q_GRID_E1M2: 3.5, FP4Q_GRID_INT4: 7.0, FP4Q_GRID_IF4: 6.0}
 
 
 @dataclass(frozen=True)

@@ -259,7 +259,6 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantArgs a) {
 // The hot path: FP32 1x16 scale, round to nearest even, codes and scales only. FLAT: the
 // tensor is contiguous and 32-byte aligned, so unit u is the 32 bytes at 32u (one 256-bit load).
 // Each thread encodes one block per iteration while the load of its next block is in flight.
-// FLAT launches also have fewer than 2^31 units, so their block counters are 32-bit.
 template <int G, bool RHT, bool FLAT>
 __device__ __forceinline__ void lean_load(const QuantArgs& a, int64_t u, uint4& lo, uint4& hi) {
   if constexpr (FLAT) load16(a.x + u * 16, true, lo, hi);
@@ -268,6 +267,17 @@ __device__ __forceinline__ void lean_load(const QuantArgs& a, int64_t u, uint4& 
 
 template <bool FLAT> struct UnitIdx { using T = int64_t; };
 template <> struct UnitIdx<true> { using T = uint32_t; };
+
+// FLAT launches index blocks with 32-bit counters and elements as u * 16 in 32 bits, so they
+// take tensors of at most 2^28 blocks (2^32 elements); larger ones take the 64-bit path.
+constexpr int64_t kFlatMaxUnits = int64_t(1) << 28;
+static_assert(kFlatMaxUnits * 16 <= (int64_t(1) << 32), "flat element offsets fit in 32 bits");
+static_assert(kFlatMaxUnits + (int64_t(1) << 24) < (int64_t(1) << 32),
+              "flat block counters plus one grid stride fit in 32 bits");
+
+__host__ __device__ inline bool flat_launch(const QuantArgs& a) {
+  return a.contiguous && a.vec32 && a.nunits <= kFlatMaxUnits;
+}
 
 template <int G, bool RHT, bool FLAT, int R>
 __global__ void __launch_bounds__(kThreads) lean_kernel(const QuantArgs a) {
@@ -703,14 +713,14 @@ cudaError_t launch_lean_nv4(const QuantArgs& a, cudaStream_t st) {
 
 template <int G, bool GROUPED = false>
 cudaError_t launch_lean_nv(const QuantArgs& a, cudaStream_t st) {
-  const bool rht = a.c != 1.0f, flat = a.contiguous && a.vec32 && a.nunits < (int64_t(1) << 31);
+  const bool rht = a.c != 1.0f, flat = flat_launch(a);
   if (rht) return flat ? launch_lean_nv4<G, true, true, GROUPED>(a, st) : launch_lean_nv4<G, true, false, GROUPED>(a, st);
   return flat ? launch_lean_nv4<G, false, true, GROUPED>(a, st) : launch_lean_nv4<G, false, false, GROUPED>(a, st);
 }
 
 template <int G, int R>
 cudaError_t launch_lean(const QuantArgs& a, cudaStream_t st) {
-  const bool rht = a.c != 1.0f, flat = a.contiguous && a.vec32 && a.nunits < (int64_t(1) << 31);
+  const bool rht = a.c != 1.0f, flat = flat_launch(a);
   if (rht) return flat ? launch_lean3<G, true, true, R>(a, st) : launch_lean3<G, true, false, R>(a, st);
   return flat ? launch_lean3<G, false, true, R>(a, st) : launch_lean3<G, false, false, R>(a, st);
 }
@@ -791,7 +801,7 @@ cudaError_t launch_amax2(const QuantArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_amax(const QuantArgs& a, cudaStream_t st) {
-  const bool rht = a.c != 1.0f, flat = a.contiguous && a.vec32 && a.nunits < (int64_t(1) << 31);
+  const bool rht = a.c != 1.0f, flat = flat_launch(a);
   if (rht) return flat ? launch_amax2<true, true>(a, st) : launch_amax2<true, false>(a, st);
   return flat ? launch_amax2<false, true>(a, st) : launch_amax2<false, false>(a, st);
 }

@@ -34,17 +34,32 @@ def _t(s):
 def test_clock_summary_uses_timed_region_samples():
     smp = bench.ClockSampler("GPU-test")
     smp.proc = _FakeSmi(_OUT)
-    c = smp.stop(_t("2026/12/02 20:45:56.050"), _t("2026/12/02 20:45:56.250"))
+    smp.source = "nvidia-smi every 100 ms"
+    smp.finish()
+    c = smp.summary(_t("2026/12/02 20:45:56.050"), _t("2026/12/02 20:45:56.250"))
     assert c == {"sm_mhz": 1837.5, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 2,
-                 "window": "timed region"}
+                 "window": "timed region", "source": "nvidia-smi every 100 ms"}
 
 
-def test_clock_summary_falls_back_to_all_samples():
+def test_clock_summary_falls_back_to_nearby_samples_only():
     smp = bench.ClockSampler("GPU-test")
     smp.proc = _FakeSmi(_OUT)
-    c = smp.stop(_t("2026/12/02 21:00:00.000"), _t("2026/12/02 21:00:01.000"))
-    assert c["samples"] == 4 and c["window"].startswith("whole run")
-    assert c["reasons"] == ["sw_power_cap"]
+    smp.finish()
+    # a region shorter than the sampling period: the samples just around it describe it
+    c = smp.summary(_t("2026/12/02 20:45:56.101"), _t("2026/12/02 20:45:56.102"), margin_s=0.05)
+    assert c["samples"] == 1 and c["window"].startswith("within 50 ms")
+    assert c["reasons"] == ["sw_power_cap"] and c["sm_mhz"] == 1830.0
+    # nothing near the region: no clock record rather than one from another part of the run
+    assert smp.summary(_t("2026/12/02 21:00:00.000"), _t("2026/12/02 21:00:01.000")) is None
+
+
+def test_nvml_reason_bits_name_the_throttle_reasons():
+    import pynvml as N
+    assert bench.REASON_BITS["sw_power_cap"] == N.nvmlClocksEventReasonSwPowerCap
+    assert bench.REASON_BITS["hw_slowdown"] == N.nvmlClocksEventReasonHwSlowdown
+    assert bench.REASON_BITS["sw_thermal_slowdown"] == N.nvmlClocksEventReasonSwThermalSlowdown
+    assert bench.REASON_BITS["hw_thermal_slowdown"] == N.nvmlClocksEventReasonHwThermalSlowdown
+    assert bench.REASON_BITS["hw_power_brake_slowdown"] == N.nvmlClocksEventReasonHwPowerBrakeSlowdown
 
 
 def _workload_choices():
@@ -91,6 +106,25 @@ def _small_dual_workload():
     return wl
 
 
+def test_oracle_arm_configs_equal_the_library_arm_configs():
+    # the oracle arm builds its workloads with the oracle's sign-mask function (so it loads no
+    # product library); the configurations must be the ones the GPU arm times
+    import oracle as O
+    for name in _workload_choices():
+        a, b = bench.make_workload(name), bench.make_workload(name, sign_mask_from_seed=O.sign_mask_from_seed)
+        for attr in ("cfg", "rc", "cc"):
+            assert getattr(a, attr, None) == getattr(b, attr, None)
+        assert a.desc == b.desc and a.kernel_key == b.kernel_key
+
+
+def test_gated_workloads_are_bench_workloads():
+    names = set(_workload_choices())
+    assert set(bench.GATED) <= names
+    # one per format and recipe of the gated configurations
+    assert {"dy8192-dual-sr", "laplace16k-nvfp4", "laplace16k-nvint4", "laplace16k-if4",
+            "laplace16k-mxfp4", "moe-experts-ufp4", "dense32k-ufp4"} <= set(bench.GATED)
+
+
 def test_oracle_sample_counts_the_elements_it_quantizes():
     # the row quantizer: one unit is one row; a partial last chunk counts only its rows
     wl = _small_row_workload()
@@ -109,7 +143,7 @@ def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
     import json
     import types
     for make in (_small_row_workload, _small_dual_workload):
-        monkeypatch.setattr(bench, "make_workload", lambda name, make=make: make())
+        monkeypatch.setattr(bench, "make_workload", lambda name, make=make, **kw: make())
         args = types.SimpleNamespace(workload="any", steps=2, warmup=3, gpus=1)
         bench.run_reference(args)
         line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
