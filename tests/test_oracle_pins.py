@@ -593,22 +593,73 @@ def test_if4_grid_and_int_lattice_blocks():
     assert abs(7 * np.float32(6 / 7) - 6) < 1e-6
 
 
-def test_if4_pseudocode_worked_example():
-    # IF4 page 3.1.1: scale = max|v|/6; int = round(v * 7/6 / scale); deq = int * scale * 6/7
-    v = np.array([6.0, 3.0, -1.2, 0.4] + [0.0] * 12, np.float32)
-    scale = np.abs(v).max() / 6
-    ints = np.rint(v * (7 / 6) / scale)
-    assert ints[:4].tolist() == [7, 4, -1, 0]
-    want = ints * scale * (6 / 7)
-    coeffs = {r[0]: eval(r[1]) for r in _golden_lines("if4_coefficients.txt")}
-    assert coeffs["FP4xINT4"] == pytest.approx(6 / 7) and coeffs["INT4xINT4"] == pytest.approx(36 / 49)
-    assert coeffs["INT4xINT4"] == pytest.approx(coeffs["FP4xINT4"] ** 2)
-    # the oracle's INT4 candidate on the same block (scale 1 via the E4M3 path: alpha * 448 * 6 = 6)
+def _if4_exact_int(y, s):
+    """The IF4 page's INT4 candidate (section 3.1.1) in exact arithmetic: the value times 7/6
+    over the block scale, rounded to the nearest integer (halves to even), limited to +-7."""
+    from fractions import Fraction
+    k = round(Fraction(float(y)) * 7 / (6 * Fraction(float(s))))
+    return max(-7, min(7, k))
+
+
+def _int4_nibbles(codes, n):
+    nib = _nib(codes).reshape(-1)[:n].astype(np.int64)
+    return np.where(nib >= 8, nib - 16, nib)
+
+
+def test_if4_worked_example_int4_block():
+    # IF4 page, section 3.1.1: an INT4 block multiplies its values by 7/6 before rounding to
+    # integers and dequantizes integer * scale * 6/7; section 3.2: the block keeps INT4 when its
+    # error is the smaller one, flagged in the scale byte's top bit.
+    # The block: 6, 3, -1.2, 0.4 (INT4 7, 4, -1, 0; 3 * 7/6 = 3.5 is a tie that goes to the even
+    # 4) and twelve values near k * 6/7, which E2M1 represents poorly and INT4 * 6/7 well.
+    head = [6.0, 3.0, -1.2, 0.4]
+    tail = [k * 6 / 7 * sg for k, sg in zip([6, 3, 5, 2, 1, 4] * 2, [1, -1] * 6)]
+    x = synth.to_bf16_bits(np.array([head + tail], np.float32))
+    y = synth.bf16_bits_to_f32(x)[0]
+    # tensor scale 2^-8 and block amax 6: Delta = 6 / (2^-8 * 6) = 256, an E4M3 value, so the
+    # block scale is s = 256 * 2^-8 = 1 exactly
     cfg = O.OracleConfig(grid=O.GRID_IF4, scale=O.SCALE_E4M3_1x16, rht=0)
-    r = O.quantize(cfg, synth.to_bf16_bits(v[None]), tensor_scale=np.float32(1 / 448), dequant=True)
-    if r["scales"][0, 0] >> 7:
-        got = synth.bf16_bits_to_f32(r["dequant"][0])
-        np.testing.assert_allclose(got[:4], want[:4], rtol=2 ** -7)
+    r = O.quantize(cfg, x, tensor_scale=np.float32(2.0 ** -8), dequant=True)
+    sbyte = int(r["scales"][0, 0])
+    assert sbyte >> 7 == 1, "the block must take INT4"
+    assert O.e4m3_decode(sbyte & 0x7F) == 256.0
+    k = _int4_nibbles(r["codes"], 16)
+    assert k[:4].tolist() == [7, 4, -1, 0]
+    assert k.tolist() == [_if4_exact_int(v, 1.0) for v in y]
+    # dequantized: integer * scale * 6/7 (bf16 output; the FP32 products differ from the exact
+    # ones by an ulp at most)
+    got = synth.bf16_bits_to_f32(r["dequant"][0]).astype(np.float64)
+    np.testing.assert_allclose(got, k * 6 / 7, rtol=2.0 ** -8, atol=0)
+    # the printed coefficient table: FP4 x INT4 blocks carry 6/7, INT4 x INT4 blocks (6/7)^2
+    coeffs = {row[0]: eval(row[1]) for row in _golden_lines("if4_coefficients.txt")}
+    assert coeffs["FP4xINT4"] == pytest.approx(6 / 7) and coeffs["INT4xINT4"] == pytest.approx(36 / 49)
+
+
+def test_if4_int_candidate_follows_the_page_rule_up_to_rounding():
+    # every INT4 block the oracle emits has the codes of the page's rule round(y * 7/6 / s) in
+    # exact arithmetic, except for values within FP32 rounding of a half-integer, where the
+    # order of the two FP32 operations decides (the oracle scales y by s first, then by 7/6)
+    from fractions import Fraction
+    x = synth.small(91, 128, 256, "laplace")
+    cfg = O.OracleConfig(grid=O.GRID_IF4, scale=O.SCALE_E4M3_1x16, rht=0)
+    r = O.quantize(cfg, x)
+    alpha = np.float32(r["tensor_scale"])
+    e4 = np.array([O.e4m3_decode(b) for b in range(128)], np.float32)
+    s = (e4[r["scales"] & 0x7F] * alpha).astype(np.float32)      # FP32 block scales
+    yb = synth.bf16_bits_to_f32(x).reshape(128, 16, 16)
+    flag = (r["scales"] >> 7).astype(bool)
+    kk = _int4_nibbles(r["codes"], x.size).reshape(128, 16, 16)
+    checked = near = 0
+    for i, j in zip(*np.nonzero(flag)):
+        for e in range(16):
+            t = Fraction(float(yb[i, j, e])) * 7 / (6 * Fraction(float(s[i, j])))
+            frac = abs(t) - math.floor(abs(t))
+            if abs(frac - Fraction(1, 2)) < Fraction(1, 2 ** 20) and abs(t) < 7:
+                near += 1
+                continue
+            assert kk[i, j, e] == _if4_exact_int(yb[i, j, e], s[i, j])
+            checked += 1
+    assert checked > 10000 and near <= checked // 1000
 
 
 # ------------------------------------------------------------------ statistics
