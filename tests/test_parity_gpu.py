@@ -14,7 +14,7 @@ import torch
 import oracle as O
 import block_scaled_bit_rht16_b200 as fq
 from block_scaled_bit_rht16_b200 import synth, _lib
-from helpers import bf16_bits, host, ocfg, to_dev
+from helpers import Canaries, bf16_bits, guarded_dual, guarded_quantized, host, ocfg, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -36,12 +36,15 @@ def _cid(c):
 
 
 def gpu_quantize(cfg, x_bits, ld=None, tensor_scale=None):
+    """The library's row quantizer on x_bits, every output (codes, scales, tensor scale,
+    dequant, workspace) between guard bands that must come back untouched."""
     x = to_dev(x_bits, ld)
-    ts = None
+    guard = Canaries()
+    out = guarded_quantized(cfg, x.shape[0], x.shape[1], guard)
     if tensor_scale is not None:
-        ts = torch.tensor([tensor_scale], dtype=torch.float32, device="cuda")
-    out = fq.rht_quantize(cfg, x, tensor_scale=ts, tensor_scale_given=tensor_scale is not None)
-    torch.cuda.synchronize()
+        out.tensor_scale.fill_(float(tensor_scale))
+    out = fq.rht_quantize(cfg, x, out=out, tensor_scale_given=tensor_scale is not None)
+    guard.check()
     return out
 
 
@@ -147,8 +150,9 @@ def test_input_only_16_byte_aligned(grid):
     t = to_dev(big)[:, 8:]
     assert t.data_ptr() % 32 == 16
     cfg = fq.Config(grid=grid, sign_mask=0x0F0F)
-    out = fq.rht_quantize(cfg, t)
-    torch.cuda.synchronize()
+    guard = Canaries()
+    out = fq.rht_quantize(cfg, t, out=guarded_quantized(cfg, 33, 256, guard))
+    guard.check()
     compare_quant(cfg, x, out)
 
 
@@ -254,8 +258,9 @@ def test_dual_matches_row_and_transposed_oracle(grid, rounds, rhts):
         rc = fq.Config(grid=grid, round=rounds[0], rht=rhts[0], sign_mask=0x3C5A, sr_seed=0x5A5A0003)
         cc = fq.Config(grid=grid, round=rounds[1], rht=rhts[1], sign_mask=0xA5C3, sr_seed=0x5A5A0003,
                        sr_stream=1)
-        out = fq.quantize_dual(rc, cc, to_dev(dy, ld))
-        torch.cuda.synchronize()
+        guard = Canaries()
+        out = fq.quantize_dual(rc, cc, to_dev(dy, ld), out=guarded_dual(M, N, guard))
+        guard.check()
         r = O.quantize(ocfg(rc), dy)
         c = O.quantize(ocfg(cc), np.ascontiguousarray(dy.T))
         np.testing.assert_array_equal(host(out.codes_row), r["codes"])
@@ -272,8 +277,9 @@ def test_dual_edge_blocks():
     dy[40:72, :13] = e.T
     rc = fq.Config(round=SR, sign_mask=0x0FF0, sr_seed=9)
     cc = fq.Config(round=SR, sign_mask=0x0FF0, sr_seed=9, sr_stream=1)
-    out = fq.quantize_dual(rc, cc, to_dev(dy))
-    torch.cuda.synchronize()
+    guard = Canaries()
+    out = fq.quantize_dual(rc, cc, to_dev(dy), out=guarded_dual(208, 64, guard))
+    guard.check()
     np.testing.assert_array_equal(host(out.codes_row), O.quantize(ocfg(rc), dy)["codes"])
     np.testing.assert_array_equal(host(out.codes_col), O.quantize(ocfg(cc), np.ascontiguousarray(dy.T))["codes"])
 
@@ -289,8 +295,10 @@ def test_dequantize(combo, inverse):
     cfg = fq.Config(grid=grid, scale=scale, round=rnd, sign_mask=0x2468, sr_seed=1)
     x = synth.small(17, 75, 320, "laplace")
     q = gpu_quantize(cfg, x)
-    d = fq.dequantize(cfg, q.codes, q.scales, q.tensor_scale, inverse_rht=inverse)
-    torch.cuda.synchronize()
+    guard = Canaries()
+    d = fq.dequantize(cfg, q.codes, q.scales, q.tensor_scale, inverse_rht=inverse,
+                      out=guard.empty((75, 320), torch.bfloat16))
+    guard.check()
     ts = float(host(q.tensor_scale)[0]) if scale == E4M3 else 0.0
     ref = O.dequantize(ocfg(cfg), host(q.codes), host(q.scales), ts, 75, 320, inverse_rht=inverse)
     np.testing.assert_array_equal(bf16_bits(d), ref)
@@ -299,8 +307,10 @@ def test_dequantize(combo, inverse):
 def test_rotation_alone():
     x = synth.small(3, 129, 2048, "t4")
     for fp32 in (True, False):
-        y = fq.rht16(to_dev(x, 2048 + 64), 0x7E57, out_fp32=fp32)
-        torch.cuda.synchronize()
+        guard = Canaries()
+        y = fq.rht16(to_dev(x, 2048 + 64), 0x7E57, out_fp32=fp32,
+                     out=guard.empty((129, 2048), torch.float32 if fp32 else torch.bfloat16))
+        guard.check()
         yf, yb = O.rht16_rows(x, 0x7E57)
         if fp32:
             np.testing.assert_array_equal(host(y).view(np.uint32), yf.view(np.uint32))
