@@ -127,7 +127,8 @@ typedef struct {
   double sum_err2;          /* sum (y - xhat)^2 */
   double sum_y_xhat;        /* sum y * xhat */
   double n;                 /* elements */
-  double cell_count[8];     /* elements per magnitude code (FP grids: code & 7; INT4: |k|) */
+  double cell_count[8];     /* elements per magnitude code (FP grids: code & 7; INT4: |k|; IF4:
+                               the chosen representation's, so FP4 and INT4 blocks share cells) */
   double cell_err[8];       /* sum (|q| - |v|) per magnitude code, in scaled (v) units */
   double if4_fp4_blocks;    /* IF4 blocks that kept FP4 */
   double blocks;            /* scale blocks */
@@ -177,8 +178,9 @@ fp4q_status fp4q_rht_quantize(const fp4q_config* cfg, const void* x, int64_t row
  *  codes_col  uint8 [N, M/2], scales_col float [N, M/16]: blocks along M, i.e. dy^T
  *             quantized along its rows (col_cfg; SR index n * M + m).
  * Both configs must use FP4Q_SCALE_FP32_1x16 and no dequant/stats outputs; M and N must be
- * multiples of 16 and M at most 65535 * 128 = 8388480 (else FP4Q_ERR_SHAPE; quantize taller dY
- * in row slices). workspace may be NULL. */
+ * multiples of 16 and at most 2^31 - 128 (else FP4Q_ERR_SHAPE). workspace may be NULL. The first
+ * call on a device, and the first with each configuration, looks up cached launch parameters;
+ * make it outside any stream capture. */
 fp4q_status fp4q_quantize_dual(const fp4q_config* row_cfg, const fp4q_config* col_cfg,
                                const void* dy, int64_t M, int64_t N, int64_t ld,
                                uint8_t* codes_row, void* scales_row, uint8_t* codes_col,
