@@ -836,6 +836,7 @@ def measure_e2e(wl, stream, world, steps=30):
 def measure_ratios(args, stream, dev, l2, fused_step_ms):
     """Time relative to quantize-only (rotation off), as the UFP4 pages report it: fused and
     unfused (rotation pass to bf16, then quantize-only), kernel time per step."""
+    import torch
     out = {}
     per = {}
     for name in ("linear1.5b-ufp4-quant-only", "linear1.5b-ufp4-unfused"):

@@ -73,9 +73,9 @@ int block_elems(const fp4q_config* cfg) { return cfg->scale == FP4Q_SCALE_UE8M0_
 
 size_t stats_bytes() { return (size_t)kStatsCtas * ST_LEN * sizeof(double); }
 
-// Largest M of fp4q_quantize_dual: its kernel puts the 128-row tiles of dY on the grid's y axis,
-// which holds at most 65535 blocks.
-constexpr int64_t kDualMaxRows = 65535ll * 128;
+// Largest M and N of fp4q_quantize_dual: its tile copies address dY with 32-bit signed
+// coordinates, and a tile reaches 128 rows / 64 columns past its start.
+constexpr int64_t kDualMaxDim = (int64_t(1) << 31) - 128;
 
 fp4q_status check_shape(int64_t rows, int64_t cols, int64_t ld, int unit) {
   if (rows < 0 || cols < 0) return FP4Q_ERR_SHAPE;
@@ -101,6 +101,7 @@ QuantArgs base_args(const fp4q_config* cfg, const void* x, int64_t rows, int64_t
   a.codes = codes;
   a.scales = scales;
   sign_words(cfg->sign_mask, cfg->rht != 0, a.sw);
+  sign_flips(a.sw, a.flip_lo, a.flip_hi);
   a.c = cfg->rht ? 4.0f : 1.0f;
   a.cinv = cfg->rht ? 0.25f : 1.0f;
   a.seedx = cfg->sr_seed ^ ((uint64_t)(cfg->sr_stream & 1u) << 63);
@@ -269,6 +270,8 @@ fp4q_status fp4q_tensor_scale(const fp4q_config* cfg, const void* x, int64_t row
     a.nunits = rows * a.units_per_row;
     a.ws = ws;
     sign_words(cfg->sign_mask, cfg->rht != 0, a.sw);
+    sign_flips(a.sw, a.flip_lo, a.flip_hi);
+  sign_flips(a.sw, a.flip_lo, a.flip_hi);
     a.c = cfg->rht ? 4.0f : 1.0f;
     a.cinv = cfg->rht ? 0.25f : 1.0f;
     a.contiguous = (ld == cols) ? 1 : 0;
@@ -309,7 +312,7 @@ fp4q_status fp4q_quantize_dual(const fp4q_config* row_cfg, const fp4q_config* co
   if (row_cfg->grid != col_cfg->grid) return FP4Q_ERR_UNSUPPORTED;
   if (row_cfg->e2m1_max != 0u || col_cfg->e2m1_max != 0u) return FP4Q_ERR_UNSUPPORTED;
   if (M < 0 || N < 0 || M % 16 != 0 || N % 16 != 0) return FP4Q_ERR_SHAPE;
-  if (M > kDualMaxRows) return FP4Q_ERR_SHAPE;   // 128-row tiles on the grid's y axis
+  if (M > kDualMaxDim || N > kDualMaxDim) return FP4Q_ERR_SHAPE;   // 32-bit tile coordinates
   if (M > 0 && N > 0 && ld < N) return FP4Q_ERR_SHAPE;
   if (M > 1 && N > 0 && ld % 8 != 0) return FP4Q_ERR_ALIGN;
   const bool empty = M == 0 || N == 0;
@@ -329,9 +332,11 @@ fp4q_status fp4q_quantize_dual(const fp4q_config* row_cfg, const fp4q_config* co
   a.scales_row = static_cast<float*>(scales_row);
   a.codes_col = codes_col;
   a.scales_col = static_cast<float*>(scales_col);
-  sign_words(row_cfg->sign_mask, row_cfg->rht != 0, a.sw_row);
+  uint32_t sw_row[8];
+  sign_words(row_cfg->sign_mask, row_cfg->rht != 0, sw_row);
+  sign_flips(sw_row, a.flip_lo_row, a.flip_hi_row);
   for (int i = 0; i < 16; ++i)
-    a.sc_col[i] = (col_cfg->rht != 0 && ((col_cfg->sign_mask >> i) & 1u)) ? 0x80008000u : 0u;
+    a.flip_col[i] = (col_cfg->rht != 0 && ((col_cfg->sign_mask >> i) & 1u)) ? 0x80000000u : 0u;
   a.vec32 = ((reinterpret_cast<uintptr_t>(dy) & 31u) == 0 && ld % 16 == 0) ? 1 : 0;
   a.col16 = (M % 64 == 0 && aligned(codes_col, 16) && aligned(scales_col, 16)) ? 1 : 0;
   a.c_row = row_cfg->rht ? 4.0f : 1.0f;
@@ -435,6 +440,14 @@ fp4q_status fp4q_check_division(uint64_t seed, uint64_t n, unsigned long long* m
 fp4q_status fp4q_device_status(int32_t* status_bits, int32_t clear, fp4q_stream_t stream) {
   if (status_bits == nullptr || (clear != 0 && clear != 1)) return FP4Q_ERR_INVALID_ARG;
   return cuda_status(read_device_status(status_bits, clear != 0, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fp4q_status fp4q_check_conversions(unsigned long long* mismatches, fp4q_stream_t stream) {
+  if (mismatches == nullptr) return FP4Q_ERR_INVALID_ARG;
+  if (!aligned(mismatches, 8)) return FP4Q_ERR_ALIGN;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(mismatches, 0, 5 * sizeof(unsigned long long), s) != cudaSuccess) return FP4Q_ERR_CUDA;
+  return cuda_status(launch_conversion_check(mismatches, s));
 }
 
 fp4q_status fp4q_check_wait_timeout(uint64_t limit_ns, fp4q_stream_t stream) {

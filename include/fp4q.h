@@ -282,6 +282,20 @@ fp4q_status fp4q_rht16(const void* x, int64_t rows, int64_t cols, int64_t ld, ui
 fp4q_status fp4q_check_division(uint64_t seed, uint64_t n, unsigned long long* mismatches,
                                 fp4q_stream_t stream);
 
+/* Diagnostic: checks the hardware conversions the encoders use, each against a rule written from
+ * the format's definition (exponent field, grid step, round half to even, saturation), over every
+ * FP32 input in the range the kernels feed it, and writes the number of inputs whose result
+ * differs in any bit to the device counters mismatches[0..4] (zeroed first; 8-byte aligned):
+ *  [0] E2M1 encode (round to nearest even, saturating at 6, sign of zero kept), every non-NaN
+ *      float ["当你的 GPU 学不会算账", section "E2M1：一块刻度不均的尺子"]
+ *  [1] E1M2 encode as the kernels form it (quarters of the scaled value through the FP6 E2M3
+ *      conversion), every float of magnitude below 15/16 ["UFP4：换一把尺子"]
+ *  [2] E4M3 encode of a block-scale quotient (round to nearest even, 448 and above -> 448), every
+ *      float >= 0 including +inf ["低精度量化技术：IF4…", section 3.2]
+ *  [3] the E2M1 decoder on all 256 bytes and the E4M3 decoder on codes 0..0x7E
+ *  [4] bf16 rounding of dequantized values (round to nearest even), every non-NaN float */
+fp4q_status fp4q_check_conversions(unsigned long long* mismatches, fp4q_stream_t stream);
+
 /* Device status word of the library on the current device: bit 0 is reserved for a bounded
  * wait inside a quantize kernel that gives up (that launch's outputs would be incomplete); the
  * current kernels read their inputs with plain loads and never wait, so it stays clear. Bit 1 is

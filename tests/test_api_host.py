@@ -139,7 +139,8 @@ def test_dual_dequant_rht_stats_validation():
         ctypes.byref(rc), ctypes.byref(cc), dy, M, N, ld, cr, FAKE, FAKE, FAKE, None, 0, None)
     assert dual(M=24) == _lib.FP4Q_ERR_SHAPE
     assert dual(N=40, ld=40) == _lib.FP4Q_ERR_SHAPE
-    assert dual(M=65535 * 128 + 16) == _lib.FP4Q_ERR_SHAPE      # beyond the tile grid's y limit
+    assert dual(M=2 ** 31) == _lib.FP4Q_ERR_SHAPE              # beyond 32-bit tile coordinates
+    assert dual(N=2 ** 31, ld=2 ** 31) == _lib.FP4Q_ERR_SHAPE
     assert dual(dy=None) == _lib.FP4Q_ERR_INVALID_ARG
     assert dual(cr=FAKE + 4) == _lib.FP4Q_ERR_ALIGN
     e2 = fq.Config(grid=fq.FP4Q_GRID_E2M1).c()

@@ -247,6 +247,18 @@ def test_division_step_matches_ieee_division():
         assert int(bad.item()) == 0
 
 
+def test_hardware_conversions_match_their_format_rules():
+    # E2M1, E1M2 (through the FP6 converter), E4M3 encode, both decoders and bf16 packing, each
+    # over every FP32 input the kernels can feed it, against rules written from the formats
+    lib = _lib.load()
+    bad = torch.zeros(5, dtype=torch.int64, device="cuda")
+    import ctypes
+    assert lib.fp4q_check_conversions(ctypes.c_void_p(bad.data_ptr()),
+                                      ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)) == 0
+    torch.cuda.synchronize()
+    assert bad.cpu().tolist() == [0, 0, 0, 0, 0]
+
+
 # ------------------------------------------------------------------ dual orientation
 
 @pytest.mark.parametrize("grid", [E1M2, E2M1, INT4])
