@@ -21,26 +21,32 @@ namespace fp4q {
 
 // ------------------------------------------------------------------ bf16 / packed helpers
 
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 // a - b as fma(b, -1, a): one rounding of the exact difference, like a plain subtraction.
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
   return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
 }
 
-// Load-side: eight 32-bit words (bf16 pairs) -> P[8], with the sign diagonal applied by
-// flipping the bf16 sign bits (exact). sw[k] holds the flips of elements 2k (bit 15) and
-// 2k+1 (bit 31).
-__device__ __forceinline__ void unpack16(const uint4& lo, const uint4& hi, const uint32_t* sw,
-                                         float2* P) {
-  const uint32_t w[8] = {lo.x ^ sw[0], lo.y ^ sw[1], lo.z ^ sw[2], lo.w ^ sw[3],
-                         hi.x ^ sw[4], hi.y ^ sw[5], hi.z ^ sw[6], hi.w ^ sw[7]};
+// The two bf16 halves of a 32-bit word as floats, each negated when its flip (0 or 0x80000000) is
+// set: the low half as w * 2^16 + flip (one integer multiply-add; adding 2^31 toggles the sign
+// bit), the high half as (w & 0xFFFF0000) ^ flip (one three-input logic operation). Plain
+// expressions, so that flips held in the kernel's parameters stay constant operands.
+__device__ __forceinline__ float bf_lo_flip(uint32_t w, uint32_t flip) {
+  return __uint_as_float(w * 65536u + flip);
+}
+__device__ __forceinline__ float bf_hi_flip(uint32_t w, uint32_t flip) {
+  return __uint_as_float((w & 0xFFFF0000u) ^ flip);
+}
+
+// Load-side: eight 32-bit words (bf16 pairs) -> P[8], with the sign diagonal applied on the way
+// (exact). flip_lo[k] / flip_hi[k] negate elements 2k / 2k+1 (bit 31).
+__device__ __forceinline__ void unpack16(const uint4& lo, const uint4& hi, const uint32_t* flip_lo,
+                                         const uint32_t* flip_hi, float2* P) {
+  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    P[2 * k] = make_float2(bf_lo(w[k]), bf_lo(w[k + 4]));
-    P[2 * k + 1] = make_float2(bf_hi(w[k]), bf_hi(w[k + 4]));
+    P[2 * k] = make_float2(bf_lo_flip(w[k], flip_lo[k]), bf_lo_flip(w[k + 4], flip_lo[k + 4]));
+    P[2 * k + 1] = make_float2(bf_hi_flip(w[k], flip_hi[k]), bf_hi_flip(w[k + 4], flip_hi[k + 4]));
   }
 }
 
@@ -296,22 +302,34 @@ constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;
 
 __device__ __forceinline__ uint64_t splitmix64(uint64_t x) { return splitmix64_mix(x + kGamma); }
 
-// 16-bit draws u[e] for the sixteen consecutive elements whose first has logical index
-// 4 * quad0 (a multiple of 4): element 4j + l takes bits 16l .. 16l+15 of output quad0 + j of
-// the SplitMix64 stream seeded with seedx = seed ^ (stream << 63), whose state for output k is
-// seedx + (k + 1) * gamma.
-__device__ __forceinline__ void sr_draws16(uint64_t seedx, uint64_t quad0, uint32_t* u) {
+// The SplitMix64 outputs that hold the draws of the sixteen consecutive elements whose first has
+// logical index 4 * quad0 (a multiple of 4), as eight 32-bit words: element 4j + l takes bits
+// 16l .. 16l+15 of output quad0 + j of the stream seeded with seedx = seed ^ (stream << 63), whose
+// state for output k is seedx + (k + 1) * gamma -- i.e. element e's draw is the low (e even) or
+// high (e odd) half of word e >> 1.
+__device__ __forceinline__ void sr_words16(uint64_t seedx, uint64_t quad0, uint32_t* d) {
   uint64_t state = seedx + (quad0 + 1u) * kGamma;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint64_t h = splitmix64_mix(state);
     state += kGamma;
-    const uint32_t lo = (uint32_t)h, hi = (uint32_t)(h >> 32);
-    u[4 * j] = lo & 0xFFFFu;
-    u[4 * j + 1] = lo >> 16;
-    u[4 * j + 2] = hi & 0xFFFFu;
-    u[4 * j + 3] = hi >> 16;
+    d[2 * j] = (uint32_t)h;
+    d[2 * j + 1] = (uint32_t)(h >> 32);
   }
+}
+
+// The same draws as sixteen 16-bit values u[e].
+__device__ __forceinline__ void sr_draws16(uint64_t seedx, uint64_t quad0, uint32_t* u) {
+  uint32_t d[8];
+  sr_words16(seedx, quad0, d);
+#pragma unroll
+  for (int e = 0; e < 16; ++e) u[e] = (e & 1) ? (d[e >> 1] >> 16) : (d[e >> 1] & 0xFFFFu);
+}
+
+// 1 + u * 2^-23 for element e's draw u (the draw in the low mantissa bits): one byte permute
+// of the word that holds it.
+__device__ __forceinline__ float sr_one_plus(const uint32_t* d, int e) {
+  return __uint_as_float(__byte_perm(d[e >> 1], 0x3F800000u, (e & 1) ? 0x7632 : 0x7610));
 }
 
 // Round-up decision r < frac with r = u * 2^-16, taken exactly as u < frac * 2^16 (both sides

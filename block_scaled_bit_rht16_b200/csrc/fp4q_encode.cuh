@@ -107,6 +107,21 @@ __device__ __forceinline__ uint32_t pack_low_nibbles(const uint32_t* t) {
   return w;
 }
 
+// E1M2 codes of eight values given as quarters (e_k = v_k / 4, |e_k| <= 7/8), element k in
+// nibble k: the FP6 E2M3 conversion of e, whose subnormal range below 1 has the uniform step 1/8,
+// so each code byte is 00s00mmm with mmm = RNE(8 |e|) = RNE(2 |v|) (ties to even, the sign of
+// zero kept). Even elements' bytes are converted into one word and odd elements' into another;
+// each byte's sign moves to bit 3 (one shift and one three-input logic operation per word, bits
+// 4..7 don't-care), and the two words interleave as low and high nibbles.
+// fp4q_check_conversions runs it over every input in that range.
+__device__ __forceinline__ uint32_t e1m2_word(const float* e) {
+  const uint32_t E = cvt_e2m3x2(e[2], e[0]) | (cvt_e2m3x2(e[6], e[4]) << 16);   // e0 e2 e4 e6
+  const uint32_t O = cvt_e2m3x2(e[3], e[1]) | (cvt_e2m3x2(e[7], e[5]) << 16);   // e1 e3 e5 e7
+  const uint32_t NE = (E & 0x07070707u) | ((E >> 2) & 0xF8F8F8F8u);
+  const uint32_t NO = (O & 0x07070707u) | ((O >> 2) & 0xF8F8F8F8u);
+  return (NE & 0x0F0F0F0Fu) | ((NO << 4) & 0xF0F0F0F0u);
+}
+
 // Codes of one block on E1M2 / INT4 / E2M1 from the (rotated) raw values P, y = P / c with
 // c = 4 under rotation and 1 without, and the block scale s. Returns the two code words.
 //
@@ -115,14 +130,17 @@ __device__ __forceinline__ uint32_t pack_low_nibbles(const uint32_t* t) {
 // i.e. in an all-zero block, which encodes as zeros anyway; without rotation the sign is copied
 // from P explicitly.
 //   E2M1: hardware round-to-nearest-even conversion of v (saturating at 6).
-//   E1M2: the FP6 E2M3 conversion of v/4: |v/4| <= 7/8 lies in E2M3's subnormal range, whose
-//         step 1/8 makes the code sign << 5 | RNE(2|v|) -- the E1M2 magnitude -- with ties to
-//         even and the sign of zero kept; a SIMD step moves the sign to bit 3 and pairs nibbles.
+//   E1M2: the FP6 E2M3 conversion of v/4 (e1m2_word): |v/4| <= 7/8 lies in E2M3's subnormal
+//         range, whose step 1/8 makes the code sign << 5 | RNE(2|v|) -- the E1M2 magnitude --
+//         with ties to even and the sign of zero kept.
 //   INT4: t = 1.5 * 2^23 + v rounds v half-to-even into t's low bits in two's complement.
 // CLAMP: saturate |v| at qmax before rounding. The FP32 scale needs none (|v| <= qmax up to an
 // ulp); E4M3 scales do (the rounded block scale, or a given tensor scale, can leave |v| > qmax).
+// amax_raw (CLAMP only): max |P|. Its quotient bounds every element's (the quotient is
+// monotonic in the numerator), so a block whose largest quotient stays below qmax + step/2
+// rounds no element above qmax, and the clamp, which could not change a code, is skipped.
 template <int G, bool RHT, bool CLAMP = false>
-__device__ __forceinline__ uint2 encode_lean(const float2* P, float s) {
+__device__ __forceinline__ uint2 encode_lean(const float2* P, float s, float amax_raw = 0.0f) {
   if (s == 0.0f) return make_uint2(0u, 0u);
   constexpr float qmax = GridInfo<G>::qmax;
   constexpr float kC = RHT ? 4.0f : 1.0f;
@@ -134,9 +152,12 @@ __device__ __forceinline__ uint2 encode_lean(const float2* P, float s) {
     for (int i = 0; i < 8; ++i) Q[i] = div2(dv, P[i]);
     if constexpr (CLAMP && !kIsE2M1<G>) {   // the E2M1 conversion saturates by itself
       constexpr float lim = qmax / kVScale;
+      constexpr float half_above = (G == kE1M2 ? 3.75f : 7.5f) / kVScale;   // qmax + step / 2
+      if (!(div2(dv, make_float2(amax_raw, amax_raw)).x < half_above)) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        Q[i] = make_float2(fminf(fmaxf(Q[i].x, -lim), lim), fminf(fmaxf(Q[i].y, -lim), lim));
+        for (int i = 0; i < 8; ++i)
+          Q[i] = make_float2(fminf(fmaxf(Q[i].x, -lim), lim), fminf(fmaxf(Q[i].y, -lim), lim));
+      }
     }
   } else {
     // scale outside the exact range of the correction step (tiny or huge data): IEEE division,
@@ -169,19 +190,10 @@ __device__ __forceinline__ uint2 encode_lean(const float2* P, float s) {
   } else if constexpr (G == kE1M2) {
 #pragma unroll
     for (int l = 0; l < 2; ++l) {
-      uint32_t x[2];
+      float e[8];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {   // elements 4h .. 4h+3 of this word
-        const int j = 2 * h;
-        const float e0 = l ? Q[2 * j].y : Q[2 * j].x, e1 = l ? Q[2 * j + 1].y : Q[2 * j + 1].x;
-        const float e2 = l ? Q[2 * j + 2].y : Q[2 * j + 2].x, e3 = l ? Q[2 * j + 3].y : Q[2 * j + 3].x;
-        const uint32_t W = cvt_e2m3x2(e1, e0) | (cvt_e2m3x2(e3, e2) << 16);   // byte k = code k
-        // byte k of W is 00s00mmm (v/4 is an E2M3 subnormal): N's low nibbles s mmm (bits 4..7
-        // of each byte are don't-care), then X's bytes 0 and 2 pair nibbles 0|1 and 2|3
-        const uint32_t N = (W & 0x07070707u) | ((W >> 2) & 0xF8F8F8F8u);
-        x[h] = (N & 0x0F0F0F0Fu) | ((N >> 4) & 0xF0F0F0F0u);
-      }
-      w[l] = __byte_perm(x[0], x[1], 0x6420);
+      for (int k = 0; k < 8; ++k) e[k] = l ? Q[k].y : Q[k].x;
+      w[l] = e1m2_word(e);
     }
   } else {
     const float2 c2 = make_float2(12582912.0f, 12582912.0f);   // 1.5 * 2^23
@@ -245,9 +257,10 @@ __device__ __forceinline__ void sr_quotients(const float2* P, float s, float c, 
   }
 }
 
-// Codes of a nonzero block from its quotients q, draws u and raw values P (for the signs).
+// Codes of a nonzero block from its quotients q, draw words d (sr_words16) and raw values P (for
+// the signs).
 template <int G>
-__device__ __forceinline__ uint2 sr_codes(const float* q, const uint32_t* u, const float2* P) {
+__device__ __forceinline__ uint2 sr_codes(const float* q, const uint32_t* d, const float2* P) {
   constexpr float qmax = GridInfo<G>::qmax;
   // sum over j = 0..7 of 0x4B400000 * 16^j, modulo 2^32
   constexpr uint32_t kBias = 0x4B400000u + (0x4B400000u << 4) + (0x4B400000u << 8) +
@@ -263,19 +276,19 @@ __device__ __forceinline__ uint2 sr_codes(const float* q, const uint32_t* u, con
       float K;
       if constexpr (kIsE2M1<G>) {
         const float a = fminf(fabsf(q[e]), qmax);
-        const float r = __fadd_rn(__uint_as_float(u[e] * 128u + 0x3F800000u), -1.0f);   // exact
+        const float r = __fmaf_rn(sr_one_plus(d, e), 128.0f, -128.0f);   // u * 2^-16, exact
         const bool lo = a < 2.0f, mid = a < 4.0f;
         const float inv_step = lo ? 2.0f : (mid ? 1.0f : 0.5f);
         const float base = lo ? 12582912.0f : (mid ? 12582914.0f : 12582916.0f);
         K = __fadd_ru(__fmaf_ru(a, inv_step, -r), base);
       } else {
         // uniform grids, t = |v| / step with qmax = 7 steps: F = 1 + u * 2^-23 (the draw in the
-        // low mantissa bits, one byte permute), c = 16.125 - 16 F = (1 - r) / 8 exactly;
+        // low mantissa bits, one byte permute of its word), c = 16.125 - 16 F = (1 - r) / 8 exactly;
         // w = min(RU((t - r + 1) / 8), 1) (the saturation is the clamp at qmax: t' = min(t, 7));
         // 8w = RU(t' - r + 1), whose ceiling is ceil(t' - r) + 1 (no integer up to 8 lies
         // between a real and its upward rounding), so K = RU(8w + 1.5 * 2^23 - 1) is
         // 1.5 * 2^23 + ceil(t' - r).
-        const float F = __uint_as_float(__byte_perm(u[e], 0x3F800000u, 0x7610));
+        const float F = sr_one_plus(d, e);
         const float c = __fmaf_rn(F, -16.0f, 16.125f);
         constexpr float inv8step = (G == kE1M2) ? 0.25f : 0.125f;
         float w;
@@ -306,9 +319,9 @@ __device__ __forceinline__ uint2 encode_sr(const float2* P, float s, float c, ui
   if (s == 0.0f) return make_uint2(0u, 0u);
   float q[16];
   sr_quotients(P, s, c, q);
-  uint32_t u[16];
-  sr_draws16(seedx, quad0, u);
-  return sr_codes<G>(q, u, P);
+  uint32_t d[8];
+  sr_words16(seedx, quad0, d);
+  return sr_codes<G>(q, d, P);
 }
 
 // IF4 block, E4M3 block scale (NVFP4's), codes only: the E2M1 candidate (round to nearest even,
@@ -318,6 +331,8 @@ __device__ __forceinline__ uint2 encode_sr(const float2* P, float s, float c, ui
 // The errors RN(value - v) are formed on magnitudes: a nonzero candidate has the sign of v and
 // RN is symmetric, so each square equals the signed one. Returns the code words; flag = 0x80 for
 // an INT4 block.
+// When even the largest |q| times RN(7/6) stays below 7.5, no INT4 candidate needs the clamp at
+// +-7 (it could not change a code) and it is skipped.
 template <bool RHT>
 __device__ __forceinline__ uint2 encode_if4(const float2* P, float s, uint32_t& flag) {
   flag = 0u;
@@ -325,6 +340,11 @@ __device__ __forceinline__ uint2 encode_if4(const float2* P, float s, uint32_t& 
   float q[16];
   sr_quotients(P, s, RHT ? 4.0f : 1.0f, q);   // exact quotients, small ones included
   const float r76 = __fdiv_rn(7.0f, 6.0f), r67 = __fdiv_rn(6.0f, 7.0f);
+  float qm = fabsf(q[0]);
+#pragma unroll
+  for (int e = 1; e < 15; e += 2) qm = max3(qm, fabsf(q[e]), fabsf(q[e + 1]));
+  qm = fmaxf(qm, fabsf(q[15]));
+  const bool clamp = !(__fmul_rn(qm, r76) < 7.5f);
   constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
   // E2M1 candidate: codes from the signed quotients (-0 keeps its sign), magnitudes decoded.
   // Byte j of word l holds elements 8l + 2j (low nibble) and 8l + 2j + 1.
@@ -352,9 +372,9 @@ __device__ __forceinline__ uint2 encode_if4(const float2* P, float s, uint32_t& 
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float2 a2 = make_float2(fabsf(q[i]), fabsf(q[i + 8]));
-    const float2 w = __fmul2_rn(make_float2(q[i], q[i + 8]), make_float2(r76, r76));
-    const float2 tw = add2(make_float2(fminf(fmaxf(w.x, -7.0f), 7.0f), fminf(fmaxf(w.y, -7.0f), 7.0f)),
-                           make_float2(kMagic, kMagic));
+    float2 w = __fmul2_rn(make_float2(q[i], q[i + 8]), make_float2(r76, r76));
+    if (clamp) w = make_float2(fminf(fmaxf(w.x, -7.0f), 7.0f), fminf(fmaxf(w.y, -7.0f), 7.0f));
+    const float2 tw = add2(w, make_float2(kMagic, kMagic));
     t0[i] = __float_as_uint(tw.x);
     t1[i] = __float_as_uint(tw.y);
     const float2 k = add2(tw, make_float2(-kMagic, -kMagic));   // exact

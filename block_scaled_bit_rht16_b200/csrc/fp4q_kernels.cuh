@@ -48,6 +48,7 @@ struct QuantArgs {
   WsHeader* ws;            // header (amax, status) or null
   double* partials;        // statistics records or null
   uint32_t sw[8];          // sign flips per bf16 pair (all 0 without rotation)
+  uint32_t flip_lo[8], flip_hi[8];   // the same flips at bit 31: element 2k / 2k+1 of a block
   float c, cinv;           // 4, 1/4 with rotation; 1, 1 without
   uint64_t seedx;          // SR: seed ^ (stream << 63)
   int contiguous;          // ld == cols
@@ -81,15 +82,25 @@ struct DualArgs {
   int64_t M, N, ld;
   uint8_t* codes_row; float* scales_row;
   uint8_t* codes_col; float* scales_col;
-  uint32_t sw_row[8];       // row blocks: sign flips per bf16 pair (elements 2j, 2j+1)
-  uint32_t sc_col[16];      // column blocks: flip of element i in both halves of a bf16 pair
+  uint32_t flip_lo_row[8], flip_hi_row[8];   // row blocks: bit 31 flips elements 2k / 2k+1
+  uint32_t flip_col[16];    // column blocks: bit 31 flips element i (both columns of a word)
   int vec32;                // dy 32-byte aligned and ld % 16 == 0: 256-bit row-block loads
   int col16;                // M % 64 == 0 and codes_col, scales_col 16-byte aligned
   float c_row, cinv_row, c_col, cinv_col;
   uint64_t seedx_row, seedx_col;
   int round_row, round_col;   // per orientation
   int grid_row, grid_col;
+  int32_t* status;            // the library's device status word (a wait that gives up sets bit 0)
 };
+
+// Host: the per-element flips at bit 31 from sign words sw (bit 15: element 2k, bit 31:
+// element 2k+1), the form unpack16 adds to the unpacked bf16 halves.
+inline void sign_flips(const uint32_t* sw, uint32_t* flip_lo, uint32_t* flip_hi) {
+  for (int k = 0; k < 8; ++k) {
+    flip_lo[k] = (sw[k] & 0x8000u) << 16;
+    flip_hi[k] = sw[k] & 0x80000000u;
+  }
+}
 
 // Bits of the device status word (defined in fp4q_row.cu): bit 0 is kept for a bounded wait in a
 // quantize kernel that gives up (the current kernels load with plain loads and never wait, so it
@@ -115,6 +126,8 @@ cudaError_t launch_dual(const DualArgs& a, cudaStream_t st);
 cudaError_t launch_division_check(uint64_t seed, uint64_t n, unsigned long long* bad,
                                   cudaStream_t st);
 cudaError_t launch_wait_timeout_check(unsigned long long limit_ns, cudaStream_t st);
+cudaError_t launch_conversion_check(unsigned long long* bad, cudaStream_t st);
 cudaError_t read_device_status(int32_t* out, bool clear, cudaStream_t st);
+cudaError_t device_status_word(int32_t** out);
 
 }  // namespace fp4q

@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantArgs a) {
       uint16_t* deq = a.deq ? a.deq + un * kUnit : nullptr;
       if constexpr (S != kUE8M0) {
         float2 P[8];
-        unpack16(buf[k][0], buf[k][1], a.sw, P);
+        unpack16(buf[k][0], buf[k][1], a.flip_lo, a.flip_hi, P);
         rotate_if(a, P);
         const float amax_y = __fmul_rn(absmax16(P), a.cinv);
         float s;
@@ -234,8 +234,8 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantArgs a) {
         }
       } else {
         float2 P[8], Q[8];
-        unpack16(buf[k][0], buf[k][1], a.sw, P);
-        unpack16(buf[k][2], buf[k][3], a.sw, Q);
+        unpack16(buf[k][0], buf[k][1], a.flip_lo, a.flip_hi, P);
+        unpack16(buf[k][2], buf[k][3], a.flip_lo, a.flip_hi, Q);
         rotate_if(a, P);
         rotate_if(a, Q);
         const float amax_y = __fmul_rn(fmaxf(absmax16(P), absmax16(Q)), a.cinv);
@@ -282,7 +282,7 @@ __host__ __device__ inline bool flat_launch(const QuantArgs& a) {
 template <int G, bool RHT, bool FLAT, int R>
 __global__ void __launch_bounds__(kThreads) lean_kernel(const QuantArgs a) {
   constexpr float kCinv = RHT ? 0.25f : 1.0f;
-  const uint32_t zero_sw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  const uint32_t zero_flip[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
   pdl_enter();
   using Idx = typename UnitIdx<FLAT>::T;
   const Idx n = (Idx)a.nunits;
@@ -295,7 +295,7 @@ __global__ void __launch_bounds__(kThreads) lean_kernel(const QuantArgs a) {
     uint4 nlo = lo, nhi = hi;
     if (u + stride < n) lean_load<G, RHT, FLAT>(a, u + stride, nlo, nhi);
     float2 P[8];
-    unpack16(lo, hi, RHT ? a.sw : zero_sw, P);
+    unpack16(lo, hi, RHT ? a.flip_lo : zero_flip, RHT ? a.flip_hi : zero_flip, P);
     if constexpr (RHT) fwht16(P);
     const float s = div_qmax<G>(__fmul_rn(absmax16(P), kCinv));
     uint2 w;
@@ -332,13 +332,14 @@ __device__ __forceinline__ int group_of(const int64_t* off, int n, int64_t r) {
 // G = kIF4: the per-block FP4 / INT4 choice, flagged in bit 7 of the scale byte.
 // GROUPED: the tensor scale is that of the block's row group (group_ts), looked up again only
 // when a thread's block leaves the rows of the group it last used.
-// Five resident CTAs per SM (46 registers, no spills) measured faster than four; IF4's two
-// candidates and the grouped variant's scale cache keep their registers (they would spill).
+// Five resident CTAs per SM (48 registers, no spills) measured faster than four; IF4's two
+// candidates are held to three CTAs per SM (no spills), the grouped variant's scale cache keeps
+// its registers.
 template <int G, bool RHT, bool FLAT, bool GROUPED = false>
-__global__ void __launch_bounds__(kThreads, (G == kIF4 || GROUPED) ? 1 : 5) lean_nv_kernel(const QuantArgs a) {
+__global__ void __launch_bounds__(kThreads, G == kIF4 ? 3 : (GROUPED ? 1 : 5)) lean_nv_kernel(const QuantArgs a) {
   constexpr float qmax = GridInfo<G>::qmax;
   constexpr float kCinv = RHT ? 0.25f : 1.0f;
-  const uint32_t zero_sw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  const uint32_t zero_flip[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
   pdl_enter();
   float alpha = 0.0f;
   if constexpr (!GROUPED) {
@@ -365,9 +366,10 @@ __global__ void __launch_bounds__(kThreads, (G == kIF4 || GROUPED) ? 1 : 5) lean
     uint4 nlo = lo, nhi = hi;
     if (u + stride < n) lean_load<G, RHT, FLAT>(a, u + stride, nlo, nhi);
     float2 P[8];
-    unpack16(lo, hi, RHT ? a.sw : zero_sw, P);
+    unpack16(lo, hi, RHT ? a.flip_lo : zero_flip, RHT ? a.flip_hi : zero_flip, P);
     if constexpr (RHT) fwht16(P);
-    const float amax_y = __fmul_rn(absmax16(P), kCinv);
+    const float amax_raw = absmax16(P);
+    const float amax_y = __fmul_rn(amax_raw, kCinv);
     if constexpr (GROUPED) {
       if ((int64_t)u < g_lo || (int64_t)u >= g_hi) {
         const int g = group_of(a.group_off, a.n_groups, (int64_t)u / a.units_per_row);
@@ -388,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, (G == kIF4 || GROUPED) ? 1 : 5) lean
     uint2 w;
     uint32_t flag = 0u;
     if constexpr (G == kIF4) w = encode_if4<RHT>(P, s, flag);
-    else w = encode_lean<G, RHT, true>(P, s);
+    else w = encode_lean<G, RHT, true>(P, s, amax_raw);
     __stcs(reinterpret_cast<uint2*>(a.codes) + u, w);
     reinterpret_cast<uint8_t*>(a.scales)[scale_slot((int64_t)u, a.units_per_row, a.mma_scales)] =
         (uint8_t)(sbyte | flag);
@@ -403,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, (G == kIF4 || GROUPED) ? 1 : 5) lean
 template <bool RHT, bool FLAT>
 __global__ void __launch_bounds__(kThreads) amax_kernel(const QuantArgs a) {
   constexpr float kCinv = RHT ? 0.25f : 1.0f;
-  const uint32_t zero_sw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  const uint32_t zero_flip[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
   pdl_enter();
   uint32_t m = 0u;
   using Idx = typename UnitIdx<FLAT>::T;
@@ -417,7 +419,7 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const QuantArgs a) {
       uint4 nlo = lo, nhi = hi;
       if (u + stride < n) lean_load<0, RHT, FLAT>(a, u + stride, nlo, nhi);
       float2 P[8];
-      unpack16(lo, hi, RHT ? a.sw : zero_sw, P);
+      unpack16(lo, hi, RHT ? a.flip_lo : zero_flip, RHT ? a.flip_hi : zero_flip, P);
       if constexpr (RHT) fwht16(P);
       m = max(m, __float_as_uint(__fmul_rn(absmax16(P), kCinv)));
       lo = nlo;
@@ -435,7 +437,7 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const QuantArgs a) {
 template <bool RHT>
 __global__ void __launch_bounds__(kThreads) grouped_amax_kernel(const QuantArgs a) {
   constexpr float kCinv = RHT ? 0.25f : 1.0f;
-  const uint32_t zero_sw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  const uint32_t zero_flip[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
   pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
@@ -445,7 +447,7 @@ __global__ void __launch_bounds__(kThreads) grouped_amax_kernel(const QuantArgs 
       uint4 lo, hi;
       load16(a.x + r * a.ld + b * 16, a.vec32 != 0, lo, hi);
       float2 P[8];
-      unpack16(lo, hi, RHT ? a.sw : zero_sw, P);
+      unpack16(lo, hi, RHT ? a.flip_lo : zero_flip, RHT ? a.flip_hi : zero_flip, P);
       if constexpr (RHT) fwht16(P);
       m = max(m, __float_as_uint(__fmul_rn(absmax16(P), kCinv)));
     }
@@ -468,7 +470,7 @@ __global__ void __launch_bounds__(kThreads) rht16_kernel(const QuantArgs a, int 
     uint4 lo, hi;
     load16(a.x + unit_offset(a, u, 16), a.vec32 != 0, lo, hi);
     float2 P[8];
-    unpack16(lo, hi, a.sw, P);
+    unpack16(lo, hi, a.flip_lo, a.flip_hi, P);
     fwht16(P);
     float y[16];
 #pragma unroll
@@ -625,6 +627,76 @@ __global__ void __launch_bounds__(kThreads) division_check_kernel(uint64_t seed,
     }
   }
   if (local) atomicAdd(bad, local);
+}
+
+// Self-check of the hardware conversions the encoders rely on, each against a rule written here
+// from the format's definition (exponent field, step, round half to even through the integer
+// conversion, saturation), over every FP32 input in the range the kernels feed it:
+//   bad[0]  E2M1 encode (cvt.rn.satfinite.e2m1x2), every non-NaN float
+//   bad[1]  E1M2 encode through the FP6 E2M3 conversion (e1m2_word), every float |e| < 15/16
+//   bad[2]  E4M3 encode of a block-scale quotient (cvt.rn.satfinite.e4m3x2), every float >= 0
+//   bad[3]  the E2M1 (all 256 byte values) and E4M3 (codes 0..0x7E) decoders
+//   bad[4]  bf16 packing of the dequantized values (cvt.rn.bf16x2.f32), every non-NaN float
+__device__ __forceinline__ uint32_t e2m1_rule(float x) {
+  const uint32_t sgn = __float_as_uint(x) >> 31;
+  const float a = fabsf(x);
+  uint32_t m;
+  if (a < 2.0f) {
+    m = (uint32_t)__float2int_rn(a * 2.0f);              // step 1/2: codes 0..4 are k / 2
+  } else if (a < 4.0f) {
+    m = (uint32_t)__float2int_rn(a) + 2u;                // step 1: 2, 3, 4 -> codes 4, 5, 6
+  } else {
+    const int k = a >= 16.0f ? 3 : __float2int_rn(a * 0.5f);   // step 2: 4, 6 -> codes 6, 7
+    m = (uint32_t)min(k, 3) + 4u;                        // saturation at 6
+  }
+  return (sgn << 3) | m;
+}
+
+__device__ __forceinline__ uint32_t e4m3_rule(float x) {   // x >= 0, not NaN
+  if (x >= 448.0f) return 0x7Eu;                           // satfinite: 448 and above -> 448
+  if (x < 0x1p-6f) return (uint32_t)__float2int_rn(x * 512.0f);   // subnormal step 2^-9
+  const int E = (int)(__float_as_uint(x) >> 23) - 127;        // 2^E <= x < 2^(E+1), E in [-6, 8]
+  const float up = __uint_as_float((uint32_t)(127 + 3 - E) << 23);   // 2^(3-E), exact scaling
+  const int m = __float2int_rn(x * up);                       // 8 .. 16
+  const uint32_t code = (uint32_t)(((E + 7) << 3) + m - 8);   // 16 carries into the exponent
+  return min(code, 0x7Eu);
+}
+
+__global__ void __launch_bounds__(kThreads) conversion_check_kernel(unsigned long long* bad) {
+  unsigned long long nb[5] = {0, 0, 0, 0, 0};
+  const uint64_t stride = (uint64_t)gridDim.x * kThreads;
+  for (uint64_t i = (uint64_t)blockIdx.x * kThreads + threadIdx.x; i < (1ull << 32); i += stride) {
+    const uint32_t u = (uint32_t)i;
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x7FFFFFu)) continue;   // NaN
+    const float x = __uint_as_float(u);
+    const uint32_t e2 = cvt_e2m1x2(x, x), want2 = e2m1_rule(x);
+    if ((e2 & 0xFu) != want2 || (e2 >> 4) != want2) ++nb[0];
+    const uint32_t bf = pack_bf16x2(x, x), wantb = (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
+    if ((bf & 0xFFFFu) != wantb || (bf >> 16) != wantb) ++nb[4];
+    if ((u & 0x7FFFFFFFu) < 0x3F700000u) {                 // |x| < 15/16
+      const float e[8] = {x, x, x, x, x, x, x, x};
+      const uint32_t want = ((u >> 31) << 3) | (uint32_t)__float2int_rn(fabsf(x) * 8.0f);
+      if (e1m2_word(e) != want * 0x11111111u) ++nb[1];
+    }
+    if ((u >> 31) == 0u && cvt_e4m3(x) != e4m3_rule(x)) ++nb[2];
+    if (i < 256) {   // the E2M1 decoder on byte i (low nibble -> .x)
+      const float2 d = e2m1x2_to_f32((uint32_t)i);
+      const float tab[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+      const uint32_t lo = (uint32_t)i & 0xFu, hi = (uint32_t)i >> 4;
+      const float wl = (lo & 8u) ? -tab[lo & 7u] : tab[lo & 7u];
+      const float wh = (hi & 8u) ? -tab[hi & 7u] : tab[hi & 7u];
+      if (__float_as_uint(d.x) != __float_as_uint(wl) || __float_as_uint(d.y) != __float_as_uint(wh)) ++nb[3];
+    }
+    if (i < 0x7F) {   // the E4M3 decoder on code i: m 2^-9 (e = 0) or (8 + m) 2^(e - 10)
+      const int e = (int)(i >> 3), m = (int)(i & 7);
+      const float want = e == 0 ? (float)m * 0x1p-9f
+                                : (float)(8 + m) * __uint_as_float((uint32_t)(127 + e - 10) << 23);
+      if (__float_as_uint(e4m3_to_f32((uint32_t)i)) != __float_as_uint(want)) ++nb[3];
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 5; ++k)
+    if (nb[k]) atomicAdd(bad + k, nb[k]);
 }
 
 // ------------------------------------------------------------------ launch helpers
@@ -826,6 +898,7 @@ cudaError_t launch_rht16(const uint16_t* x, int64_t rows, int64_t cols, int64_t 
   a.nunits = rows * a.units_per_row;
   a.contiguous = (ld == cols);
   for (int k = 0; k < 8; ++k) a.sw[k] = sw[k];
+  sign_flips(a.sw, a.flip_lo, a.flip_hi);
   a.c = 4.0f;
   a.cinv = 0.25f;
   a.vec32 = (reinterpret_cast<uintptr_t>(x) % 32 == 0) && (rows == 1 || ld % 16 == 0);
@@ -877,9 +950,34 @@ cudaError_t launch_division_check(uint64_t seed, uint64_t n, unsigned long long*
   return cudaGetLastError();
 }
 
+cudaError_t launch_conversion_check(unsigned long long* bad, cudaStream_t st) {
+  conversion_check_kernel<<<resident_ctas(conversion_check_kernel), kThreads, 0, st>>>(bad);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_wait_timeout_check(unsigned long long limit_ns, cudaStream_t st) {
   wait_timeout_kernel<<<1, 1, 0, st>>>(limit_ns);
   return cudaGetLastError();
+}
+
+// Device address of the status word on the current device (looked up once per device; kernels
+// of other translation units receive it as an argument).
+cudaError_t device_status_word(int32_t** out) {
+  static std::mutex mu;
+  static std::map<int, int32_t*> cache;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(dev);
+  if (it == cache.end()) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_device_status);
+    if (e != cudaSuccess) return e;
+    it = cache.emplace(dev, static_cast<int32_t*>(p)).first;
+  }
+  *out = it->second;
+  return cudaSuccess;
 }
 
 cudaError_t read_device_status(int32_t* out, bool clear, cudaStream_t st) {
