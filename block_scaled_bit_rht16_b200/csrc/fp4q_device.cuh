@@ -159,6 +159,11 @@ __device__ __forceinline__ float2 div2(const Divider& d, float2 a) {
 
 // ------------------------------------------------------------------ grids
 
+// RN(7/6) and RN(6/7) in binary32 (1.16666663, 0.857142866): the IF4 INT4 candidate's scaling
+// and dequantization factors.
+constexpr float kR76 = 0x1.2aaaaap+0f;
+constexpr float kR67 = 0x1.b6db6ep-1f;
+
 template <int G> struct GridInfo;
 template <> struct GridInfo<kE2M1> { static constexpr float qmax = 6.0f; };
 template <> struct GridInfo<kE1M2> { static constexpr float qmax = 3.5f; };
@@ -229,9 +234,9 @@ __device__ __forceinline__ void pdl_enter() {
 
 // ------------------------------------------------------------------ bulk copies and barriers
 //
-// Global -> shared bulk copies (cp.async.bulk, no multicast) complete on an mbarrier with a
-// transaction count. Every wait is bounded by the global timer: a wait that gives up sets a
-// bit in the library's device status word and returns false, so no kernel can hang.
+// Tile copies into shared memory complete on an mbarrier with a transaction count. Every wait is
+// bounded by the global timer: a wait that gives up returns false (the caller records it in the
+// library's device status word), so no kernel can hang.
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
 
@@ -279,13 +284,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63u) == 0u && global_ns() - t0 > limit_ns) return false;
   }
-}
-
-// bytes (multiple of 16) from global src (16-byte aligned) to shared dst (16-byte aligned).
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
 
 // ------------------------------------------------------------------ stochastic rounding source

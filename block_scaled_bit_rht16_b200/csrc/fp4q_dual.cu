@@ -7,7 +7,7 @@
 // section 三 on bwd_dx / bwd_dw).
 //
 // Persistent kernel over 128 x 64 tiles of dY (tile t: rows 128 (t / tiles_n), columns
-// 64 (t % tiles_n)). Each CTA takes every gridDim.x-th tile. The tiles reach shared memory through
+// 64 (t % tiles_n)). Each CTA takes every gridDim.x-th tile, starting at tile blockIdx.x. The tiles reach shared memory through
 // a ring of kStages buffers filled by 2-D bulk tensor copies (TMA, this GPU's memory only, no
 // multicast) that complete on one mbarrier per buffer, so a CTA's next tiles are in flight
 // while it encodes the current one; out-of-range rows and columns of edge tiles arrive as zeros.
@@ -86,26 +86,39 @@ __global__ void __launch_bounds__(kThreads, 3)
   __syncthreads();
   pdl_enter();
 
-  auto issue = [&](int64_t tile, int s) {
-    mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
-    tma_load_tile(sm.tile[s], &tmap, (int)((tile % tiles_n) * kTileN), (int)((tile / tiles_n) * kTileM),
-                  &sm.full[s]);
+  // Tile t is (t / tiles_n, t % tiles_n); walking t by gridDim.x moves that pair by
+  // (step_m, step_n) with one carry, so no division is left in the loop.
+  const int64_t step_m = gridDim.x / tiles_n, step_n = gridDim.x % tiles_n;
+  auto advance = [&](int64_t& tm, int64_t& tn) {
+    tm += step_m;
+    tn += step_n;
+    if (tn >= tiles_n) {
+      tn -= tiles_n;
+      ++tm;
+    }
   };
+  const int64_t tm0 = blockIdx.x / tiles_n, tn0 = blockIdx.x % tiles_n;
+  auto issue = [&](int64_t tm, int64_t tn, int s) {
+    mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
+    tma_load_tile(sm.tile[s], &tmap, (int)(tn * kTileN), (int)(tm * kTileM), &sm.full[s]);
+  };
+  // the tile kStages ahead of the current one (the copy that refills its buffer)
+  int64_t am = tm0, an = tn0;
   if (t == 0) {
     for (int s = 0; s < kStages; ++s) {
-      const int64_t tile = blockIdx.x + (int64_t)s * gridDim.x;
-      if (tile < tiles) issue(tile, s);
+      if (am * tiles_n + an < tiles) issue(am, an, s);
+      advance(am, an);
     }
   }
 
-  int64_t it = 0;
-  for (;; ++it) {
-    const int64_t tile = blockIdx.x + it * gridDim.x;
+  int64_t it = 0, tm = tm0, tn = tn0;
+  for (;; ++it, advance(tm, tn)) {
+    const int64_t tile = tm * tiles_n + tn;
     if (tile >= tiles) break;
     const int s = (int)(it % kStages);
     const uint32_t parity = (uint32_t)((it / kStages) & 1);
     const int fail = mbar_wait(&sm.full[s], parity) ? 0 : 1;
-    const int64_t m0 = (tile / tiles_n) * kTileM, n0 = (tile % tiles_n) * kTileN;
+    const int64_t m0 = tm * kTileM, n0 = tn * kTileN;
     const uint8_t* T = reinterpret_cast<const uint8_t*>(sm.tile[s]);
 
     // row blocks: rows 8 (2 wp + k) + lane % 8, block lane / 8 (columns 16 (lane / 8) ..)
@@ -163,8 +176,8 @@ __global__ void __launch_bounds__(kThreads, 3)
     if (__syncthreads_or(fail)) break;
     // every thread is done with ring buffer s: refill it with the tile kStages ahead
     if (t == 0) {
-      const int64_t next = tile + (int64_t)kStages * gridDim.x;
-      if (next < tiles) issue(next, s);
+      if (am * tiles_n + an < tiles) issue(am, an, s);
+      advance(am, an);
     }
 
     // column c's blocks for rows m0 .. m0+127 are kGroups consecutive entries of codes_col /
@@ -205,13 +218,12 @@ __global__ void __launch_bounds__(kThreads, 3)
     }
   }
 
-  if (it * gridDim.x + blockIdx.x < tiles && t == 0) {
+  if (tm * tiles_n + tn < tiles && t == 0) {
     // a wait gave up: record it, then wait (bounded) for every copy this CTA still has in flight
     // so that none lands in shared memory after the CTA has ended
     atomicOr(a.status, kStatusWaitTimeout);
-    for (int64_t j = it; j < it + kStages; ++j) {
-      const int64_t tile = blockIdx.x + j * gridDim.x;
-      if (tile >= tiles) break;
+    for (int64_t j = it; j < it + kStages; ++j, advance(tm, tn)) {
+      if (tm * tiles_n + tn >= tiles) break;
       mbar_wait(&sm.full[j % kStages], (uint32_t)((j / kStages) & 1));
     }
   }

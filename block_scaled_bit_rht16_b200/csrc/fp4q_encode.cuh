@@ -139,13 +139,18 @@ __device__ __forceinline__ uint32_t e1m2_word(const float* e) {
 // amax_raw (CLAMP only): max |P|. Its quotient bounds every element's (the quotient is
 // monotonic in the numerator), so a block whose largest quotient stays below qmax + step/2
 // rounds no element above qmax, and the clamp, which could not change a code, is skipped.
+// The divisor of encode_lean's quotients: c * s, times 4 for E1M2 (whose codes come from v / 4).
+template <int G, bool RHT>
+constexpr float lean_divisor_factor() { return (RHT ? 4.0f : 1.0f) * (G == kE1M2 ? 4.0f : 1.0f); }
+
+// encode_lean with the block's Divider of s * lean_divisor_factor<G, RHT>() given.
 template <int G, bool RHT, bool CLAMP = false>
-__device__ __forceinline__ uint2 encode_lean(const float2* P, float s, float amax_raw = 0.0f) {
+__device__ __forceinline__ uint2 encode_lean_dv(const float2* P, float s, const Divider& dv,
+                                                float amax_raw = 0.0f) {
   if (s == 0.0f) return make_uint2(0u, 0u);
   constexpr float qmax = GridInfo<G>::qmax;
   constexpr float kC = RHT ? 4.0f : 1.0f;
   constexpr float kVScale = (G == kE1M2) ? 4.0f : 1.0f;   // quotients of v / kVScale
-  const Divider dv = make_divider(s, kC * kVScale);
   float2 Q[8];
   if (dv.fast) {
 #pragma unroll
@@ -210,6 +215,12 @@ __device__ __forceinline__ uint2 encode_lean(const float2* P, float s, float ama
   return make_uint2(w[0], w[1]);
 }
 
+template <int G, bool RHT, bool CLAMP = false>
+__device__ __forceinline__ uint2 encode_lean(const float2* P, float s, float amax_raw = 0.0f) {
+  if (s == 0.0f) return make_uint2(0u, 0u);
+  return encode_lean_dv<G, RHT, CLAMP>(P, s, make_divider(s, lean_divisor_factor<G, RHT>()), amax_raw);
+}
+
 // Stochastic rounding, FP32 1x16 scale, codes only; runtime rotation factor c (4 or 1).
 // Element e (0..15) of the block has logical index 4*quad0 + e and the 16-bit draw u_e.
 //
@@ -226,10 +237,10 @@ __device__ __forceinline__ uint2 encode_lean(const float2* P, float s, float ama
 // Codes: sign-magnitude (E1M2, E2M1) takes the input's sign bit as bit 3; INT4 takes -k in
 // two's complement for a negative input.
 
-// Quotients v_e = RN(P_e / (c * s)) of a nonzero block, exact.
-__device__ __forceinline__ void sr_quotients(const float2* P, float s, float c, float* q) {
+// Quotients v_e = RN(P_e / (c * s)) of a nonzero block, exact, with dv the Divider of c * s.
+__device__ __forceinline__ void sr_quotients_dv(const float2* P, float s, float c, const Divider& dv,
+                                                float* q) {
   const float cinv = __frcp_rn(c);   // exact: c is 4 or 1
-  const Divider dv = make_divider(s, c);
   if (dv.fast) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -255,6 +266,10 @@ __device__ __forceinline__ void sr_quotients(const float2* P, float s, float c, 
 #pragma unroll
     for (int e = 0; e < 16; ++e) q[e] = __fdiv_rn(__fmul_rn(elem_x(P, e), cinv), s);
   }
+}
+
+__device__ __forceinline__ void sr_quotients(const float2* P, float s, float c, float* q) {
+  sr_quotients_dv(P, s, c, make_divider(s, c), q);
 }
 
 // Codes of a nonzero block from its quotients q, draw words d (sr_words16) and raw values P (for
@@ -328,28 +343,27 @@ __device__ __forceinline__ uint2 encode_sr(const float2* P, float s, float c, ui
 // saturating) and the INT4 candidate k = RNE(RN(v * RN(7/6))) clamped to +-7 with value
 // RN(k * RN(6/7)); INT4 is kept iff its squared error, summed in FP32 over the balanced pairwise
 // tree of elements 0..15, is strictly smaller ("低精度量化技术：IF4…", sections 3.1-3.2).
-// The errors RN(value - v) are formed on magnitudes: a nonzero candidate has the sign of v and
-// RN is symmetric, so each square equals the signed one. Returns the code words; flag = 0x80 for
-// an INT4 block.
+// Returns the code words; flag = 0x80 for an INT4 block.
 // When even the largest |q| times RN(7/6) stays below 7.5, no INT4 candidate needs the clamp at
 // +-7 (it could not change a code) and it is skipped.
+// dv: the Divider of c * s (c = 4 with rotation, else 1).
 template <bool RHT>
-__device__ __forceinline__ uint2 encode_if4(const float2* P, float s, uint32_t& flag) {
+__device__ __forceinline__ uint2 encode_if4(const float2* P, float s, const Divider& dv, uint32_t& flag) {
   flag = 0u;
   if (s == 0.0f) return make_uint2(0u, 0u);
   float q[16];
-  sr_quotients(P, s, RHT ? 4.0f : 1.0f, q);   // exact quotients, small ones included
-  const float r76 = __fdiv_rn(7.0f, 6.0f), r67 = __fdiv_rn(6.0f, 7.0f);
+  sr_quotients_dv(P, s, RHT ? 4.0f : 1.0f, dv, q);   // exact quotients, small ones included
+  const float r76 = kR76, r67 = kR67;
   float qm = fabsf(q[0]);
 #pragma unroll
   for (int e = 1; e < 15; e += 2) qm = max3(qm, fabsf(q[e]), fabsf(q[e + 1]));
   qm = fmaxf(qm, fabsf(q[15]));
   const bool clamp = !(__fmul_rn(qm, r76) < 7.5f);
   constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
-  // E2M1 candidate: codes from the signed quotients (-0 keeps its sign), magnitudes decoded.
+  // E2M1 candidate: codes from the signed quotients (-0 keeps its sign), decoded with signs.
   // Byte j of word l holds elements 8l + 2j (low nibble) and 8l + 2j + 1.
   uint32_t fw[2] = {0u, 0u};
-  float gabs[16];
+  float g[16];
 #pragma unroll
   for (int l = 0; l < 2; ++l) {
 #pragma unroll
@@ -359,28 +373,31 @@ __device__ __forceinline__ uint2 encode_if4(const float2* P, float s, uint32_t& 
       const float v1 = RHT ? q[e + 1] : with_sign_of(q[e + 1], elem_x(P, e + 1));
       const uint32_t b = cvt_e2m1x2(v1, v0);
       fw[l] |= b << (8 * j);
-      const float2 g = e2m1x2_to_f32(b);
-      gabs[e] = fabsf(g.x);
-      gabs[e + 1] = fabsf(g.y);
+      const float2 d = e2m1x2_to_f32(b);
+      g[e] = d.x;
+      g[e + 1] = d.y;
     }
   }
   // INT4 candidate and both squared errors, two elements (i, i+8) per float2: w = RN(v * 7/6)
   // clamped to +-7 and rounded half-even by the 1.5 * 2^23 add (its low nibble is the two's
-  // complement code), the magnitude k back as an exact float.
+  // complement code), k back as an exact signed float. The errors are formed on signed values:
+  // each candidate value has the sign of v (or is a zero), and RN is symmetric, so
+  // RN(RN(k * 6/7) - v) and RN(g - v) have the magnitudes of the errors on magnitudes, and the
+  // same squares.
   uint32_t t0[8], t1[8];
   float2 Sf[8], Si[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float2 a2 = make_float2(fabsf(q[i]), fabsf(q[i + 8]));
-    float2 w = __fmul2_rn(make_float2(q[i], q[i + 8]), make_float2(r76, r76));
+    const float2 q2 = make_float2(q[i], q[i + 8]);
+    float2 w = __fmul2_rn(q2, make_float2(r76, r76));
     if (clamp) w = make_float2(fminf(fmaxf(w.x, -7.0f), 7.0f), fminf(fmaxf(w.y, -7.0f), 7.0f));
     const float2 tw = add2(w, make_float2(kMagic, kMagic));
     t0[i] = __float_as_uint(tw.x);
     t1[i] = __float_as_uint(tw.y);
     const float2 k = add2(tw, make_float2(-kMagic, -kMagic));   // exact
-    const float2 vint = __fmul2_rn(make_float2(fabsf(k.x), fabsf(k.y)), make_float2(r67, r67));
-    const float2 dint = sub2(vint, a2);
-    const float2 dfp = sub2(make_float2(gabs[i], gabs[i + 8]), a2);
+    const float2 vint = __fmul2_rn(k, make_float2(r67, r67));
+    const float2 dint = sub2(vint, q2);
+    const float2 dfp = sub2(make_float2(g[i], g[i + 8]), q2);
     Sf[i] = __fmul2_rn(dfp, dfp);
     Si[i] = __fmul2_rn(dint, dint);
   }
@@ -513,7 +530,7 @@ __device__ __forceinline__ uint32_t encode16(const EncCtx& ctx, const float2* P,
       }
     }
     if constexpr (G == kIF4) {
-      const float r76 = __fdiv_rn(7.0f, 6.0f), r67 = __fdiv_rn(6.0f, 7.0f);
+      const float r76 = kR76, r67 = kR67;
       float vint[16];
       uint32_t mint[16];
       uint32_t i0 = 0u, i1 = 0u;

@@ -102,9 +102,9 @@ inline void sign_flips(const uint32_t* sw, uint32_t* flip_lo, uint32_t* flip_hi)
   }
 }
 
-// Bits of the device status word (defined in fp4q_row.cu): bit 0 is kept for a bounded wait in a
-// quantize kernel that gives up (the current kernels load with plain loads and never wait, so it
-// stays clear), bit 1 the timeout self-test fired. Sticky until read with clear.
+// Bits of the device status word (defined in fp4q_row.cu): bit 0 a bounded wait in a quantize
+// kernel gave up (the dual kernel's waits on its tile copies), bit 1 the timeout self-test fired.
+// Sticky until read with clear.
 constexpr int32_t kStatusWaitTimeout = 1;
 constexpr int32_t kStatusSelfTest = 2;
 

@@ -354,6 +354,19 @@ __global__ void __launch_bounds__(kThreads, G == kIF4 ? 3 : (GROUPED ? 1 : 5)) l
   // RN(amax / denom) for every block through the correction step on one reciprocal (exact for
   // quotients in [2^-20, 2^64); the E4M3 conversion sends anything below 2^-11 to 0 either way)
   Divider dd = make_divider(denom, 1.0f);
+  // One tensor scale for the launch: a block scale is RN(decode(d8) * alpha) for one of the 127
+  // E4M3 codes d8, so each code's scale and the Divider of its element quotients are formed
+  // once per CTA (the same operations as per block) and looked up by code.
+  constexpr float kFactor = G == kIF4 ? (RHT ? 4.0f : 1.0f) : lean_divisor_factor<G, RHT>();
+  __shared__ float4 s_tab[128];
+  if constexpr (!GROUPED) {
+    if (threadIdx.x < 128) {
+      const float sd = __fmul_rn(e4m3_to_f32(threadIdx.x), alpha);
+      const Divider dv = make_divider(sd, kFactor);
+      s_tab[threadIdx.x] = make_float4(sd, dv.S, dv.R, dv.fast ? 1.0f : 0.0f);
+    }
+    __syncthreads();
+  }
   int64_t g_lo = 0, g_hi = 0;   // blocks of the group whose scale is loaded (none yet)
   using Idx = typename UnitIdx<FLAT>::T;
   const Idx n = (Idx)a.nunits;
@@ -386,11 +399,24 @@ __global__ void __launch_bounds__(kThreads, G == kIF4 ? 3 : (GROUPED ? 1 : 5)) l
     // tensor scale may be tiny), the IEEE division
     if ((!dd.fast || !(delta < 0x1p+64f)) && denom > 0.0f) delta = __fdiv_rn(amax_y, denom);
     const uint32_t sbyte = cvt_e4m3(delta);
-    const float s = __fmul_rn(e4m3_to_f32(sbyte), alpha);
+    float s;
+    Divider dv;
+    if constexpr (GROUPED) {
+      s = __fmul_rn(e4m3_to_f32(sbyte), alpha);
+      dv = make_divider(s, kFactor);
+    } else {
+      const float4 e = s_tab[sbyte];
+      s = e.x;
+      dv.S = e.y;
+      dv.R = e.z;
+      dv.fast = e.w != 0.0f;
+      dv.R2 = make_float2(dv.R, dv.R);
+      dv.nS2 = make_float2(-dv.S, -dv.S);
+    }
     uint2 w;
     uint32_t flag = 0u;
-    if constexpr (G == kIF4) w = encode_if4<RHT>(P, s, flag);
-    else w = encode_lean<G, RHT, true>(P, s, amax_raw);
+    if constexpr (G == kIF4) w = encode_if4<RHT>(P, s, dv, flag);
+    else w = encode_lean_dv<G, RHT, true>(P, s, dv, amax_raw);
     __stcs(reinterpret_cast<uint2*>(a.codes) + u, w);
     reinterpret_cast<uint8_t*>(a.scales)[scale_slot((int64_t)u, a.units_per_row, a.mma_scales)] =
         (uint8_t)(sbyte | flag);
@@ -508,7 +534,7 @@ struct DeqArgs {
 template <int G, int S>
 __global__ void __launch_bounds__(kThreads) dequant_kernel(const DeqArgs a) {
   const float alpha = (S == kE4M3) ? *a.ts : 0.0f;
-  const float r67 = __fdiv_rn(6.0f, 7.0f);
+  const float r67 = kR67;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < a.nunits; u += stride) {
     const uint2 cw = __ldcs(reinterpret_cast<const uint2*>(a.codes) + u);
@@ -635,7 +661,8 @@ __global__ void __launch_bounds__(kThreads) division_check_kernel(uint64_t seed,
 //   bad[0]  E2M1 encode (cvt.rn.satfinite.e2m1x2), every non-NaN float
 //   bad[1]  E1M2 encode through the FP6 E2M3 conversion (e1m2_word), every float |e| < 15/16
 //   bad[2]  E4M3 encode of a block-scale quotient (cvt.rn.satfinite.e4m3x2), every float >= 0
-//   bad[3]  the E2M1 (all 256 byte values) and E4M3 (codes 0..0x7E) decoders
+//   bad[3]  the E2M1 (all 256 byte values) and E4M3 (codes 0..0x7E) decoders, and the IF4
+//           factors RN(7/6), RN(6/7) against the IEEE quotients
 //   bad[4]  bf16 packing of the dequantized values (cvt.rn.bf16x2.f32), every non-NaN float
 __device__ __forceinline__ uint32_t e2m1_rule(float x) {
   const uint32_t sgn = __float_as_uint(x) >> 31;
@@ -687,6 +714,9 @@ __global__ void __launch_bounds__(kThreads) conversion_check_kernel(unsigned lon
       const float wh = (hi & 8u) ? -tab[hi & 7u] : tab[hi & 7u];
       if (__float_as_uint(d.x) != __float_as_uint(wl) || __float_as_uint(d.y) != __float_as_uint(wh)) ++nb[3];
     }
+    if (i == 0 && (__float_as_uint(__fdiv_rn(7.0f, 6.0f)) != __float_as_uint(kR76) ||
+                   __float_as_uint(__fdiv_rn(6.0f, 7.0f)) != __float_as_uint(kR67)))
+      ++nb[3];   // the IF4 factors are the IEEE quotients
     if (i < 0x7F) {   // the E4M3 decoder on code i: m 2^-9 (e = 0) or (8 + m) 2^(e - 10)
       const int e = (int)(i >> 3), m = (int)(i & 7);
       const float want = e == 0 ? (float)m * 0x1p-9f

@@ -139,8 +139,8 @@ typedef struct {
   double nmse;              /* sum_err2 / sum_y2 */
   double cell_mean_err[8];  /* cell_err / cell_count (NaN for an empty cell): shrinkage bias */
   double if4_fp4_fraction;  /* if4_fp4_blocks / blocks */
-  int32_t status;           /* FP4Q_OK, or FP4Q_ERR_TIMEOUT if a device wait gave up (no
-                               current kernel waits: always FP4Q_OK) */
+  int32_t status;           /* FP4Q_OK, or FP4Q_ERR_TIMEOUT if a device wait gave up (the
+                               statistics-producing kernels do not wait: FP4Q_OK) */
   int32_t reserved;
 } fp4q_stats_t;
 
@@ -292,15 +292,16 @@ fp4q_status fp4q_check_division(uint64_t seed, uint64_t n, unsigned long long* m
  *      conversion), every float of magnitude below 15/16 ["UFP4：换一把尺子"]
  *  [2] E4M3 encode of a block-scale quotient (round to nearest even, 448 and above -> 448), every
  *      float >= 0 including +inf ["低精度量化技术：IF4…", section 3.2]
- *  [3] the E2M1 decoder on all 256 bytes and the E4M3 decoder on codes 0..0x7E
+ *  [3] the E2M1 decoder on all 256 bytes, the E4M3 decoder on codes 0..0x7E, and IF4's
+ *      factors RN(7/6), RN(6/7) against the IEEE quotients
  *  [4] bf16 rounding of dequantized values (round to nearest even), every non-NaN float */
 fp4q_status fp4q_check_conversions(unsigned long long* mismatches, fp4q_stream_t stream);
 
-/* Device status word of the library on the current device: bit 0 is reserved for a bounded
- * wait inside a quantize kernel that gives up (that launch's outputs would be incomplete); the
- * current kernels read their inputs with plain loads and never wait, so it stays clear. Bit 1 is
- * set by fp4q_check_wait_timeout. Copies the word to *status_bits (host), clears it when
- * `clear` is 1, and synchronizes `stream`. */
+/* Device status word of the library on the current device: bit 0 is set when a bounded wait
+ * inside a quantize kernel gives up (fp4q_quantize_dual waits on the tile copies it has issued,
+ * at most 2 s each; that launch's outputs are then incomplete); the row quantizers read their
+ * inputs with plain loads and never wait. Bit 1 is set by fp4q_check_wait_timeout. Copies the
+ * word to *status_bits (host), clears it when `clear` is 1, and synchronizes `stream`. */
 fp4q_status fp4q_device_status(int32_t* status_bits, int32_t clear, fp4q_stream_t stream);
 
 /* Diagnostic: launches one thread that waits, with a limit of limit_ns (1 ns .. 1 s), on a

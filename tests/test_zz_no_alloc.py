@@ -46,6 +46,26 @@ def test_noalloc_matches_workspace_entry_point_twice(grid):
         np.testing.assert_array_equal(bf16_bits(deq), bf16_bits(ref.dequant))
 
 
+@pytest.mark.parametrize("cfg", [
+    fq.Config(grid=fq.FP4Q_GRID_E1M2, round=fq.FP4Q_ROUND_SR, sign_mask=0x0FF0, sr_seed=0x5A5A0003),
+    fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=fq.FP4Q_SCALE_UE8M0_1x32, sign_mask=0x1234, dequant=True)],
+    ids=["fp32-sr", "ue8m0-rtne"])
+def test_noalloc_configurations_without_scratch(cfg):
+    # FP32 and UE8M0 scales need no scratch at all: the entry point passes no workspace and must
+    # still give the workspace entry point's results, stochastic rounding included
+    for bits in [synth.small(7, 130, 512, "t4"), synth.small(8, 64, 1024, "normal", 1e-3)]:
+        x = to_dev(bits)
+        ref = fq.rht_quantize(cfg, x)
+        codes, scales = torch.empty_like(ref.codes), torch.empty_like(ref.scales)
+        deq = torch.empty_like(ref.dequant) if cfg.dequant else None
+        assert _noalloc(cfg, x, codes, scales, None, deq) == 0
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(host(codes), host(ref.codes))
+        np.testing.assert_array_equal(host(scales), host(ref.scales))
+        if cfg.dequant:
+            np.testing.assert_array_equal(bf16_bits(deq), bf16_bits(ref.dequant))
+
+
 def test_noalloc_rejects_statistics():
     cfg = fq.Config(stats=True)
     x = torch.zeros((16, 64), dtype=torch.bfloat16, device="cuda")
