@@ -50,6 +50,20 @@ __device__ __forceinline__ void unpack16(const uint4& lo, const uint4& hi, const
   }
 }
 
+// Two blocks at once (words lo0/hi0 of block 0, lo1/hi1 of block 1) as A[i] = (element i of
+// block 0, element i of block 1), with the same sign flips for both.
+__device__ __forceinline__ void unpack16_pair(const uint4& lo0, const uint4& hi0, const uint4& lo1,
+                                              const uint4& hi1, const uint32_t* flip_lo,
+                                              const uint32_t* flip_hi, float2* A) {
+  const uint32_t w0[8] = {lo0.x, lo0.y, lo0.z, lo0.w, hi0.x, hi0.y, hi0.z, hi0.w};
+  const uint32_t w1[8] = {lo1.x, lo1.y, lo1.z, lo1.w, hi1.x, hi1.y, hi1.z, hi1.w};
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    A[2 * k] = make_float2(bf_lo_flip(w0[k], flip_lo[k]), bf_lo_flip(w1[k], flip_lo[k]));
+    A[2 * k + 1] = make_float2(bf_hi_flip(w0[k], flip_hi[k]), bf_hi_flip(w1[k], flip_hi[k]));
+  }
+}
+
 __device__ __forceinline__ uint4 ld_stream(const uint16_t* p) {
   return __ldcs(reinterpret_cast<const uint4*>(p));
 }

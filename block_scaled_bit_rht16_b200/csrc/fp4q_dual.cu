@@ -122,6 +122,30 @@ __global__ void __launch_bounds__(kThreads, 3)
     const uint8_t* T = reinterpret_cast<const uint8_t*>(sm.tile[s]);
 
     // row blocks: rows 8 (2 wp + k) + lane % 8, block lane / 8 (columns 16 (lane / 8) ..)
+    if constexpr (RR == kSR) {
+      // both of the thread's row blocks at once (rows r and r + 8: the 16-row group 16 wp is in
+      // range or out of range as a whole, M % 16 == 0)
+      const int r = 16 * wp + (lane & 7), b = lane >> 3;
+      const int64_t m = m0 + r, n = n0 + 16 * b;
+      if (m < a.M && n < a.N) {
+        float2 A[16];
+        unpack16_pair(*reinterpret_cast<const uint4*>(T + swz(r, 2 * b)),
+                      *reinterpret_cast<const uint4*>(T + swz(r, 2 * b + 1)),
+                      *reinterpret_cast<const uint4*>(T + swz(r + 8, 2 * b)),
+                      *reinterpret_cast<const uint4*>(T + swz(r + 8, 2 * b + 1)), a.flip_lo_row,
+                      a.flip_hi_row, A);
+        if (rot_row) fwht16_pair(A);
+        const float2 am = absmax16_pair(A);
+        const float2 sc = make_float2(div_qmax<G>(__fmul_rn(am.x, cinv_row)), div_qmax<G>(__fmul_rn(am.y, cinv_row)));
+        const int64_t u0 = (m * a.N + n) >> 4, u1 = ((m + 8) * a.N + n) >> 4;
+        uint2 w0, w1;
+        encode_sr_pair<G>(A, sc, c_row, a.seedx_row, (uint64_t)u0 * 4u, (uint64_t)u1 * 4u, w0, w1);
+        __stcs(reinterpret_cast<uint2*>(a.codes_row) + u0, w0);
+        __stcs(a.scales_row + u0, sc.x);
+        __stcs(reinterpret_cast<uint2*>(a.codes_row) + u1, w1);
+        __stcs(a.scales_row + u1, sc.y);
+      }
+    } else {
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int r = 8 * (2 * wp + k) + (lane & 7), b = lane >> 3;
@@ -140,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 3)
       __stcs(reinterpret_cast<uint2*>(a.codes_row) + u, w);
       __stcs(a.scales_row + u, sc);
     }
+    }
 
     // column blocks: rows 16 wp .. 16 wp + 15, columns 2 lane + h (N % 16 == 0, M % 16 == 0: a
     // column pair and a group of 16 rows are in range or out of range as a whole)
@@ -153,6 +178,23 @@ __global__ void __launch_bounds__(kThreads, 3)
           const int r = 16 * wp + i;
           wd[i] = *reinterpret_cast<const uint32_t*>(T + swz(r, lane >> 2) + 4 * (lane & 3));
         }
+        if constexpr (RC == kSR) {
+          // both columns at once: A[i] = (column 2 lane, column 2 lane + 1) of row 16 wp + i
+          float2 A[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            A[i] = make_float2(bf_lo_flip(wd[i], a.flip_col[i]), bf_hi_flip(wd[i], a.flip_col[i]));
+          if (rot_col) fwht16_pair(A);
+          const float2 am = absmax16_pair(A);
+          const float2 sc = make_float2(div_qmax<G>(__fmul_rn(am.x, cinv_col)), div_qmax<G>(__fmul_rn(am.y, cinv_col)));
+          const int64_t u0 = (nA * a.M + m) >> 4, u1 = ((nA + 1) * a.M + m) >> 4;
+          uint2 w0, w1;
+          encode_sr_pair<G>(A, sc, c_col, a.seedx_col, (uint64_t)u0 * 4u, (uint64_t)u1 * 4u, w0, w1);
+          sm.stage_codes[buf][(2 * lane) * kCodePitch + wp] = w0;
+          sm.stage_scales[buf][(2 * lane) * kScalePitch + wp] = sc.x;
+          sm.stage_codes[buf][(2 * lane + 1) * kCodePitch + wp] = w1;
+          sm.stage_scales[buf][(2 * lane + 1) * kScalePitch + wp] = sc.y;
+        } else {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           float2 P[8];
@@ -169,6 +211,7 @@ __global__ void __launch_bounds__(kThreads, 3)
           const int c = 2 * lane + h;
           sm.stage_codes[buf][c * kCodePitch + wp] = w;
           sm.stage_scales[buf][c * kScalePitch + wp] = sc;
+        }
         }
       }
     }

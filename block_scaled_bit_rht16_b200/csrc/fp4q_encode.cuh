@@ -272,58 +272,72 @@ __device__ __forceinline__ void sr_quotients(const float2* P, float s, float c, 
   sr_quotients_dv(P, s, c, make_divider(s, c), q);
 }
 
-// Codes of a nonzero block from its quotients q, draw words d (sr_words16) and raw values P (for
-// the signs).
+// Bit pattern 0x4B400000 + k of the stochastically rounded magnitude code k of one quotient q
+// (element e of its block, draw words d from sr_words16).
 template <int G>
-__device__ __forceinline__ uint2 sr_codes(const float* q, const uint32_t* d, const float2* P) {
+__device__ __forceinline__ uint32_t sr_bits(float q, const uint32_t* d, int e) {
   constexpr float qmax = GridInfo<G>::qmax;
-  // sum over j = 0..7 of 0x4B400000 * 16^j, modulo 2^32
-  constexpr uint32_t kBias = 0x4B400000u + (0x4B400000u << 4) + (0x4B400000u << 8) +
+  float K;
+  if constexpr (kIsE2M1<G>) {
+    const float a = fminf(fabsf(q), qmax);
+    const float r = __fmaf_rn(sr_one_plus(d, e), 128.0f, -128.0f);   // u * 2^-16, exact
+    const bool lo = a < 2.0f, mid = a < 4.0f;
+    const float inv_step = lo ? 2.0f : (mid ? 1.0f : 0.5f);
+    const float base = lo ? 12582912.0f : (mid ? 12582914.0f : 12582916.0f);
+    K = __fadd_ru(__fmaf_ru(a, inv_step, -r), base);
+  } else {
+    // uniform grids, t = |v| / step with qmax = 7 steps: F = 1 + u * 2^-23 (the draw in the
+    // low mantissa bits, one byte permute of its word), c = 16.125 - 16 F = (1 - r) / 8 exactly;
+    // w = min(RU((t - r + 1) / 8), 1) (the saturation is the clamp at qmax: t' = min(t, 7));
+    // 8w = RU(t' - r + 1), whose ceiling is ceil(t' - r) + 1 (no integer up to 8 lies
+    // between a real and its upward rounding), so K = RU(8w + 1.5 * 2^23 - 1) is
+    // 1.5 * 2^23 + ceil(t' - r).
+    const float F = sr_one_plus(d, e);
+    const float c = __fmaf_rn(F, -16.0f, 16.125f);
+    constexpr float inv8step = (G == kE1M2) ? 0.25f : 0.125f;
+    float w;
+    asm("fma.rp.sat.f32 %0, %1, %2, %3;" : "=f"(w) : "f"(fabsf(q)), "f"(inv8step), "f"(c));
+    K = __fmaf_ru(w, 8.0f, 12582911.0f);
+  }
+  return __float_as_uint(K);
+}
+
+// sum over j = 0..7 of 0x4B400000 * 16^j, modulo 2^32
+constexpr uint32_t kSrBias = 0x4B400000u + (0x4B400000u << 4) + (0x4B400000u << 8) +
                              (0x4B400000u << 12) + (0x4B400000u << 16) + (0x4B400000u << 20) +
                              (0x4B400000u << 24) + (0x4B400000u << 28);
+
+// Appends element e's code to a word built from element 7 down to 0: mags accumulates
+// sum bits_j * 16^j, signs the raw values' sign bits at bit 3 of each nibble (sign-magnitude
+// grids); INT4 takes -k in two's complement for a negative raw value.
+template <int G>
+__device__ __forceinline__ void sr_append(uint32_t bits, float raw, uint32_t& mags, uint32_t& signs) {
+  if constexpr (G == kINT4) {
+    const uint32_t m = (uint32_t)((int32_t)__float_as_uint(raw) >> 31);
+    mags = mags * 16u + (((bits ^ m) - m) & 0xFu);
+  } else {
+    mags = mags * 16u + bits;
+    signs = __funnelshift_l(__float_as_uint(raw), signs, 4);
+  }
+}
+
+template <int G>
+__device__ __forceinline__ uint32_t sr_word(uint32_t mags, uint32_t signs) {
+  if constexpr (G == kINT4) return mags;
+  else return (mags - kSrBias) | (signs & 0x88888888u);
+}
+
+// Codes of a nonzero block from its quotients q, draw words d (sr_words16) and raw values raw
+// (element e of the block, for the signs).
+template <int G>
+__device__ __forceinline__ uint2 sr_codes(const float* q, const uint32_t* d, const float* raw) {
   uint32_t w[2];
 #pragma unroll
   for (int l = 0; l < 2; ++l) {
     uint32_t mags = 0u, signs = 0u;
 #pragma unroll
-    for (int j = 7; j >= 0; --j) {
-      const int e = 8 * l + j;
-      float K;
-      if constexpr (kIsE2M1<G>) {
-        const float a = fminf(fabsf(q[e]), qmax);
-        const float r = __fmaf_rn(sr_one_plus(d, e), 128.0f, -128.0f);   // u * 2^-16, exact
-        const bool lo = a < 2.0f, mid = a < 4.0f;
-        const float inv_step = lo ? 2.0f : (mid ? 1.0f : 0.5f);
-        const float base = lo ? 12582912.0f : (mid ? 12582914.0f : 12582916.0f);
-        K = __fadd_ru(__fmaf_ru(a, inv_step, -r), base);
-      } else {
-        // uniform grids, t = |v| / step with qmax = 7 steps: F = 1 + u * 2^-23 (the draw in the
-        // low mantissa bits, one byte permute of its word), c = 16.125 - 16 F = (1 - r) / 8 exactly;
-        // w = min(RU((t - r + 1) / 8), 1) (the saturation is the clamp at qmax: t' = min(t, 7));
-        // 8w = RU(t' - r + 1), whose ceiling is ceil(t' - r) + 1 (no integer up to 8 lies
-        // between a real and its upward rounding), so K = RU(8w + 1.5 * 2^23 - 1) is
-        // 1.5 * 2^23 + ceil(t' - r).
-        const float F = sr_one_plus(d, e);
-        const float c = __fmaf_rn(F, -16.0f, 16.125f);
-        constexpr float inv8step = (G == kE1M2) ? 0.25f : 0.125f;
-        float w;
-        asm("fma.rp.sat.f32 %0, %1, %2, %3;" : "=f"(w) : "f"(fabsf(q[e])), "f"(inv8step), "f"(c));
-        K = __fmaf_ru(w, 8.0f, 12582911.0f);
-      }
-      const uint32_t bits = __float_as_uint(K);   // 0x4B400000 + magnitude code
-      if constexpr (G == kINT4) {
-        const uint32_t m = (uint32_t)((int32_t)__float_as_uint(elem_x(P, e)) >> 31);
-        mags = mags * 16u + (((bits ^ m) - m) & 0xFu);   // two's complement nibble
-      } else {
-        mags = mags * 16u + bits;
-        signs = __funnelshift_l(__float_as_uint(elem_x(P, e)), signs, 4);
-      }
-    }
-    if constexpr (G == kINT4) {
-      w[l] = mags;
-    } else {
-      w[l] = (mags - kBias) | (signs & 0x88888888u);
-    }
+    for (int j = 7; j >= 0; --j) sr_append<G>(sr_bits<G>(q[8 * l + j], d, 8 * l + j), raw[8 * l + j], mags, signs);
+    w[l] = sr_word<G>(mags, signs);
   }
   return make_uint2(w[0], w[1]);
 }
@@ -332,11 +346,110 @@ template <int G>
 __device__ __forceinline__ uint2 encode_sr(const float2* P, float s, float c, uint64_t seedx,
                                           uint64_t quad0) {
   if (s == 0.0f) return make_uint2(0u, 0u);
-  float q[16];
+  float q[16], raw[16];
   sr_quotients(P, s, c, q);
+#pragma unroll
+  for (int e = 0; e < 16; ++e) raw[e] = elem_x(P, e);
   uint32_t d[8];
   sr_words16(seedx, quad0, d);
-  return sr_codes<G>(q, d, P);
+  return sr_codes<G>(q, d, raw);
+}
+
+// ------------------------------------------------------------------ two blocks at once
+//
+// Two blocks of one thread held as A[i] = (element i of block 0, element i of block 1),
+// i = 0..15: every butterfly stage pairs A[i] with A[i+h] and runs as packed f32x2 operations
+// (the same IEEE operations in the same stage order as fwht16, for both blocks at once), and the
+// quotients of both blocks come from one packed correction step with a divisor per lane.
+
+__device__ __forceinline__ void fwht16_pair(float2* A) {
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if ((i & h) == 0) {
+        const float2 a = A[i], b = A[i + h];
+        A[i] = add2(a, b);
+        A[i + h] = sub2(a, b);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ float2 absmax16_pair(const float2* A) {
+  float m0 = max3(fabsf(A[0].x), fabsf(A[1].x), fabsf(A[2].x));
+  float m1 = max3(fabsf(A[0].y), fabsf(A[1].y), fabsf(A[2].y));
+#pragma unroll
+  for (int i = 3; i < 15; i += 2) {
+    m0 = max3(m0, fabsf(A[i].x), fabsf(A[i + 1].x));
+    m1 = max3(m1, fabsf(A[i].y), fabsf(A[i + 1].y));
+  }
+  return make_float2(fmaxf(m0, fabsf(A[15].x)), fmaxf(m1, fabsf(A[15].y)));
+}
+
+// Stochastic-rounding codes of one block given as lane h of A, exactly as encode_sr gives them
+// (the path for blocks with quotients below the correction step's exact range).
+// Not inlined: the rare path must not take registers from the common one.
+template <int G>
+__device__ __noinline__ uint2 encode_sr_lane(const float2* A, int h, float s, float c,
+                                             uint64_t seedx, uint64_t quad0) {
+  if (s == 0.0f) return make_uint2(0u, 0u);
+  float2 P[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    P[i] = h ? make_float2(A[i].y, A[i + 8].y) : make_float2(A[i].x, A[i + 8].x);
+  return encode_sr<G>(P, s, c, seedx, quad0);
+}
+
+// Stochastic-rounding codes of the two blocks in A (block k: scale s.k, first logical index
+// 4 quad0_k), each exactly what encode_sr gives for it alone; c: 4 with rotation, else 1. Both
+// blocks' quotients come from one packed correction step and go straight into their decisions;
+// a block with a quotient below the step's exact range (2^-19, rare) is redone by encode_sr.
+template <int G>
+__device__ __forceinline__ void encode_sr_pair(const float2* A, float2 s, float c, uint64_t seedx,
+                                               uint64_t quad0_0, uint64_t quad0_1, uint2& w0,
+                                               uint2& w1) {
+  const bool z0 = s.x == 0.0f, z1 = s.y == 0.0f;
+  // a zero block's lane divides by 1 (its codes are zeros whatever its quotients)
+  const Divider d0 = make_divider(z0 ? 1.0f : s.x, c), d1 = make_divider(z1 ? 1.0f : s.y, c);
+  if (!(d0.fast && d1.fast)) {
+    w0 = encode_sr_lane<G>(A, 0, s.x, c, seedx, quad0_0);
+    w1 = encode_sr_lane<G>(A, 1, s.y, c, seedx, quad0_1);
+    return;
+  }
+  uint32_t r0[8], r1[8];
+  sr_words16(seedx, quad0_0, r0);
+  sr_words16(seedx, quad0_1, r1);
+  const float2 R2 = make_float2(d0.R, d1.R), nS2 = make_float2(-d0.S, -d1.S);
+  float m0 = 0x1p+30f, m1 = 0x1p+30f;
+  uint32_t c0[2], c1[2];
+#pragma unroll
+  for (int l = 0; l < 2; ++l) {
+    uint32_t ma0 = 0u, sg0 = 0u, ma1 = 0u, sg1 = 0u;
+#pragma unroll
+    for (int j = 7; j >= 0; j -= 2) {
+      const int e = 8 * l + j;
+      float2 q[2];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const float2 q0 = __fmul2_rn(A[e - t], R2);
+        q[t] = __ffma2_rn(__ffma2_rn(q0, nS2, A[e - t]), R2, q0);
+      }
+      m0 = min3(m0, fabsf(q[0].x), fabsf(q[1].x));
+      m1 = min3(m1, fabsf(q[0].y), fabsf(q[1].y));
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        sr_append<G>(sr_bits<G>(q[t].x, r0, e - t), A[e - t].x, ma0, sg0);
+        sr_append<G>(sr_bits<G>(q[t].y, r1, e - t), A[e - t].y, ma1, sg1);
+      }
+    }
+    c0[l] = sr_word<G>(ma0, sg0);
+    c1[l] = sr_word<G>(ma1, sg1);
+  }
+  w0 = z0 ? make_uint2(0u, 0u) : make_uint2(c0[0], c0[1]);
+  w1 = z1 ? make_uint2(0u, 0u) : make_uint2(c1[0], c1[1]);
+  if (m0 < 0x1p-19f && !z0) w0 = encode_sr_lane<G>(A, 0, s.x, c, seedx, quad0_0);
+  if (m1 < 0x1p-19f && !z1) w1 = encode_sr_lane<G>(A, 1, s.y, c, seedx, quad0_1);
 }
 
 // IF4 block, E4M3 block scale (NVFP4's), codes only: the E2M1 candidate (round to nearest even,
