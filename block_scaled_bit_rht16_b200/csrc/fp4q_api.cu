@@ -1,6 +1,7 @@
 // fp4q_api.cu -- the C ABI declared in include/fp4q.h: host-side validation, workspace layout
 // and kernel dispatch. Every argument is checked before anything is enqueued; a rejected call
 // launches nothing.
+#include <climits>
 #include <cmath>
 #include <cstring>
 
@@ -73,8 +74,8 @@ int block_elems(const fp4q_config* cfg) { return cfg->scale == FP4Q_SCALE_UE8M0_
 
 size_t stats_bytes() { return (size_t)kStatsCtas * ST_LEN * sizeof(double); }
 
-// Largest M and N of fp4q_quantize_dual: its tile copies address dY with 32-bit signed
-// coordinates, and a tile reaches 128 rows / 64 columns past its start.
+// Largest M and N of fp4q_quantize_dual (and its 128 x 64 tiles must number below 2^31: one CTA
+// each on the grid's x axis).
 constexpr int64_t kDualMaxDim = (int64_t(1) << 31) - 128;
 
 fp4q_status check_shape(int64_t rows, int64_t cols, int64_t ld, int unit) {
@@ -312,7 +313,8 @@ fp4q_status fp4q_quantize_dual(const fp4q_config* row_cfg, const fp4q_config* co
   if (row_cfg->grid != col_cfg->grid) return FP4Q_ERR_UNSUPPORTED;
   if (row_cfg->e2m1_max != 0u || col_cfg->e2m1_max != 0u) return FP4Q_ERR_UNSUPPORTED;
   if (M < 0 || N < 0 || M % 16 != 0 || N % 16 != 0) return FP4Q_ERR_SHAPE;
-  if (M > kDualMaxDim || N > kDualMaxDim) return FP4Q_ERR_SHAPE;   // 32-bit tile coordinates
+  if (M > kDualMaxDim || N > kDualMaxDim) return FP4Q_ERR_SHAPE;
+  if (((M + 127) / 128) * ((N + 63) / 64) > INT32_MAX) return FP4Q_ERR_SHAPE;   // one CTA per tile
   if (M > 0 && N > 0 && ld < N) return FP4Q_ERR_SHAPE;
   if (M > 1 && N > 0 && ld % 8 != 0) return FP4Q_ERR_ALIGN;
   const bool empty = M == 0 || N == 0;
@@ -440,6 +442,25 @@ fp4q_status fp4q_check_division(uint64_t seed, uint64_t n, unsigned long long* m
 fp4q_status fp4q_device_status(int32_t* status_bits, int32_t clear, fp4q_stream_t stream) {
   if (status_bits == nullptr || (clear != 0 && clear != 1)) return FP4Q_ERR_INVALID_ARG;
   return cuda_status(read_device_status(status_bits, clear != 0, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fp4q_status fp4q_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_tensor_scale,
+                            const uint8_t* b_codes, const uint8_t* b_scales, const float* b_tensor_scale,
+                            int64_t M, int64_t N, int64_t K, void* out, int64_t ldo,
+                            fp4q_stream_t stream) {
+  if (M < 0 || N < 0 || K < 256 || M % 128 != 0 || N % 128 != 0 || K % 256 != 0) return FP4Q_ERR_SHAPE;
+  if (M / 128 > 65535 || K > (int64_t(1) << 31)) return FP4Q_ERR_SHAPE;
+  if (M > 0 && N > 0 && ldo < N) return FP4Q_ERR_SHAPE;
+  if (M == 0 || N == 0) return FP4Q_OK;
+  if (a_codes == nullptr || a_scales == nullptr || a_tensor_scale == nullptr || b_codes == nullptr ||
+      b_scales == nullptr || b_tensor_scale == nullptr || out == nullptr)
+    return FP4Q_ERR_INVALID_ARG;
+  if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_scales, 16) || !aligned(b_scales, 16) ||
+      !aligned(out, 16) || ldo % 8 != 0 || !aligned(a_tensor_scale, 4) || !aligned(b_tensor_scale, 4))
+    return FP4Q_ERR_ALIGN;
+  return cuda_status(launch_gemm_nvfp4(a_codes, a_scales, a_tensor_scale, b_codes, b_scales, b_tensor_scale,
+                                       M, N, K, static_cast<uint16_t*>(out), ldo,
+                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
 fp4q_status fp4q_check_conversions(unsigned long long* mismatches, fp4q_stream_t stream) {

@@ -90,7 +90,6 @@ struct DualArgs {
   uint64_t seedx_row, seedx_col;
   int round_row, round_col;   // per orientation
   int grid_row, grid_col;
-  int32_t* status;            // the library's device status word (a wait that gives up sets bit 0)
 };
 
 // Host: the per-element flips at bit 31 from sign words sw (bit 15: element 2k, bit 31:
@@ -102,9 +101,9 @@ inline void sign_flips(const uint32_t* sw, uint32_t* flip_lo, uint32_t* flip_hi)
   }
 }
 
-// Bits of the device status word (defined in fp4q_row.cu): bit 0 a bounded wait in a quantize
-// kernel gave up (the dual kernel's waits on its tile copies), bit 1 the timeout self-test fired.
-// Sticky until read with clear.
+// Bits of the device status word (defined in fp4q_row.cu): bit 0 a bounded wait in a kernel gave
+// up (the GEMM's waits on its tile copies and MMAs), bit 1 the timeout self-test fired. Sticky
+// until read with clear.
 constexpr int32_t kStatusWaitTimeout = 1;
 constexpr int32_t kStatusSelfTest = 2;
 
@@ -129,5 +128,9 @@ cudaError_t launch_wait_timeout_check(unsigned long long limit_ns, cudaStream_t 
 cudaError_t launch_conversion_check(unsigned long long* bad, cudaStream_t st);
 cudaError_t read_device_status(int32_t* out, bool clear, cudaStream_t st);
 cudaError_t device_status_word(int32_t** out);
+cudaError_t launch_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_ts,
+                              const uint8_t* b_codes, const uint8_t* b_scales, const float* b_ts,
+                              int64_t M, int64_t N, int64_t K, uint16_t* out, int64_t ldo,
+                              cudaStream_t st);
 
 }  // namespace fp4q

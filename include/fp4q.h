@@ -178,9 +178,8 @@ fp4q_status fp4q_rht_quantize(const fp4q_config* cfg, const void* x, int64_t row
  *  codes_col  uint8 [N, M/2], scales_col float [N, M/16]: blocks along M, i.e. dy^T
  *             quantized along its rows (col_cfg; SR index n * M + m).
  * Both configs must use FP4Q_SCALE_FP32_1x16 and no dequant/stats outputs; M and N must be
- * multiples of 16 and at most 2^31 - 128 (else FP4Q_ERR_SHAPE). workspace may be NULL. The first
- * call on a device, and the first with each configuration, looks up cached launch parameters;
- * make it outside any stream capture. */
+ * multiples of 16, at most 2^31 - 128, and (M/128) * (N/64) (rounded up) below 2^31 (else
+ * FP4Q_ERR_SHAPE). workspace may be NULL. */
 fp4q_status fp4q_quantize_dual(const fp4q_config* row_cfg, const fp4q_config* col_cfg,
                                const void* dy, int64_t M, int64_t N, int64_t ld,
                                uint8_t* codes_row, void* scales_row, uint8_t* codes_col,
@@ -257,6 +256,25 @@ fp4q_status fp4q_rht_quantize_grouped(const fp4q_config* cfg, const void* x, int
                                       float* tensor_scales, int32_t tensor_scales_given,
                                       void* workspace, size_t workspace_bytes,
                                       fp4q_stream_t stream);
+
+/* NVFP4 GEMM on the tensor cores (tcgen05 block-scaled MMA, sm_100a), consuming the quantizer's
+ * outputs unchanged: out[m, n] = alpha_a * alpha_b * sum_k A[m, k] B[n, k] (bf16, RNE), where A and B
+ * are the E2M1 codes of two NVFP4 quantizations along K (fp4q_rht_quantize with grid E2M1,
+ * FP4Q_SCALE_E4M3_1x16_TENSOR and FP4Q_OUT_SCALES_MMA) times their E4M3 block scales, and alpha_a,
+ * alpha_b their FP32 tensor scales ("低精度量化技术：IF4…", section 3.2: the two-level NVFP4 scale
+ * of the hardware path; both operands rotated with the same sign mask keep A B^T, since the
+ * 16-point rotation is orthogonal). Products accumulate in FP32.
+ *  a_codes uint8 [M, K/2], a_scales uint8 [M, K/16] in the MMA layout, a_tensor_scale one device
+ *  float; b_* the same with N rows; out bf16 [M, ldo], ldo >= N, ldo % 8 == 0.
+ *  M and N multiples of 128 (M at most 65535 * 128), K a multiple of 256 (else FP4Q_ERR_SHAPE);
+ *  every pointer 16-byte aligned (tensor scales 4) (else FP4Q_ERR_ALIGN); a null pointer:
+ *  FP4Q_ERR_INVALID_ARG. The first call on a device looks up cached launch parameters; make it
+ *  outside any stream capture. A tile whose bounded waits (2 s) give up is left incomplete and
+ *  sets bit 0 of the device status word (fp4q_device_status). */
+fp4q_status fp4q_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales,
+                            const float* a_tensor_scale, const uint8_t* b_codes,
+                            const uint8_t* b_scales, const float* b_tensor_scale, int64_t M,
+                            int64_t N, int64_t K, void* out, int64_t ldo, fp4q_stream_t stream);
 
 /* Reduce the statistics a previous fp4q_rht_quantize / fp4q_if4_select call with
  * FP4Q_OUT_STATS left in `workspace` (in a fixed order, FP64), copy them to *host_out and

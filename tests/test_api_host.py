@@ -139,8 +139,9 @@ def test_dual_dequant_rht_stats_validation():
         ctypes.byref(rc), ctypes.byref(cc), dy, M, N, ld, cr, FAKE, FAKE, FAKE, None, 0, None)
     assert dual(M=24) == _lib.FP4Q_ERR_SHAPE
     assert dual(N=40, ld=40) == _lib.FP4Q_ERR_SHAPE
-    assert dual(M=2 ** 31) == _lib.FP4Q_ERR_SHAPE              # beyond 32-bit tile coordinates
+    assert dual(M=2 ** 31) == _lib.FP4Q_ERR_SHAPE
     assert dual(N=2 ** 31, ld=2 ** 31) == _lib.FP4Q_ERR_SHAPE
+    assert dual(M=2 ** 24, N=2 ** 24, ld=2 ** 24) == _lib.FP4Q_ERR_SHAPE   # 2^35 tiles: one CTA each
     assert dual(dy=None) == _lib.FP4Q_ERR_INVALID_ARG
     assert dual(cr=FAKE + 4) == _lib.FP4Q_ERR_ALIGN
     e2 = fq.Config(grid=fq.FP4Q_GRID_E2M1).c()
@@ -264,3 +265,21 @@ def test_binding_rejects_host_tensors_before_any_call():
         fq.stats(torch.zeros(256, dtype=torch.uint8))
     with pytest.raises(TypeError):
         fq.rht_quantize(cfg, torch.zeros((4, 32), dtype=torch.float32))
+
+
+def test_gemm_validation():
+    lib = _lib.load()
+    g = lambda M=128, N=128, K=256, ldo=128, a=FAKE, sa=FAKE, out=FAKE, ts=FAKE: lib.fp4q_gemm_nvfp4(
+        a, sa, ts, FAKE, FAKE, FAKE, M, N, K, out, ldo, None)
+    assert g(M=100) == _lib.FP4Q_ERR_SHAPE            # M not a multiple of 128
+    assert g(N=64) == _lib.FP4Q_ERR_SHAPE
+    assert g(K=128) == _lib.FP4Q_ERR_SHAPE            # K not a multiple of 256
+    assert g(K=0) == _lib.FP4Q_ERR_SHAPE
+    assert g(ldo=64) == _lib.FP4Q_ERR_SHAPE           # ldo < N
+    assert g(M=65536 * 128) == _lib.FP4Q_ERR_SHAPE    # beyond the tile grid's y limit
+    assert g(a=None) == _lib.FP4Q_ERR_INVALID_ARG
+    assert g(ts=None) == _lib.FP4Q_ERR_INVALID_ARG
+    assert g(a=FAKE + 8) == _lib.FP4Q_ERR_ALIGN       # codes 16-byte aligned
+    assert g(sa=FAKE + 4) == _lib.FP4Q_ERR_ALIGN
+    assert g(ldo=132) == _lib.FP4Q_ERR_ALIGN          # 16-byte output rows
+    assert g(M=0) == _lib.FP4Q_OK                     # empty: nothing to do
