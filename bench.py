@@ -513,7 +513,7 @@ def make_workload(name, sign_mask_from_seed=None):
         if name == "linear1.5b-ufp4-unfused":
             return RowWorkload(name, desc + " -- unfused: rotation pass to bf16, then quantize",
                                stacked_operands, cfg, "rht16_kernel+lean_kernel", unfused=True)
-        return RowWorkload(name, desc, stacked_operands, cfg, "lean_kernel<E1M2,rotation,flat>")
+        return RowWorkload(name, desc, stacked_operands, cfg, "lean_pair_kernel<E1M2,rotation>")
     if name == "dy8192-row-sr":
         mask = sign_mask_from_seed(synth.sign_seed(3))
         rc = fq.recipe("ufp4", "bwd_dx", "dy", sign_mask=mask, sr_seed=synth.SR_SEED)
@@ -575,8 +575,8 @@ def make_workload(name, sign_mask_from_seed=None):
             inp = dense_inp
             desc = "dense [32768,8192] N(0,1)"
         desc += ", %s fwd_y" % ("UFP4 RHT16+E1M2" if ufp4 else "E2M1 baseline (no rotation)")
-        return RowWorkload(name, desc, inp, cfg, "lean_kernel<%s,%s,flat>" % ("E1M2" if ufp4 else "E2M1",
-                                                                            "rotation" if ufp4 else "no-rotation"))
+        key = "lean_pair_kernel<E1M2,rotation>" if ufp4 else "lean_kernel<E2M1,no-rotation,flat>"
+        return RowWorkload(name, desc, inp, cfg, key)
     raise ValueError(name)
 
 

@@ -338,10 +338,14 @@ __device__ __forceinline__ void sr_draws16(uint64_t seedx, uint64_t quad0, uint3
   for (int e = 0; e < 16; ++e) u[e] = (e & 1) ? (d[e >> 1] >> 16) : (d[e >> 1] & 0xFFFFu);
 }
 
-// 1 + u * 2^-23 for element e's draw u (the draw in the low mantissa bits): one byte permute
-// of the word that holds it.
+// 1 + u * 2^-23 for element e's draw u (the draw in the low mantissa bits). The 16-bit field is
+// extracted with the integer multiplier (x * 2^16 to drop the high half, the high word of
+// x * 2^16 to shift it down) rather than a byte permute: the pass that uses it is bound by the
+// integer ALU pipe, and the multiplies issue on the FMA pipe.
 __device__ __forceinline__ float sr_one_plus(const uint32_t* d, int e) {
-  return __uint_as_float(__byte_perm(d[e >> 1], 0x3F800000u, (e & 1) ? 0x7632 : 0x7610));
+  const uint32_t w = d[e >> 1];
+  const uint32_t x = (e & 1) ? w : w * 65536u;
+  return __uint_as_float(__umulhi(x, 65536u) + 0x3F800000u);
 }
 
 // Round-up decision r < frac with r = u * 2^-16, taken exactly as u < frac * 2^16 (both sides

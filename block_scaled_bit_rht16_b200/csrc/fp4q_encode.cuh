@@ -215,6 +215,40 @@ __device__ __forceinline__ uint2 encode_lean_dv(const float2* P, float s, const 
   return make_uint2(w[0], w[1]);
 }
 
+// Round-to-nearest codes of a nonzero block from its exact quotients q[e] (v / 4 for E1M2, the
+// divisor of lean_divisor_factor) and raw values raw[e] (for the signs without rotation): the
+// code step of encode_lean_dv for the FP32 scale, on quotients computed elsewhere.
+template <int G, bool RHT>
+__device__ __forceinline__ uint2 lean_codes(const float* q, const float* raw) {
+  float v[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) v[e] = (!RHT && G != kINT4) ? with_sign_of(q[e], raw[e]) : q[e];
+  uint32_t w[2];
+  if constexpr (kIsE2M1<G>) {
+#pragma unroll
+    for (int l = 0; l < 2; ++l) {
+      uint32_t b[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = cvt_e2m1x2(v[8 * l + 2 * j + 1], v[8 * l + 2 * j]);
+      w[l] = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+    }
+  } else if constexpr (G == kE1M2) {
+    w[0] = e1m2_word(v);
+    w[1] = e1m2_word(v + 8);
+  } else {
+    uint32_t t0[8], t1[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 t = __fadd2_rn(make_float2(v[i], v[i + 8]), make_float2(12582912.0f, 12582912.0f));
+      t0[i] = __float_as_uint(t.x);
+      t1[i] = __float_as_uint(t.y);
+    }
+    w[0] = pack_low_nibbles(t0);
+    w[1] = pack_low_nibbles(t1);
+  }
+  return make_uint2(w[0], w[1]);
+}
+
 template <int G, bool RHT, bool CLAMP = false>
 __device__ __forceinline__ uint2 encode_lean(const float2* P, float s, float amax_raw = 0.0f) {
   if (s == 0.0f) return make_uint2(0u, 0u);

@@ -9,16 +9,19 @@
 // scale); "FP4 训练 vs FP4 推理" (reports.10n1j.top) notes that Blackwell's FP4 tensor-core path
 // is E2M1-only.
 //
-// One CTA computes a 128 x 128 tile of D with 128 threads. Thread 0 streams the K dimension in
-// 256-element steps through a ring of kStages shared-memory buffers: per step the A and B code
-// tiles (128 rows x 128 bytes each) arrive by 2-D TMA copies with the 128-byte swizzle, and the
-// two 2 KB scale blocks (four 512-byte MMA-layout tiles each) by 1-D bulk copies, all completing
-// on the buffer's mbarrier. It then copies the scales into tensor memory (tcgen05.cp, 32 lanes x
-// 128 bits, replicated to the four lane quarters) and issues four MMAs of K = 64
-// (tcgen05.mma kind::mxf4nvf4, block16 scaling, M = 128, N = 128), and tcgen05.commit arrives
-// on the buffer's release barrier when they have read it. The accumulator is 128 lanes x 128
-// FP32 columns of tensor memory; after the last step every warp reads its 32 lanes back
-// (tcgen05.ld), scales by alpha_A alpha_B and stores bf16. Every mbarrier wait is bounded by the
+// One CTA computes a 128 x BN tile of D (BN = 256 when N allows, else 128) with 128 threads,
+// one CTA per SM (217 KB of shared memory, 512 tensor-memory columns). The K dimension streams in
+// 256-element steps through a ring of shared-memory buffers, with two specialised threads:
+//   thread 0 (producer): per step the A and B code tiles (128 / BN rows x 128 bytes) by 2-D TMA
+//     copies with the 128-byte swizzle, and the scale blocks (four 512-byte MMA-layout tiles per
+//     128 rows) by 1-D bulk copies, all completing on the buffer's `full` mbarrier; a buffer is
+//     refilled once its `empty` barrier says the MMAs that read it have completed;
+//   thread 32 (MMA issuer, warp 1): copies the step's scales into tensor memory (tcgen05.cp,
+//     32 lanes x 128 bits, replicated to the four lane quarters), issues four MMAs of K = 64
+//     (tcgen05.mma kind::mxf4nvf4, block16 scaling, M = 128, N = BN) and commits them to the
+//     buffer's `empty` barrier.
+// The accumulator is 128 lanes x BN FP32 columns of tensor memory; after the last step every warp
+// reads its 32 lanes back (tcgen05.ld), scales by alpha_A alpha_B and stores bf16. Every mbarrier wait is bounded by the
 // global timer; a wait that gives up sets bit 0 of the library's device status word and the CTA
 // skips the rest of its work (its outputs are then incomplete), releasing its tensor memory.
 // No copy uses cluster multicast.
@@ -36,25 +39,39 @@
 namespace fp4q {
 namespace {
 
-constexpr int kBM = 128, kBN = 128, kBKBytes = 128;   // 256 FP4 values per row per step
-constexpr int kGStages = 4;
+constexpr int kBM = 128, kBKBytes = 128;   // 256 FP4 values per row per step
 constexpr int kGThreads = 128;
-constexpr uint32_t kTileA = kBM * kBKBytes, kTileB = kBN * kBKBytes;   // 16 KB each
-constexpr uint32_t kSfBytes = 4 * 512;                                 // 4 K-blocks of 64
-constexpr uint32_t kStageTx = kTileA + kTileB + 2 * kSfBytes;
-constexpr uint32_t kTmemCols = 256;   // 128 accumulator + kGStages x 2 x 16 scale columns
+constexpr uint32_t kTileA = kBM * kBKBytes;   // 16 KB
+constexpr uint32_t kSfTile = 4 * 512;         // one 128-row scale tile row: 4 K-blocks of 64
 
+// Per tile width BN (128 or 256): stages, shared memory, tensor memory.
+template <int BN>
+struct GemmCfg {
+  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr uint32_t kTileB = BN * kBKBytes;
+  static constexpr uint32_t kSfB = (BN / 128) * kSfTile;
+  static constexpr uint32_t kStageTx = kTileA + kTileB + kSfTile + kSfB;
+  static constexpr uint32_t kSfCols = 16 + BN / 8;   // A: 4 K-blocks x 4 columns; B: 4 x BN/32
+  static constexpr uint32_t kTmemCols = (BN + kStages * kSfCols) <= 256 ? 256 : 512;
+  // kind::mxf4nvf4: E2M1 A and B (format 1), K-major, N / 8 in bits 17-22, UE4M3 scales (bit 23
+  // = 0), M / 16 in bits 24-28, scale-factor ids 0, K = 64
+  static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+};
+
+template <int BN>
 struct GemmSmem {
-  uint8_t a[kGStages][kTileA];      // 1024-byte aligned (swizzle period)
-  uint8_t b[kGStages][kTileB];
-  uint8_t sfa[kGStages][kSfBytes];
-  uint8_t sfb[kGStages][kSfBytes];
-  uint64_t full[kGStages];
-  uint64_t empty[kGStages];
+  using C = GemmCfg<BN>;
+  uint8_t a[C::kStages][kTileA];      // 1024-byte aligned (swizzle period)
+  uint8_t b[C::kStages][C::kTileB];
+  uint8_t sfa[C::kStages][kSfTile];
+  uint8_t sfb[C::kStages][C::kSfB];
+  uint64_t full[C::kStages];
+  uint64_t empty[C::kStages];
   uint64_t done;
   uint32_t tmem_base;
 };
-constexpr size_t kGemmSmemBytes = sizeof(GemmSmem) + 1024;
+template <int BN>
+constexpr size_t gemm_smem_bytes() { return sizeof(GemmSmem<BN>) + 1024; }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(
@@ -79,25 +96,29 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
 }
 
-// Instruction descriptor of kind::mxf4nvf4 with E2M1 A and B (format 1), K-major A and B, N / 8
-// in bits 17-22, UE4M3 scales (bit 23 = 0), M / 16 in bits 24-28, scale-factor ids 0, K = 64.
-constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               ::"r"(smem_u32(bar)) : "memory");
+}
 
+template <int BN>
 __global__ void __launch_bounds__(kGThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb,
                       const float* __restrict__ ts_a, const float* __restrict__ ts_b,
                       __nv_bfloat16* __restrict__ out, int64_t ldo, int64_t K, int32_t* status) {
+  using C = GemmCfg<BN>;
+  constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
-  GemmSmem& sm = *reinterpret_cast<GemmSmem*>(
+  GemmSmem<BN>& sm = *reinterpret_cast<GemmSmem<BN>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int64_t m0 = (int64_t)blockIdx.y * kBM, n0 = (int64_t)blockIdx.x * kBN;
+  const int64_t m0 = (int64_t)blockIdx.y * kBM, n0 = (int64_t)blockIdx.x * BN;
   const int ksteps = (int)(K / 256);
   const int64_t kb64 = K / 64;   // scale tiles (of 4 K-blocks of 16) per 128-row tile row
 
   if (t == 0) {
-    for (int s = 0; s < kGStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
     }
@@ -106,7 +127,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
   }
   if (warp == 0) {   // tensor memory for the accumulator and the staged scales
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                 ::"r"(smem_u32(&sm.tmem_base)), "r"(kTmemCols) : "memory");
+                 ::"r"(smem_u32(&sm.tmem_base)), "r"(C::kTmemCols) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -114,36 +135,44 @@ __global__ void __launch_bounds__(kGThreads, 1)
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   pdl_enter();
   const uint32_t tmem = sm.tmem_base;
-  const uint32_t tmem_acc = tmem;                 // lanes 0..127, columns 0..127
-  const uint32_t tmem_sf = tmem + kBN;            // then kGStages x (A: 16, B: 16) columns
+  const uint32_t tmem_acc = tmem;                 // lanes 0..127, columns 0..BN-1
+  const uint32_t tmem_sf = tmem + BN;             // then S x (A: 16, B: BN/8) columns
 
   int fail = 0;
+  int issued = 0;   // producer: steps whose copies have been issued
   if (t == 0) {
+    // producer: refills a buffer once the MMAs that read it have completed
     const uint8_t* sfa_row = sfa + (m0 / 128) * kb64 * 512;
-    const uint8_t* sfb_row = sfb + (n0 / 128) * kb64 * 512;
-    auto issue = [&](int kt, int s) {
-      mbar_arrive_expect_tx(&sm.full[s], kStageTx);
+    for (int kt = 0; kt < ksteps; ++kt, ++issued) {
+      const int s = kt % S;
+      if (kt >= S && !mbar_wait(&sm.empty[s], (uint32_t)(((kt / S) - 1) & 1))) { fail = 1; break; }
+      mbar_arrive_expect_tx(&sm.full[s], C::kStageTx);
       tma_load_2d(sm.a[s], &tmA, kt * kBKBytes, (int)m0, &sm.full[s]);
       tma_load_2d(sm.b[s], &tmB, kt * kBKBytes, (int)n0, &sm.full[s]);
-      bulk_load_1d(sm.sfa[s], sfa_row + (int64_t)kt * kSfBytes, kSfBytes, &sm.full[s]);
-      bulk_load_1d(sm.sfb[s], sfb_row + (int64_t)kt * kSfBytes, kSfBytes, &sm.full[s]);
-    };
-    int issued = 0;   // steps whose copies have been issued
-    for (; issued < kGStages && issued < ksteps; ++issued) issue(issued, issued);
-    int kt = 0;
-    for (; kt < ksteps; ++kt) {
-      const int s = kt % kGStages;
-      const uint32_t ph = (uint32_t)((kt / kGStages) & 1);
-      if (!mbar_wait(&sm.full[s], ph)) { fail = 1; break; }
+      bulk_load_1d(sm.sfa[s], sfa_row + (int64_t)kt * kSfTile, kSfTile, &sm.full[s]);
+#pragma unroll
+      for (int j = 0; j < BN / 128; ++j)
+        bulk_load_1d(sm.sfb[s] + j * kSfTile, sfb + ((n0 / 128 + j) * kb64 * 512) + (int64_t)kt * kSfTile,
+                     kSfTile, &sm.full[s]);
+    }
+  } else if (t == 32) {
+    // MMA issuer: scales into tensor memory, four MMAs of K = 64 per step
+    for (int kt = 0; kt < ksteps; ++kt) {
+      const int s = kt % S;
+      if (!mbar_wait(&sm.full[s], (uint32_t)((kt / S) & 1))) { fail = 1; break; }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t sa = tmem_sf + (uint32_t)s * 32u, sb = sa + 16u;
+      const uint32_t sa = tmem_sf + (uint32_t)s * C::kSfCols, sb = sa + 16u;
 #pragma unroll
       for (int kb = 0; kb < 4; ++kb) {
-        // 512 bytes = 32 rows of 16 bytes, 8-row groups 128 bytes apart
+        // a 512-byte scale tile = 32 rows of 16 bytes, 8-row groups 128 bytes apart
         const uint64_t da = smem_desc(smem_u32(sm.sfa[s] + kb * 512), 16u, 128u, 0u);
-        const uint64_t db = smem_desc(smem_u32(sm.sfb[s] + kb * 512), 16u, 128u, 0u);
         asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(sa + 4u * kb), "l"(da) : "memory");
-        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(sb + 4u * kb), "l"(db) : "memory");
+#pragma unroll
+        for (int j = 0; j < BN / 128; ++j) {
+          const uint64_t db = smem_desc(smem_u32(sm.sfb[s] + j * kSfTile + kb * 512), 16u, 128u, 0u);
+          asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
+                       ::"r"(sb + (uint32_t)(BN / 32) * kb + 4u * j), "l"(db) : "memory");
+        }
       }
 #pragma unroll
       for (int kb = 0; kb < 4; ++kb) {
@@ -154,32 +183,24 @@ __global__ void __launch_bounds__(kGThreads, 1)
         asm volatile(
             "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-            ::"r"(tmem_acc), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(acc), "r"(sa + 4u * kb), "r"(sb + 4u * kb)
+            ::"r"(tmem_acc), "l"(adesc), "l"(bdesc), "r"(C::kIdesc), "r"(acc), "r"(sa + 4u * kb),
+              "r"(sb + (uint32_t)(BN / 32) * kb)
             : "memory");
       }
-      // the buffer is free again once these MMAs have read it
-      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                   ::"r"(smem_u32(&sm.empty[s])) : "memory");
-      if (issued < ksteps) {
-        if (!mbar_wait(&sm.empty[s], ph)) { fail = 1; break; }
-        issue(issued, s);
-        ++issued;
-      }
-    }
-    if (fail) {
-      // drain: the copies still in flight (steps kt + 1 .. issued - 1, and kt's own if its wait
-      // gave up), each wait bounded again
-      for (int j = kt; j < issued; ++j) mbar_wait(&sm.full[j % kGStages], (uint32_t)((j / kGStages) & 1));
+      umma_commit(&sm.empty[s]);   // the buffer is free again once these MMAs have read it
     }
     // arrives when every MMA and scale copy issued above has completed
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                 ::"r"(smem_u32(&sm.done)) : "memory");
+    umma_commit(&sm.done);
   }
-  // the other threads wait at the barrier (not spinning beside thread 0) until every step is
-  // issued; then all wait for the last MMAs (bounded), and a failed wait anywhere reaches every
-  // thread through the second barrier (then nothing reads tensor memory)
+  // the other threads wait at the barrier; a failed wait of the producer or the MMA issuer
+  // reaches every thread through it
   fail = __syncthreads_or(fail);
-  if (!mbar_wait(&sm.done, 0u)) fail = 1;   // thread 0 commits `done` on every path
+  if (fail && t == 0) {
+    // drain: wait (bounded) for the last fill issued into each buffer, steps issued - S ..
+    // issued - 1 (a fill the MMA issuer has consumed has completed, and its wait returns at once)
+    for (int j = issued > S ? issued - S : 0; j < issued; ++j) mbar_wait(&sm.full[j % S], (uint32_t)((j / S) & 1));
+  }
+  if (!mbar_wait(&sm.done, 0u)) fail = 1;   // the MMA issuer commits `done` on every path
   fail = __syncthreads_or(fail);
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   if (fail) {
@@ -187,8 +208,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
   } else {
     const float alpha = __fmul_rn(*ts_a, *ts_b);
     const int64_t row = m0 + 32 * warp + lane;
-#pragma unroll
-    for (int c0 = 0; c0 < kBN; c0 += 32) {
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 32) {
       uint32_t v[32];
       asm volatile(
           "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -214,7 +235,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols) : "memory");
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 gemm_tensor_map_encoder() {
@@ -230,13 +251,13 @@ PFN_cuTensorMapEncodeTiled_v12000 gemm_tensor_map_encoder() {
   return fn;
 }
 
-// 2-D map of a code matrix (uint8 [rows, K/2]) with 128-byte x 128-row boxes, 128-byte swizzle.
-cudaError_t make_codes_map(const uint8_t* codes, int64_t rows, int64_t K, CUtensorMap* map) {
+// 2-D map of a code matrix (uint8 [rows, K/2]) with 128-byte x box_rows boxes, 128-byte swizzle.
+cudaError_t make_codes_map(const uint8_t* codes, int64_t rows, int64_t K, int box_rows, CUtensorMap* map) {
   auto enc = gemm_tensor_map_encoder();
   if (enc == nullptr) return cudaErrorNotSupported;
   const cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-  const cuuint32_t box[2] = {(cuuint32_t)kBKBytes, (cuuint32_t)kBM};
+  const cuuint32_t box[2] = {(cuuint32_t)kBKBytes, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides,
                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -244,7 +265,9 @@ cudaError_t make_codes_map(const uint8_t* codes, int64_t rows, int64_t K, CUtens
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t gemm_prepare(int* ok) {
+// Raises the kernel's shared-memory limit once per (tile width, device).
+template <int BN>
+cudaError_t gemm_prepare() {
   static std::mutex mu;
   static std::map<int, cudaError_t> done;
   int dev = 0;
@@ -253,10 +276,38 @@ cudaError_t gemm_prepare(int* ok) {
   std::lock_guard<std::mutex> lock(mu);
   auto it = done.find(dev);
   if (it == done.end())
-    it = done.emplace(dev, cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                (int)kGemmSmemBytes)).first;
-  *ok = it->second == cudaSuccess;
+    it = done.emplace(dev, cudaFuncSetAttribute(nvfp4_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                (int)gemm_smem_bytes<BN>())).first;
   return it->second;
+}
+
+template <int BN>
+cudaError_t launch_gemm_bn(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_ts,
+                           const uint8_t* b_codes, const uint8_t* b_scales, const float* b_ts,
+                           int64_t M, int64_t N, int64_t K, uint16_t* out, int64_t ldo, cudaStream_t st) {
+  alignas(64) CUtensorMap ma, mb;
+  cudaError_t e = make_codes_map(a_codes, M, K, kBM, &ma);
+  if (e != cudaSuccess) return e;
+  e = make_codes_map(b_codes, N, K, BN, &mb);
+  if (e != cudaSuccess) return e;
+  e = gemm_prepare<BN>();
+  if (e != cudaSuccess) return e;
+  int32_t* status = nullptr;
+  e = device_status_word(&status);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(N / BN), (unsigned)(M / kBM));
+  cfg.blockDim = dim3(kGThreads);
+  cfg.dynamicSmemBytes = gemm_smem_bytes<BN>();
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<BN>, ma, mb, a_scales, b_scales, a_ts, b_ts,
+                         reinterpret_cast<__nv_bfloat16*>(out), ldo, K, status);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace
@@ -266,30 +317,9 @@ cudaError_t launch_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales, c
                               int64_t M, int64_t N, int64_t K, uint16_t* out, int64_t ldo,
                               cudaStream_t st) {
   if (M == 0 || N == 0) return cudaSuccess;
-  alignas(64) CUtensorMap ma, mb;
-  cudaError_t e = make_codes_map(a_codes, M, K, &ma);
-  if (e != cudaSuccess) return e;
-  e = make_codes_map(b_codes, N, K, &mb);
-  if (e != cudaSuccess) return e;
-  int ok = 0;
-  e = gemm_prepare(&ok);
-  if (e != cudaSuccess) return e;
-  int32_t* status = nullptr;
-  e = device_status_word(&status);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(N / kBN), (unsigned)(M / kBM));
-  cfg.blockDim = dim3(kGThreads);
-  cfg.dynamicSmemBytes = kGemmSmemBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel, ma, mb, a_scales, b_scales, a_ts, b_ts,
-                         reinterpret_cast<__nv_bfloat16*>(out), ldo, K, status);
-  return e != cudaSuccess ? e : cudaGetLastError();
+  if (N % 256 == 0)
+    return launch_gemm_bn<256>(a_codes, a_scales, a_ts, b_codes, b_scales, b_ts, M, N, K, out, ldo, st);
+  return launch_gemm_bn<128>(a_codes, a_scales, a_ts, b_codes, b_scales, b_ts, M, N, K, out, ldo, st);
 }
 
 }  // namespace fp4q

@@ -279,6 +279,11 @@ __host__ __device__ inline bool flat_launch(const QuantArgs& a) {
   return a.contiguous && a.vec32 && a.nunits <= kFlatMaxUnits;
 }
 
+// The two-block kernel stores a pair's codes as one 16-byte word and its scales as one 8-byte word.
+inline bool pair_aligned(const QuantArgs& a) {
+  return reinterpret_cast<uintptr_t>(a.codes) % 16 == 0 && reinterpret_cast<uintptr_t>(a.scales) % 8 == 0;
+}
+
 template <int G, bool RHT, bool FLAT, int R>
 __global__ void __launch_bounds__(kThreads) lean_kernel(const QuantArgs a) {
   constexpr float kCinv = RHT ? 0.25f : 1.0f;
@@ -305,6 +310,85 @@ __global__ void __launch_bounds__(kThreads) lean_kernel(const QuantArgs a) {
     __stcs(reinterpret_cast<float*>(a.scales) + u, s);
     lo = nlo;
     hi = nhi;
+  }
+}
+
+// The hot path for a flat tensor with round to nearest: two adjacent blocks per thread per
+// iteration (64 contiguous bytes: two 256-bit loads, one 16-byte code store, one 8-byte scale
+// store), held as A[i] = (element i of the first block, element i of the second) so that every
+// butterfly stage and every quotient step runs as packed f32x2 operations for both blocks -- the
+// same IEEE operations, in the same order, as the one-block kernel. The next pair's loads are in
+// flight while the current pair encodes.
+template <int G, bool RHT>
+__global__ void __launch_bounds__(kThreads) lean_pair_kernel(const QuantArgs a) {
+  constexpr float kCinv = RHT ? 0.25f : 1.0f;
+  constexpr float kF = lean_divisor_factor<G, RHT>();
+  const uint32_t zero_flip[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  pdl_enter();
+  const uint32_t npairs = (uint32_t)(a.nunits >> 1);
+  const uint32_t stride = gridDim.x * kThreads;
+  uint32_t p = blockIdx.x * kThreads + threadIdx.x;
+  uint4 v[4];
+  if (p < npairs) {
+    load16(a.x + (size_t)p * 32, true, v[0], v[1]);
+    load16(a.x + (size_t)p * 32 + 16, true, v[2], v[3]);
+  }
+  for (; p < npairs; p += stride) {
+    uint4 nv[4] = {v[0], v[1], v[2], v[3]};
+    if (p + stride < npairs) {
+      load16(a.x + (size_t)(p + stride) * 32, true, nv[0], nv[1]);
+      load16(a.x + (size_t)(p + stride) * 32 + 16, true, nv[2], nv[3]);
+    }
+    float2 A[16];
+    unpack16_pair(v[0], v[1], v[2], v[3], RHT ? a.flip_lo : zero_flip, RHT ? a.flip_hi : zero_flip, A);
+    if constexpr (RHT) fwht16_pair(A);
+    const float2 am = absmax16_pair(A);
+    const float s0 = div_qmax<G>(__fmul_rn(am.x, kCinv)), s1 = div_qmax<G>(__fmul_rn(am.y, kCinv));
+    // a zero block's lane divides by 1 (its codes are zeros whatever its quotients)
+    const Divider d0 = make_divider(s0 == 0.0f ? 1.0f : s0, kF), d1 = make_divider(s1 == 0.0f ? 1.0f : s1, kF);
+    uint2 w0, w1;
+    if (d0.fast && d1.fast) {
+      const float2 R2 = make_float2(d0.R, d1.R), nS2 = make_float2(-d0.S, -d1.S);
+      float q0[16], q1[16], r0[16], r1[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float2 qa = __fmul2_rn(A[e], R2);
+        const float2 q = __ffma2_rn(__ffma2_rn(qa, nS2, A[e]), R2, qa);
+        q0[e] = q.x;
+        q1[e] = q.y;
+        r0[e] = A[e].x;
+        r1[e] = A[e].y;
+      }
+      w0 = s0 == 0.0f ? make_uint2(0u, 0u) : lean_codes<G, RHT>(q0, r0);
+      w1 = s1 == 0.0f ? make_uint2(0u, 0u) : lean_codes<G, RHT>(q1, r1);
+    } else {
+      float2 P0[8], P1[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        P0[i] = make_float2(A[i].x, A[i + 8].x);
+        P1[i] = make_float2(A[i].y, A[i + 8].y);
+      }
+      w0 = encode_lean<G, RHT>(P0, s0);
+      w1 = encode_lean<G, RHT>(P1, s1);
+    }
+    __stcs(reinterpret_cast<uint4*>(a.codes) + p, make_uint4(w0.x, w0.y, w1.x, w1.y));
+    __stcs(reinterpret_cast<float2*>(a.scales) + p, make_float2(s0, s1));
+    v[0] = nv[0];
+    v[1] = nv[1];
+    v[2] = nv[2];
+    v[3] = nv[3];
+  }
+  // an odd last block
+  if ((a.nunits & 1) && blockIdx.x == 0 && threadIdx.x == 0) {
+    const uint32_t u = (uint32_t)a.nunits - 1u;
+    uint4 lo, hi;
+    load16(a.x + (size_t)u * 16, true, lo, hi);
+    float2 P[8];
+    unpack16(lo, hi, RHT ? a.flip_lo : zero_flip, RHT ? a.flip_hi : zero_flip, P);
+    if constexpr (RHT) fwht16(P);
+    const float s = div_qmax<G>(__fmul_rn(absmax16(P), kCinv));
+    __stcs(reinterpret_cast<uint2*>(a.codes) + u, encode_lean<G, RHT>(P, s));
+    __stcs(reinterpret_cast<float*>(a.scales) + u, s);
   }
 }
 
@@ -820,9 +904,20 @@ cudaError_t launch_lean_nv(const QuantArgs& a, cudaStream_t st) {
   return flat ? launch_lean_nv4<G, false, true, GROUPED>(a, st) : launch_lean_nv4<G, false, false, GROUPED>(a, st);
 }
 
+template <int G, bool RHT>
+cudaError_t launch_lean_pair(const QuantArgs& a, cudaStream_t st) {
+  auto k = lean_pair_kernel<G, RHT>;
+  const cudaError_t e = launch_pdl(k, persistent_grid(k, (a.nunits + 1) / 2), st, a);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 template <int G, int R>
 cudaError_t launch_lean(const QuantArgs& a, cudaStream_t st) {
   const bool rht = a.c != 1.0f, flat = flat_launch(a);
+  // rotated, flat and round to nearest: two blocks per thread when the pair stores are aligned
+  // (79 registers, three CTAs per SM; without the rotation the sign copies push the pair kernel
+  // to 98 registers, so unrotated tensors stay on one block per thread)
+  if (R == kRTNE && rht && flat && pair_aligned(a)) return launch_lean_pair<G, true>(a, st);
   if (rht) return flat ? launch_lean3<G, true, true, R>(a, st) : launch_lean3<G, true, false, R>(a, st);
   return flat ? launch_lean3<G, false, true, R>(a, st) : launch_lean3<G, false, false, R>(a, st);
 }
