@@ -207,26 +207,45 @@ def canonical_code(src):
     return "\n".join(ln for ln in lines if ln)
 
 
-def kernel_source_sha(csrc=None):
-    """Fingerprint of the device sources, to tell whether committed ncu counters still apply.
-    Comments and layout are left out: they cannot change what a kernel does."""
+# The device sources each recorded kernel is built from (its translation unit and the headers
+# it includes); a record's fingerprint covers only these, so that a change to an unrelated
+# kernel leaves it valid.
+ROW_SOURCES = ("fp4q_row.cu", "fp4q_device.cuh", "fp4q_encode.cuh", "fp4q_kernels.cuh")
+DUAL_SOURCES = ("fp4q_dual.cu", "fp4q_device.cuh", "fp4q_encode.cuh", "fp4q_kernels.cuh")
+GEMM_SOURCES = ("fp4q_gemm.cu", "fp4q_device.cuh", "fp4q_kernels.cuh")
+
+
+def kernel_sources(kernel_key):
+    """The device source files of a recorded kernel (by the name the bench reports)."""
+    if kernel_key.startswith("dual_kernel"):
+        return DUAL_SOURCES
+    if kernel_key.startswith("nvfp4_gemm"):
+        return GEMM_SOURCES
+    return ROW_SOURCES
+
+
+def kernel_source_sha(csrc=None, files=None):
+    """Fingerprint of device sources (all of them, or the given files), to tell whether
+    committed ncu counters still apply. Comments and layout are left out: they cannot change
+    what a kernel does."""
     h = hashlib.sha256()
     csrc = csrc or os.path.join(ROOT, "block_scaled_bit_rht16_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")) and name not in HOST_ONLY_SOURCES:
-            with open(os.path.join(csrc, name), encoding="utf-8") as f:
-                code = canonical_code(f.read())
-            h.update(name.encode() + b"\0" + code.encode())
+    names = sorted(files) if files is not None else sorted(
+        n for n in os.listdir(csrc) if n.endswith((".cu", ".cuh")) and n not in HOST_ONLY_SOURCES)
+    for name in names:
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            code = canonical_code(f.read())
+        h.update(name.encode() + b"\0" + code.encode())
     return h.hexdigest()[:16]
 
 
 def profiled_record(kernel_key):
     """The committed ncu record of a kernel (profiles/traffic.json), if it was taken on the
-    current device sources; else None."""
+    kernel's current device sources; else None."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f).get(kernel_key)
-        if rec and rec.get("source_sha") == kernel_source_sha():
+        if rec and rec.get("source_sha") == kernel_source_sha(files=kernel_sources(kernel_key)):
             return rec
     except Exception:
         pass

@@ -412,6 +412,17 @@ __device__ __forceinline__ int group_of(const int64_t* off, int n, int64_t r) {
   return lo;
 }
 
+// The Divider stored in a scale table entry (scale, S, R, fast).
+__device__ __forceinline__ Divider table_divider(const float4& e) {
+  Divider dv;
+  dv.S = e.y;
+  dv.R = e.z;
+  dv.fast = e.w != 0.0f;
+  dv.R2 = make_float2(dv.R, dv.R);
+  dv.nS2 = make_float2(-dv.S, -dv.S);
+  return dv;
+}
+
 // E4M3 block scale + FP32 tensor scale, round to nearest even, codes and scale bytes only.
 // G = kIF4: the per-block FP4 / INT4 choice, flagged in bit 7 of the scale byte.
 // GROUPED: the tensor scale is that of the block's row group (group_ts), looked up again only
@@ -491,11 +502,7 @@ __global__ void __launch_bounds__(kThreads, G == kIF4 ? 3 : (GROUPED ? 1 : 5)) l
     } else {
       const float4 e = s_tab[sbyte];
       s = e.x;
-      dv.S = e.y;
-      dv.R = e.z;
-      dv.fast = e.w != 0.0f;
-      dv.R2 = make_float2(dv.R, dv.R);
-      dv.nS2 = make_float2(-dv.S, -dv.S);
+      dv = table_divider(e);
     }
     uint2 w;
     uint32_t flag = 0u;

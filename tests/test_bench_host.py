@@ -165,6 +165,17 @@ def test_kernel_fingerprint_ignores_comments_and_layout_only():
     assert bench.canonical_code(a) != bench.canonical_code(a.replace("x * 2", "x * 3"))
 
 
+def test_kernel_fingerprint_covers_only_its_sources(tmp_path):
+    for name in ("fp4q_row.cu", "fp4q_device.cuh", "fp4q_encode.cuh", "fp4q_kernels.cuh", "fp4q_gemm.cu"):
+        (tmp_path / name).write_text("int %s_v = 1;\n" % name.split(".")[0])
+    row = bench.kernel_source_sha(str(tmp_path), bench.kernel_sources("lean_pair_kernel<E1M2,rotation>"))
+    (tmp_path / "fp4q_gemm.cu").write_text("int changed = 2;\n")
+    assert bench.kernel_source_sha(str(tmp_path), bench.ROW_SOURCES) == row
+    (tmp_path / "fp4q_encode.cuh").write_text("int changed = 3;\n")
+    assert bench.kernel_source_sha(str(tmp_path), bench.ROW_SOURCES) != row
+    assert bench.kernel_sources("dual_kernel<E1M2,SR,SR>") == bench.DUAL_SOURCES
+
+
 def test_issue_roofline_arithmetic():
     r = bench.issue_roofline(115174472, 0.1396, 148, 1965.0)
     assert r["peak_per_s"] == round(148 * 4 * 1965e6 / 1e9, 1)

@@ -93,7 +93,11 @@ def test_small_ragged(combo, rht, outs):
     full = outs == "all"
     cfg = fq.Config(grid=grid, scale=scale, round=rnd, rht=rht, sign_mask=MASK, sr_seed=0x1234ABCD,
                     dequant=full, stats=full)
-    for rows, cols, kind in [(1, 32, "normal"), (37, 96, "t4"), (130, 1056, "laplace")]:
+    # odd block counts (3, 185) end the two-blocks-per-thread kernels on a single block
+    for rows, cols, kind in [(1, 32, "normal"), (37, 96, "t4"), (130, 1056, "laplace"),
+                             (3, 16, "normal"), (37, 80, "t4")]:
+        if scale == UE8M0 and cols % 32:
+            continue   # 32-element blocks
         x = synth.small(rows * 7 + cols, rows, cols, kind)
         compare_quant(cfg, x, gpu_quantize(cfg, x))
 
