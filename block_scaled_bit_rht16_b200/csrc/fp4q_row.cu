@@ -319,8 +319,24 @@ __global__ void __launch_bounds__(kThreads) lean_kernel(const QuantArgs a) {
 // butterfly stage and every quotient step runs as packed f32x2 operations for both blocks -- the
 // same IEEE operations, in the same order, as the one-block kernel. The next pair's loads are in
 // flight while the current pair encodes.
+// Codes of block u of a flat tensor with FP32 scale s, recomputed from the input (the same loads
+// and operations as the pair kernel's) for a scale outside the correction step's exact range.
+// Not inlined, and handed only the arguments' address (a grid constant) and scalars, so that the
+// rare path takes neither registers nor a stack frame from the common one: the common path then
+// fits 64 registers, four CTAs per SM.
 template <int G, bool RHT>
-__global__ void __launch_bounds__(kThreads) lean_pair_kernel(const QuantArgs a) {
+__device__ __noinline__ uint2 lean_block_slow(const QuantArgs* a, uint32_t u, float s) {
+  const uint32_t zero_flip[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  uint4 lo, hi;
+  load16(a->x + (size_t)u * 16, true, lo, hi);
+  float2 P[8];
+  unpack16(lo, hi, RHT ? a->flip_lo : zero_flip, RHT ? a->flip_hi : zero_flip, P);
+  if constexpr (RHT) fwht16(P);
+  return encode_lean<G, RHT>(P, s);
+}
+
+template <int G, bool RHT>
+__global__ void __launch_bounds__(kThreads, 4) lean_pair_kernel(const __grid_constant__ QuantArgs a) {
   constexpr float kCinv = RHT ? 0.25f : 1.0f;
   constexpr float kF = lean_divisor_factor<G, RHT>();
   const uint32_t zero_flip[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
@@ -362,14 +378,8 @@ __global__ void __launch_bounds__(kThreads) lean_pair_kernel(const QuantArgs a) 
       w0 = s0 == 0.0f ? make_uint2(0u, 0u) : lean_codes<G, RHT>(q0, r0);
       w1 = s1 == 0.0f ? make_uint2(0u, 0u) : lean_codes<G, RHT>(q1, r1);
     } else {
-      float2 P0[8], P1[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        P0[i] = make_float2(A[i].x, A[i + 8].x);
-        P1[i] = make_float2(A[i].y, A[i + 8].y);
-      }
-      w0 = encode_lean<G, RHT>(P0, s0);
-      w1 = encode_lean<G, RHT>(P1, s1);
+      w0 = lean_block_slow<G, RHT>(&a, 2 * p, s0);
+      w1 = lean_block_slow<G, RHT>(&a, 2 * p + 1, s1);
     }
     __stcs(reinterpret_cast<uint4*>(a.codes) + p, make_uint4(w0.x, w0.y, w1.x, w1.y));
     __stcs(reinterpret_cast<float2*>(a.scales) + p, make_float2(s0, s1));
@@ -922,8 +932,8 @@ template <int G, int R>
 cudaError_t launch_lean(const QuantArgs& a, cudaStream_t st) {
   const bool rht = a.c != 1.0f, flat = flat_launch(a);
   // rotated, flat and round to nearest: two blocks per thread when the pair stores are aligned
-  // (79 registers, three CTAs per SM; without the rotation the sign copies push the pair kernel
-  // to 98 registers, so unrotated tensors stay on one block per thread)
+  // (without the rotation the sign copies take the pair kernel past 64 registers, so unrotated
+  // tensors stay on one block per thread)
   if (R == kRTNE && rht && flat && pair_aligned(a)) return launch_lean_pair<G, true>(a, st);
   if (rht) return flat ? launch_lean3<G, true, true, R>(a, st) : launch_lean3<G, true, false, R>(a, st);
   return flat ? launch_lean3<G, false, true, R>(a, st) : launch_lean3<G, false, false, R>(a, st);
