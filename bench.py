@@ -252,6 +252,13 @@ def profiled_record(kernel_key):
     return None
 
 
+def traffic_detail(rec):
+    """The parts of a record's traffic: DRAM reads and writes during the launch, and the bytes of
+    stores the kernel issued to L2 (written back to DRAM as L2 evicts them, partly after the
+    launch ends)."""
+    return {k: rec[k] for k in ("dram_read_bytes", "dram_write_bytes", "l2_write_bytes") if k in rec}
+
+
 def profiled_traffic(kernel_key):
     """DRAM bytes per launch from the committed ncu summary, if taken on the current sources."""
     rec = profiled_record(kernel_key)
@@ -685,6 +692,10 @@ def measure_gated(args, stream, dev, l2, peak):
                      "steps": steps, "launches_per_step": wl.launches_per_step,
                      "bytes_per_element": round(wl.bytes_per_step() / wl.elements(), 5),
                      "kernel": wl.kernel_key}
+        rec = profiled_record(wl.kernel_key)
+        if rec:   # one launch per step: the committed ncu record of that kernel applies
+            out[name]["traffic"] = rec["bytes_per_launch"]
+            out[name]["traffic_detail"] = traffic_detail(rec)
         del g_main, g_rem, wl
         torch.cuda.empty_cache()
     _INPUTS.clear()
@@ -740,6 +751,8 @@ def run_ours(args):
                 "algorithmic_bytes_per_launch": bytes_step / wl.launches_per_step}
     try:   # the second roofline, where the committed capture recorded the instruction count
         rec = profiled_record(wl.kernel_key)
+        if rec:
+            roofline["traffic_detail"] = traffic_detail(rec)
         if rec and rec.get("warp_instructions_per_launch"):
             roofline["issue"] = issue_roofline(rec["warp_instructions_per_launch"], launch_ms,
                                                props.multi_processor_count, max_sm_mhz(clocks))

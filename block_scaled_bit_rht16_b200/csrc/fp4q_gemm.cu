@@ -9,26 +9,31 @@
 // scale); "FP4 训练 vs FP4 推理" (reports.10n1j.top) notes that Blackwell's FP4 tensor-core path
 // is E2M1-only.
 //
-// One CTA computes a 128 x BN tile of D (BN = 256 when N allows, else 128) with 128 threads,
-// one CTA per SM (217 KB of shared memory, 512 tensor-memory columns). The K dimension streams in
-// 256-element steps through a ring of shared-memory buffers, with two specialised threads:
+// A persistent kernel: one CTA per SM (217 KB of shared memory, 512 tensor-memory columns)
+// walks the 128 x BN tiles of D (BN = 256 when N allows, else 128), tile i of a CTA being
+// blockIdx.x + i * gridDim.x with m fastest. The K dimension streams in 256-element steps through
+// a ring of shared-memory buffers that runs on across tiles. Six warps, three roles:
 //   thread 0 (producer): per step the A and B code tiles (128 / BN rows x 128 bytes) by 2-D TMA
 //     copies with the 128-byte swizzle, and the scale blocks (four 512-byte MMA-layout tiles per
 //     128 rows) by 1-D bulk copies, all completing on the buffer's `full` mbarrier; a buffer is
-//     refilled once its `empty` barrier says the MMAs that read it have completed;
-//   thread 32 (MMA issuer, warp 1): copies the step's scales into tensor memory (tcgen05.cp,
-//     32 lanes x 128 bits, replicated to the four lane quarters), issues four MMAs of K = 64
-//     (tcgen05.mma kind::mxf4nvf4, block16 scaling, M = 128, N = BN) and commits them to the
-//     buffer's `empty` barrier.
-// The accumulator is 128 lanes x BN FP32 columns of tensor memory; after the last step every warp
-// reads its 32 lanes back (tcgen05.ld), scales by alpha_A alpha_B and stores bf16. Every mbarrier wait is bounded by the
-// global timer; a wait that gives up sets bit 0 of the library's device status word and the CTA
-// skips the rest of its work (its outputs are then incomplete), releasing its tensor memory.
+//     refilled once its `empty` barrier says the MMAs that read it have completed, so the next
+//     tile's operands load while the current tile drains;
+//   thread 32 (MMA issuer): per tile, once `acc_empty` says the epilogue has read the previous
+//     accumulator, copies each step's scales into tensor memory (tcgen05.cp, 32 lanes x 128 bits,
+//     replicated to the four lane quarters), issues four MMAs of K = 64 (tcgen05.mma
+//     kind::mxf4nvf4, block16 scaling, M = 128, N = BN) and commits them to the buffer's `empty`
+//     barrier; the tile's last commit goes to `acc_full`;
+//   warps 2-5 (epilogue): warp w reads tensor-memory lanes 32 (w % 4) .. +31 (tcgen05.ld, 32
+//     columns at a time), scales by alpha_A alpha_B, stores bf16 rows, and arrives on `acc_empty`.
+// Every mbarrier wait is bounded by the global timer; a wait that gives up sets bit 0 of the
+// library's device status word and the CTA stops (its outputs are then incomplete), draining its
+// copies in flight and releasing its tensor memory.
 // No copy uses cluster multicast.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -40,7 +45,7 @@ namespace fp4q {
 namespace {
 
 constexpr int kBM = 128, kBKBytes = 128;   // 256 FP4 values per row per step
-constexpr int kGThreads = 128;
+constexpr int kGThreads = 192;   // warp 0 producer, warp 1 MMA issuer, warps 2-5 epilogue
 constexpr uint32_t kTileA = kBM * kBKBytes;   // 16 KB
 constexpr uint32_t kSfTile = 4 * 512;         // one 128-row scale tile row: 4 K-blocks of 64
 
@@ -67,7 +72,9 @@ struct GemmSmem {
   uint8_t sfb[C::kStages][C::kSfB];
   uint64_t full[C::kStages];
   uint64_t empty[C::kStages];
-  uint64_t done;
+  uint64_t acc_full;    // the MMAs of a tile have completed (tcgen05.commit)
+  uint64_t acc_empty;   // the epilogue warps have read the accumulator (one arrival per warp)
+  uint64_t done;        // every MMA and scale copy issued has completed
   uint32_t tmem_base;
 };
 template <int BN>
@@ -106,14 +113,16 @@ __global__ void __launch_bounds__(kGThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb,
                       const float* __restrict__ ts_a, const float* __restrict__ ts_b,
-                      __nv_bfloat16* __restrict__ out, int64_t ldo, int64_t K, int32_t* status) {
+                      __nv_bfloat16* __restrict__ out, int64_t ldo, int64_t M, int64_t N, int64_t K,
+                      int32_t* status) {
   using C = GemmCfg<BN>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   GemmSmem<BN>& sm = *reinterpret_cast<GemmSmem<BN>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int64_t m0 = (int64_t)blockIdx.y * kBM, n0 = (int64_t)blockIdx.x * BN;
+  const int tiles_m = (int)(M / kBM);
+  const int ntiles = tiles_m * (int)(N / BN);
   const int ksteps = (int)(K / 256);
   const int64_t kb64 = K / 64;   // scale tiles (of 4 K-blocks of 16) per 128-row tile row
 
@@ -122,10 +131,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
     }
+    mbar_init(&sm.acc_full, 1);
+    mbar_init(&sm.acc_empty, 4);
     mbar_init(&sm.done, 1);
     fence_mbar_init();
   }
-  if (warp == 0) {   // tensor memory for the accumulator and the staged scales
+  if (warp == 1) {   // tensor memory for the accumulator and the staged scales
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  ::"r"(smem_u32(&sm.tmem_base)), "r"(C::kTmemCols) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -138,103 +149,125 @@ __global__ void __launch_bounds__(kGThreads, 1)
   const uint32_t tmem_acc = tmem;                 // lanes 0..127, columns 0..BN-1
   const uint32_t tmem_sf = tmem + BN;             // then S x (A: 16, B: BN/8) columns
 
+  // Tiles are visited in the same order by every role: tile i of this CTA is
+  // blockIdx.x + i * gridDim.x, m fastest (CTAs in flight share B tiles in L2).
   int fail = 0;
   int issued = 0;   // producer: steps whose copies have been issued
   if (t == 0) {
     // producer: refills a buffer once the MMAs that read it have completed
-    const uint8_t* sfa_row = sfa + (m0 / 128) * kb64 * 512;
-    for (int kt = 0; kt < ksteps; ++kt, ++issued) {
-      const int s = kt % S;
-      if (kt >= S && !mbar_wait(&sm.empty[s], (uint32_t)(((kt / S) - 1) & 1))) { fail = 1; break; }
-      mbar_arrive_expect_tx(&sm.full[s], C::kStageTx);
-      tma_load_2d(sm.a[s], &tmA, kt * kBKBytes, (int)m0, &sm.full[s]);
-      tma_load_2d(sm.b[s], &tmB, kt * kBKBytes, (int)n0, &sm.full[s]);
-      bulk_load_1d(sm.sfa[s], sfa_row + (int64_t)kt * kSfTile, kSfTile, &sm.full[s]);
+    for (int tile = blockIdx.x; tile < ntiles && !fail; tile += gridDim.x) {
+      const int64_t m0 = (int64_t)(tile % tiles_m) * kBM, n0 = (int64_t)(tile / tiles_m) * BN;
+      const uint8_t* sfa_row = sfa + (m0 / 128) * kb64 * 512;
+      for (int kt = 0; kt < ksteps; ++kt, ++issued) {
+        const int s = issued % S;
+        if (issued >= S && !mbar_wait(&sm.empty[s], (uint32_t)(((issued / S) - 1) & 1))) { fail = 1; break; }
+        mbar_arrive_expect_tx(&sm.full[s], C::kStageTx);
+        tma_load_2d(sm.a[s], &tmA, kt * kBKBytes, (int)m0, &sm.full[s]);
+        tma_load_2d(sm.b[s], &tmB, kt * kBKBytes, (int)n0, &sm.full[s]);
+        bulk_load_1d(sm.sfa[s], sfa_row + (int64_t)kt * kSfTile, kSfTile, &sm.full[s]);
 #pragma unroll
-      for (int j = 0; j < BN / 128; ++j)
-        bulk_load_1d(sm.sfb[s] + j * kSfTile, sfb + ((n0 / 128 + j) * kb64 * 512) + (int64_t)kt * kSfTile,
-                     kSfTile, &sm.full[s]);
+        for (int j = 0; j < BN / 128; ++j)
+          bulk_load_1d(sm.sfb[s] + j * kSfTile, sfb + ((n0 / 128 + j) * kb64 * 512) + (int64_t)kt * kSfTile,
+                       kSfTile, &sm.full[s]);
+      }
     }
   } else if (t == 32) {
-    // MMA issuer: scales into tensor memory, four MMAs of K = 64 per step
-    for (int kt = 0; kt < ksteps; ++kt) {
-      const int s = kt % S;
-      if (!mbar_wait(&sm.full[s], (uint32_t)((kt / S) & 1))) { fail = 1; break; }
+    // MMA issuer: per tile, once the epilogue has read the previous accumulator, scales into
+    // tensor memory and four MMAs of K = 64 per step; the tile's last commit goes to acc_full
+    int it = 0;
+    int j = 0;
+    for (int tile = blockIdx.x; tile < ntiles && !fail; tile += gridDim.x, ++j) {
+      if (j > 0 && !mbar_wait(&sm.acc_empty, (uint32_t)((j - 1) & 1))) { fail = 1; break; }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t sa = tmem_sf + (uint32_t)s * C::kSfCols, sb = sa + 16u;
+      for (int kt = 0; kt < ksteps; ++kt, ++it) {
+        const int s = it % S;
+        if (!mbar_wait(&sm.full[s], (uint32_t)((it / S) & 1))) { fail = 1; break; }
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t sa = tmem_sf + (uint32_t)s * C::kSfCols, sb = sa + 16u;
 #pragma unroll
-      for (int kb = 0; kb < 4; ++kb) {
-        // a 512-byte scale tile = 32 rows of 16 bytes, 8-row groups 128 bytes apart
-        const uint64_t da = smem_desc(smem_u32(sm.sfa[s] + kb * 512), 16u, 128u, 0u);
-        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(sa + 4u * kb), "l"(da) : "memory");
+        for (int kb = 0; kb < 4; ++kb) {
+          // a 512-byte scale tile = 32 rows of 16 bytes, 8-row groups 128 bytes apart
+          const uint64_t da = smem_desc(smem_u32(sm.sfa[s] + kb * 512), 16u, 128u, 0u);
+          asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(sa + 4u * kb), "l"(da) : "memory");
 #pragma unroll
-        for (int j = 0; j < BN / 128; ++j) {
-          const uint64_t db = smem_desc(smem_u32(sm.sfb[s] + j * kSfTile + kb * 512), 16u, 128u, 0u);
-          asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
-                       ::"r"(sb + (uint32_t)(BN / 32) * kb + 4u * j), "l"(db) : "memory");
+          for (int jb = 0; jb < BN / 128; ++jb) {
+            const uint64_t db = smem_desc(smem_u32(sm.sfb[s] + jb * kSfTile + kb * 512), 16u, 128u, 0u);
+            asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
+                         ::"r"(sb + (uint32_t)(BN / 32) * kb + 4u * jb), "l"(db) : "memory");
+          }
         }
-      }
 #pragma unroll
-      for (int kb = 0; kb < 4; ++kb) {
-        // K-major, 128-byte swizzle: 8-row groups 1024 bytes apart; K-block kb starts 32 bytes in
-        const uint64_t adesc = smem_desc(smem_u32(sm.a[s]) + 32u * kb, 16u, 1024u, 2u);
-        const uint64_t bdesc = smem_desc(smem_u32(sm.b[s]) + 32u * kb, 16u, 1024u, 2u);
-        const uint32_t acc = (kt > 0 || kb > 0) ? 1u : 0u;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-            ::"r"(tmem_acc), "l"(adesc), "l"(bdesc), "r"(C::kIdesc), "r"(acc), "r"(sa + 4u * kb),
-              "r"(sb + (uint32_t)(BN / 32) * kb)
-            : "memory");
+        for (int kb = 0; kb < 4; ++kb) {
+          // K-major, 128-byte swizzle: 8-row groups 1024 bytes apart; K-block kb starts 32 bytes in
+          const uint64_t adesc = smem_desc(smem_u32(sm.a[s]) + 32u * kb, 16u, 1024u, 2u);
+          const uint64_t bdesc = smem_desc(smem_u32(sm.b[s]) + 32u * kb, 16u, 1024u, 2u);
+          const uint32_t acc = (kt > 0 || kb > 0) ? 1u : 0u;
+          asm volatile(
+              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+              "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+              ::"r"(tmem_acc), "l"(adesc), "l"(bdesc), "r"(C::kIdesc), "r"(acc), "r"(sa + 4u * kb),
+                "r"(sb + (uint32_t)(BN / 32) * kb)
+              : "memory");
+        }
+        umma_commit(&sm.empty[s]);   // the buffer is free again once these MMAs have read it
       }
-      umma_commit(&sm.empty[s]);   // the buffer is free again once these MMAs have read it
+      if (fail) break;
+      umma_commit(&sm.acc_full);     // the tile's accumulator is complete once these have run
     }
     // arrives when every MMA and scale copy issued above has completed
     umma_commit(&sm.done);
+  } else if (warp >= 2) {
+    // epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. +31 (rows of the tile) 32 columns
+    // at a time, stores them as bf16 x alpha, and releases the accumulator to the next tile's
+    // MMAs (the producer has kept loading the next tile's operands meanwhile)
+    const float alpha = __fmul_rn(*ts_a, *ts_b);
+    const int quarter = warp & 3;
+    int j = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
+      const int64_t m0 = (int64_t)(tile % tiles_m) * kBM, n0 = (int64_t)(tile / tiles_m) * BN;
+      if (!mbar_wait(&sm.acc_full, (uint32_t)(j & 1))) { fail = 1; break; }
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      uint4* dst = reinterpret_cast<uint4*>(out + (m0 + 32 * quarter + lane) * ldo + n0);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v[32];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+            "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+              "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+              "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+            : "r"(tmem_acc + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t o[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            o[i] = pack_bf16x2(__fmul_rn(__uint_as_float(v[8 * q + 2 * i]), alpha),
+                               __fmul_rn(__uint_as_float(v[8 * q + 2 * i + 1]), alpha));
+          dst[c0 / 8 + q] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+      // the stores need nothing more from tensor memory: release the accumulator
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.acc_empty);
+    }
   }
-  // the other threads wait at the barrier; a failed wait of the producer or the MMA issuer
-  // reaches every thread through it
+  // a failed wait of any role reaches every thread through the barrier
   fail = __syncthreads_or(fail);
   if (fail && t == 0) {
     // drain: wait (bounded) for the last fill issued into each buffer, steps issued - S ..
     // issued - 1 (a fill the MMA issuer has consumed has completed, and its wait returns at once)
-    for (int j = issued > S ? issued - S : 0; j < issued; ++j) mbar_wait(&sm.full[j % S], (uint32_t)((j / S) & 1));
+    for (int i = issued > S ? issued - S : 0; i < issued; ++i) mbar_wait(&sm.full[i % S], (uint32_t)((i / S) & 1));
   }
   if (!mbar_wait(&sm.done, 0u)) fail = 1;   // the MMA issuer commits `done` on every path
   fail = __syncthreads_or(fail);
+  if (fail && t == 0) atomicOr(status, kStatusWaitTimeout);
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  if (fail) {
-    if (t == 0) atomicOr(status, kStatusWaitTimeout);
-  } else {
-    const float alpha = __fmul_rn(*ts_a, *ts_b);
-    const int64_t row = m0 + 32 * warp + lane;
-#pragma unroll 1
-    for (int c0 = 0; c0 < BN; c0 += 32) {
-      uint32_t v[32];
-      asm volatile(
-          "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-          "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-          : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-            "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
-            "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
-            "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-          : "r"(tmem_acc + ((uint32_t)(32 * warp) << 16) + (uint32_t)c0));
-      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-      uint4* dst = reinterpret_cast<uint4*>(out + row * ldo + n0 + c0);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint4 o;
-        o.x = pack_bf16x2(__fmul_rn(__uint_as_float(v[8 * q + 0]), alpha), __fmul_rn(__uint_as_float(v[8 * q + 1]), alpha));
-        o.y = pack_bf16x2(__fmul_rn(__uint_as_float(v[8 * q + 2]), alpha), __fmul_rn(__uint_as_float(v[8 * q + 3]), alpha));
-        o.z = pack_bf16x2(__fmul_rn(__uint_as_float(v[8 * q + 4]), alpha), __fmul_rn(__uint_as_float(v[8 * q + 5]), alpha));
-        o.w = pack_bf16x2(__fmul_rn(__uint_as_float(v[8 * q + 6]), alpha), __fmul_rn(__uint_as_float(v[8 * q + 7]), alpha));
-        dst[q] = o;
-      }
-    }
-  }
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-  __syncthreads();
-  if (warp == 0)
+  if (warp == 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols) : "memory");
 }
 
@@ -296,7 +329,13 @@ cudaError_t launch_gemm_bn(const uint8_t* a_codes, const uint8_t* a_scales, cons
   e = device_status_word(&status);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(N / BN), (unsigned)(M / kBM));
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = (M / kBM) * (N / BN);
+  cfg.gridDim = dim3((unsigned)std::min<int64_t>(tiles, sms));   // one persistent CTA per SM
   cfg.blockDim = dim3(kGThreads);
   cfg.dynamicSmemBytes = gemm_smem_bytes<BN>();
   cfg.stream = st;
@@ -306,7 +345,7 @@ cudaError_t launch_gemm_bn(const uint8_t* a_codes, const uint8_t* a_scales, cons
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<BN>, ma, mb, a_scales, b_scales, a_ts, b_ts,
-                         reinterpret_cast<__nv_bfloat16*>(out), ldo, K, status);
+                         reinterpret_cast<__nv_bfloat16*>(out), ldo, M, N, K, status);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -34,7 +34,8 @@ def _sqnr(ref, got):
     return 10 * math.log10(float((ref ** 2).sum()) / max(float(((got - ref) ** 2).sum()), 1e-300))
 
 
-@pytest.mark.parametrize("shape", [(128, 128, 256), (256, 384, 768), (1024, 512, 2048), (128, 768, 4096)])
+@pytest.mark.parametrize("shape", [(128, 128, 256), (256, 384, 768), (1024, 512, 2048), (128, 768, 4096),
+                                   (4096, 1280, 512), (4096, 1152, 256)])   # more tiles than SMs
 def test_gemm_matches_the_decoded_product(shape):
     import torch
     from dataclasses import replace
