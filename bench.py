@@ -239,13 +239,15 @@ def kernel_source_sha(csrc=None, files=None):
     return h.hexdigest()[:16]
 
 
-def profiled_record(kernel_key):
-    """The committed ncu record of a kernel (profiles/traffic.json), if it was taken on the
-    kernel's current device sources; else None."""
+def profiled_record(kernel_key, workload):
+    """The committed ncu record of a kernel on a workload (profiles/traffic.json: per-launch
+    counters hold for the launch size they were captured on), if it was taken on the kernel's
+    current device sources; else None."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f).get(kernel_key)
-        if rec and rec.get("source_sha") == kernel_source_sha(files=kernel_sources(kernel_key)):
+        if rec and rec.get("workload") == workload and \
+                rec.get("source_sha") == kernel_source_sha(files=kernel_sources(kernel_key)):
             return rec
     except Exception:
         pass
@@ -259,9 +261,10 @@ def traffic_detail(rec):
     return {k: rec[k] for k in ("dram_read_bytes", "dram_write_bytes", "l2_write_bytes") if k in rec}
 
 
-def profiled_traffic(kernel_key):
-    """DRAM bytes per launch from the committed ncu summary, if taken on the current sources."""
-    rec = profiled_record(kernel_key)
+def profiled_traffic(kernel_key, workload):
+    """DRAM bytes per launch from the committed ncu summary, if taken on this workload and the
+    current sources."""
+    rec = profiled_record(kernel_key, workload)
     return rec["bytes_per_launch"] if rec else None
 
 
@@ -692,8 +695,8 @@ def measure_gated(args, stream, dev, l2, peak):
                      "steps": steps, "launches_per_step": wl.launches_per_step,
                      "bytes_per_element": round(wl.bytes_per_step() / wl.elements(), 5),
                      "kernel": wl.kernel_key}
-        rec = profiled_record(wl.kernel_key)
-        if rec:   # one launch per step: the committed ncu record of that kernel applies
+        rec = profiled_record(wl.kernel_key, name)
+        if rec:   # the committed ncu record of this workload's one launch per step
             out[name]["traffic"] = rec["bytes_per_launch"]
             out[name]["traffic_detail"] = traffic_detail(rec)
         del g_main, g_rem, wl
@@ -745,12 +748,12 @@ def run_ours(args):
     peak, peak_src = hbm_peak()
     achieved = bytes_step / wl.launches_per_step / (launch_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": profiled_traffic(wl.kernel_key),
+                "frac": round(achieved / peak, 4), "traffic": profiled_traffic(wl.kernel_key, wl.name),
                 "kernel": wl.kernel_key, "peak_source": peak_src,
                 "launch_us": round(launch_ms * 1e3, 3),
                 "algorithmic_bytes_per_launch": bytes_step / wl.launches_per_step}
     try:   # the second roofline, where the committed capture recorded the instruction count
-        rec = profiled_record(wl.kernel_key)
+        rec = profiled_record(wl.kernel_key, wl.name)
         if rec:
             roofline["traffic_detail"] = traffic_detail(rec)
         if rec and rec.get("warp_instructions_per_launch"):

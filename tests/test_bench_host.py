@@ -86,7 +86,10 @@ def test_every_workload_constructs():
     # the committed ncu traffic record names kernels that the bench reports
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     with open(os.path.join(root, "profiles", "traffic.json")) as f:
-        assert set(json.load(f)) <= keys
+        recs = json.load(f)
+    assert set(recs) <= keys
+    for key, rec in recs.items():   # each record names the workload whose launch it measured
+        assert bench.make_workload(rec["workload"]).kernel_key == key
 
 
 _MAKE_WORKLOAD = bench.make_workload
