@@ -376,3 +376,36 @@ def gemm_nvfp4(a: Quantized, b: Quantized, *, out=None, stream=None):
                                          _stream_ptr(stream, dev))
     _lib.check(st, "fp4q_gemm_nvfp4")
     return out
+
+
+
+def gemm_mxfp4(a: Quantized, b: Quantized, *, out=None, stream=None):
+    """fp4q_gemm_mxfp4: out[m, n] = sum_k A[m, k] B[n, k] in bf16, from two MXFP4 quantizations
+    (E2M1 codes, UE8M0 scales in the MMA layout) used unchanged."""
+    torch = _torch()
+    for name, q in (("a", a), ("b", b)):
+        if not isinstance(q, Quantized):
+            raise TypeError("%s must be the Quantized result of an MXFP4 quantization" % name)
+    M, K2 = a.codes.shape
+    N = b.codes.shape[0]
+    K = 2 * K2
+    dev = a.codes.device
+    _check_buf(a.codes, "a.codes", torch.uint8, M * K2, dev)
+    _check_buf(b.codes, "b.codes", torch.uint8, N * K2, dev)
+    _check_buf(a.scales, "a.scales", torch.uint8, M * (K // 32), dev)
+    _check_buf(b.scales, "b.scales", torch.uint8, N * (K // 32), dev)
+    if b.codes.shape[1] != K2:
+        raise ValueError("a and b must have the same K")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    if not (isinstance(out, torch.Tensor) and out.is_cuda and out.dtype == torch.bfloat16 and out.dim() == 2
+            and out.stride(1) == 1 and out.shape[0] == M and out.shape[1] == N):
+        raise TypeError("out must be a bf16 CUDA tensor [M, N] with unit column stride")
+    if out.device != dev:
+        raise ValueError("out is on %s but the operands are on %s" % (out.device, dev))
+    ldo = out.stride(0) if M > 1 else N
+    with torch.cuda.device(dev):
+        st = _lib.load().fp4q_gemm_mxfp4(_ptr(a.codes), _ptr(a.scales), _ptr(b.codes), _ptr(b.scales), M, N, K,
+                                         _ptr(out), ldo, _stream_ptr(stream, dev))
+    _lib.check(st, "fp4q_gemm_mxfp4")
+    return out

@@ -21,7 +21,7 @@ EXPORTS = ["fp4q_status_string", "fp4q_sign_mask_from_seed", "fp4q_workspace_siz
            "fp4q_stats", "fp4q_rht16", "fp4q_check_division", "fp4q_device_status",
            "fp4q_check_wait_timeout", "fp4q_tensor_scale", "fp4q_rht_quantize_noalloc",
            "fp4q_grouped_workspace_size", "fp4q_rht_quantize_grouped", "fp4q_check_conversions",
-           "fp4q_gemm_nvfp4"]
+           "fp4q_gemm_nvfp4", "fp4q_gemm_mxfp4"]
 
 
 class fp4q_config(ctypes.Structure):
@@ -61,6 +61,7 @@ SIGNATURES = {
     "fp4q_check_division": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_uint64, _P, _P]),
     "fp4q_check_conversions": (ctypes.c_int, [_P, _P]),
     "fp4q_gemm_nvfp4": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P]),
+    "fp4q_gemm_mxfp4": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P]),
     "fp4q_device_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int32), ctypes.c_int32, _P]),
     "fp4q_check_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
     "fp4q_tensor_scale": (ctypes.c_int, [_CFG, _P, _I64, _I64, _I64, _P, _P, ctypes.c_size_t, _P]),

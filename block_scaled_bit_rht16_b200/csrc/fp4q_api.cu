@@ -463,6 +463,22 @@ fp4q_status fp4q_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales, con
                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
+fp4q_status fp4q_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
+                            const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, void* out, int64_t ldo,
+                            fp4q_stream_t stream) {
+  if (M < 0 || N < 0 || K < 256 || M % 128 != 0 || N % 128 != 0 || K % 256 != 0) return FP4Q_ERR_SHAPE;
+  if (M / 128 > 65535 || K > (int64_t(1) << 31)) return FP4Q_ERR_SHAPE;
+  if (M > 0 && N > 0 && ldo < N) return FP4Q_ERR_SHAPE;
+  if (M == 0 || N == 0) return FP4Q_OK;
+  if (a_codes == nullptr || a_scales == nullptr || b_codes == nullptr || b_scales == nullptr || out == nullptr)
+    return FP4Q_ERR_INVALID_ARG;
+  if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_scales, 16) || !aligned(b_scales, 16) ||
+      !aligned(out, 16) || ldo % 8 != 0)
+    return FP4Q_ERR_ALIGN;
+  return cuda_status(launch_gemm_mxfp4(a_codes, a_scales, b_codes, b_scales, M, N, K, static_cast<uint16_t*>(out),
+                                       ldo, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 fp4q_status fp4q_check_conversions(unsigned long long* mismatches, fp4q_stream_t stream) {
   if (mismatches == nullptr) return FP4Q_ERR_INVALID_ARG;
   if (!aligned(mismatches, 8)) return FP4Q_ERR_ALIGN;

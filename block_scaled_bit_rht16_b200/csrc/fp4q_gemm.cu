@@ -47,28 +47,33 @@ namespace {
 constexpr int kBM = 128, kBKBytes = 128;   // 256 FP4 values per row per step
 constexpr int kGThreads = 192;   // warp 0 producer, warp 1 MMA issuer, warps 2-5 epilogue
 constexpr uint32_t kTileA = kBM * kBKBytes;   // 16 KB
-constexpr uint32_t kSfTile = 4 * 512;         // one 128-row scale tile row: 4 K-blocks of 64
-
-// Per tile width BN (128 or 256): stages, shared memory, tensor memory.
-template <int BN>
+// Per tile width BN (128 or 256) and scale kind (MX: UE8M0 per 32 elements, else E4M3 per 16):
+// stages, shared memory, tensor memory. A 512-byte MMA-layout scale tile covers 128 rows and
+// 4 scale columns: K = 64 (NVFP4) or 128 (MXFP4), so a 256-deep step takes 4 or 2 of them per 128
+// rows.
+template <int BN, bool MX>
 struct GemmCfg {
   static constexpr int kStages = BN == 256 ? 4 : 6;
   static constexpr uint32_t kTileB = BN * kBKBytes;
-  static constexpr uint32_t kSfB = (BN / 128) * kSfTile;
-  static constexpr uint32_t kStageTx = kTileA + kTileB + kSfTile + kSfB;
-  static constexpr uint32_t kSfCols = 16 + BN / 8;   // A: 4 K-blocks x 4 columns; B: 4 x BN/32
+  static constexpr int kSfTiles = MX ? 2 : 4;                     // per 128 rows per step
+  static constexpr uint32_t kSfA = kSfTiles * 512;
+  static constexpr uint32_t kSfB = (BN / 128) * kSfA;
+  static constexpr uint32_t kStageTx = kTileA + kTileB + kSfA + kSfB;
+  static constexpr uint32_t kSfCols = 4 * kSfTiles * (1 + BN / 128);   // A then B, 4 columns a tile
   static constexpr uint32_t kTmemCols = (BN + kStages * kSfCols) <= 256 ? 256 : 512;
-  // kind::mxf4nvf4: E2M1 A and B (format 1), K-major, N / 8 in bits 17-22, UE4M3 scales (bit 23
-  // = 0), M / 16 in bits 24-28, scale-factor ids 0, K = 64
-  static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+  // kind::mxf4nvf4: E2M1 A and B (format 1), K-major, N / 8 in bits 17-22, scale type in bit 23
+  // (0 UE4M3, 1 UE8M0), M / 16 in bits 24-28, K = 64; the scale-factor ids (which byte pair of a
+  // 32-bit scale column a 32-element-block MMA reads: 0 or 2) in bits 4-5 (B) and 29-30 (A)
+  static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                     ((MX ? 1u : 0u) << 23) | ((uint32_t)(kBM >> 4) << 24);
 };
 
-template <int BN>
+template <int BN, bool MX>
 struct GemmSmem {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, MX>;
   uint8_t a[C::kStages][kTileA];      // 1024-byte aligned (swizzle period)
   uint8_t b[C::kStages][C::kTileB];
-  uint8_t sfa[C::kStages][kSfTile];
+  uint8_t sfa[C::kStages][C::kSfA];
   uint8_t sfb[C::kStages][C::kSfB];
   uint64_t full[C::kStages];
   uint64_t empty[C::kStages];
@@ -77,8 +82,8 @@ struct GemmSmem {
   uint64_t done;        // every MMA and scale copy issued has completed
   uint32_t tmem_base;
 };
-template <int BN>
-constexpr size_t gemm_smem_bytes() { return sizeof(GemmSmem<BN>) + 1024; }
+template <int BN, bool MX>
+constexpr size_t gemm_smem_bytes() { return sizeof(GemmSmem<BN, MX>) + 1024; }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(
@@ -108,23 +113,23 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                ::"r"(smem_u32(bar)) : "memory");
 }
 
-template <int BN>
+template <int BN, bool MX>
 __global__ void __launch_bounds__(kGThreads, 1)
-    nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+    fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                       const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb,
                       const float* __restrict__ ts_a, const float* __restrict__ ts_b,
                       __nv_bfloat16* __restrict__ out, int64_t ldo, int64_t M, int64_t N, int64_t K,
                       int32_t* status) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, MX>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
-  GemmSmem<BN>& sm = *reinterpret_cast<GemmSmem<BN>*>(
+  GemmSmem<BN, MX>& sm = *reinterpret_cast<GemmSmem<BN, MX>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int tiles_m = (int)(M / kBM);
   const int ntiles = tiles_m * (int)(N / BN);
   const int ksteps = (int)(K / 256);
-  const int64_t kb64 = K / 64;   // scale tiles (of 4 K-blocks of 16) per 128-row tile row
+  const int64_t row_tiles = K / (MX ? 128 : 64);   // 512-byte scale tiles per 128-row tile row
 
   if (t == 0) {
     for (int s = 0; s < S; ++s) {
@@ -157,18 +162,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
     // producer: refills a buffer once the MMAs that read it have completed
     for (int tile = blockIdx.x; tile < ntiles && !fail; tile += gridDim.x) {
       const int64_t m0 = (int64_t)(tile % tiles_m) * kBM, n0 = (int64_t)(tile / tiles_m) * BN;
-      const uint8_t* sfa_row = sfa + (m0 / 128) * kb64 * 512;
+      const uint8_t* sfa_row = sfa + (m0 / 128) * row_tiles * 512;
       for (int kt = 0; kt < ksteps; ++kt, ++issued) {
         const int s = issued % S;
         if (issued >= S && !mbar_wait(&sm.empty[s], (uint32_t)(((issued / S) - 1) & 1))) { fail = 1; break; }
         mbar_arrive_expect_tx(&sm.full[s], C::kStageTx);
         tma_load_2d(sm.a[s], &tmA, kt * kBKBytes, (int)m0, &sm.full[s]);
         tma_load_2d(sm.b[s], &tmB, kt * kBKBytes, (int)n0, &sm.full[s]);
-        bulk_load_1d(sm.sfa[s], sfa_row + (int64_t)kt * kSfTile, kSfTile, &sm.full[s]);
+        bulk_load_1d(sm.sfa[s], sfa_row + (int64_t)kt * C::kSfA, C::kSfA, &sm.full[s]);
 #pragma unroll
         for (int j = 0; j < BN / 128; ++j)
-          bulk_load_1d(sm.sfb[s] + j * kSfTile, sfb + ((n0 / 128 + j) * kb64 * 512) + (int64_t)kt * kSfTile,
-                       kSfTile, &sm.full[s]);
+          bulk_load_1d(sm.sfb[s] + j * C::kSfA, sfb + ((n0 / 128 + j) * row_tiles * 512) + (int64_t)kt * C::kSfA,
+                       C::kSfA, &sm.full[s]);
       }
     }
   } else if (t == 32) {
@@ -183,17 +188,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
         const int s = it % S;
         if (!mbar_wait(&sm.full[s], (uint32_t)((it / S) & 1))) { fail = 1; break; }
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t sa = tmem_sf + (uint32_t)s * C::kSfCols, sb = sa + 16u;
+        // scale tile t of A at columns sa + 4t; tile t of B's 128-row group j at sb + 4 (BN/128) t + 4j
+        const uint32_t sa = tmem_sf + (uint32_t)s * C::kSfCols, sb = sa + 4u * C::kSfTiles;
 #pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
+        for (int tt = 0; tt < C::kSfTiles; ++tt) {
           // a 512-byte scale tile = 32 rows of 16 bytes, 8-row groups 128 bytes apart
-          const uint64_t da = smem_desc(smem_u32(sm.sfa[s] + kb * 512), 16u, 128u, 0u);
-          asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(sa + 4u * kb), "l"(da) : "memory");
+          const uint64_t da = smem_desc(smem_u32(sm.sfa[s] + tt * 512), 16u, 128u, 0u);
+          asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(sa + 4u * tt), "l"(da) : "memory");
 #pragma unroll
           for (int jb = 0; jb < BN / 128; ++jb) {
-            const uint64_t db = smem_desc(smem_u32(sm.sfb[s] + jb * kSfTile + kb * 512), 16u, 128u, 0u);
+            const uint64_t db = smem_desc(smem_u32(sm.sfb[s] + jb * C::kSfA + tt * 512), 16u, 128u, 0u);
             asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
-                         ::"r"(sb + (uint32_t)(BN / 32) * kb + 4u * jb), "l"(db) : "memory");
+                         ::"r"(sb + 4u * (uint32_t)(BN / 128) * tt + 4u * jb), "l"(db) : "memory");
           }
         }
 #pragma unroll
@@ -202,12 +208,24 @@ __global__ void __launch_bounds__(kGThreads, 1)
           const uint64_t adesc = smem_desc(smem_u32(sm.a[s]) + 32u * kb, 16u, 1024u, 2u);
           const uint64_t bdesc = smem_desc(smem_u32(sm.b[s]) + 32u * kb, 16u, 1024u, 2u);
           const uint32_t acc = (kt > 0 || kb > 0) ? 1u : 0u;
-          asm volatile(
-              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-              "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-              ::"r"(tmem_acc), "l"(adesc), "l"(bdesc), "r"(C::kIdesc), "r"(acc), "r"(sa + 4u * kb),
-                "r"(sb + (uint32_t)(BN / 32) * kb)
-              : "memory");
+          // NVFP4: tile kb, all four bytes of each scale column; MXFP4: tile kb / 2, bytes
+          // 2 (kb % 2) and 2 (kb % 2) + 1 (the scale-factor ids)
+          const int tt = MX ? kb >> 1 : kb;
+          const uint32_t id = MX ? 2u * (uint32_t)(kb & 1) : 0u;
+          const uint32_t idesc = C::kIdesc | (id << 4) | (id << 29);
+          const uint32_t sfa_col = sa + 4u * tt, sfb_col = sb + 4u * (uint32_t)(BN / 128) * tt;
+          if constexpr (MX)
+            asm volatile(
+                "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+                ::"r"(tmem_acc), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(sfa_col), "r"(sfb_col)
+                : "memory");
+          else
+            asm volatile(
+                "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+                ::"r"(tmem_acc), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(sfa_col), "r"(sfb_col)
+                : "memory");
         }
         umma_commit(&sm.empty[s]);   // the buffer is free again once these MMAs have read it
       }
@@ -220,7 +238,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     // epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. +31 (rows of the tile) 32 columns
     // at a time, stores them as bf16 x alpha, and releases the accumulator to the next tile's
     // MMAs (the producer has kept loading the next tile's operands meanwhile)
-    const float alpha = __fmul_rn(*ts_a, *ts_b);
+    const float alpha = MX ? 1.0f : __fmul_rn(*ts_a, *ts_b);   // MXFP4 has no tensor scale
     const int quarter = warp & 3;
     int j = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
@@ -298,8 +316,8 @@ cudaError_t make_codes_map(const uint8_t* codes, int64_t rows, int64_t K, int bo
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// Raises the kernel's shared-memory limit once per (tile width, device).
-template <int BN>
+// Raises the kernel's shared-memory limit once per (kernel, device).
+template <int BN, bool MX>
 cudaError_t gemm_prepare() {
   static std::mutex mu;
   static std::map<int, cudaError_t> done;
@@ -309,12 +327,12 @@ cudaError_t gemm_prepare() {
   std::lock_guard<std::mutex> lock(mu);
   auto it = done.find(dev);
   if (it == done.end())
-    it = done.emplace(dev, cudaFuncSetAttribute(nvfp4_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                (int)gemm_smem_bytes<BN>())).first;
+    it = done.emplace(dev, cudaFuncSetAttribute(fp4_gemm_kernel<BN, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                (int)gemm_smem_bytes<BN, MX>())).first;
   return it->second;
 }
 
-template <int BN>
+template <int BN, bool MX>
 cudaError_t launch_gemm_bn(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_ts,
                            const uint8_t* b_codes, const uint8_t* b_scales, const float* b_ts,
                            int64_t M, int64_t N, int64_t K, uint16_t* out, int64_t ldo, cudaStream_t st) {
@@ -323,7 +341,7 @@ cudaError_t launch_gemm_bn(const uint8_t* a_codes, const uint8_t* a_scales, cons
   if (e != cudaSuccess) return e;
   e = make_codes_map(b_codes, N, K, BN, &mb);
   if (e != cudaSuccess) return e;
-  e = gemm_prepare<BN>();
+  e = gemm_prepare<BN, MX>();
   if (e != cudaSuccess) return e;
   int32_t* status = nullptr;
   e = device_status_word(&status);
@@ -337,14 +355,14 @@ cudaError_t launch_gemm_bn(const uint8_t* a_codes, const uint8_t* a_scales, cons
   const int64_t tiles = (M / kBM) * (N / BN);
   cfg.gridDim = dim3((unsigned)std::min<int64_t>(tiles, sms));   // one persistent CTA per SM
   cfg.blockDim = dim3(kGThreads);
-  cfg.dynamicSmemBytes = gemm_smem_bytes<BN>();
+  cfg.dynamicSmemBytes = gemm_smem_bytes<BN, MX>();
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<BN>, ma, mb, a_scales, b_scales, a_ts, b_ts,
+  e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, MX>, ma, mb, a_scales, b_scales, a_ts, b_ts,
                          reinterpret_cast<__nv_bfloat16*>(out), ldo, M, N, K, status);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -357,8 +375,17 @@ cudaError_t launch_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales, c
                               cudaStream_t st) {
   if (M == 0 || N == 0) return cudaSuccess;
   if (N % 256 == 0)
-    return launch_gemm_bn<256>(a_codes, a_scales, a_ts, b_codes, b_scales, b_ts, M, N, K, out, ldo, st);
-  return launch_gemm_bn<128>(a_codes, a_scales, a_ts, b_codes, b_scales, b_ts, M, N, K, out, ldo, st);
+    return launch_gemm_bn<256, false>(a_codes, a_scales, a_ts, b_codes, b_scales, b_ts, M, N, K, out, ldo, st);
+  return launch_gemm_bn<128, false>(a_codes, a_scales, a_ts, b_codes, b_scales, b_ts, M, N, K, out, ldo, st);
+}
+
+cudaError_t launch_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
+                              const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, uint16_t* out,
+                              int64_t ldo, cudaStream_t st) {
+  if (M == 0 || N == 0) return cudaSuccess;
+  if (N % 256 == 0)
+    return launch_gemm_bn<256, true>(a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, M, N, K, out, ldo, st);
+  return launch_gemm_bn<128, true>(a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, M, N, K, out, ldo, st);
 }
 
 }  // namespace fp4q

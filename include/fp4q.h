@@ -276,6 +276,19 @@ fp4q_status fp4q_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales,
                             const uint8_t* b_scales, const float* b_tensor_scale, int64_t M,
                             int64_t N, int64_t K, void* out, int64_t ldo, fp4q_stream_t stream);
 
+/* MXFP4 GEMM on the tensor cores (tcgen05 block-scaled MMA with 32-element blocks, sm_100a),
+ * consuming the quantizer's outputs unchanged: out[m, n] = sum_k A[m, k] B[n, k] (bf16, RNE), where
+ * A and B are the E2M1 codes of two MXFP4 quantizations along K (fp4q_rht_quantize with grid E2M1,
+ * FP4Q_SCALE_UE8M0_1x32 and FP4Q_OUT_SCALES_MMA) times their UE8M0 block scales
+ * ("AMD全新研究揭示：FP4训练不稳定性源于结构误差而非随机性不足", cannews.ca/article/21387: MXFP4 = 32-element
+ * blocks sharing one power-of-two scale; no tensor scale). Products accumulate in FP32.
+ *  a_codes uint8 [M, K/2], a_scales uint8 [M, K/32] in the MMA layout; b_* the same with N rows;
+ *  out bf16 [M, ldo], ldo >= N, ldo % 8 == 0.
+ *  Shapes, alignment, errors, the first call and the bounded waits as fp4q_gemm_nvfp4. */
+fp4q_status fp4q_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
+                            const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, void* out, int64_t ldo,
+                            fp4q_stream_t stream);
+
 /* Reduce the statistics a previous fp4q_rht_quantize / fp4q_if4_select call with
  * FP4Q_OUT_STATS left in `workspace` (in a fixed order, FP64), copy them to *host_out and
  * derive SQNR, alpha, MSE and the per-cell mean error [UFP4-A "E2M1", "复利效应的反向版本",

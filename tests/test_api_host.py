@@ -283,3 +283,11 @@ def test_gemm_validation():
     assert g(sa=FAKE + 4) == _lib.FP4Q_ERR_ALIGN
     assert g(ldo=132) == _lib.FP4Q_ERR_ALIGN          # 16-byte output rows
     assert g(M=0) == _lib.FP4Q_OK                     # empty: nothing to do
+    mx = lambda M=128, N=128, K=256, ldo=128, a=FAKE, sa=FAKE, out=FAKE: lib.fp4q_gemm_mxfp4(
+        a, sa, FAKE, FAKE, M, N, K, out, ldo, None)
+    assert mx(M=100) == _lib.FP4Q_ERR_SHAPE
+    assert mx(K=128) == _lib.FP4Q_ERR_SHAPE
+    assert mx(ldo=64) == _lib.FP4Q_ERR_SHAPE
+    assert mx(sa=None) == _lib.FP4Q_ERR_INVALID_ARG
+    assert mx(sa=FAKE + 4) == _lib.FP4Q_ERR_ALIGN
+    assert mx(M=0) == _lib.FP4Q_OK
