@@ -51,12 +51,18 @@ constexpr uint32_t kTileA = kBM * kBKBytes;   // 16 KB
 // stages, shared memory, tensor memory. A 512-byte MMA-layout scale tile covers 128 rows and
 // 4 scale columns: K = 64 (NVFP4) or 128 (MXFP4), so a 256-deep step takes 4 or 2 of them per 128
 // rows.
+// In shared memory each scale tile lands four times in a row (kSfRep: the tensor map repeats
+// it along a zero-stride dimension), so that one 128x256b tcgen05.cp (128 lanes x 8 columns;
+// rows r and r + 32k read the same bytes) puts two tiles into tensor memory exactly as two
+// 32x128b.warpx4 copies would: the copies, which run in the tensor pipe in issue order with the
+// MMAs, are halved.
+constexpr uint32_t kSfRep = 4 * 512;
 template <int BN, bool MX>
 struct GemmCfg {
-  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kStages = BN == 256 ? 3 : (MX ? 5 : 4);
   static constexpr uint32_t kTileB = BN * kBKBytes;
   static constexpr int kSfTiles = MX ? 2 : 4;                     // per 128 rows per step
-  static constexpr uint32_t kSfA = kSfTiles * 512;
+  static constexpr uint32_t kSfA = kSfTiles * kSfRep;
   static constexpr uint32_t kSfB = (BN / 128) * kSfA;
   static constexpr uint32_t kStageTx = kTileA + kTileB + kSfA + kSfB;
   static constexpr uint32_t kSfCols = 4 * kSfTiles * (1 + BN / 128);   // A then B, 4 columns a tile
@@ -71,10 +77,10 @@ struct GemmCfg {
 template <int BN, bool MX>
 struct GemmSmem {
   using C = GemmCfg<BN, MX>;
+  uint8_t sfa[C::kStages][C::kSfA];   // first: every copy descriptor's reach stays inside the struct
+  uint8_t sfb[C::kStages][C::kSfB];
   uint8_t a[C::kStages][kTileA];      // 1024-byte aligned (swizzle period)
   uint8_t b[C::kStages][C::kTileB];
-  uint8_t sfa[C::kStages][C::kSfA];
-  uint8_t sfb[C::kStages][C::kSfB];
   uint64_t full[C::kStages];
   uint64_t empty[C::kStages];
   uint64_t acc_full;    // the MMAs of a tile have completed (tcgen05.commit)
@@ -93,10 +99,11 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-__device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -116,7 +123,7 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 template <int BN, bool MX>
 __global__ void __launch_bounds__(kGThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const uint8_t* __restrict__ sfa, const uint8_t* __restrict__ sfb,
+                      const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
                       const float* __restrict__ ts_a, const float* __restrict__ ts_b,
                       __nv_bfloat16* __restrict__ out, int64_t ldo, int64_t M, int64_t N, int64_t K,
                       int32_t* status) {
@@ -129,7 +136,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
   const int tiles_m = (int)(M / kBM);
   const int ntiles = tiles_m * (int)(N / BN);
   const int ksteps = (int)(K / 256);
-  const int64_t row_tiles = K / (MX ? 128 : 64);   // 512-byte scale tiles per 128-row tile row
+  const int row_tiles = (int)(K / (MX ? 128 : 64));   // 512-byte scale tiles per 128-row tile row
 
   if (t == 0) {
     for (int s = 0; s < S; ++s) {
@@ -162,18 +169,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
     // producer: refills a buffer once the MMAs that read it have completed
     for (int tile = blockIdx.x; tile < ntiles && !fail; tile += gridDim.x) {
       const int64_t m0 = (int64_t)(tile % tiles_m) * kBM, n0 = (int64_t)(tile / tiles_m) * BN;
-      const uint8_t* sfa_row = sfa + (m0 / 128) * row_tiles * 512;
       for (int kt = 0; kt < ksteps; ++kt, ++issued) {
         const int s = issued % S;
         if (issued >= S && !mbar_wait(&sm.empty[s], (uint32_t)(((issued / S) - 1) & 1))) { fail = 1; break; }
         mbar_arrive_expect_tx(&sm.full[s], C::kStageTx);
         tma_load_2d(sm.a[s], &tmA, kt * kBKBytes, (int)m0, &sm.full[s]);
         tma_load_2d(sm.b[s], &tmB, kt * kBKBytes, (int)n0, &sm.full[s]);
-        bulk_load_1d(sm.sfa[s], sfa_row + (int64_t)kt * C::kSfA, C::kSfA, &sm.full[s]);
+        // the step's kSfTiles scale tiles of A and of each 128-row group of B, each four times
+        tma_load_3d(sm.sfa[s], &tmSA, 0, 0, (int)(m0 / 128) * row_tiles + kt * C::kSfTiles, &sm.full[s]);
 #pragma unroll
         for (int j = 0; j < BN / 128; ++j)
-          bulk_load_1d(sm.sfb[s] + j * C::kSfA, sfb + ((n0 / 128 + j) * row_tiles * 512) + (int64_t)kt * C::kSfA,
-                       C::kSfA, &sm.full[s]);
+          tma_load_3d(sm.sfb[s] + j * C::kSfA, &tmSB, 0, 0, (int)(n0 / 128 + j) * row_tiles + kt * C::kSfTiles,
+                      &sm.full[s]);
       }
     }
   } else if (t == 32) {
@@ -190,16 +197,25 @@ __global__ void __launch_bounds__(kGThreads, 1)
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         // scale tile t of A at columns sa + 4t; tile t of B's 128-row group j at sb + 4 (BN/128) t + 4j
         const uint32_t sa = tmem_sf + (uint32_t)s * C::kSfCols, sb = sa + 4u * C::kSfTiles;
+        // a copy's source: 128 rows of 32 bytes = 8-row groups 128 bytes apart (SBO) within one
+        // repeated tile, the second 16 bytes of each row (the second tile) LBO further on. A and
+        // BN = 128 pair tiles (2p, 2p + 1); BN = 256 pairs the two row groups' tile tt.
 #pragma unroll
-        for (int tt = 0; tt < C::kSfTiles; ++tt) {
-          // a 512-byte scale tile = 32 rows of 16 bytes, 8-row groups 128 bytes apart
-          const uint64_t da = smem_desc(smem_u32(sm.sfa[s] + tt * 512), 16u, 128u, 0u);
-          asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(sa + 4u * tt), "l"(da) : "memory");
+        for (int p = 0; p < C::kSfTiles / 2; ++p) {
+          const uint64_t da = smem_desc(smem_u32(sm.sfa[s] + p * 2 * kSfRep), kSfRep, 128u, 0u);
+          asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(sa + 8u * p), "l"(da) : "memory");
+        }
+        if constexpr (BN == 256) {
 #pragma unroll
-          for (int jb = 0; jb < BN / 128; ++jb) {
-            const uint64_t db = smem_desc(smem_u32(sm.sfb[s] + jb * C::kSfA + tt * 512), 16u, 128u, 0u);
-            asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
-                         ::"r"(sb + 4u * (uint32_t)(BN / 128) * tt + 4u * jb), "l"(db) : "memory");
+          for (int tt = 0; tt < C::kSfTiles; ++tt) {
+            const uint64_t db = smem_desc(smem_u32(sm.sfb[s] + tt * kSfRep), C::kSfA, 128u, 0u);
+            asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(sb + 8u * tt), "l"(db) : "memory");
+          }
+        } else {
+#pragma unroll
+          for (int p = 0; p < C::kSfTiles / 2; ++p) {
+            const uint64_t db = smem_desc(smem_u32(sm.sfb[s] + p * 2 * kSfRep), kSfRep, 128u, 0u);
+            asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(sb + 8u * p), "l"(db) : "memory");
           }
         }
 #pragma unroll
@@ -316,6 +332,22 @@ cudaError_t make_codes_map(const uint8_t* codes, int64_t rows, int64_t K, int bo
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// 3-D map of MMA-layout scales (uint8 [rows / 128 * row_tiles] tiles of 512 bytes) as 32-bit words:
+// 128 words of a tile, the tile repeated four times (a zero stride), the tiles; a box of
+// `tiles` consecutive tiles lands as tile 0 x4, tile 1 x4, ... in shared memory.
+cudaError_t make_scales_map(const uint8_t* scales, int64_t total_tiles, int tiles, CUtensorMap* map) {
+  auto enc = gemm_tensor_map_encoder();
+  if (enc == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {128, 4, (cuuint64_t)total_tiles};
+  const cuuint64_t strides[2] = {0, 512};
+  const cuuint32_t box[3] = {128, 4, (cuuint32_t)tiles};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t*>(scales), dims, strides,
+                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 // Raises the kernel's shared-memory limit once per (kernel, device).
 template <int BN, bool MX>
 cudaError_t gemm_prepare() {
@@ -336,10 +368,16 @@ template <int BN, bool MX>
 cudaError_t launch_gemm_bn(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_ts,
                            const uint8_t* b_codes, const uint8_t* b_scales, const float* b_ts,
                            int64_t M, int64_t N, int64_t K, uint16_t* out, int64_t ldo, cudaStream_t st) {
-  alignas(64) CUtensorMap ma, mb;
+  using C = GemmCfg<BN, MX>;
+  alignas(64) CUtensorMap ma, mb, msa, msb;
   cudaError_t e = make_codes_map(a_codes, M, K, kBM, &ma);
   if (e != cudaSuccess) return e;
   e = make_codes_map(b_codes, N, K, BN, &mb);
+  if (e != cudaSuccess) return e;
+  const int64_t row_tiles = K / (MX ? 128 : 64);
+  e = make_scales_map(a_scales, M / 128 * row_tiles, C::kSfTiles, &msa);
+  if (e != cudaSuccess) return e;
+  e = make_scales_map(b_scales, N / 128 * row_tiles, C::kSfTiles, &msb);
   if (e != cudaSuccess) return e;
   e = gemm_prepare<BN, MX>();
   if (e != cudaSuccess) return e;
@@ -362,7 +400,7 @@ cudaError_t launch_gemm_bn(const uint8_t* a_codes, const uint8_t* a_scales, cons
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, MX>, ma, mb, a_scales, b_scales, a_ts, b_ts,
+  e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, MX>, ma, mb, msa, msb, a_ts, b_ts,
                          reinterpret_cast<__nv_bfloat16*>(out), ldo, M, N, K, status);
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -283,6 +283,7 @@ def test_gemm_validation():
     assert g(a=FAKE + 8) == _lib.FP4Q_ERR_ALIGN       # codes 16-byte aligned
     assert g(sa=FAKE + 4) == _lib.FP4Q_ERR_ALIGN
     assert g(ldo=132) == _lib.FP4Q_ERR_ALIGN          # 16-byte output rows
+    assert g(M=1 << 16, K=1 << 31) == _lib.FP4Q_ERR_SHAPE   # over 2^31 - 1 scale tiles
     assert g(M=0) == _lib.FP4Q_OK                     # empty: nothing to do
     mx = lambda M=128, N=128, K=256, ldo=128, a=FAKE, sa=FAKE, out=FAKE: lib.fp4q_gemm_mxfp4(
         a, sa, FAKE, FAKE, M, N, K, out, ldo, None)
