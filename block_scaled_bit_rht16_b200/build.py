@@ -40,7 +40,7 @@ def _stale(target, deps):
 
 def build(force: bool = False, verbose: bool = False) -> str:
     """Compile every csrc/*.cu and link libfp4q.so; returns its path."""
-    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + \
+    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
         [os.path.join(HERE, "..", "include", "fp4q.h"), __file__]
     if not force and not _stale(LIB, deps):
         return LIB

@@ -7,6 +7,7 @@
 
 #include "../../include/fp4q.h"
 #include "fp4q_kernels.cuh"
+#include "fp4q_launch.h"
 
 using namespace fp4q;
 

@@ -12,6 +12,7 @@
 
 #include "../../include/fp4q.h"
 #include "fp4q_kernels.cuh"
+#include "fp4q_launch.h"
 
 namespace {
 

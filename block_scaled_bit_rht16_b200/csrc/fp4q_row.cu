@@ -23,6 +23,7 @@
 #include "fp4q_device.cuh"
 #include "fp4q_encode.cuh"
 #include "fp4q_kernels.cuh"
+#include "fp4q_launch.h"
 
 namespace fp4q {
 
