@@ -70,6 +70,22 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback (earlier measurement on this pool)"
 
 
+FALLBACK_BF16_TFLOPS = 1590.0   # earlier cuBLAS bf16 burst measurement on this machine
+FP4_OVER_BF16 = 4.0             # dense FP4 / bf16 tensor rate, B200 nominal (9 / 2.25 PFLOP/s)
+
+
+def fp4_tensor_peak():
+    """Dense FP4 tensor peak in TFLOP/s: the measured bf16 burst GEMM rate times the nominal
+    FP4/bf16 ratio."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]) * FP4_OVER_BF16, \
+                "measured bf16 burst (MEASURED_PEAKS.json bf16_tflops) x 4, the nominal FP4/bf16 ratio"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS * FP4_OVER_BF16, "fallback bf16 burst (earlier measurement on this pool) x 4"
+
+
 REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
                "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
@@ -780,6 +796,7 @@ def run_ours(args):
     del g_main, g_rem
     if world == 1 and not args.no_extras and args.workload == "linear1.5b-ufp4":
         extras["gated"] = measure_gated(args, stream, dev, l2, peak)
+        extras["consumer_gemm"] = measure_consumer_gemm(stream)
     if sampler:
         sampler.finish()
     if world > 1:
@@ -803,8 +820,8 @@ def run_ours(args):
         "clocks": clocks,
         "sustained": sustained,
     }
-    line.update({k: v for k, v in extras.items() if k not in ("ratios", "gated")})
-    for k in ("ratios", "gated"):
+    line.update({k: v for k, v in extras.items() if k not in ("ratios", "gated", "consumer_gemm")})
+    for k in ("ratios", "gated", "consumer_gemm"):
         if k in extras:
             line[k] = extras[k]
     if rank == 0 and world == 1 and not args.no_extras:
@@ -866,6 +883,72 @@ def measure_e2e(wl, stream, world, steps=30):
     return {"value": round(world * wl.bytes_per_step() / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": round(ms, 4), "pipelined": "upload, compute, download on 3 streams"}
+
+
+def measure_consumer_gemm(stream):
+    """The library's NVFP4 and MXFP4 GEMMs (the quantizer's consumers on the tensor cores) on
+    4096 x 4096 x 8192 operands quantized by the library, timed with CUDA events beside cuBLASLt's
+    FP4 GEMM on the same codes and scales, and checked to agree with it."""
+    import numpy as np
+    import torch
+    import torch.nn.functional as F
+    import block_scaled_bit_rht16_b200 as fq
+    from block_scaled_bit_rht16_b200 import synth
+    M = N = 4096
+    K = 8192
+    peak, peak_src = fp4_tensor_peak()
+    a_bits = synth.small(61, M, K, "t4")
+    b_bits = synth.small(62, N, K, "normal", 0.02)
+
+    def dev(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+
+    out = {}
+    with torch.cuda.stream(stream):
+        xa, xb = dev(a_bits), dev(b_bits)
+        mask = fq.sign_mask_from_seed(synth.sign_seed(2))
+        for fmt in ("nvfp4", "mxfp4"):
+            nv = fmt == "nvfp4"
+            cfg = fq.Config(grid=fq.FP4Q_GRID_E2M1, rht=1, sign_mask=mask, mma_scales=True,
+                            scale=fq.FP4Q_SCALE_E4M3_1x16_TENSOR if nv else fq.FP4Q_SCALE_UE8M0_1x32)
+            qa, qb = fq.rht_quantize(cfg, xa, stream=stream), fq.rht_quantize(cfg, xb, stream=stream)
+            ours = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            blk, sdt = (16, torch.float8_e4m3fn) if nv else (32, torch.float8_e8m0fnu)
+            recipe = F.ScalingType.BlockWise1x16 if nv else F.ScalingType.BlockWise1x32
+            sa = [qa.scales.view(sdt).reshape(M, K // blk)] + ([qa.tensor_scale] if nv else [])
+            sb = [qb.scales.view(sdt).reshape(K // blk, N)] + ([qb.tensor_scale] if nv else [])
+            rs = [recipe] + ([F.ScalingType.TensorWise] if nv else [])
+
+            def lib():
+                (fq.gemm_nvfp4 if nv else fq.gemm_mxfp4)(qa, qb, out=ours, stream=stream)
+
+            def cublaslt():
+                return F.scaled_mm(qa.codes.view(torch.float4_e2m1fn_x2), qb.codes.view(torch.float4_e2m1fn_x2).t(),
+                                   sa, rs, sb, rs, swizzle_a=[F.SwizzleType.SWIZZLE_32_4_4],
+                                   swizzle_b=[F.SwizzleType.SWIZZLE_32_4_4], output_dtype=torch.bfloat16)
+            lib()
+            same = bool(torch.equal(ours, cublaslt()))
+            ms = {}
+            for name, fn in (("library", lib), ("cublaslt", cublaslt)):
+                for _ in range(3):
+                    fn()
+                t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize()
+                t0.record(stream)
+                for _ in range(20):
+                    fn()
+                t1.record(stream)
+                torch.cuda.synchronize()
+                ms[name] = t0.elapsed_time(t1) / 20
+            tf = 2.0 * M * N * K / (ms["library"] * 1e-3) / 1e12
+            out[fmt] = {"shape": [M, N, K], "ms": round(ms["library"], 4), "tflops": round(tf, 1),
+                        "cublaslt_ms": round(ms["cublaslt"], 4),
+                        "vs_cublaslt": round(ms["cublaslt"] / ms["library"], 3),
+                        "identical_to_cublaslt": same,
+                        "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak, "unit": "TFLOP/s",
+                                     "frac": round(tf / peak, 4), "peak_source": peak_src}}
+            del qa, qb, ours
+    return out
 
 
 def measure_ratios(args, stream, dev, l2, fused_step_ms):

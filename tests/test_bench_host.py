@@ -185,3 +185,13 @@ def test_issue_roofline_arithmetic():
     assert abs(r["frac"] - 115174472 / 0.1396e-3 / (148 * 4 * 1965e6)) < 1e-4
     assert r["warp_instructions_per_launch"] == 115174472
     assert bench.max_sm_mhz({"sm_max_mhz": 1800.0}) > 0
+
+
+def test_fp4_tensor_peak_from_the_measured_bf16_rate(tmp_path, monkeypatch):
+    import json
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6540.2, "bf16_tflops": 1600.0}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peak, src = bench.fp4_tensor_peak()
+    assert peak == 6400.0 and "measured" in src
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path / "absent"))
+    assert bench.fp4_tensor_peak()[0] == bench.FALLBACK_BF16_TFLOPS * 4
