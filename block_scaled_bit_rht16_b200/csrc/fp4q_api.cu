@@ -450,7 +450,7 @@ fp4q_status fp4q_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales, con
                             int64_t M, int64_t N, int64_t K, void* out, int64_t ldo,
                             fp4q_stream_t stream) {
   if (M < 0 || N < 0 || K < 256 || M % 128 != 0 || N % 128 != 0 || K % 256 != 0) return FP4Q_ERR_SHAPE;
-  if (M / 128 > 65535 || K > (int64_t(1) << 31) || (M / 128) * (N / 128) > INT32_MAX) return FP4Q_ERR_SHAPE;
+  if (M / 128 > 65535 || K > (int64_t(1) << 31) || (M / 128) * (N / 128) > (int64_t(1) << 30)) return FP4Q_ERR_SHAPE;
   if ((M / 128) * (K / 64) > INT32_MAX || (N / 128) * (K / 64) > INT32_MAX) return FP4Q_ERR_SHAPE;   // scale tiles
   if (M > 0 && N > 0 && ldo < N) return FP4Q_ERR_SHAPE;
   if (M == 0 || N == 0) return FP4Q_OK;
@@ -469,7 +469,7 @@ fp4q_status fp4q_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, con
                             const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, void* out, int64_t ldo,
                             fp4q_stream_t stream) {
   if (M < 0 || N < 0 || K < 256 || M % 128 != 0 || N % 128 != 0 || K % 256 != 0) return FP4Q_ERR_SHAPE;
-  if (M / 128 > 65535 || K > (int64_t(1) << 31) || (M / 128) * (N / 128) > INT32_MAX) return FP4Q_ERR_SHAPE;
+  if (M / 128 > 65535 || K > (int64_t(1) << 31) || (M / 128) * (N / 128) > (int64_t(1) << 30)) return FP4Q_ERR_SHAPE;
   if ((M / 128) * (K / 64) > INT32_MAX || (N / 128) * (K / 64) > INT32_MAX) return FP4Q_ERR_SHAPE;   // scale tiles
   if (M > 0 && N > 0 && ldo < N) return FP4Q_ERR_SHAPE;
   if (M == 0 || N == 0) return FP4Q_OK;

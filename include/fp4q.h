@@ -266,7 +266,7 @@ fp4q_status fp4q_rht_quantize_grouped(const fp4q_config* cfg, const void* x, int
  * 16-point rotation is orthogonal). Products accumulate in FP32.
  *  a_codes uint8 [M, K/2], a_scales uint8 [M, K/16] in the MMA layout, a_tensor_scale one device
  *  float; b_* the same with N rows; out bf16 [M, ldo], ldo >= N, ldo % 8 == 0.
- *  M and N multiples of 128 (M at most 65535 * 128, at most 2^31 - 1 tiles of 128 x 128, and
+ *  M and N multiples of 128 (M at most 65535 * 128, at most 2^30 tiles of 128 x 128, and
  *  M / 128 * K / 64 and N / 128 * K / 64 at most 2^31 - 1), K a multiple of 256 up to 2^31 (else
  *  FP4Q_ERR_SHAPE);
  *  every pointer 16-byte aligned (tensor scales 4) (else FP4Q_ERR_ALIGN); a null pointer:

@@ -277,7 +277,7 @@ def test_gemm_validation():
     assert g(K=0) == _lib.FP4Q_ERR_SHAPE
     assert g(ldo=64) == _lib.FP4Q_ERR_SHAPE           # ldo < N
     assert g(M=65536 * 128) == _lib.FP4Q_ERR_SHAPE    # beyond the tile grid's y limit
-    assert g(M=65535 * 128, N=(1 << 16) * 128, ldo=(1 << 16) * 128) == _lib.FP4Q_ERR_SHAPE   # over 2^31 - 1 tiles
+    assert g(M=65535 * 128, N=(1 << 16) * 128, ldo=(1 << 16) * 128) == _lib.FP4Q_ERR_SHAPE   # over 2^30 tiles
     assert g(a=None) == _lib.FP4Q_ERR_INVALID_ARG
     assert g(ts=None) == _lib.FP4Q_ERR_INVALID_ARG
     assert g(a=FAKE + 8) == _lib.FP4Q_ERR_ALIGN       # codes 16-byte aligned
