@@ -796,6 +796,11 @@ def run_ours(args):
     del g_main, g_rem
     if world == 1 and not args.no_extras and args.workload == "linear1.5b-ufp4":
         extras["gated"] = measure_gated(args, stream, dev, l2, peak)
+        g = extras["gated"]
+        if "ratios" in extras and "laplace16k-if4" in g and "laplace16k-nvfp4" in g:
+            # IF4's selection against NVFP4, both with the tensor scale computed (the IF4 page: ~+15%)
+            extras["ratios"]["if4_over_nvfp4"] = round(g["laplace16k-if4"]["us_per_step"] /
+                                                       g["laplace16k-nvfp4"]["us_per_step"], 3)
         extras["consumer_gemm"] = measure_consumer_gemm(stream)
     if sampler:
         sampler.finish()
