@@ -98,3 +98,22 @@ def test_mxfp4_gemm_agrees_with_cublaslt_and_timing():
                                          tf["cublaslt"], sq))
     # both accumulate exact products in FP32 (in different orders) and round to bf16
     assert sq > 45.0
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+def test_gemm_into_a_row_pitched_output(fmt):
+    # out with ldo = N + 64: the result equals the contiguous one, the pad columns stay untouched
+    import torch
+    M, N, K = 512, 512, 1024
+    scale = fq.FP4Q_SCALE_E4M3_1x16_TENSOR if fmt == "nvfp4" else fq.FP4Q_SCALE_UE8M0_1x32
+    cfg = fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=scale, rht=1,
+                    sign_mask=fq.sign_mask_from_seed(synth.sign_seed(2)), mma_scales=True)
+    qa = fq.rht_quantize(cfg, to_dev(synth.small(91, M, K, "t4")))
+    qb = fq.rht_quantize(cfg, to_dev(synth.small(92, N, K, "normal", 0.02)))
+    gemm = fq.gemm_nvfp4 if fmt == "nvfp4" else fq.gemm_mxfp4
+    ref = gemm(qa, qb)
+    wide = torch.full((M, N + 64), -7.0, dtype=torch.bfloat16, device="cuda")
+    gemm(qa, qb, out=wide[:, :N])
+    torch.cuda.synchronize()
+    assert torch.equal(wide[:, :N], ref)
+    assert bool((wide[:, N:] == -7.0).all())
