@@ -168,7 +168,11 @@ fp4q_status fp4q_rht_quantize(const fp4q_config* cfg, const void* x, int64_t row
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   WsHeader* ws = reinterpret_cast<WsHeader*>(workspace);
-  if (need > 0) {
+  // the header is read only for a computed tensor scale (its amax) and for statistics; with a
+  // given scale the quantize kernel is the call's only work (no memset between back-to-back
+  // launches, which would also cut their programmatic overlap)
+  const bool use_ws = compute_alpha || want_stats;
+  if (use_ws) {
     if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), s) != cudaSuccess) return FP4Q_ERR_CUDA;
   }
   if (empty) {
@@ -181,7 +185,7 @@ fp4q_status fp4q_rht_quantize(const fp4q_config* cfg, const void* x, int64_t row
   a.deq = want_deq ? static_cast<uint16_t*>(dequant) : nullptr;
   a.ts_in = (nv && tensor_scale_given) ? tensor_scale : nullptr;
   a.ts_out = compute_alpha ? tensor_scale : nullptr;
-  a.ws = need > 0 ? ws : nullptr;
+  a.ws = use_ws ? ws : nullptr;
   a.partials = want_stats ? reinterpret_cast<double*>(static_cast<char*>(workspace) + sizeof(WsHeader)) : nullptr;
 
   if (compute_alpha) {
