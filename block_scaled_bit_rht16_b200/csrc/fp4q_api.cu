@@ -173,7 +173,7 @@ fp4q_status fp4q_rht_quantize(const fp4q_config* cfg, const void* x, int64_t row
   // launches, which would also cut their programmatic overlap)
   const bool use_ws = compute_alpha || want_stats;
   if (use_ws) {
-    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), s) != cudaSuccess) return FP4Q_ERR_CUDA;
+    if (launch_ws_reset(ws, s) != cudaSuccess) return FP4Q_ERR_CUDA;
   }
   if (empty) {
     if (compute_alpha && cudaMemsetAsync(tensor_scale, 0, sizeof(float), s) != cudaSuccess)
@@ -265,7 +265,7 @@ fp4q_status fp4q_tensor_scale(const fp4q_config* cfg, const void* x, int64_t row
   if (workspace == nullptr || workspace_bytes < sizeof(WsHeader)) return FP4Q_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   WsHeader* ws = reinterpret_cast<WsHeader*>(workspace);
-  if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), s) != cudaSuccess) return FP4Q_ERR_CUDA;
+  if (launch_ws_reset(ws, s) != cudaSuccess) return FP4Q_ERR_CUDA;
   if (!empty) {
     QuantArgs a{};
     a.x = static_cast<const uint16_t*>(x);
