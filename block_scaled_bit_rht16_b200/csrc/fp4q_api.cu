@@ -173,7 +173,7 @@ fp4q_status fp4q_rht_quantize(const fp4q_config* cfg, const void* x, int64_t row
   // launches, which would also cut their programmatic overlap)
   const bool use_ws = compute_alpha || want_stats;
   if (use_ws) {
-    if (launch_ws_reset(ws, s) != cudaSuccess) return FP4Q_ERR_CUDA;
+    if (launch_ws_clear(ws, sizeof(WsHeader), s) != cudaSuccess) return FP4Q_ERR_CUDA;
   }
   if (empty) {
     if (compute_alpha && cudaMemsetAsync(tensor_scale, 0, sizeof(float), s) != cudaSuccess)
@@ -235,7 +235,7 @@ fp4q_status fp4q_rht_quantize_grouped(const fp4q_config* cfg, const void* x, int
   const size_t need = given ? 0 : fp4q_grouped_workspace_size(cfg, n_groups);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return FP4Q_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (!given && cudaMemsetAsync(workspace, 0, need, s) != cudaSuccess) return FP4Q_ERR_CUDA;
+  if (!given && launch_ws_clear(workspace, need, s) != cudaSuccess) return FP4Q_ERR_CUDA;
   QuantArgs a = base_args(cfg, x, rows, cols, ld, codes, scales);
   a.group_off = group_offsets;
   a.n_groups = n_groups;
@@ -265,7 +265,7 @@ fp4q_status fp4q_tensor_scale(const fp4q_config* cfg, const void* x, int64_t row
   if (workspace == nullptr || workspace_bytes < sizeof(WsHeader)) return FP4Q_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   WsHeader* ws = reinterpret_cast<WsHeader*>(workspace);
-  if (launch_ws_reset(ws, s) != cudaSuccess) return FP4Q_ERR_CUDA;
+  if (launch_ws_clear(ws, sizeof(WsHeader), s) != cudaSuccess) return FP4Q_ERR_CUDA;
   if (!empty) {
     QuantArgs a{};
     a.x = static_cast<const uint16_t*>(x);

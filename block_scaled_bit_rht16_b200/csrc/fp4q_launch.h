@@ -35,6 +35,6 @@ cudaError_t launch_gemm_mxfp4(const uint8_t* a_codes, const uint8_t* a_scales, c
                               const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, uint16_t* out,
                               int64_t ldo, cudaStream_t st);
 
-cudaError_t launch_ws_reset(WsHeader* ws, cudaStream_t st);   // fp4q_workspace.cu
+cudaError_t launch_ws_clear(void* p, size_t bytes, cudaStream_t st);   // fp4q_workspace.cu; bytes % 16 == 0
 
 }  // namespace fp4q

@@ -1,7 +1,8 @@
-// fp4q_workspace.cu -- clearing the workspace header before a call that accumulates into it (the
-// rotated tensor's amax for a computed E4M3 tensor scale, the statistics record counts).
+// fp4q_workspace.cu -- clearing workspace before a call that accumulates into it (the header's
+// rotated-tensor amax for a computed E4M3 tensor scale and its statistics record counts; the
+// grouped call's per-group amax slots).
 //
-// A one-CTA kernel rather than a memset: launched with programmatic stream serialization like
+// A kernel rather than a memset: launched with programmatic stream serialization like
 // the quantize kernels, it keeps a chain of back-to-back calls (quantize, clear, amax, quantize,
 // ...) free of the copy-engine node a memset would put between them. It waits for the preceding
 // kernel on the stream (which may still be reading the header) before it clears it.
@@ -12,18 +13,22 @@
 namespace fp4q {
 namespace {
 
-__global__ void __launch_bounds__(kThreads) ws_reset_kernel(WsHeader* ws) {
+// Zeroes n16 16-byte words at p, grid-stride.
+__global__ void __launch_bounds__(kThreads) ws_clear_kernel(uint4* p, size_t n16) {
   pdl_enter();
-  constexpr int kWords = (int)(sizeof(WsHeader) / sizeof(uint32_t));
-  static_assert(kWords <= kThreads, "one word per thread");
-  if (threadIdx.x < kWords) reinterpret_cast<uint32_t*>(ws)[threadIdx.x] = 0u;
+  const size_t stride = (size_t)gridDim.x * kThreads;
+  for (size_t i = (size_t)blockIdx.x * kThreads + threadIdx.x; i < n16; i += stride) p[i] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 }  // namespace
 
-cudaError_t launch_ws_reset(WsHeader* ws, cudaStream_t st) {
+cudaError_t launch_ws_clear(void* p, size_t bytes, cudaStream_t st) {
+  if (bytes == 0) return cudaSuccess;
+  if (bytes % 16 != 0 || reinterpret_cast<uintptr_t>(p) % 16 != 0) return cudaErrorInvalidValue;
+  const size_t n16 = bytes / 16;
+  const size_t blocks = (n16 + kThreads - 1) / kThreads;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(1);
+  cfg.gridDim = dim3((unsigned)(blocks < 592 ? blocks : 592));
   cfg.blockDim = dim3(kThreads);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -31,7 +36,7 @@ cudaError_t launch_ws_reset(WsHeader* ws, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, ws_reset_kernel, ws);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, ws_clear_kernel, reinterpret_cast<uint4*>(p), n16);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
