@@ -375,7 +375,7 @@ class RowWorkload(Workload):
             y = torch.empty_like(x) if self.unfused else None
             self.sets.append((x, out, y))
         if self.cfg.scale == fq.FP4Q_SCALE_E4M3_1x16_TENSOR and not self.given:
-            self.launches_per_step = 2   # amax pass + quantize pass
+            self.launches_per_step = 3   # workspace clear + amax pass + quantize pass
 
     def elements(self):
         return self.rows * self.cols
@@ -455,7 +455,7 @@ class GroupedWorkload(RowWorkload):
         for _, out, _ in self.sets:
             out.tensor_scale = torch.zeros(n, dtype=torch.float32, device=device)
             out.workspace = torch.empty(nws, dtype=torch.uint8, device=device)
-        self.launches_per_step = 3   # grouped amax, per-group alpha, quantize
+        self.launches_per_step = 4   # slot clear, grouped amax, per-group alpha, quantize
 
     def enqueue(self, i, stream):
         x, out, _ = self.sets[i % self.R]
