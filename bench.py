@@ -584,7 +584,7 @@ def make_workload(name, sign_mask_from_seed=None):
                 "if4": fq.FP4Q_GRID_IF4}[fmt]
         scale = fq.FP4Q_SCALE_UE8M0_1x32 if kind == "mxfp4" else fq.FP4Q_SCALE_E4M3_1x16_TENSOR
         cfg = fq.Config(grid=grid, scale=scale, rht=1, sign_mask=mask)
-        key = {"nvfp4": "lean_nv_kernel<E2M1,rotation,flat>", "nvint4": "lean_nv_kernel<INT4,rotation,flat>",
+        key = {"nvfp4": "lean_nv_pair_kernel<E2M1,rotation>", "nvint4": "lean_nv_pair_kernel<INT4,rotation>",
                "if4": "lean_nv_kernel<IF4,rotation,flat>", "mxfp4": "quantize_kernel<E2M1,UE8M0>"}[fmt]
         if kind in ("nvfp4", "nvint4", "if4"):
             key += "+amax_kernel<rotation,flat>"

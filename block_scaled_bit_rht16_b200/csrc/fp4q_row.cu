@@ -527,6 +527,140 @@ __global__ void __launch_bounds__(kThreads, G == kIF4 ? 3 : (GROUPED ? 1 : 5)) l
   }
 }
 
+// Codes of rotated block u of a flat tensor from its scale table entry e, recomputed from the
+// input (the same loads and operations as the pair kernel's): encode_lean_dv with the clamp, for
+// scales outside the correction step's exact range. Not inlined, and handed only the arguments'
+// address (a grid constant) and scalars, so that the rare path takes neither registers nor a
+// stack frame from the common one.
+template <int G>
+__device__ __noinline__ uint2 nv_block_slow(const QuantArgs* a, uint32_t u, float4 e) {
+  uint4 lo, hi;
+  load16(a->x + (size_t)u * 16, true, lo, hi);
+  float2 P[8];
+  unpack16(lo, hi, a->flip_lo, a->flip_hi, P);
+  fwht16(P);
+  return encode_lean_dv<G, true, true>(P, e.x, table_divider(e), absmax16(P));
+}
+
+// lean_nv_kernel for a rotated flat tensor with one tensor scale (E2M1, E1M2, INT4): two
+// adjacent blocks per thread per iteration, as lean_pair_kernel does for the FP32 scale. The
+// block-scale quotients of the pair come from one packed correction step and one paired E4M3
+// conversion; the element quotients from packed steps on the two blocks' dividers (looked up by
+// scale code in the CTA's table); the same IEEE operations in the same order as the one-block
+// kernel. The pair's two scale bytes are adjacent in either scale layout (the MMA layout has a
+// multiple of four blocks per row), so they leave as one 16-bit store.
+template <int G>
+__global__ void __launch_bounds__(kThreads) lean_nv_pair_kernel(const __grid_constant__ QuantArgs a) {
+  constexpr float qmax = GridInfo<G>::qmax;
+  constexpr float kF = lean_divisor_factor<G, true>();
+  constexpr float kVScale = (G == kE1M2) ? 4.0f : 1.0f;
+  pdl_enter();
+  float alpha;
+  if (a.ts_in != nullptr) {
+    alpha = *a.ts_in;
+  } else {
+    alpha = __fdiv_rn(__uint_as_float(a.ws->amax_bits), __fmul_rn(qmax, 448.0f));
+    if (a.ts_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *a.ts_out = alpha;
+  }
+  const float denom = __fmul_rn(alpha, qmax);
+  const Divider dd = make_divider(denom, 1.0f);
+  __shared__ float4 s_tab[128];
+  if (threadIdx.x < 128) {
+    const float sd = __fmul_rn(e4m3_to_f32(threadIdx.x), alpha);
+    const Divider dv = make_divider(sd, kF);
+    s_tab[threadIdx.x] = make_float4(sd, dv.S, dv.R, dv.fast ? 1.0f : 0.0f);
+  }
+  __syncthreads();
+  const uint32_t npairs = (uint32_t)(a.nunits >> 1);
+  const uint32_t stride = gridDim.x * kThreads;
+  uint32_t p = blockIdx.x * kThreads + threadIdx.x;
+  uint4 v[4];
+  if (p < npairs) {
+    load16(a.x + (size_t)p * 32, true, v[0], v[1]);
+    load16(a.x + (size_t)p * 32 + 16, true, v[2], v[3]);
+  }
+  for (; p < npairs; p += stride) {
+    uint4 nv[4] = {v[0], v[1], v[2], v[3]};
+    if (p + stride < npairs) {
+      load16(a.x + (size_t)(p + stride) * 32, true, nv[0], nv[1]);
+      load16(a.x + (size_t)(p + stride) * 32 + 16, true, nv[2], nv[3]);
+    }
+    float2 A[16];
+    unpack16_pair(v[0], v[1], v[2], v[3], a.flip_lo, a.flip_hi, A);
+    fwht16_pair(A);
+    const float2 am = absmax16_pair(A);   // amax of the raw butterfly outputs
+    const float2 ay = __fmul2_rn(am, make_float2(0.25f, 0.25f));
+    float2 delta = dd.fast ? div2(dd, ay) : make_float2(0.0f, 0.0f);
+    // outside the fast range, and for quotients too large for the correction step, the IEEE
+    // division (as in the one-block kernel)
+    if ((!dd.fast || !(delta.x < 0x1p+64f)) && denom > 0.0f) delta.x = __fdiv_rn(ay.x, denom);
+    if ((!dd.fast || !(delta.y < 0x1p+64f)) && denom > 0.0f) delta.y = __fdiv_rn(ay.y, denom);
+    uint16_t sb2;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(sb2) : "f"(delta.y), "f"(delta.x));
+    // the quotients are non-negative, so both codes are in 0..126
+    const float4 e0 = s_tab[sb2 & 0x7Fu], e1 = s_tab[(sb2 >> 8) & 0x7Fu];
+    uint2 w0, w1;
+    if ((e0.w != 0.0f || e0.x == 0.0f) && (e1.w != 0.0f || e1.x == 0.0f)) {
+      // a zero-scale lane divides by 1 (its codes are zeros whatever its quotients)
+      const float2 R2 = make_float2(e0.x == 0.0f ? 1.0f : e0.z, e1.x == 0.0f ? 1.0f : e1.z);
+      const float2 nS2 = make_float2(e0.x == 0.0f ? -1.0f : -e0.y, e1.x == 0.0f ? -1.0f : -e1.y);
+      float q0[16], q1[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float2 qa = __fmul2_rn(A[e], R2);
+        const float2 q = __ffma2_rn(__ffma2_rn(qa, nS2, A[e]), R2, qa);
+        q0[e] = q.x;
+        q1[e] = q.y;
+      }
+      if constexpr (!kIsE2M1<G>) {   // the E2M1 conversion saturates by itself
+        constexpr float lim = qmax / kVScale;
+        constexpr float half_above = (G == kE1M2 ? 3.75f : 7.5f) / kVScale;   // qmax + step / 2
+        const float2 qa = __fmul2_rn(am, R2);
+        const float2 qm = __ffma2_rn(__ffma2_rn(qa, nS2, am), R2, qa);
+        if (!(qm.x < half_above)) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) q0[e] = fminf(fmaxf(q0[e], -lim), lim);
+        }
+        if (!(qm.y < half_above)) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) q1[e] = fminf(fmaxf(q1[e], -lim), lim);
+        }
+      }
+      w0 = e0.x == 0.0f ? make_uint2(0u, 0u) : lean_codes<G, true>(q0, q0);
+      w1 = e1.x == 0.0f ? make_uint2(0u, 0u) : lean_codes<G, true>(q1, q1);
+    } else {
+      // a scale outside the correction step's exact range (tiny or huge data)
+      w0 = nv_block_slow<G>(&a, 2 * p, e0);
+      w1 = nv_block_slow<G>(&a, 2 * p + 1, e1);
+    }
+    __stcs(reinterpret_cast<uint4*>(a.codes) + p, make_uint4(w0.x, w0.y, w1.x, w1.y));
+    const int64_t slot = scale_slot((int64_t)p * 2, a.units_per_row, a.mma_scales);
+    *reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(a.scales) + slot) = sb2;
+    v[0] = nv[0];
+    v[1] = nv[1];
+    v[2] = nv[2];
+    v[3] = nv[3];
+  }
+  // an odd last block (row-major scales only: the MMA layout has an even count)
+  if ((a.nunits & 1) && blockIdx.x == 0 && threadIdx.x == 0) {
+    const uint32_t u = (uint32_t)a.nunits - 1u;
+    uint4 lo, hi;
+    load16(a.x + (size_t)u * 16, true, lo, hi);
+    float2 P[8];
+    unpack16(lo, hi, a.flip_lo, a.flip_hi, P);
+    fwht16(P);
+    const float amax_raw = absmax16(P);
+    const float amax_y = __fmul_rn(amax_raw, 0.25f);
+    float delta = 0.0f;
+    if (dd.fast) delta = div2(dd, make_float2(amax_y, 0.0f)).x;
+    if ((!dd.fast || !(delta < 0x1p+64f)) && denom > 0.0f) delta = __fdiv_rn(amax_y, denom);
+    const uint32_t sbyte = cvt_e4m3(delta);
+    const float4 e = s_tab[sbyte];
+    __stcs(reinterpret_cast<uint2*>(a.codes) + u, encode_lean_dv<G, true, true>(P, e.x, table_divider(e), amax_raw));
+    reinterpret_cast<uint8_t*>(a.scales)[scale_slot((int64_t)u, a.units_per_row, a.mma_scales)] = (uint8_t)sbyte;
+  }
+}
+
 // Amax of the rotated tensor: per-warp maximum of the bit patterns (non-negative floats order
 // like unsigned integers), one atomicMax per warp into the workspace header. Like the lean
 // kernels: rotation and layout fixed at compile time, the next block's load in flight.
@@ -915,9 +1049,21 @@ cudaError_t launch_lean_nv4(const QuantArgs& a, cudaStream_t st) {
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
+template <int G>
+cudaError_t launch_lean_nv_pair(const QuantArgs& a, cudaStream_t st) {
+  auto k = lean_nv_pair_kernel<G>;
+  const cudaError_t e = launch_pdl(k, persistent_grid(k, (a.nunits + 1) / 2), st, a);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 template <int G, bool GROUPED = false>
 cudaError_t launch_lean_nv(const QuantArgs& a, cudaStream_t st) {
   const bool rht = a.c != 1.0f, flat = flat_launch(a);
+  // one tensor scale, rotated, flat: two blocks per thread (IF4's two candidates stay on one)
+  if constexpr (!GROUPED && G != kIF4) {
+    if (rht && flat && reinterpret_cast<uintptr_t>(a.codes) % 16 == 0 && reinterpret_cast<uintptr_t>(a.scales) % 2 == 0)
+      return launch_lean_nv_pair<G>(a, st);
+  }
   if (rht) return flat ? launch_lean_nv4<G, true, true, GROUPED>(a, st) : launch_lean_nv4<G, true, false, GROUPED>(a, st);
   return flat ? launch_lean_nv4<G, false, true, GROUPED>(a, st) : launch_lean_nv4<G, false, false, GROUPED>(a, st);
 }
