@@ -549,8 +549,8 @@ __device__ __noinline__ uint2 nv_block_slow(const QuantArgs* a, uint32_t u, floa
 // scale code in the CTA's table); the same IEEE operations in the same order as the one-block
 // kernel. The pair's two scale bytes are adjacent in either scale layout (the MMA layout has a
 // multiple of four blocks per row), so they leave as one 16-bit store.
-template <int G>
-__global__ void __launch_bounds__(kThreads) lean_nv_pair_kernel(const __grid_constant__ QuantArgs a) {
+template <int G, int TH>
+__global__ void __launch_bounds__(TH) lean_nv_pair_kernel(const __grid_constant__ QuantArgs a) {
   constexpr float qmax = GridInfo<G>::qmax;
   constexpr float kF = lean_divisor_factor<G, true>();
   constexpr float kVScale = (G == kE1M2) ? 4.0f : 1.0f;
@@ -565,6 +565,7 @@ __global__ void __launch_bounds__(kThreads) lean_nv_pair_kernel(const __grid_con
   const float denom = __fmul_rn(alpha, qmax);
   const Divider dd = make_divider(denom, 1.0f);
   __shared__ float4 s_tab[128];
+  static_assert(TH >= 128, "one table entry per thread");
   if (threadIdx.x < 128) {
     const float sd = __fmul_rn(e4m3_to_f32(threadIdx.x), alpha);
     const Divider dv = make_divider(sd, kF);
@@ -572,8 +573,8 @@ __global__ void __launch_bounds__(kThreads) lean_nv_pair_kernel(const __grid_con
   }
   __syncthreads();
   const uint32_t npairs = (uint32_t)(a.nunits >> 1);
-  const uint32_t stride = gridDim.x * kThreads;
-  uint32_t p = blockIdx.x * kThreads + threadIdx.x;
+  const uint32_t stride = gridDim.x * TH;
+  uint32_t p = blockIdx.x * TH + threadIdx.x;
   uint4 v[4];
   if (p < npairs) {
     load16(a.x + (size_t)p * 32, true, v[0], v[1]);
@@ -970,18 +971,18 @@ __global__ void __launch_bounds__(kThreads) conversion_check_kernel(unsigned lon
 // Resident CTAs of `kernel` on the current device (SM count x occupancy), queried once per
 // (kernel, device) and cached, so that launches inside a stream capture do no queries.
 template <class K>
-int resident_ctas(K kernel) {
+int resident_ctas(K kernel, int threads = kThreads) {
   static std::mutex mu;
   static std::map<std::pair<const void*, int>, int> cache;
   int dev = 0;
   cudaGetDevice(&dev);
-  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+  const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev * 4096 + threads);
   std::lock_guard<std::mutex> lock(mu);
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
   int sms = 148, per_sm = 1;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0);
   const int n = sms * std::max(per_sm, 1);
   cache.emplace(key, n);
   return n;
@@ -989,10 +990,10 @@ int resident_ctas(K kernel) {
 
 // Launch with programmatic stream serialization (the kernels call pdl_enter() first).
 template <class... Args>
-cudaError_t launch_pdl(void (*kernel)(Args...), int grid, cudaStream_t st, Args... args) {
+cudaError_t launch_pdl_n(void (*kernel)(Args...), int grid, int threads, cudaStream_t st, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3((unsigned)threads);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1002,10 +1003,15 @@ cudaError_t launch_pdl(void (*kernel)(Args...), int grid, cudaStream_t st, Args.
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+template <class... Args>
+cudaError_t launch_pdl(void (*kernel)(Args...), int grid, cudaStream_t st, Args... args) {
+  return launch_pdl_n(kernel, grid, kThreads, st, args...);
+}
+
 template <class K>
-int persistent_grid(K kernel, int64_t work_threads) {
-  const int64_t need = (work_threads + kThreads - 1) / kThreads;
-  return (int)std::max<int64_t>(1, std::min<int64_t>(need, resident_ctas(kernel)));
+int persistent_grid(K kernel, int64_t work_threads, int threads = kThreads) {
+  const int64_t need = (work_threads + threads - 1) / threads;
+  return (int)std::max<int64_t>(1, std::min<int64_t>(need, resident_ctas(kernel, threads)));
 }
 
 template <int G, int S, int R, bool STATS>
@@ -1051,8 +1057,12 @@ cudaError_t launch_lean_nv4(const QuantArgs& a, cudaStream_t st) {
 
 template <int G>
 cudaError_t launch_lean_nv_pair(const QuantArgs& a, cudaStream_t st) {
-  auto k = lean_nv_pair_kernel<G>;
-  const cudaError_t e = launch_pdl(k, persistent_grid(k, (a.nunits + 1) / 2), st, a);
+  // E2M1 takes 72 registers a thread, at which 128-thread CTAs let 28 warps reside per SM against
+  // 24 in three 256-thread CTAs (measured 40.0 against 41.0 us on a 16384 x 5120 tensor); E1M2
+  // and INT4 take 80, where smaller CTAs gain no warps (43.3 against 42.3 us for INT4)
+  constexpr int kTh = G == kE2M1 ? 128 : 256;
+  auto k = lean_nv_pair_kernel<G, kTh>;
+  const cudaError_t e = launch_pdl_n(k, persistent_grid(k, (a.nunits + 1) / 2, kTh), kTh, st, a);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
