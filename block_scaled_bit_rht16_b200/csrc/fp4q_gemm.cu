@@ -1,28 +1,32 @@
-// fp4q_gemm.cu -- NVFP4 GEMM on the 5th-generation tensor cores (tcgen05, sm_100a) consuming the
-// quantizer's outputs unchanged: E2M1 codes (two per byte, element 2j in the low nibble) and
-// E4M3 block scales in the block-scaled MMA layout (FP4Q_OUT_SCALES_MMA), plus each operand's
-// FP32 tensor scale. D[m, n] = alpha_A alpha_B sum_k A[m, k] B[n, k], A and B both K-major
+// fp4q_gemm.cu -- NVFP4 and MXFP4 GEMMs on the 5th-generation tensor cores (tcgen05, sm_100a)
+// consuming the quantizer's outputs unchanged: E2M1 codes (two per byte, element 2j in the low
+// nibble) and block scales in the block-scaled MMA layout (FP4Q_OUT_SCALES_MMA): E4M3 per 16
+// elements plus each operand's FP32 tensor scale (NVFP4), or UE8M0 per 32 elements (MXFP4).
+// D[m, n] = alpha_A alpha_B sum_k A[m, k] B[n, k] (alpha = 1 for MXFP4), A and B both K-major
 // (rows of the quantized tensors), accumulated in FP32 in tensor memory, stored as bf16.
 //
 // The NVFP4 recipe is the hardware path of "低精度量化技术：IF4自适应数据类型的原理与应用"
 // (bxzpzcl.cn/news/2320061), section 3.2 (E4M3 block scale per 16 elements + FP32 tensor
-// scale); "FP4 训练 vs FP4 推理" (reports.10n1j.top) notes that Blackwell's FP4 tensor-core path
-// is E2M1-only.
+// scale); MXFP4 is the 32-element power-of-two block of "AMD全新研究揭示：FP4训练不稳定性源于结构误差
+// 而非随机性不足" (cannews.ca/article/21387); "FP4 训练 vs FP4 推理" (reports.10n1j.top) notes that
+// Blackwell's FP4 tensor-core path is E2M1-only.
 //
-// A persistent kernel: one CTA per SM (217 KB of shared memory, 512 tensor-memory columns)
-// walks the 128 x BN tiles of D (BN = 256 when N allows, else 128), tile i of a CTA being
-// blockIdx.x + i * gridDim.x with m fastest. The K dimension streams in 256-element steps through
-// a ring of shared-memory buffers that runs on across tiles. Six warps, three roles:
+// A persistent kernel: one CTA per SM (up to 217 KB of shared memory, 256 or 512 tensor-memory
+// columns) walks the 128 x BN tiles of D (BN = 256 when N allows, else 128), tile i of a CTA
+// being blockIdx.x + i * gridDim.x with m fastest. The K dimension streams in 256-element steps
+// through a ring of shared-memory buffers that runs on across tiles. Six warps, three roles:
 //   thread 0 (producer): per step the A and B code tiles (128 / BN rows x 128 bytes) by 2-D TMA
-//     copies with the 128-byte swizzle, and the scale blocks (four 512-byte MMA-layout tiles per
-//     128 rows) by 1-D bulk copies, all completing on the buffer's `full` mbarrier; a buffer is
-//     refilled once its `empty` barrier says the MMAs that read it have completed, so the next
-//     tile's operands load while the current tile drains;
+//     copies with the 128-byte swizzle, and the step's 512-byte MMA-layout scale tiles (per 128
+//     rows: four for NVFP4, two for MXFP4) by 3-D TMA copies whose zero-stride middle dimension
+//     lands each tile four times in a row (kSfRep), all completing on the buffer's `full`
+//     mbarrier; a buffer is refilled once its `empty` barrier says the MMAs that read it have
+//     completed, so the next tile's operands load while the current tile drains;
 //   thread 32 (MMA issuer): per tile, once `acc_empty` says the epilogue has read the previous
-//     accumulator, copies each step's scales into tensor memory (tcgen05.cp, 32 lanes x 128 bits,
-//     replicated to the four lane quarters), issues four MMAs of K = 64 (tcgen05.mma
-//     kind::mxf4nvf4, block16 scaling, M = 128, N = BN) and commits them to the buffer's `empty`
-//     barrier; the tile's last commit goes to `acc_full`;
+//     accumulator, copies each step's scales into tensor memory two tiles at a time
+//     (tcgen05.cp .128x256b: the replicated rows fill all four lane quarters), issues four MMAs
+//     of K = 64 (tcgen05.mma kind::mxf4nvf4, block16 with E4M3 or block32 with UE8M0 scales,
+//     M = 128, N = BN) and commits them to the buffer's `empty` barrier; the tile's last commit
+//     goes to `acc_full`;
 //   warps 2-5 (epilogue): warp w reads tensor-memory lanes 32 (w % 4) .. +31 (tcgen05.ld, 32
 //     columns at a time), scales by alpha_A alpha_B, stores bf16 rows, and arrives on `acc_empty`.
 // Every mbarrier wait is bounded by the global timer; a wait that gives up sets bit 0 of the
