@@ -421,71 +421,6 @@ __device__ __forceinline__ float2 absmax16_pair(const float2* A) {
   return make_float2(fmaxf(m0, fabsf(A[15].x)), fmaxf(m1, fabsf(A[15].y)));
 }
 
-// Stochastic-rounding codes of one block given as lane h of A, exactly as encode_sr gives them
-// (the path for blocks with quotients below the correction step's exact range).
-// Not inlined: the rare path must not take registers from the common one.
-template <int G>
-__device__ __noinline__ uint2 encode_sr_lane(const float2* A, int h, float s, float c,
-                                             uint64_t seedx, uint64_t quad0) {
-  if (s == 0.0f) return make_uint2(0u, 0u);
-  float2 P[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    P[i] = h ? make_float2(A[i].y, A[i + 8].y) : make_float2(A[i].x, A[i + 8].x);
-  return encode_sr<G>(P, s, c, seedx, quad0);
-}
-
-// Stochastic-rounding codes of the two blocks in A (block k: scale s.k, first logical index
-// 4 quad0_k), each exactly what encode_sr gives for it alone; c: 4 with rotation, else 1. Both
-// blocks' quotients come from one packed correction step and go straight into their decisions;
-// a block with a quotient below the step's exact range (2^-19, rare) is redone by encode_sr.
-template <int G>
-__device__ __forceinline__ void encode_sr_pair(const float2* A, float2 s, float c, uint64_t seedx,
-                                               uint64_t quad0_0, uint64_t quad0_1, uint2& w0,
-                                               uint2& w1) {
-  const bool z0 = s.x == 0.0f, z1 = s.y == 0.0f;
-  // a zero block's lane divides by 1 (its codes are zeros whatever its quotients)
-  const Divider d0 = make_divider(z0 ? 1.0f : s.x, c), d1 = make_divider(z1 ? 1.0f : s.y, c);
-  if (!(d0.fast && d1.fast)) {
-    w0 = encode_sr_lane<G>(A, 0, s.x, c, seedx, quad0_0);
-    w1 = encode_sr_lane<G>(A, 1, s.y, c, seedx, quad0_1);
-    return;
-  }
-  uint32_t r0[8], r1[8];
-  sr_words16(seedx, quad0_0, r0);
-  sr_words16(seedx, quad0_1, r1);
-  const float2 R2 = make_float2(d0.R, d1.R), nS2 = make_float2(-d0.S, -d1.S);
-  float m0 = 0x1p+30f, m1 = 0x1p+30f;
-  uint32_t c0[2], c1[2];
-#pragma unroll
-  for (int l = 0; l < 2; ++l) {
-    uint32_t ma0 = 0u, sg0 = 0u, ma1 = 0u, sg1 = 0u;
-#pragma unroll
-    for (int j = 7; j >= 0; j -= 2) {
-      const int e = 8 * l + j;
-      float2 q[2];
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const float2 q0 = __fmul2_rn(A[e - t], R2);
-        q[t] = __ffma2_rn(__ffma2_rn(q0, nS2, A[e - t]), R2, q0);
-      }
-      m0 = min3(m0, fabsf(q[0].x), fabsf(q[1].x));
-      m1 = min3(m1, fabsf(q[0].y), fabsf(q[1].y));
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        sr_append<G>(sr_bits<G>(q[t].x, r0, e - t), A[e - t].x, ma0, sg0);
-        sr_append<G>(sr_bits<G>(q[t].y, r1, e - t), A[e - t].y, ma1, sg1);
-      }
-    }
-    c0[l] = sr_word<G>(ma0, sg0);
-    c1[l] = sr_word<G>(ma1, sg1);
-  }
-  w0 = z0 ? make_uint2(0u, 0u) : make_uint2(c0[0], c0[1]);
-  w1 = z1 ? make_uint2(0u, 0u) : make_uint2(c1[0], c1[1]);
-  if (m0 < 0x1p-19f && !z0) w0 = encode_sr_lane<G>(A, 0, s.x, c, seedx, quad0_0);
-  if (m1 < 0x1p-19f && !z1) w1 = encode_sr_lane<G>(A, 1, s.y, c, seedx, quad0_1);
-}
-
 // IF4 block, E4M3 block scale (NVFP4's), codes only: the E2M1 candidate (round to nearest even,
 // saturating) and the INT4 candidate k = RNE(RN(v * RN(7/6))) clamped to +-7 with value
 // RN(k * RN(6/7)); INT4 is kept iff its squared error, summed in FP32 over the balanced pairwise

@@ -92,6 +92,18 @@ def test_every_workload_constructs():
         assert bench.make_workload(rec["workload"]).kernel_key == key
 
 
+def test_traffic_records_match_the_current_kernel_sources():
+    import json
+    # every committed ncu record was taken on the kernel sources in the tree: a kernel change
+    # without a new capture would make the bench report traffic as null
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    with open(os.path.join(root, "profiles", "traffic.json")) as f:
+        recs = json.load(f)
+    for key, rec in recs.items():
+        assert list(rec["sources"]) == list(bench.kernel_sources(key)), key
+        assert rec["source_sha"] == bench.kernel_source_sha(files=bench.kernel_sources(key)), key
+
+
 _MAKE_WORKLOAD = bench.make_workload
 
 
