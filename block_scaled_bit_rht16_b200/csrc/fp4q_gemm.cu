@@ -14,19 +14,21 @@
 // A persistent kernel: one CTA per SM (up to 217 KB of shared memory, 256 or 512 tensor-memory
 // columns) walks the 128 x BN tiles of D (BN = 256 when N allows, else 128), tile i of a CTA
 // being blockIdx.x + i * gridDim.x with m fastest. The K dimension streams in 256-element steps
-// through a ring of shared-memory buffers that runs on across tiles. Six warps, three roles:
-//   thread 0 (producer): per step the A and B code tiles (128 / BN rows x 128 bytes) by 2-D TMA
-//     copies with the 128-byte swizzle, and the step's 512-byte MMA-layout scale tiles (per 128
-//     rows: four for NVFP4, two for MXFP4) by 3-D TMA copies whose zero-stride middle dimension
-//     lands each tile four times in a row (kSfRep), all completing on the buffer's `full`
+// through a ring of shared-memory buffers that runs on across tiles. Ten warps, four roles:
+//   thread 0 (producer): per step the A and B code tiles (128 / BN rows x 128 bytes) and the
+//     step's 512-byte MMA-layout scale tiles (per 128 rows: four for NVFP4, two for MXFP4) by
+//     2-D TMA copies (codes with the 128-byte swizzle), all completing on the buffer's `full`
 //     mbarrier; a buffer is refilled once its `empty` barrier says the MMAs that read it have
 //     completed, so the next tile's operands load while the current tile drains;
+//   warps 6-9 (scales): per step, warp w writes row l of each scale tile into tensor-memory
+//     lane 32 (w % 4) + l of the stage's scale columns (tcgen05.st), so that the four warps
+//     together fill the four lane quarters with the same 32 rows, the layout the block-scaled
+//     MMA reads, and arrive on the buffer's `sf_full` barrier;
 //   thread 32 (MMA issuer): per tile, once `acc_empty` says the epilogue has read the previous
-//     accumulator, copies each step's scales into tensor memory two tiles at a time
-//     (tcgen05.cp .128x256b: the replicated rows fill all four lane quarters), issues four MMAs
-//     of K = 64 (tcgen05.mma kind::mxf4nvf4, block16 with E4M3 or block32 with UE8M0 scales,
-//     M = 128, N = BN) and commits them to the buffer's `empty` barrier; the tile's last commit
-//     goes to `acc_full`;
+//     accumulator, per step waits for `full` and `sf_full`, issues four MMAs of K = 64
+//     (tcgen05.mma kind::mxf4nvf4, block16 with E4M3 or block32 with UE8M0 scales, M = 128,
+//     N = BN) and commits them to the buffer's `empty` barrier; the tile's last commit goes to
+//     `acc_full`;
 //   warps 2-5 (epilogue): warp w reads tensor-memory lanes 32 (w % 4) .. +31 (tcgen05.ld, 32
 //     columns at a time), scales by alpha_A alpha_B, stores bf16 rows, and arrives on `acc_empty`.
 // Every mbarrier wait is bounded by the global timer; a wait that gives up sets bit 0 of the
@@ -50,24 +52,19 @@ namespace fp4q {
 namespace {
 
 constexpr int kBM = 128, kBKBytes = 128;   // 256 FP4 values per row per step
-constexpr int kGThreads = 192;   // warp 0 producer, warp 1 MMA issuer, warps 2-5 epilogue
+constexpr int kGThreads = 320;   // warp 0 producer, warp 1 MMA issuer, warps 2-5 epilogue, 6-9 scales
 constexpr uint32_t kTileA = kBM * kBKBytes;   // 16 KB
 // Per tile width BN (128 or 256) and scale kind (MX: UE8M0 per 32 elements, else E4M3 per 16):
 // stages, shared memory, tensor memory. A 512-byte MMA-layout scale tile covers 128 rows and
 // 4 scale columns: K = 64 (NVFP4) or 128 (MXFP4), so a 256-deep step takes 4 or 2 of them per 128
 // rows.
-// In shared memory each scale tile lands four times in a row (kSfRep: the tensor map repeats
-// it along a zero-stride dimension), so that one 128x256b tcgen05.cp (128 lanes x 8 columns;
-// rows r and r + 32k read the same bytes) puts two tiles into tensor memory exactly as two
-// 32x128b.warpx4 copies would: the copies, which run in the tensor pipe in issue order with the
-// MMAs, are halved.
-constexpr uint32_t kSfRep = 4 * 512;
+constexpr uint32_t kSfTile = 512;
 template <int BN, bool MX>
 struct GemmCfg {
-  static constexpr int kStages = BN == 256 ? 3 : (MX ? 5 : 4);
+  static constexpr int kStages = BN == 256 ? 4 : 6;
   static constexpr uint32_t kTileB = BN * kBKBytes;
   static constexpr int kSfTiles = MX ? 2 : 4;                     // per 128 rows per step
-  static constexpr uint32_t kSfA = kSfTiles * kSfRep;
+  static constexpr uint32_t kSfA = kSfTiles * kSfTile;
   static constexpr uint32_t kSfB = (BN / 128) * kSfA;
   static constexpr uint32_t kStageTx = kTileA + kTileB + kSfA + kSfB;
   static constexpr uint32_t kSfCols = 4 * kSfTiles * (1 + BN / 128);   // A then B, 4 columns a tile
@@ -88,6 +85,7 @@ struct GemmSmem {
   uint8_t b[C::kStages][C::kTileB];
   uint64_t full[C::kStages];
   uint64_t empty[C::kStages];
+  uint64_t sf_full[C::kStages];   // the step's scales are in tensor memory (one arrival per scale warp)
   uint64_t acc_full;    // the MMAs of a tile have completed (tcgen05.commit)
   uint64_t acc_empty;   // the epilogue warps have read the accumulator (one arrival per warp)
   uint64_t done;        // every MMA and scale copy issued has completed
@@ -95,20 +93,23 @@ struct GemmSmem {
 };
 template <int BN, bool MX>
 constexpr size_t gemm_smem_bytes() { return sizeof(GemmSmem<BN, MX>) + 1024; }
+// The code tiles start on the 128-byte swizzle's 1024-byte period (the scale buffers before them
+// fill whole periods), shared memory fits one CTA (227 KB) and the accumulator plus every stage's
+// scale columns fit the tensor memory allocated.
+template <int BN, bool MX>
+constexpr bool gemm_layout_ok() {
+  using C = GemmCfg<BN, MX>;
+  return (C::kStages * (C::kSfA + C::kSfB)) % 1024 == 0 && gemm_smem_bytes<BN, MX>() <= 232448 &&
+         BN + C::kStages * C::kSfCols <= C::kTmemCols && C::kTmemCols <= 512;
+}
+static_assert(gemm_layout_ok<256, false>() && gemm_layout_ok<256, true>() && gemm_layout_ok<128, false>() &&
+              gemm_layout_ok<128, true>(), "GEMM shared- or tensor-memory layout");
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3}], [%4];"
       ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];"
-      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -123,6 +124,47 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                ::"r"(smem_u32(bar)) : "memory");
+}
+
+// N consecutive 32-bit tensor-memory columns of the warp's 32 lanes from r[0..N) (tcgen05.st
+// 32x32b: thread l writes lane quarter base + l); the caller waits with tcgen05.wait::st.
+template <int N>
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t* r);
+template <>
+__device__ __forceinline__ void tmem_st<8>(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+               ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_st<16>(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+               ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+                 "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+               : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_st<32>(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+               "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+               ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+                 "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+                 "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+                 "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+               : "memory");
+}
+
+// The 16 bytes of row `lane` of each of n 512-byte scale tiles (tile i at src + i * stride) into
+// r[4 i .. 4 i + 3].
+__device__ __forceinline__ void load_sf_rows(const uint8_t* src, uint32_t stride, int n, int lane, uint32_t* r) {
+#pragma unroll
+  for (int i = 0; i < n; ++i) {
+    const uint4 v = *reinterpret_cast<const uint4*>(src + i * stride + 16 * lane);
+    r[4 * i] = v.x;
+    r[4 * i + 1] = v.y;
+    r[4 * i + 2] = v.z;
+    r[4 * i + 3] = v.w;
+  }
 }
 
 template <int BN, bool MX>
@@ -147,6 +189,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
+      mbar_init(&sm.sf_full[s], 4);
     }
     mbar_init(&sm.acc_full, 1);
     mbar_init(&sm.acc_empty, 4);
@@ -180,11 +223,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
         mbar_arrive_expect_tx(&sm.full[s], C::kStageTx);
         tma_load_2d(sm.a[s], &tmA, kt * kBKBytes, (int)m0, &sm.full[s]);
         tma_load_2d(sm.b[s], &tmB, kt * kBKBytes, (int)n0, &sm.full[s]);
-        // the step's kSfTiles scale tiles of A and of each 128-row group of B, each four times
-        tma_load_3d(sm.sfa[s], &tmSA, 0, 0, (int)(m0 / 128) * row_tiles + kt * C::kSfTiles, &sm.full[s]);
+        // the step's kSfTiles scale tiles of A and of each 128-row group of B
+        tma_load_2d(sm.sfa[s], &tmSA, 0, (int)(m0 / 128) * row_tiles + kt * C::kSfTiles, &sm.full[s]);
 #pragma unroll
         for (int j = 0; j < BN / 128; ++j)
-          tma_load_3d(sm.sfb[s] + j * C::kSfA, &tmSB, 0, 0, (int)(n0 / 128 + j) * row_tiles + kt * C::kSfTiles,
+          tma_load_2d(sm.sfb[s] + j * C::kSfA, &tmSB, 0, (int)(n0 / 128 + j) * row_tiles + kt * C::kSfTiles,
                       &sm.full[s]);
       }
     }
@@ -199,30 +242,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
       for (int kt = 0; kt < ksteps; ++kt, ++it) {
         const int s = it % S;
         if (!mbar_wait(&sm.full[s], (uint32_t)((it / S) & 1))) { fail = 1; break; }
+        if (!mbar_wait(&sm.sf_full[s], (uint32_t)((it / S) & 1))) { fail = 1; break; }
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         // scale tile t of A at columns sa + 4t; tile t of B's 128-row group j at sb + 4 (BN/128) t + 4j
         const uint32_t sa = tmem_sf + (uint32_t)s * C::kSfCols, sb = sa + 4u * C::kSfTiles;
-        // a copy's source: 128 rows of 32 bytes = 8-row groups 128 bytes apart (SBO) within one
-        // repeated tile, the second 16 bytes of each row (the second tile) LBO further on. A and
-        // BN = 128 pair tiles (2p, 2p + 1); BN = 256 pairs the two row groups' tile tt.
-#pragma unroll
-        for (int p = 0; p < C::kSfTiles / 2; ++p) {
-          const uint64_t da = smem_desc(smem_u32(sm.sfa[s] + p * 2 * kSfRep), kSfRep, 128u, 0u);
-          asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(sa + 8u * p), "l"(da) : "memory");
-        }
-        if constexpr (BN == 256) {
-#pragma unroll
-          for (int tt = 0; tt < C::kSfTiles; ++tt) {
-            const uint64_t db = smem_desc(smem_u32(sm.sfb[s] + tt * kSfRep), C::kSfA, 128u, 0u);
-            asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(sb + 8u * tt), "l"(db) : "memory");
-          }
-        } else {
-#pragma unroll
-          for (int p = 0; p < C::kSfTiles / 2; ++p) {
-            const uint64_t db = smem_desc(smem_u32(sm.sfb[s] + p * 2 * kSfRep), kSfRep, 128u, 0u);
-            asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(sb + 8u * p), "l"(db) : "memory");
-          }
-        }
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb) {
           // K-major, 128-byte swizzle: 8-row groups 1024 bytes apart; K-block kb starts 32 bytes in
@@ -255,6 +278,47 @@ __global__ void __launch_bounds__(kGThreads, 1)
     }
     // arrives when every MMA and scale copy issued above has completed
     umma_commit(&sm.done);
+  } else if (warp >= 6) {
+    // scale warps: warp w writes tensor-memory lanes 32 (w % 4) .. +31. Per step, once the
+    // buffer's copies have landed (and so the MMAs that last read the stage's scale columns have
+    // completed: the buffer was refilled only after them), row l of each of the step's 512-byte
+    // scale tiles (its first repeat) goes to lane l of the tile's four columns; the four warps
+    // together fill all four lane quarters with the same rows, the layout the MMAs read.
+    const uint32_t quarter_base = (uint32_t)(32 * (warp & 3)) << 16;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < ntiles && !fail; tile += gridDim.x) {
+      for (int kt = 0; kt < ksteps; ++kt, ++it) {
+        const int s = it % S;
+        // warp-uniform: every lane takes the same branch before the collective stores
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.full[s], (uint32_t)((it / S) & 1)))) { fail = 1; break; }
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t sa = tmem_sf + quarter_base + (uint32_t)s * C::kSfCols, sb = sa + 4u * C::kSfTiles;
+        {
+          uint32_t r[4 * C::kSfTiles];   // A: tile t at columns sa + 4t
+          load_sf_rows(sm.sfa[s], kSfTile, C::kSfTiles, lane, r);
+          tmem_st<4 * C::kSfTiles>(sa, r);
+        }
+        {
+          // B: tile t of 128-row group j at columns sb + 4 (BN / 128) t + 4 j
+          constexpr int kG = BN / 128;
+          uint32_t r[4 * C::kSfTiles * kG];
+#pragma unroll
+          for (int j = 0; j < kG; ++j) {
+            uint32_t g[4 * C::kSfTiles];
+            load_sf_rows(sm.sfb[s] + j * C::kSfA, kSfTile, C::kSfTiles, lane, g);
+#pragma unroll
+            for (int tt = 0; tt < C::kSfTiles; ++tt)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) r[4 * (kG * tt + j) + i] = g[4 * tt + i];
+          }
+          tmem_st<4 * C::kSfTiles * kG>(sb, r);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.sf_full[s]);
+      }
+    }
   } else if (warp >= 2) {
     // epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. +31 (rows of the tile) 32 columns
     // at a time, stores them as bf16 x alpha, and releases the accumulator to the next tile's
@@ -264,7 +328,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
     int j = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
       const int64_t m0 = (int64_t)(tile % tiles_m) * kBM, n0 = (int64_t)(tile / tiles_m) * BN;
-      if (!mbar_wait(&sm.acc_full, (uint32_t)(j & 1))) { fail = 1; break; }
+      // warp-uniform: every lane takes the same branch before the collective loads
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.acc_full, (uint32_t)(j & 1)))) { fail = 1; break; }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       uint4* dst = reinterpret_cast<uint4*>(out + (m0 + 32 * quarter + lane) * ldo + n0);
 #pragma unroll 1
@@ -337,17 +402,16 @@ cudaError_t make_codes_map(const uint8_t* codes, int64_t rows, int64_t K, int bo
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// 3-D map of MMA-layout scales (uint8 [rows / 128 * row_tiles] tiles of 512 bytes) as 32-bit words:
-// 128 words of a tile, the tile repeated four times (a zero stride), the tiles; a box of
-// `tiles` consecutive tiles lands as tile 0 x4, tile 1 x4, ... in shared memory.
+// 2-D map of MMA-layout scales (uint8 [rows / 128 * row_tiles] tiles of 512 bytes) as 32-bit words:
+// 128 words of a tile, the tiles; a box of `tiles` consecutive tiles lands contiguously.
 cudaError_t make_scales_map(const uint8_t* scales, int64_t total_tiles, int tiles, CUtensorMap* map) {
   auto enc = gemm_tensor_map_encoder();
   if (enc == nullptr) return cudaErrorNotSupported;
-  const cuuint64_t dims[3] = {128, 4, (cuuint64_t)total_tiles};
-  const cuuint64_t strides[2] = {0, 512};
-  const cuuint32_t box[3] = {128, 4, (cuuint32_t)tiles};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t*>(scales), dims, strides,
+  const cuuint64_t dims[2] = {128, (cuuint64_t)total_tiles};
+  const cuuint64_t strides[1] = {512};
+  const cuuint32_t box[2] = {128, (cuuint32_t)tiles};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t*>(scales), dims, strides,
                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
