@@ -13,7 +13,8 @@
 //
 // A persistent kernel: one CTA per SM (up to 217 KB of shared memory, 256 or 512 tensor-memory
 // columns) walks the 128 x BN tiles of D (BN = 256 when N allows, else 128), tile i of a CTA
-// being blockIdx.x + i * gridDim.x with m fastest. The K dimension streams in 256-element steps
+// being blockIdx.x + i * gridDim.x with m fastest; when the last round's tiles fit the grid twice
+// over, each of them is split into two 128 x 128 halves on two CTAs (GemmItem). The K dimension streams in 256-element steps
 // through a ring of shared-memory buffers that runs on across tiles. Ten warps, four roles:
 //   thread 0 (producer): per step the A and B code tiles (128 / BN rows x 128 bytes) and the
 //     step's 512-byte MMA-layout scale tiles (per 128 rows: four for NVFP4, two for MXFP4) by
@@ -67,6 +68,7 @@ struct GemmCfg {
   static constexpr uint32_t kSfA = kSfTiles * kSfTile;
   static constexpr uint32_t kSfB = (BN / 128) * kSfA;
   static constexpr uint32_t kStageTx = kTileA + kTileB + kSfA + kSfB;
+  static constexpr uint32_t kStageTxHalf = kTileA + kTileB / 2 + kSfA + kSfB / 2;   // a half tile (BN = 256)
   static constexpr uint32_t kSfCols = 4 * kSfTiles * (1 + BN / 128);   // A then B, 4 columns a tile
   static constexpr uint32_t kTmemCols = (BN + kStages * kSfCols) <= 256 ? 256 : 512;
   // kind::mxf4nvf4: E2M1 A and B (format 1), K-major, N / 8 in bits 17-22, scale type in bit 23
@@ -74,6 +76,8 @@ struct GemmCfg {
   // 32-bit scale column a 32-element-block MMA reads: 0 or 2) in bits 4-5 (B) and 29-30 (A)
   static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                      ((MX ? 1u : 0u) << 23) | ((uint32_t)(kBM >> 4) << 24);
+  // the same with N = BN / 2 (a half tile)
+  static constexpr uint32_t kIdescHalf = (kIdesc & ~(0x3Fu << 17)) | ((uint32_t)(BN >> 4) << 17);
 };
 
 template <int BN, bool MX>
@@ -167,9 +171,34 @@ __device__ __forceinline__ void load_sf_rows(const uint8_t* src, uint32_t stride
   }
 }
 
+// Work item i of a launch over ntiles tiles on `grid` CTAs: tile i (m fastest), except that when
+// BN = 256 and the last round's rem = ntiles % grid tiles fit the grid twice over, each of those
+// tiles becomes two items of half its width (BN / 2 columns at n0 and n0 + BN / 2), so that the
+// last round takes about half as long. Every role walks the same items.
+struct GemmItem {
+  int64_t m0, n0;
+  int half;   // 1: a half tile
+};
+template <int BN>
+__device__ __forceinline__ int gemm_split_tiles(int ntiles, int grid) {
+  const int rem = ntiles % grid;
+  return (BN == 256 && ntiles > grid && 2 * rem <= grid) ? rem : 0;
+}
+template <int BN>
+__device__ __forceinline__ GemmItem gemm_item(int i, int tiles_m, int ntiles, int split) {
+  GemmItem w;
+  const int nfull = ntiles - split;
+  const int tile = i < nfull ? i : nfull + ((i - nfull) >> 1);
+  w.half = i < nfull ? 0 : 1;
+  w.m0 = (int64_t)(tile % tiles_m) * kBM;
+  w.n0 = (int64_t)(tile / tiles_m) * BN + (w.half ? (int64_t)((i - nfull) & 1) * (BN / 2) : 0);
+  return w;
+}
+
 template <int BN, bool MX>
 __global__ void __launch_bounds__(kGThreads, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const __grid_constant__ CUtensorMap tmBh,
                       const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
                       const float* __restrict__ ts_a, const float* __restrict__ ts_b,
                       __nv_bfloat16* __restrict__ out, int64_t ldo, int64_t M, int64_t N, int64_t K,
@@ -182,6 +211,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int tiles_m = (int)(M / kBM);
   const int ntiles = tiles_m * (int)(N / BN);
+  const int split = gemm_split_tiles<BN>(ntiles, (int)gridDim.x);
+  const int nitems = ntiles + split;
   const int ksteps = (int)(K / 256);
   const int row_tiles = (int)(K / (MX ? 128 : 64));   // 512-byte scale tiles per 128-row tile row
 
@@ -209,25 +240,25 @@ __global__ void __launch_bounds__(kGThreads, 1)
   const uint32_t tmem_acc = tmem;                 // lanes 0..127, columns 0..BN-1
   const uint32_t tmem_sf = tmem + BN;             // then S x (A: 16, B: BN/8) columns
 
-  // Tiles are visited in the same order by every role: tile i of this CTA is
-  // blockIdx.x + i * gridDim.x, m fastest (CTAs in flight share B tiles in L2).
+  // Items are visited in the same order by every role: item i of this CTA is
+  // blockIdx.x + i * gridDim.x (tiles m fastest: CTAs in flight share B tiles in L2).
   int fail = 0;
   int issued = 0;   // producer: steps whose copies have been issued
   if (t == 0) {
     // producer: refills a buffer once the MMAs that read it have completed
-    for (int tile = blockIdx.x; tile < ntiles && !fail; tile += gridDim.x) {
-      const int64_t m0 = (int64_t)(tile % tiles_m) * kBM, n0 = (int64_t)(tile / tiles_m) * BN;
+    for (int i = blockIdx.x; i < nitems && !fail; i += gridDim.x) {
+      const GemmItem w = gemm_item<BN>(i, tiles_m, ntiles, split);
+      const int groups = w.half ? BN / 256 : BN / 128;   // 128-row groups of B in the item
       for (int kt = 0; kt < ksteps; ++kt, ++issued) {
         const int s = issued % S;
         if (issued >= S && !mbar_wait(&sm.empty[s], (uint32_t)(((issued / S) - 1) & 1))) { fail = 1; break; }
-        mbar_arrive_expect_tx(&sm.full[s], C::kStageTx);
-        tma_load_2d(sm.a[s], &tmA, kt * kBKBytes, (int)m0, &sm.full[s]);
-        tma_load_2d(sm.b[s], &tmB, kt * kBKBytes, (int)n0, &sm.full[s]);
+        mbar_arrive_expect_tx(&sm.full[s], w.half ? C::kStageTxHalf : C::kStageTx);
+        tma_load_2d(sm.a[s], &tmA, kt * kBKBytes, (int)w.m0, &sm.full[s]);
+        tma_load_2d(sm.b[s], w.half ? &tmBh : &tmB, kt * kBKBytes, (int)w.n0, &sm.full[s]);
         // the step's kSfTiles scale tiles of A and of each 128-row group of B
-        tma_load_2d(sm.sfa[s], &tmSA, 0, (int)(m0 / 128) * row_tiles + kt * C::kSfTiles, &sm.full[s]);
-#pragma unroll
-        for (int j = 0; j < BN / 128; ++j)
-          tma_load_2d(sm.sfb[s] + j * C::kSfA, &tmSB, 0, (int)(n0 / 128 + j) * row_tiles + kt * C::kSfTiles,
+        tma_load_2d(sm.sfa[s], &tmSA, 0, (int)(w.m0 / 128) * row_tiles + kt * C::kSfTiles, &sm.full[s]);
+        for (int j = 0; j < groups; ++j)
+          tma_load_2d(sm.sfb[s] + j * C::kSfA, &tmSB, 0, (int)(w.n0 / 128 + j) * row_tiles + kt * C::kSfTiles,
                       &sm.full[s]);
       }
     }
@@ -236,7 +267,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
     // tensor memory and four MMAs of K = 64 per step; the tile's last commit goes to acc_full
     int it = 0;
     int j = 0;
-    for (int tile = blockIdx.x; tile < ntiles && !fail; tile += gridDim.x, ++j) {
+    for (int i = blockIdx.x; i < nitems && !fail; i += gridDim.x, ++j) {
+      const bool half = i >= ntiles - split;
+      // a half tile: N = BN / 2, B's scales in the one-group layout (tile t at sb + 4t)
+      const uint32_t idesc_base = half ? C::kIdescHalf : C::kIdesc;
+      const uint32_t sfb_stride = half ? 4u : 4u * (uint32_t)(BN / 128);
       if (j > 0 && !mbar_wait(&sm.acc_empty, (uint32_t)((j - 1) & 1))) { fail = 1; break; }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       for (int kt = 0; kt < ksteps; ++kt, ++it) {
@@ -256,8 +291,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
           // 2 (kb % 2) and 2 (kb % 2) + 1 (the scale-factor ids)
           const int tt = MX ? kb >> 1 : kb;
           const uint32_t id = MX ? 2u * (uint32_t)(kb & 1) : 0u;
-          const uint32_t idesc = C::kIdesc | (id << 4) | (id << 29);
-          const uint32_t sfa_col = sa + 4u * tt, sfb_col = sb + 4u * (uint32_t)(BN / 128) * tt;
+          const uint32_t idesc = idesc_base | (id << 4) | (id << 29);
+          const uint32_t sfa_col = sa + 4u * tt, sfb_col = sb + sfb_stride * tt;
           if constexpr (MX)
             asm volatile(
                 "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
@@ -282,11 +317,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
     // scale warps: warp w writes tensor-memory lanes 32 (w % 4) .. +31. Per step, once the
     // buffer's copies have landed (and so the MMAs that last read the stage's scale columns have
     // completed: the buffer was refilled only after them), row l of each of the step's 512-byte
-    // scale tiles (its first repeat) goes to lane l of the tile's four columns; the four warps
-    // together fill all four lane quarters with the same rows, the layout the MMAs read.
+    // scale tiles goes to lane l of the tile's four columns; the four warps together fill all four
+    // lane quarters with the same rows, the layout the MMAs read.
     const uint32_t quarter_base = (uint32_t)(32 * (warp & 3)) << 16;
     int it = 0;
-    for (int tile = blockIdx.x; tile < ntiles && !fail; tile += gridDim.x) {
+    for (int i = blockIdx.x; i < nitems && !fail; i += gridDim.x) {
+      const bool half = i >= ntiles - split;
       for (int kt = 0; kt < ksteps; ++kt, ++it) {
         const int s = it % S;
         // warp-uniform: every lane takes the same branch before the collective stores
@@ -298,7 +334,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
           load_sf_rows(sm.sfa[s], kSfTile, C::kSfTiles, lane, r);
           tmem_st<4 * C::kSfTiles>(sa, r);
         }
-        {
+        if (BN == 256 && half) {
+          // a half tile's one 128-row group of B: tile t at columns sb + 4t
+          uint32_t r[4 * C::kSfTiles];
+          load_sf_rows(sm.sfb[s], kSfTile, C::kSfTiles, lane, r);
+          tmem_st<4 * C::kSfTiles>(sb, r);
+        } else {
           // B: tile t of 128-row group j at columns sb + 4 (BN / 128) t + 4 j
           constexpr int kG = BN / 128;
           uint32_t r[4 * C::kSfTiles * kG];
@@ -309,7 +350,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
 #pragma unroll
             for (int tt = 0; tt < C::kSfTiles; ++tt)
 #pragma unroll
-              for (int i = 0; i < 4; ++i) r[4 * (kG * tt + j) + i] = g[4 * tt + i];
+              for (int q = 0; q < 4; ++q) r[4 * (kG * tt + j) + q] = g[4 * tt + q];
           }
           tmem_st<4 * C::kSfTiles * kG>(sb, r);
         }
@@ -326,14 +367,16 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const float alpha = MX ? 1.0f : __fmul_rn(*ts_a, *ts_b);   // MXFP4 has no tensor scale
     const int quarter = warp & 3;
     int j = 0;
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
-      const int64_t m0 = (int64_t)(tile % tiles_m) * kBM, n0 = (int64_t)(tile / tiles_m) * BN;
+    for (int i = blockIdx.x; i < nitems; i += gridDim.x, ++j) {
+      const GemmItem w = gemm_item<BN>(i, tiles_m, ntiles, split);
+      const int64_t m0 = w.m0, n0 = w.n0;
+      const int cols = w.half ? BN / 2 : BN;
       // warp-uniform: every lane takes the same branch before the collective loads
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(&sm.acc_full, (uint32_t)(j & 1)))) { fail = 1; break; }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       uint4* dst = reinterpret_cast<uint4*>(out + (m0 + 32 * quarter + lane) * ldo + n0);
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      for (int c0 = 0; c0 < cols; c0 += 32) {
         uint32_t v[32];
         asm volatile(
             "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -438,10 +481,12 @@ cudaError_t launch_gemm_bn(const uint8_t* a_codes, const uint8_t* a_scales, cons
                            const uint8_t* b_codes, const uint8_t* b_scales, const float* b_ts,
                            int64_t M, int64_t N, int64_t K, uint16_t* out, int64_t ldo, cudaStream_t st) {
   using C = GemmCfg<BN, MX>;
-  alignas(64) CUtensorMap ma, mb, msa, msb;
+  alignas(64) CUtensorMap ma, mb, mbh, msa, msb;
   cudaError_t e = make_codes_map(a_codes, M, K, kBM, &ma);
   if (e != cudaSuccess) return e;
   e = make_codes_map(b_codes, N, K, BN, &mb);
+  if (e != cudaSuccess) return e;
+  e = make_codes_map(b_codes, N, K, BN / 2, &mbh);   // half tiles' B (used only when BN = 256)
   if (e != cudaSuccess) return e;
   const int64_t row_tiles = K / (MX ? 128 : 64);
   e = make_scales_map(a_scales, M / 128 * row_tiles, C::kSfTiles, &msa);
@@ -469,7 +514,7 @@ cudaError_t launch_gemm_bn(const uint8_t* a_codes, const uint8_t* a_scales, cons
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, MX>, ma, mb, msa, msb, a_ts, b_ts,
+  e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, MX>, ma, mb, mbh, msa, msb, a_ts, b_ts,
                          reinterpret_cast<__nv_bfloat16*>(out), ldo, M, N, K, status);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
