@@ -103,3 +103,30 @@ def test_gemm_agrees_with_cublaslt_and_timing():
                                          tf["cublaslt"], sq))
     # both accumulate exact products in FP32 (in different orders) and round to bf16
     assert sq > 45.0
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+def test_half_tiles_of_the_last_round_equal_whole_tiles(fmt):
+    # 4096 x 1280: 160 tiles of 128 x 256 on at most 148 CTAs, so the last round's tiles run as
+    # 128 x 128 halves; the column blocks [0, 1024) and [1024, 1280) as GEMMs of their own (128
+    # and 32 tiles) run as whole tiles. Each output element is the same sum in the same order.
+    import torch
+    M, N, K = 4096, 1280, 512
+    scale = fq.FP4Q_SCALE_E4M3_1x16_TENSOR if fmt == "nvfp4" else fq.FP4Q_SCALE_UE8M0_1x32
+    cfg = fq.Config(grid=fq.FP4Q_GRID_E2M1, scale=scale, rht=1,
+                    sign_mask=fq.sign_mask_from_seed(synth.sign_seed(2)), mma_scales=True)
+    gemm = fq.gemm_nvfp4 if fmt == "nvfp4" else fq.gemm_mxfp4
+    qa = fq.rht_quantize(cfg, to_dev(synth.small(93, M, K, "t4")))
+    b = to_dev(synth.small(94, N, K, "normal", 0.02))
+    qb = fq.rht_quantize(cfg, b)
+    whole = gemm(qa, qb)
+    parts = []
+    for c0, c1 in ((0, 1024), (1024, N)):
+        # the rows of B quantized alone, with the whole B's tensor scale (NVFP4): the same codes
+        # and block scales as those rows of qb
+        q = fq.rht_quantize(cfg, b[c0:c1].contiguous(), tensor_scale=qb.tensor_scale,
+                            tensor_scale_given=fmt == "nvfp4")
+        parts.append(gemm(qa, q))
+    torch.cuda.synchronize()
+    assert torch.equal(whole[:, :1024], parts[0])
+    assert torch.equal(whole[:, 1024:], parts[1])
